@@ -1,0 +1,603 @@
+// C ABI of the HiKVP knowledge-graph attention library (see include/atlaskv.h).
+//
+// Host side: argument validation, workspace planning and kernel launches.  All
+// device work of atlaskv_attend runs in the kernels of descend.cuh,
+// staging.cuh and attend.cuh; nothing here computes on the host.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "atlaskv.h"
+#include "attend.cuh"
+#include "descend.cuh"
+#include "staging.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+atlaskv_status fail(atlaskv_status st, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+#define AKV_CUDA(call)                                                                                 \
+    do {                                                                                               \
+        cudaError_t e_ = (call);                                                                       \
+        if (e_ != cudaSuccess) return fail(ATLASKV_ECUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+    } while (0)
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+int pow2_at_least(long long x, int floor_)
+{
+    int p = floor_;
+    while (p < x) p <<= 1;
+    return p;
+}
+
+constexpr int kMaxCandidates = 8192;   // per level and traversal (shared-memory bound of the descent CTA)
+constexpr int kNumEvents = 6;
+
+}  // namespace
+
+struct atlaskv_tree {
+    atlaskv_tree_desc d;
+    long long rows[3];
+    const void *leaf_keys_dev;     // device-accessible leaf pointers (mapped for host leaves)
+    const void *leaf_values_dev;
+    float *norm_bound;             // device [3][H_kv]
+    int *status;                   // device sticky status word
+    bool profiling;
+    bool timed;                    // the last attend recorded events
+    bool host_mode_last;
+    cudaEvent_t ev[kNumEvents];
+};
+
+namespace {
+
+size_t esize(int dtype) { return dtype == ATLASKV_F32 ? 4 : 2; }
+
+struct Layout {
+    size_t s_ws, anorm_ws, kept[3], leaf_slot, kept_leaf_row, vslot, umid, ucount_mid, uleaf, ucount_leaf,
+        key_pool, val_pool, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Layout plan(const atlaskv_tree *t, const atlaskv_params *p, int B, int N, int H, int T)
+{
+    (void)N;
+    (void)T;
+    Layout L{};
+    const size_t BH = (size_t)B * H;
+    const int D = t->d.head_dim;
+    const bool host = t->d.leaf_location == ATLASKV_LEAVES_HOST_PINNED;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    L.s_ws = take(BH * D * 4);
+    L.anorm_ws = take(BH * 4);
+    for (int l = 0; l < 3; ++l) L.kept[l] = take(BH * (size_t)(l == 0 ? p->K_root : l == 1 ? p->K_mid : p->K_leaf) * 4);
+    if (host) {
+        const int G = H / t->d.n_kv_heads;
+        const size_t groups = (size_t)B * t->d.n_kv_heads;
+        const size_t n_mid = (size_t)G * p->K_mid, n_leaf = (size_t)G * p->K_leaf;
+        L.leaf_slot = take(BH * p->K_mid * 4);
+        L.kept_leaf_row = take(BH * p->K_leaf * 4);
+        L.vslot = take(BH * p->K_leaf * 4);
+        L.umid = take(groups * n_mid * 4);
+        L.ucount_mid = take(groups * 4);
+        L.uleaf = take(groups * n_leaf * 4);
+        L.ucount_leaf = take(groups * 4);
+        L.key_pool = take(groups * n_mid * (size_t)t->d.fanout[2] * D * esize(t->d.dtype));
+        L.val_pool = take(groups * n_leaf * D * esize(t->d.dtype));
+    }
+    L.total = off;
+    return L;
+}
+
+atlaskv_status check_params(const atlaskv_tree *t, const atlaskv_params *p, int B, int N, int H, int T)
+{
+    if (!t || !p) return fail(ATLASKV_EINVAL, "null tree or params");
+    const int *fo = t->d.fanout;
+    if (B < 0) return fail(ATLASKV_EINVAL, "B = %d < 0", B);
+    if (H < 1 || H % t->d.n_kv_heads != 0)
+        return fail(ATLASKV_EINVAL, "H = %d is not a positive multiple of H_kv = %d", H, t->d.n_kv_heads);
+    if (N < 1 || N > T) return fail(ATLASKV_EINVAL, "need 1 <= N <= T (N = %d, T = %d)", N, T);
+    if (N > 65535) return fail(ATLASKV_EUNSUPPORTED, "N = %d above 65535", N);
+    if (p->K_root < 1 || p->K_root > fo[0]) return fail(ATLASKV_EINVAL, "K_root = %d not in [1, b_R = %d]", p->K_root, fo[0]);
+    if (p->K_mid < 1 || (long long)p->K_mid > (long long)p->K_root * fo[1])
+        return fail(ATLASKV_EINVAL, "K_mid = %d not in [1, K_root * b_I = %lld]", p->K_mid, (long long)p->K_root * fo[1]);
+    if (p->K_leaf < 1 || (long long)p->K_leaf > (long long)p->K_mid * fo[2])
+        return fail(ATLASKV_EINVAL, "K_leaf = %d not in [1, K_mid * b_L = %lld]", p->K_leaf, (long long)p->K_mid * fo[2]);
+    const long long c1 = (long long)p->K_root * fo[1], c2 = (long long)p->K_mid * fo[2];
+    if (fo[0] > kMaxCandidates || c1 > kMaxCandidates || c2 > kMaxCandidates)
+        return fail(ATLASKV_EUNSUPPORTED, "a level has more than %d candidates per traversal (%d, %lld, %lld)",
+                    kMaxCandidates, fo[0], c1, c2);
+    if (!(p->scale >= 0.f) || std::isinf(p->scale)) return fail(ATLASKV_EINVAL, "scale must be finite and >= 0");
+    if ((long long)B * H > (1LL << 31) - 1) return fail(ATLASKV_EUNSUPPORTED, "B * H too large");
+    return ATLASKV_OK;
+}
+
+template <typename T, int D>
+atlaskv_status launch_norms(const atlaskv_tree *t, const void *keys, long long rows, int level, cudaStream_t s)
+{
+    dim3 grid((unsigned)std::min<long long>((rows + 7) / 8, 4096), t->d.n_kv_heads);
+    akv::key_norm_kernel<T, D><<<grid, 256, 0, s>>>(reinterpret_cast<const T *>(keys), rows,
+                                                    reinterpret_cast<unsigned int *>(t->norm_bound) +
+                                                        (size_t)level * t->d.n_kv_heads);
+    AKV_CUDA(cudaGetLastError());
+    return ATLASKV_OK;
+}
+
+template <typename T, int D>
+atlaskv_status tree_norms(const atlaskv_tree *t, cudaStream_t s)
+{
+    const void *lv[3] = {t->d.root_keys, t->d.mid_keys, t->leaf_keys_dev};
+    for (int l = 0; l < 3; ++l) {
+        atlaskv_status st = launch_norms<T, D>(t, lv[l], t->rows[l], l, s);
+        if (st != ATLASKV_OK) return st;
+    }
+    return ATLASKV_OK;
+}
+
+atlaskv_status dispatch_norms(const atlaskv_tree *t, cudaStream_t s)
+{
+    const int D = t->d.head_dim;
+    if (t->d.dtype == ATLASKV_F32) return D == 64 ? tree_norms<float, 64>(t, s) : tree_norms<float, 128>(t, s);
+    return D == 64 ? tree_norms<__nv_bfloat16, 64>(t, s) : tree_norms<__nv_bfloat16, 128>(t, s);
+}
+
+atlaskv_status check_table(const int32_t *tab, long long entries_per_head, int H_kv, long long child_rows, int *status,
+                           cudaStream_t s)
+{
+    unsigned int *hits = nullptr;
+    const size_t n = (size_t)H_kv * child_rows;
+    AKV_CUDA(cudaMallocAsync(&hits, n * sizeof(unsigned int), s));
+    AKV_CUDA(cudaMemsetAsync(hits, 0, n * sizeof(unsigned int), s));
+    akv::child_table_check_kernel<<<2048, 256, 0, s>>>(tab, entries_per_head, H_kv, child_rows, hits, status);
+    akv::hits_check_kernel<<<2048, 256, 0, s>>>(hits, (long long)n, status);
+    AKV_CUDA(cudaGetLastError());
+    AKV_CUDA(cudaFreeAsync(hits, s));
+    return ATLASKV_OK;
+}
+
+// ---- descent launch -------------------------------------------------------
+template <typename T, int D>
+atlaskv_status launch_descend(const akv::DescendParams &dp, int grid, cudaStream_t s)
+{
+    const size_t smem = akv::DescendSmem<D>::bytes(dp.cap, dp.kcap);
+    static size_t configured = 0;
+    if (smem > configured) {
+        AKV_CUDA(cudaFuncSetAttribute(akv::descend_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        configured = smem;
+    }
+    akv::descend_kernel<T, D><<<grid, akv::kDescendThreads, smem, s>>>(dp);
+    AKV_CUDA(cudaGetLastError());
+    return ATLASKV_OK;
+}
+
+atlaskv_status dispatch_descend(int dtype, int D, const akv::DescendParams &dp, int grid, cudaStream_t s)
+{
+    if (dtype == ATLASKV_F32)
+        return D == 64 ? launch_descend<float, 64>(dp, grid, s) : launch_descend<float, 128>(dp, grid, s);
+    return D == 64 ? launch_descend<__nv_bfloat16, 64>(dp, grid, s) : launch_descend<__nv_bfloat16, 128>(dp, grid, s);
+}
+
+// ---- attention launch -----------------------------------------------------
+template <int D>
+atlaskv_status launch_attend_bf16(const akv::AttnParams &ap, cudaStream_t s)
+{
+    const int nchunks = (ap.N + 15) / 16;
+    const int bpg = (ap.G * nchunks + akv::kAttnWarps - 1) / akv::kAttnWarps;
+    const long long grid = (long long)ap.B * ap.H_kv * bpg;
+    if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "attention grid too large");
+    const int smem = akv::AttnSmem<D>::BYTES;
+    static bool configured = false;
+    if (!configured) {
+        AKV_CUDA(cudaFuncSetAttribute(akv::attend_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+        configured = true;
+    }
+    akv::attend_bf16_kernel<D><<<(unsigned)grid, akv::kAttnWarps * 32, smem, s>>>(ap, bpg);
+    AKV_CUDA(cudaGetLastError());
+    return ATLASKV_OK;
+}
+
+template <int D>
+atlaskv_status launch_attend_f32(const akv::AttnParams &ap, cudaStream_t s)
+{
+    const long long rows = (long long)ap.B * ap.N * ap.H;
+    const long long grid = (rows + 3) / 4;
+    if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "attention grid too large");
+    akv::attend_f32_kernel<D><<<(unsigned)grid, 128, 0, s>>>(ap);
+    AKV_CUDA(cudaGetLastError());
+    return ATLASKV_OK;
+}
+
+atlaskv_status dispatch_attend(int dtype, int D, const akv::AttnParams &ap, cudaStream_t s)
+{
+    if (dtype == ATLASKV_F32) return D == 64 ? launch_attend_f32<64>(ap, s) : launch_attend_f32<128>(ap, s);
+    return D == 64 ? launch_attend_bf16<64>(ap, s) : launch_attend_bf16<128>(ap, s);
+}
+
+// ---- staging launches -----------------------------------------------------
+atlaskv_status launch_dedupe(const int32_t *ids, int n, int groups, int32_t *uniq, int32_t *slot, int32_t *count,
+                             cudaStream_t s)
+{
+    const int n2 = pow2_at_least(n, 2);
+    const size_t smem = (size_t)n2 * 12;
+    static size_t configured = 0;
+    if (smem > 48 * 1024 && smem > configured) {
+        AKV_CUDA(cudaFuncSetAttribute(akv::dedupe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        configured = smem;
+    }
+    akv::dedupe_kernel<<<groups, akv::kDedupeThreads, smem, s>>>(ids, n, n2, uniq, slot, count);
+    AKV_CUDA(cudaGetLastError());
+    return ATLASKV_OK;
+}
+
+template <typename T, int D>
+atlaskv_status stage_keys(const atlaskv_tree *t, const int32_t *umid, const int32_t *cnt, int n, int groups,
+                          void *pool, cudaStream_t s)
+{
+    akv::stage_leaf_blocks_kernel<T, D><<<592, 256, 0, s>>>(
+        reinterpret_cast<const T *>(t->leaf_keys_dev), t->d.mid_child, t->rows[1], t->rows[2], t->d.fanout[2],
+        t->d.n_kv_heads, umid, cnt, n, groups, reinterpret_cast<T *>(pool), t->status);
+    AKV_CUDA(cudaGetLastError());
+    return ATLASKV_OK;
+}
+
+template <typename T, int D>
+atlaskv_status stage_values(const atlaskv_tree *t, const int32_t *uleaf, const int32_t *cnt, int n, int groups,
+                            void *vpool, cudaStream_t s)
+{
+    akv::stage_value_rows_kernel<T, D><<<592, 256, 0, s>>>(reinterpret_cast<const T *>(t->leaf_values_dev), t->rows[2],
+                                                          t->d.n_kv_heads, uleaf, cnt, n, groups,
+                                                          reinterpret_cast<T *>(vpool));
+    AKV_CUDA(cudaGetLastError());
+    return ATLASKV_OK;
+}
+
+atlaskv_status dispatch_stage_keys(const atlaskv_tree *t, const int32_t *umid, const int32_t *cnt, int n, int groups,
+                                   void *pool, cudaStream_t s)
+{
+    const int D = t->d.head_dim;
+    if (t->d.dtype == ATLASKV_F32)
+        return D == 64 ? stage_keys<float, 64>(t, umid, cnt, n, groups, pool, s)
+                       : stage_keys<float, 128>(t, umid, cnt, n, groups, pool, s);
+    return D == 64 ? stage_keys<__nv_bfloat16, 64>(t, umid, cnt, n, groups, pool, s)
+                   : stage_keys<__nv_bfloat16, 128>(t, umid, cnt, n, groups, pool, s);
+}
+
+atlaskv_status dispatch_stage_values(const atlaskv_tree *t, const int32_t *uleaf, const int32_t *cnt, int n,
+                                     int groups, void *vpool, cudaStream_t s)
+{
+    const int D = t->d.head_dim;
+    if (t->d.dtype == ATLASKV_F32)
+        return D == 64 ? stage_values<float, 64>(t, uleaf, cnt, n, groups, vpool, s)
+                       : stage_values<float, 128>(t, uleaf, cnt, n, groups, vpool, s);
+    return D == 64 ? stage_values<__nv_bfloat16, 64>(t, uleaf, cnt, n, groups, vpool, s)
+                   : stage_values<__nv_bfloat16, 128>(t, uleaf, cnt, n, groups, vpool, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *atlaskv_last_error(void) { return g_last_error.c_str(); }
+
+atlaskv_status atlaskv_create_tree(const atlaskv_tree_desc *d, void *stream, atlaskv_tree **out)
+{
+    if (!d || !out) return fail(ATLASKV_EINVAL, "null desc or out");
+    if (d->dtype != ATLASKV_F32 && d->dtype != ATLASKV_BF16) return fail(ATLASKV_EINVAL, "unknown dtype %d", d->dtype);
+    if (d->head_dim != 64 && d->head_dim != 128)
+        return fail(ATLASKV_EUNSUPPORTED, "head_dim %d not supported (64 or 128)", d->head_dim);
+    if (d->n_kv_heads < 1) return fail(ATLASKV_EINVAL, "n_kv_heads = %d", d->n_kv_heads);
+    for (int i = 0; i < 3; ++i)
+        if (d->fanout[i] < 1) return fail(ATLASKV_EINVAL, "fanout[%d] = %d", i, d->fanout[i]);
+    const long long n_root = d->fanout[0], n_mid = n_root * d->fanout[1], n_leaf = n_mid * d->fanout[2];
+    if (n_leaf > (1LL << 31) - 1 || n_leaf * d->n_kv_heads > (1LL << 31) - 1)
+        return fail(ATLASKV_EUNSUPPORTED, "H_kv * M = %lld rows above 2^31 - 1", n_leaf * d->n_kv_heads);
+    if (!d->root_keys || !d->mid_keys || !d->leaf_keys || !d->leaf_values)
+        return fail(ATLASKV_EINVAL, "null key/value pointer");
+    if (!aligned16(d->root_keys) || !aligned16(d->mid_keys) || !aligned16(d->leaf_keys) || !aligned16(d->leaf_values))
+        return fail(ATLASKV_EINVAL, "key/value buffers must be 16-byte aligned");
+    if (d->leaf_location != ATLASKV_LEAVES_DEVICE && d->leaf_location != ATLASKV_LEAVES_HOST_PINNED)
+        return fail(ATLASKV_EINVAL, "unknown leaf_location %d", d->leaf_location);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    atlaskv_tree *t = new (std::nothrow) atlaskv_tree();
+    if (!t) return fail(ATLASKV_ENOMEM, "host allocation failed");
+    t->d = *d;
+    t->rows[0] = n_root;
+    t->rows[1] = n_mid;
+    t->rows[2] = n_leaf;
+    t->leaf_keys_dev = d->leaf_keys;
+    t->leaf_values_dev = d->leaf_values;
+    auto bail = [&](atlaskv_status st) {
+        std::string msg = g_last_error;
+        atlaskv_destroy(t);
+        g_last_error = msg;
+        return st;
+    };
+    if (d->leaf_location == ATLASKV_LEAVES_HOST_PINNED) {
+        void *pk = nullptr, *pv = nullptr;
+        if (cudaHostGetDevicePointer(&pk, const_cast<void *>(d->leaf_keys), 0) != cudaSuccess ||
+            cudaHostGetDevicePointer(&pv, const_cast<void *>(d->leaf_values), 0) != cudaSuccess) {
+            cudaGetLastError();
+            return bail(fail(ATLASKV_EINVAL, "leaf buffers are not pinned (page-locked, mapped) host memory"));
+        }
+        t->leaf_keys_dev = pk;
+        t->leaf_values_dev = pv;
+    }
+    if (cudaMalloc(&t->norm_bound, 3 * sizeof(float) * d->n_kv_heads) != cudaSuccess ||
+        cudaMalloc(&t->status, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return bail(fail(ATLASKV_ECUDA, "device allocation of the tree's bound/status words failed"));
+    }
+    atlaskv_status st;
+#define AKV_TRY(x)                             \
+    do {                                       \
+        st = (x);                              \
+        if (st != ATLASKV_OK) return bail(st); \
+    } while (0)
+#define AKV_TRYC(x)                                                                              \
+    do {                                                                                         \
+        cudaError_t e_ = (x);                                                                    \
+        if (e_ != cudaSuccess) return bail(fail(ATLASKV_ECUDA, "%s: %s", #x, cudaGetErrorString(e_))); \
+    } while (0)
+    AKV_TRYC(cudaMemsetAsync(t->norm_bound, 0, 3 * sizeof(float) * d->n_kv_heads, s));
+    AKV_TRYC(cudaMemsetAsync(t->status, 0, sizeof(int), s));
+    AKV_TRY(dispatch_norms(t, s));
+    if (d->root_child) AKV_TRY(check_table(d->root_child, n_mid, d->n_kv_heads, n_mid, t->status, s));
+    if (d->mid_child) AKV_TRY(check_table(d->mid_child, n_leaf, d->n_kv_heads, n_leaf, t->status, s));
+    int dev_status = 0;
+    AKV_TRYC(cudaMemcpyAsync(&dev_status, t->status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    AKV_TRYC(cudaStreamSynchronize(s));
+    if (dev_status != akv::kDevOk)
+        return bail(fail(ATLASKV_EINVAL, "child table has an out-of-range id or is not a permutation"));
+    // inflate the norm bounds slightly (they were rounded up already)
+    {
+        float hb[3 * 64];
+        const int nb = 3 * d->n_kv_heads;
+        float *tmp = nb <= 192 ? hb : new (std::nothrow) float[nb];
+        if (!tmp) return bail(fail(ATLASKV_ENOMEM, "host allocation failed"));
+        AKV_TRYC(cudaMemcpy(tmp, t->norm_bound, nb * sizeof(float), cudaMemcpyDeviceToHost));
+        for (int i = 0; i < nb; ++i) tmp[i] = nextafterf(tmp[i] * (1.0f + 0x1p-20f), INFINITY);
+        AKV_TRYC(cudaMemcpy(t->norm_bound, tmp, nb * sizeof(float), cudaMemcpyHostToDevice));
+        if (tmp != hb) delete[] tmp;
+    }
+#undef AKV_TRY
+#undef AKV_TRYC
+    *out = t;
+    return ATLASKV_OK;
+}
+
+atlaskv_status atlaskv_workspace_size(const atlaskv_tree *t, const atlaskv_params *p, int32_t B, int32_t N, int32_t H,
+                                      int32_t T, size_t *bytes)
+{
+    if (!bytes) return fail(ATLASKV_EINVAL, "null bytes");
+    atlaskv_status st = check_params(t, p, B, N, H, T);
+    if (st != ATLASKV_OK) return st;
+    *bytes = plan(t, p, B, N, H, T).total;
+    return ATLASKV_OK;
+}
+
+atlaskv_status atlaskv_attend(atlaskv_tree *t, const atlaskv_params *p, const atlaskv_io *io, void *workspace,
+                              size_t ws_bytes, void *stream)
+{
+    if (!io) return fail(ATLASKV_EINVAL, "null io");
+    atlaskv_status st = check_params(t, p, io->B, io->N, io->H, io->T);
+    if (st != ATLASKV_OK) return st;
+    if (io->B == 0) return ATLASKV_OK;
+    if (!io->q_kg || !io->q_seq || !io->k_seq || !io->v_seq || !io->out)
+        return fail(ATLASKV_EINVAL, "null q_kg/q_seq/k_seq/v_seq/out");
+    const void *ptrs[] = {io->q_kg, io->q_seq, io->k_seq, io->v_seq, io->out, io->lse, io->kept_root, io->kept_mid,
+                          io->kept_leaf};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return fail(ATLASKV_EINVAL, "io buffers must be 16-byte aligned");
+    const Layout L = plan(t, p, io->B, io->N, io->H, io->T);
+    if (!workspace || ((uintptr_t)workspace & 255u)) return fail(ATLASKV_EINVAL, "workspace must be 256-byte aligned");
+    if (ws_bytes < L.total)
+        return fail(ATLASKV_ENOMEM, "workspace of %zu bytes, %zu needed", ws_bytes, L.total);
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+    const int D = t->d.head_dim;
+    const int H_kv = t->d.n_kv_heads;
+    const int G = io->H / H_kv;
+    const bool host = t->d.leaf_location == ATLASKV_LEAVES_HOST_PINNED;
+    const int BH = io->B * io->H;
+    int32_t *kept[3] = {io->kept_root ? io->kept_root : reinterpret_cast<int32_t *>(ws + L.kept[0]),
+                        io->kept_mid ? io->kept_mid : reinterpret_cast<int32_t *>(ws + L.kept[1]),
+                        io->kept_leaf ? io->kept_leaf : reinterpret_cast<int32_t *>(ws + L.kept[2])};
+
+    akv::DescendParams dp{};
+    dp.q_kg = io->q_kg;
+    dp.B = io->B;
+    dp.N = io->N;
+    dp.H = io->H;
+    dp.H_kv = H_kv;
+    dp.G = G;
+    dp.keys[0] = t->d.root_keys;
+    dp.keys[1] = t->d.mid_keys;
+    dp.keys[2] = t->leaf_keys_dev;
+    for (int l = 0; l < 3; ++l) {
+        dp.rows[l] = t->rows[l];
+        dp.fanout[l] = t->d.fanout[l];
+        dp.kept[l] = kept[l];
+    }
+    dp.child[0] = t->d.root_child;
+    dp.child[1] = t->d.mid_child;
+    dp.norm_bound = t->norm_bound;
+    dp.K[0] = p->K_root;
+    dp.K[1] = p->K_mid;
+    dp.K[2] = p->K_leaf;
+    dp.s_ws = reinterpret_cast<float *>(ws + L.s_ws);
+    dp.anorm_ws = reinterpret_cast<float *>(ws + L.anorm_ws);
+    const long long cmax = std::max<long long>(t->d.fanout[0], std::max<long long>((long long)p->K_root * t->d.fanout[1],
+                                                                                  (long long)p->K_mid * t->d.fanout[2]));
+    dp.cap = pow2_at_least(cmax, 64);
+    dp.kcap = pow2_at_least(std::max(p->K_root, std::max(p->K_mid, p->K_leaf)), 64);
+    dp.status = t->status;
+
+    const float scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)D);
+    akv::AttnParams ap{};
+    ap.q_kg = io->q_kg;
+    ap.q_seq = io->q_seq;
+    ap.k_seq = io->k_seq;
+    ap.v_seq = io->v_seq;
+    ap.out = io->out;
+    ap.lse = io->lse;
+    ap.B = io->B;
+    ap.N = io->N;
+    ap.H = io->H;
+    ap.H_kv = H_kv;
+    ap.G = G;
+    ap.T = io->T;
+    ap.K_L = p->K_leaf;
+    ap.scale_log2 = scale * 1.4426950408889634f;
+
+    const bool prof = t->profiling;
+    auto mark = [&](int i) -> atlaskv_status {
+        if (prof) AKV_CUDA(cudaEventRecord(t->ev[i], s));
+        return ATLASKV_OK;
+    };
+#define AKV_STEP(x)                            \
+    do {                                       \
+        atlaskv_status st_ = (x);              \
+        if (st_ != ATLASKV_OK) return st_;     \
+    } while (0)
+
+    if (!host) {
+        AKV_STEP(mark(0));
+        dp.first_level = 0;
+        dp.last_level = 2;
+        dp.s_ws = nullptr;   // fused: token sums stay in shared memory
+        AKV_STEP(dispatch_descend(t->d.dtype, D, dp, BH, s));
+        AKV_STEP(mark(1));
+        ap.lk_base = t->d.leaf_keys;
+        ap.lv_base = t->d.leaf_values;
+        ap.lk_idx = kept[2];
+        ap.lv_idx = kept[2];
+        ap.leaf_head_stride = t->rows[2];
+        AKV_STEP(dispatch_attend(t->d.dtype, D, ap, s));
+        AKV_STEP(mark(2));
+    } else {
+        const int groups = io->B * H_kv;
+        const int n_mid = G * p->K_mid, n_leaf = G * p->K_leaf;
+        int32_t *leaf_slot = reinterpret_cast<int32_t *>(ws + L.leaf_slot);
+        int32_t *kept_leaf_row = reinterpret_cast<int32_t *>(ws + L.kept_leaf_row);
+        int32_t *vslot = reinterpret_cast<int32_t *>(ws + L.vslot);
+        int32_t *umid = reinterpret_cast<int32_t *>(ws + L.umid);
+        int32_t *cmid = reinterpret_cast<int32_t *>(ws + L.ucount_mid);
+        int32_t *uleaf = reinterpret_cast<int32_t *>(ws + L.uleaf);
+        int32_t *cleaf = reinterpret_cast<int32_t *>(ws + L.ucount_leaf);
+        void *pool = ws + L.key_pool;
+        void *vpool = ws + L.val_pool;
+        AKV_STEP(mark(0));
+        dp.first_level = 0;
+        dp.last_level = 1;
+        AKV_STEP(dispatch_descend(t->d.dtype, D, dp, BH, s));
+        AKV_STEP(mark(1));
+        AKV_STEP(launch_dedupe(kept[1], n_mid, groups, umid, leaf_slot, cmid, s));
+        AKV_STEP(dispatch_stage_keys(t, umid, cmid, n_mid, groups, pool, s));
+        AKV_STEP(mark(2));
+        dp.first_level = 2;
+        dp.last_level = 2;
+        dp.keys[2] = pool;
+        dp.leaf_slot = leaf_slot;
+        dp.kept_leaf_row = kept_leaf_row;
+        AKV_STEP(dispatch_descend(t->d.dtype, D, dp, BH, s));
+        AKV_STEP(mark(3));
+        AKV_STEP(launch_dedupe(kept[2], n_leaf, groups, uleaf, vslot, cleaf, s));
+        AKV_STEP(dispatch_stage_values(t, uleaf, cleaf, n_leaf, groups, vpool, s));
+        AKV_STEP(mark(4));
+        ap.lk_base = pool;
+        ap.lv_base = vpool;
+        ap.lk_idx = kept_leaf_row;
+        ap.lv_idx = vslot;
+        ap.leaf_head_stride = 0;
+        AKV_STEP(dispatch_attend(t->d.dtype, D, ap, s));
+        AKV_STEP(mark(5));
+    }
+#undef AKV_STEP
+    t->timed = prof;
+    t->host_mode_last = host;
+    return ATLASKV_OK;
+}
+
+atlaskv_status atlaskv_sync_status(atlaskv_tree *t, void *stream)
+{
+    if (!t) return fail(ATLASKV_EINVAL, "null tree");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int v = 0;
+    AKV_CUDA(cudaMemcpyAsync(&v, t->status, sizeof(int), cudaMemcpyDeviceToHost, s));
+    AKV_CUDA(cudaStreamSynchronize(s));
+    if (v == akv::kDevBadChild) return fail(ATLASKV_EDEVICE, "a child id was out of range on the device");
+    if (v == akv::kDevTimeout) return fail(ATLASKV_ETIMEOUT, "a bounded device wait gave up");
+    if (v != akv::kDevOk) return fail(ATLASKV_EDEVICE, "device status %d", v);
+    return ATLASKV_OK;
+}
+
+atlaskv_status atlaskv_set_profiling(atlaskv_tree *t, int32_t enable)
+{
+    if (!t) return fail(ATLASKV_EINVAL, "null tree");
+    if (enable && !t->ev[0])
+        for (int i = 0; i < kNumEvents; ++i) AKV_CUDA(cudaEventCreate(&t->ev[i]));
+    t->profiling = enable != 0;
+    return ATLASKV_OK;
+}
+
+atlaskv_status atlaskv_stage_times(atlaskv_tree *t, float *ms, int32_t n)
+{
+    if (!t || !ms || n < 1) return fail(ATLASKV_EINVAL, "null tree/ms or n < 1");
+    if (!t->timed) return fail(ATLASKV_EINVAL, "no attend call was timed (enable profiling first)");
+    float v[3] = {0.f, 0.f, 0.f};
+    if (!t->host_mode_last) {
+        AKV_CUDA(cudaEventSynchronize(t->ev[2]));
+        AKV_CUDA(cudaEventElapsedTime(&v[0], t->ev[0], t->ev[1]));
+        AKV_CUDA(cudaEventElapsedTime(&v[2], t->ev[1], t->ev[2]));
+    } else {
+        float a, b2, c, d2, e;
+        AKV_CUDA(cudaEventSynchronize(t->ev[5]));
+        AKV_CUDA(cudaEventElapsedTime(&a, t->ev[0], t->ev[1]));
+        AKV_CUDA(cudaEventElapsedTime(&b2, t->ev[1], t->ev[2]));
+        AKV_CUDA(cudaEventElapsedTime(&c, t->ev[2], t->ev[3]));
+        AKV_CUDA(cudaEventElapsedTime(&d2, t->ev[3], t->ev[4]));
+        AKV_CUDA(cudaEventElapsedTime(&e, t->ev[4], t->ev[5]));
+        v[0] = a + c;
+        v[1] = b2 + d2;
+        v[2] = e;
+    }
+    for (int i = 0; i < n && i < 3; ++i) ms[i] = v[i];
+    return ATLASKV_OK;
+}
+
+atlaskv_status atlaskv_destroy(atlaskv_tree *t)
+{
+    if (!t) return ATLASKV_OK;
+    if (t->norm_bound) cudaFree(t->norm_bound);
+    if (t->status) cudaFree(t->status);
+    for (int i = 0; i < kNumEvents; ++i)
+        if (t->ev[i]) cudaEventDestroy(t->ev[i]);
+    delete t;
+    return ATLASKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,143 @@
+// Host-leaf staging: bring the leaf-key blocks of the kept mids, and later the
+// kept leaves' value rows, from pinned host memory into HBM.
+//
+// "AtlasKV: Augmenting LLMs with Billion-Scale Knowledge Graphs in 20GB VRAM",
+// section "Quick read / How it works": only the root keys need to stay on the
+// GPU; after each level's pruning the next level's keys are loaded from CPU
+// memory.  Section "Quick read / Results" names the cost: CPU-GPU movement
+// between levels adds I/O latency.  So every block crosses the host link once
+// per query: the G query heads of a query share one staged copy.
+#pragma once
+
+#include "common.cuh"
+
+namespace akv {
+
+constexpr int kDedupeThreads = 256;
+
+// Per group q (one query and one KV head: the kept lists of its G query heads
+// are contiguous): the n ids ids[q*n .. q*n+n) -> unique ids
+// uniq[q*n .. q*n+count[q]) in ascending order, and slot[q*n + i] = q*n + rank
+// of ids[q*n+i] among them.  Dynamic shared memory: n2 (power of two >= n)
+// uint64 + n2 int32.
+__global__ void __launch_bounds__(kDedupeThreads) dedupe_kernel(const int32_t *__restrict__ ids, int n, int n2,
+                                                                 int32_t *uniq, int32_t *slot, int32_t *count)
+{
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint64_t *buf = reinterpret_cast<uint64_t *>(smem_raw);
+    int32_t *flag = reinterpret_cast<int32_t *>(buf + n2);   // [n2] inclusive scan of "first of a run"
+    const int b = blockIdx.x;   // group q
+    const int32_t *src = ids + (size_t)b * n;
+    for (int i = threadIdx.x; i < n2; i += blockDim.x)
+        buf[i] = i < n ? ((uint64_t)(uint32_t)src[i] << 32) | (uint32_t)i : ~0ull;
+    // bitonic sort ascending
+    for (int size = 2; size <= n2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            __syncthreads();
+            for (int i = threadIdx.x; i < n2 / 2; i += blockDim.x) {
+                const int lo = 2 * i - (i & (stride - 1));
+                const int hi = lo + stride;
+                const bool asc = (lo & size) == 0;
+                const uint64_t x = buf[lo], y = buf[hi];
+                if ((x > y) == asc) {
+                    buf[lo] = y;
+                    buf[hi] = x;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n2; i += blockDim.x)
+        flag[i] = (i < n && (i == 0 || (buf[i] >> 32) != (buf[i - 1] >> 32))) ? 1 : 0;
+    __syncthreads();
+    // inclusive scan of flag: each thread scans a contiguous segment, then
+    // the per-thread totals are scanned by warp 0
+    __shared__ int seg_tot[kDedupeThreads];
+    const int seg = (n2 + blockDim.x - 1) / blockDim.x;
+    const int s0 = threadIdx.x * seg, s1 = min(n2, s0 + seg);
+    int run = 0;
+    for (int i = s0; i < s1; ++i) {
+        run += flag[i];
+        flag[i] = run;
+    }
+    seg_tot[threadIdx.x] = run;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int t = 0; t < (int)blockDim.x; ++t) {
+            const int v = seg_tot[t];
+            seg_tot[t] = acc;
+            acc += v;
+        }
+    }
+    __syncthreads();
+    for (int i = s0; i < s1; ++i) flag[i] += seg_tot[threadIdx.x];
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int u = flag[i] - 1;
+        const int32_t id = (int32_t)(buf[i] >> 32);
+        const int orig = (int)(buf[i] & 0xffffffffu);
+        slot[(size_t)b * n + orig] = b * n + u;
+        if (i == 0 || (buf[i] >> 32) != (buf[i - 1] >> 32)) uniq[(size_t)b * n + u] = id;
+    }
+    if (threadIdx.x == 0) count[b] = flag[n - 1];
+}
+
+// Copy the b_L leaf-key rows of every unique kept mid of every group into the
+// key pool: pool row (q*n + u) * b_L + j <- host leaf row child(mid, j) of KV
+// head q % H_kv.  One warp per (block, row); 16-byte loads from mapped host
+// memory.
+template <typename T, int D>
+__global__ void stage_leaf_blocks_kernel(const T *__restrict__ host_leaf_keys, const int32_t *__restrict__ mid_child,
+                                         long long n_mid, long long n_leaf, int b_leaf, int H_kv,
+                                         const int32_t *__restrict__ uniq, const int32_t *__restrict__ count,
+                                         int n, int n_groups, T *pool, int *status)
+{
+    constexpr int VPR = D * (int)sizeof(T) / 16;   // 16-byte vectors per row
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    const long long total = (long long)n_groups * n * b_leaf;
+    for (long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
+        const long long blk = w / b_leaf;
+        const int j = (int)(w - blk * b_leaf);
+        const int b = (int)(blk / n);
+        const int u = (int)(blk - (long long)b * n);
+        if (u >= count[b]) continue;
+        const int hkv = b % H_kv;   // group b = query * H_kv + hkv
+        const long long mid = uniq[blk];
+        const long long leaf = mid_child ? (long long)mid_child[((size_t)hkv * n_mid + mid) * b_leaf + j]
+                                         : mid * b_leaf + j;
+        if (leaf < 0 || leaf >= n_leaf) {
+            if (lane == 0) set_status(status, kDevBadChild);
+            continue;
+        }
+        const uint4 *src = reinterpret_cast<const uint4 *>(host_leaf_keys + ((size_t)hkv * n_leaf + leaf) * D);
+        uint4 *dst = reinterpret_cast<uint4 *>(pool + ((size_t)blk * b_leaf + j) * D);
+        for (int v = lane; v < VPR; v += 32) dst[v] = src[v];
+    }
+}
+
+// Copy value rows: vpool row (q*n + u) <- host leaf value row uniq[q*n + u]
+// of KV head q % H_kv.
+template <typename T, int D>
+__global__ void stage_value_rows_kernel(const T *__restrict__ host_leaf_values, long long n_leaf, int H_kv,
+                                        const int32_t *__restrict__ uniq, const int32_t *__restrict__ count, int n,
+                                        int n_groups, T *vpool)
+{
+    constexpr int VPR = D * (int)sizeof(T) / 16;
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    const long long total = (long long)n_groups * n;
+    for (long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
+        const int b = (int)(w / n);
+        const int u = (int)(w - (long long)b * n);
+        if (u >= count[b]) continue;
+        const int hkv = b % H_kv;
+        const long long leaf = uniq[w];
+        const uint4 *src = reinterpret_cast<const uint4 *>(host_leaf_values + ((size_t)hkv * n_leaf + leaf) * D);
+        uint4 *dst = reinterpret_cast<uint4 *>(vpool + (size_t)w * D);
+        for (int v = lane; v < VPR; v += 32) dst[v] = src[v];
+    }
+}
+
+}  // namespace akv

@@ -1,0 +1,170 @@
+/*
+ * atlaskv.h -- C ABI of the B200 (sm_100a) HiKVP knowledge-graph attention library.
+ *
+ * HiKVP = hierarchical key-value pruning from "AtlasKV: Augmenting LLMs with
+ * Billion-Scale Knowledge Graphs in 20GB VRAM" (ICLR 2026).  For every query b
+ * and query head h (a "traversal"; KV head hkv = h / (H / H_kv)):
+ *
+ *   1. score the query against all root keys and keep the top K_root roots;
+ *   2. score the children of the kept roots, keep the top K_mid mids;
+ *   3. score the children of the kept mids (the leaves), keep the top K_leaf;
+ *   4. attend over the kept leaves (knowledge part) and over the causal
+ *      sequence, and merge the two with lambda weights;
+ *   (section "Quick read / How it works" of the paper notes; leaves may live in
+ *   pinned host memory and are then staged into HBM on demand.)
+ *
+ * Node score: the mean over the query's N tokens of <q_kg[n], k> / sqrt(D).
+ * Ranking uses the EXACT real value of that score computed from the stored
+ * numbers (the library filters in fp32 with a rigorous error bound and settles
+ * the candidates the bound cannot separate with exact integer arithmetic), so
+ * the kept sets depend on the inputs only.  Equal exact scores go to the lower
+ * storage row id.  Kept ids are returned in ascending order.
+ *
+ * Merge ("Quick read / How it works" merge equation; "Method details /
+ * Equivalent attention"):  y = lam_kg * Softmax(l_kg) V_kg + lam_seq *
+ * Softmax(l_seq) V_seq with lam_kg = e^{LSE_kg} / (e^{LSE_kg} + e^{LSE_seq}),
+ * lam_seq = 1 - lam_kg, which equals one softmax over the kept leaves and the
+ * visible sequence keys ("Background / Rectangular attention in KBLaM").  The N
+ * query tokens are the last N positions of the T-token sequence: token n sees
+ * sequence positions 0..T-N+n ("Background / Self-attention" equation) and
+ * every kept leaf.
+ *
+ * Layouts (all row-major, D contiguous, every base pointer 16-byte aligned):
+ *   root_keys   [H_kv][b_R][D]            device
+ *   mid_keys    [H_kv][b_R*b_I][D]        device
+ *   leaf_keys   [H_kv][b_R*b_I*b_L][D]    device, or pinned host memory
+ *   leaf_values [H_kv][b_R*b_I*b_L][D]    same location as leaf_keys
+ *   root_child  [H_kv][b_R][b_I]    int32 mid row ids, or NULL: child(r,j) = r*b_I + j
+ *   mid_child   [H_kv][b_R*b_I][b_L] int32 leaf row ids, or NULL: child(m,j) = m*b_L + j
+ *   q_kg, q_seq [B][N][H][D]              device
+ *   k_seq, v_seq [B][T][H_kv][D]          device
+ *   out         [B][N][H][D]              device, tree dtype
+ *   lse         [B][N][H] float32         device, optional (natural log, of the union)
+ *   kept_root   [B][H][K_root] int32      device, optional (likewise kept_mid, kept_leaf)
+ *
+ * Ownership: the library borrows every buffer; the caller keeps them alive and
+ * unmodified while a tree exists (tree buffers) or until the attend call's work
+ * on its stream has finished (io buffers and workspace).  The library never
+ * allocates device memory inside atlaskv_attend; the caller passes a workspace
+ * of atlaskv_workspace_size() bytes (256-byte aligned).
+ *
+ * Errors: every call returns an atlaskv_status; on a non-OK return nothing was
+ * enqueued and no output was written, and atlaskv_last_error() gives a
+ * thread-local message.  atlaskv_attend is asynchronous: OK means validated and
+ * enqueued on `stream`.  Errors found on the device (a child-table entry out of
+ * range, a bounded wait that gave up) set a sticky status word in the tree,
+ * read by atlaskv_sync_status().  No call aborts the process or traps the GPU.
+ */
+#ifndef ATLASKV_H
+#define ATLASKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATLASKV_OK = 0,
+    ATLASKV_EINVAL = 1,        /* bad argument: shape, K, pointer, alignment */
+    ATLASKV_ENOMEM = 2,        /* workspace too small / host allocation failed */
+    ATLASKV_ECUDA = 3,         /* a CUDA runtime call failed */
+    ATLASKV_EUNSUPPORTED = 4,  /* valid but outside what this build supports */
+    ATLASKV_ETIMEOUT = 5,      /* a bounded device wait gave up */
+    ATLASKV_EDEVICE = 6        /* device-side check failed (child id out of range) */
+} atlaskv_status;
+
+typedef enum { ATLASKV_F32 = 0, ATLASKV_BF16 = 1 } atlaskv_dtype;
+
+typedef enum {
+    ATLASKV_LEAVES_DEVICE = 0,       /* leaf keys/values in HBM */
+    ATLASKV_LEAVES_HOST_PINNED = 1   /* leaf keys/values in pinned (page-locked) host memory */
+} atlaskv_leaf_location;
+
+/* Tree description ("Method details / Hierarchical clustering of KGKVs": three
+ * levels, root / intermediate / leaf; only leaves carry values). */
+typedef struct {
+    int32_t dtype;             /* atlaskv_dtype of every key/value/query buffer */
+    int32_t n_kv_heads;        /* H_kv >= 1: one tree per KV head */
+    int32_t head_dim;          /* D: 64 or 128 */
+    int32_t fanout[3];         /* b_R roots, b_I mids per root, b_L leaves per mid; each >= 1 */
+    const void *root_keys;
+    const void *mid_keys;
+    const void *leaf_keys;
+    const void *leaf_values;
+    int32_t leaf_location;     /* atlaskv_leaf_location */
+    const int32_t *root_child; /* device, optional */
+    const int32_t *mid_child;  /* device, optional */
+} atlaskv_tree_desc;
+
+typedef struct {
+    int32_t K_root;            /* 1 <= K_root <= b_R */
+    int32_t K_mid;             /* 1 <= K_mid  <= K_root * b_I */
+    int32_t K_leaf;            /* 1 <= K_leaf <= K_mid * b_L */
+    float scale;               /* logit scale; 0 means 1/sqrt(D) */
+} atlaskv_params;
+
+typedef struct {
+    int32_t B;                 /* independent queries, >= 0 (0: nothing to do) */
+    int32_t N;                 /* query tokens per query, 1 <= N <= T */
+    int32_t H;                 /* query heads, a multiple of H_kv */
+    int32_t T;                 /* causal sequence length */
+    const void *q_kg;          /* KG query (knowledge part and node scores) */
+    const void *q_seq;         /* sequence query */
+    const void *k_seq;
+    const void *v_seq;
+    void *out;
+    float *lse;                /* optional */
+    int32_t *kept_root;        /* optional */
+    int32_t *kept_mid;         /* optional */
+    int32_t *kept_leaf;        /* optional */
+} atlaskv_io;
+
+typedef struct atlaskv_tree atlaskv_tree;
+
+/* Validate a tree description and build the handle.  Checks child tables on
+ * the device (every id in range, each level's table a permutation) and computes
+ * per-level key-norm bounds used by the ranking filter; this reads every key
+ * once (host-pinned leaves are read over the host link) and synchronises
+ * `stream` (a cudaStream_t, or NULL for the legacy default stream).
+ * Returns EINVAL for a bad description or table, EUNSUPPORTED for D not in
+ * {64, 128}, ECUDA if a CUDA call fails.  *out is set only on OK. */
+atlaskv_status atlaskv_create_tree(const atlaskv_tree_desc *desc, void *stream, atlaskv_tree **out);
+
+/* Bytes of workspace atlaskv_attend needs for these sizes (EINVAL on bad sizes). */
+atlaskv_status atlaskv_workspace_size(const atlaskv_tree *tree, const atlaskv_params *params,
+                                      int32_t B, int32_t N, int32_t H, int32_t T, size_t *bytes);
+
+/* Enqueue the whole path on `stream`: descent (3 levels, staging of host
+ * leaves when the tree's leaves are in host memory), knowledge + sequence
+ * attention and merge.  `workspace` is device memory of at least
+ * atlaskv_workspace_size() bytes, 256-byte aligned, not shared with a
+ * concurrent call.  Returns EINVAL / ENOMEM (workspace too small) /
+ * EUNSUPPORTED without enqueuing anything. */
+atlaskv_status atlaskv_attend(atlaskv_tree *tree, const atlaskv_params *params, const atlaskv_io *io,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* Synchronise `stream` and return the tree's sticky device status (OK,
+ * EDEVICE or ETIMEOUT), or ECUDA if the stream reports a CUDA error. */
+atlaskv_status atlaskv_sync_status(atlaskv_tree *tree, void *stream);
+
+/* Per-stage device times (ms) of the most recent attend call made while
+ * profiling was on: [0] descent levels, [1] host-leaf staging (0 when leaves
+ * are in HBM), [2] attention + merge.  Synchronises the stream of that call.
+ * n is the capacity of ms; returns EINVAL if profiling was never enabled. */
+atlaskv_status atlaskv_set_profiling(atlaskv_tree *tree, int32_t enable);
+atlaskv_status atlaskv_stage_times(atlaskv_tree *tree, float *ms, int32_t n);
+
+/* Release the handle and the small device buffers it owns; the caller's
+ * buffers are untouched.  NULL is accepted. */
+atlaskv_status atlaskv_destroy(atlaskv_tree *tree);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char *atlaskv_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATLASKV_H */

@@ -1,0 +1,291 @@
+"""Parity of the CUDA path (through the C ABI) with the oracle.
+
+Kept node and leaf sets must be bit-exact.  Outputs: float32 within
+1e-5 * max|y_ref| (max-abs), bfloat16 within 2e-2 max-abs on unit-scale
+outputs; LSE within 1e-4 (float32) / 2e-3 (bfloat16, logits from bfloat16
+inputs accumulated in fp32).  Full-size shapes are checked on sampled
+traversals against the oracle and on every traversal by properties that hold
+at any size (ascending, distinct, in range, nested).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hierarchical_kv_pruning_b200 import synth
+from hierarchical_kv_pruning_b200.binding import AtlaskvError, HikvpTree
+from tests._util import oracle_inputs, oracle_tree, storage
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "tiny_fp32_10x10x10.npz")
+BF16_TOL = 2e-2
+LSE_TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-3}
+
+
+def gpu_run(w, K, scale=0.0, tree=None):
+    own = tree is None
+    if own:
+        tree = HikvpTree.from_workload(w)
+    r = tree.attend(w.q_kg, w.q_seq, w.k_seq, w.v_seq, K, scale=scale)
+    tree.sync_status()
+    out = {k: (v.cpu() if torch.is_tensor(v) and k != "workspace" else v) for k, v in r.items()}
+    if own:
+        tree.close()
+    return out
+
+
+def to_device(w, device="cuda"):
+    f = {}
+    for name in ("root_keys", "mid_keys", "leaf_keys", "leaf_values", "root_child", "mid_child", "q_kg", "q_seq",
+                 "k_seq", "v_seq", "targets"):
+        v = getattr(w, name)
+        f[name] = None if v is None else v.to(device)
+    return synth.Workload(w.shape, **f)
+
+
+def sample_traversals(B, H, n, seed=0):
+    rng = np.random.default_rng(seed)
+    pairs = {(0, 0), (B - 1, H - 1)}
+    while len(pairs) < min(n, B * H):
+        pairs.add((int(rng.integers(B)), int(rng.integers(H))))
+    return sorted(pairs)
+
+
+def compare(w, K, g, traversals=None, scale=None):
+    sh = w.shape
+    t = oracle_tree(w)
+    inp = oracle_inputs(w)
+    r = oracle.hikvp(t, inp["q_kg"], inp["q_seq"], inp["k_seq"], inp["v_seq"], K, traversals, scale)
+    worst = 0.0
+    for i, (b, h) in enumerate(r["traversals"]):
+        assert g["kept_root"][b, h].tolist() == r["kept_root"][i].tolist(), ("root", b, h)
+        assert g["kept_mid"][b, h].tolist() == r["kept_mid"][i].tolist(), ("mid", b, h)
+        assert g["kept_leaf"][b, h].tolist() == r["kept_leaf"][i].tolist(), ("leaf", b, h)
+        y = g["out"][b, :, h, :].double().numpy()
+        err = np.max(np.abs(y - r["y"][i]))
+        if sh.dtype == torch.float32:
+            assert err <= 1e-5 * np.max(np.abs(r["y"][i])), (b, h, err)
+        else:
+            assert err <= BF16_TOL, (b, h, err)
+        lerr = np.max(np.abs(g["lse"][b, :, h].double().numpy() - r["lse"][i]))
+        assert lerr <= LSE_TOL[sh.dtype], (b, h, lerr)
+        worst = max(worst, err)
+    return worst
+
+
+def check_structure(w, K, g):
+    """Properties of every traversal: ascending distinct ids in range, nesting."""
+    sh = w.shape
+    bR, bI, bL = sh.fanout
+    kr, km, kl = g["kept_root"], g["kept_mid"], g["kept_leaf"]
+    for a, hi in ((kr, bR), (km, bR * bI), (kl, sh.n_leaves)):
+        assert int(a.min()) >= 0 and int(a.max()) < hi
+        assert bool((a[..., 1:] > a[..., :-1]).all())
+    G = sh.group
+    hkv = torch.arange(sh.n_heads) // G
+    if w.root_child is None:
+        parent_mid = km // bI
+        parent_leaf = kl // bL
+    else:
+        inv_mid = torch.empty(sh.n_kv_heads, bR * bI, dtype=torch.int64)
+        inv_leaf = torch.empty(sh.n_kv_heads, bR * bI * bL, dtype=torch.int64)
+        rc, mc = w.root_child.cpu().long(), w.mid_child.cpu().long()
+        for hk in range(sh.n_kv_heads):
+            inv_mid[hk, rc[hk].flatten()] = torch.arange(bR).repeat_interleave(bI)
+            inv_leaf[hk, mc[hk].flatten()] = torch.arange(bR * bI).repeat_interleave(bL)
+        parent_mid = inv_mid[hkv[None, :, None].expand_as(km), km.long()]
+        parent_leaf = inv_leaf[hkv[None, :, None].expand_as(kl), kl.long()]
+    # every kept mid's parent is a kept root, every kept leaf's parent a kept mid
+    assert bool((parent_mid[..., :, None] == kr[..., None, :].long()).any(-1).all())
+    assert bool((parent_leaf[..., :, None] == km[..., None, :].long()).any(-1).all())
+    assert torch.isfinite(g["out"].float()).all()
+
+
+# ---------------------------------------------------------------------------
+
+def test_tiny_fp32_matches_golden():
+    gold = np.load(GOLDEN)
+    sh = synth.shape(0)
+    w = to_device(synth.make_workload(sh, "cpu", 1000))
+    assert np.array_equal(storage(w.q_kg), gold["q_kg"])
+    g = gpu_run(w, sh.keep)
+    assert g["kept_root"][0, 0].tolist() == gold["kept_root"][0].tolist()
+    assert g["kept_mid"][0, 0].tolist() == gold["kept_mid"][0].tolist()
+    assert g["kept_leaf"][0, 0].tolist() == gold["kept_leaf"][0].tolist()
+    y = g["out"][0, :, 0, :].double().numpy()
+    assert np.max(np.abs(y - gold["y"][0])) <= 1e-5 * np.max(np.abs(gold["y"][0]))
+    assert np.max(np.abs(g["lse"][0, :, 0].double().numpy() - gold["lse"][0])) <= 1e-4
+
+
+SMALL = [
+    # (dtype, H, H_kv, D, fanout, K, B, N, T, permuted)
+    (torch.float32, 1, 1, 64, (10, 10, 10), (2, 2, 4), 1, 16, 16, False),
+    (torch.float32, 4, 2, 128, (6, 5, 7), (3, 4, 9), 3, 5, 11, True),
+    (torch.bfloat16, 4, 1, 64, (9, 8, 7), (3, 5, 20), 2, 16, 40, False),
+    (torch.bfloat16, 8, 2, 128, (12, 11, 10), (4, 6, 17), 3, 20, 37, False),    # ragged N, T
+    (torch.bfloat16, 6, 3, 128, (7, 9, 11), (2, 7, 33), 2, 33, 33, True),      # N = T, permuted
+    (torch.bfloat16, 2, 1, 128, (5, 4, 3), (5, 20, 60), 2, 3, 70, False),      # full K: nothing pruned
+    (torch.bfloat16, 32, 8, 128, (20, 20, 20), (8, 8, 32), 2, 128, 130, False),
+    (torch.bfloat16, 32, 1, 128, (16, 16, 17), (16, 16, 64), 3, 32, 96, True),
+    (torch.float32, 2, 2, 64, (30, 30, 9), (16, 200, 1000), 1, 1, 1, False),    # K above 128 and 1000 leaves
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[str(i) for i in range(len(SMALL))])
+def test_small_trees(case):
+    dtype, H, H_kv, D, fanout, K, B, N, T, perm = case
+    sh = synth.custom(dtype=dtype, n_heads=H, n_kv_heads=H_kv, head_dim=D, fanout=fanout, keep=K, batch=B,
+                      n_tokens=N, seq_len=T, permuted=perm)
+    w = synth.make_workload(sh, "cuda", 4242)
+    g = gpu_run(w, K)
+    check_structure(w, K, g)
+    compare(w, K, g)
+
+
+def test_balanced_lambda_regime():
+    # KG queries scaled so the KG and sequence log-sum-exps are comparable and
+    # both lambda weights matter.
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(10, 10, 10),
+                      keep=(4, 4, 16), batch=2, n_tokens=32, seq_len=64)
+    w = synth.make_workload(sh, "cuda", 7)
+    w.q_kg.mul_(0.15)
+    g = gpu_run(w, sh.keep)
+    compare(w, sh.keep, g)
+
+
+def test_scale_argument():
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=4, n_kv_heads=1, head_dim=64, fanout=(6, 6, 6),
+                      keep=(2, 3, 8), batch=2, n_tokens=16, seq_len=24)
+    w = synth.make_workload(sh, "cuda", 8)
+    g = gpu_run(w, sh.keep, scale=0.05)
+    compare(w, sh.keep, g, scale=0.05)
+
+
+def test_all_keys_identical_mass_ties():
+    # Every score ties exactly; more ambiguous candidates than one refinement
+    # chunk: the lowest row ids must win at every level.
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=2, n_kv_heads=1, head_dim=128, fanout=(40, 30, 20),
+                      keep=(5, 70, 150), batch=2, n_tokens=4, seq_len=8, permuted=True)
+    w = synth.make_workload(sh, "cuda", 9)
+    for t in (w.root_keys, w.mid_keys, w.leaf_keys):
+        t.copy_(w.leaf_keys[0, 0].expand_as(t))
+    g = gpu_run(w, sh.keep)
+    compare(w, sh.keep, g)
+    assert g["kept_root"][0, 0].tolist() == list(range(5))
+
+
+def test_zero_queries():
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=2, n_kv_heads=1, head_dim=128, fanout=(8, 8, 8),
+                      keep=(3, 5, 7), batch=2, n_tokens=4, seq_len=8)
+    w = synth.make_workload(sh, "cuda", 10)
+    w.q_kg.zero_()
+    g = gpu_run(w, sh.keep)
+    compare(w, sh.keep, g)
+    assert g["kept_leaf"][0, 0].tolist() == list(range(7))
+
+
+def test_near_ties_need_exact_arithmetic():
+    # Pairs of float32 keys that differ in one component by one unit in the
+    # last place, and duplicated keys: the fp32 filter cannot order them,
+    # exact arithmetic must.
+    sh = synth.custom(dtype=torch.float32, n_heads=2, n_kv_heads=1, head_dim=64, fanout=(16, 8, 8),
+                      keep=(5, 11, 23), batch=3, n_tokens=7, seq_len=9)
+    w = synth.make_workload(sh, "cuda", 11)
+    for keys in (w.root_keys, w.mid_keys, w.leaf_keys):
+        k = keys[0]
+        n = k.shape[0]
+        for i in range(1, n, 2):
+            k[i] = k[i - 1]
+            j = i % sh.head_dim
+            k[i, j] = torch.nextafter(k[i - 1, j], torch.tensor(float("inf"), device=k.device))
+        for i in range(3, n, 7):
+            k[i] = k[i - 3]
+    g = gpu_run(w, sh.keep)
+    compare(w, sh.keep, g)
+
+
+def test_leaves_in_pinned_host_memory_small():
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(12, 10, 9),
+                      keep=(3, 4, 16), batch=3, n_tokens=16, seq_len=48, permuted=True)
+    w = synth.make_workload(sh, "cuda", 12)
+    g_dev = gpu_run(w, sh.keep)
+    hw = synth.Workload(sh, w.root_keys, w.mid_keys, w.leaf_keys.cpu().pin_memory(),
+                        w.leaf_values.cpu().pin_memory(), w.root_child, w.mid_child, w.q_kg, w.q_seq, w.k_seq,
+                        w.v_seq, w.targets)
+    g_host = gpu_run(hw, sh.keep)
+    for k in ("kept_root", "kept_mid", "kept_leaf", "out", "lse"):
+        assert torch.equal(g_dev[k], g_host[k]), k
+    compare(w, sh.keep, g_host)
+
+
+def test_deterministic_and_b0():
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(10, 10, 10),
+                      keep=(3, 4, 16), batch=4, n_tokens=32, seq_len=64)
+    w = synth.make_workload(sh, "cuda", 13)
+    with HikvpTree.from_workload(w) as tree:
+        a = gpu_run(w, sh.keep, tree=tree)
+        b = gpu_run(w, sh.keep, tree=tree)
+        for k in ("kept_root", "kept_mid", "kept_leaf", "out", "lse"):
+            assert torch.equal(a[k], b[k]), k
+        e = tree.attend(w.q_kg[:0], w.q_seq[:0], w.k_seq[:0], w.v_seq[:0], sh.keep)
+        tree.sync_status()
+        assert e["out"].numel() == 0
+
+
+def test_device_errors_are_reported():
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=2, n_kv_heads=1, head_dim=128, fanout=(4, 4, 4),
+                      keep=(2, 2, 2), batch=1, n_tokens=2, seq_len=2, permuted=True)
+    w = synth.make_workload(sh, "cuda", 14)
+    bad = w.mid_child.clone()
+    bad[0, 0, 0] = bad[0, 0, 1]          # not a permutation
+    with pytest.raises(AtlaskvError) as ei:
+        HikvpTree(w.root_keys, w.mid_keys, w.leaf_keys, w.leaf_values, sh.fanout, w.root_child, bad)
+    assert ei.value.status == 1
+    bad2 = w.root_child.clone()
+    bad2[0, 1, 1] = 99                    # out of range
+    with pytest.raises(AtlaskvError):
+        HikvpTree(w.root_keys, w.mid_keys, w.leaf_keys, w.leaf_values, sh.fanout, bad2, w.mid_child)
+    with HikvpTree.from_workload(w) as tree:
+        small = torch.empty(256, dtype=torch.uint8, device="cuda")
+        with pytest.raises(AtlaskvError) as ei:
+            tree.attend(w.q_kg, w.q_seq, w.k_seq, w.v_seq, sh.keep, workspace=small)
+        assert ei.value.status == 2
+        with pytest.raises(AtlaskvError) as ei:
+            tree.attend(w.q_kg, w.q_seq, w.k_seq, w.v_seq, (2, 9, 2))
+        assert ei.value.status == 1
+
+
+# ---- benchmark shapes at full size ----------------------------------------
+
+@pytest.fixture(scope="module")
+def full_cache():
+    return {}
+
+
+@pytest.mark.parametrize("i", [1, 2, 3])
+def test_full_size_shapes(i, full_cache):
+    sh = synth.shape(i)
+    w = synth.make_workload(sh, "cuda", 1000 + i)
+    g = gpu_run(w, sh.keep)
+    check_structure(w, sh.keep, g)
+    trav = sample_traversals(sh.batch, sh.n_heads, 10, seed=i)
+    compare(w, sh.keep, g, trav)
+    del w
+    torch.cuda.empty_cache()
+
+
+def test_full_size_host_leaves():
+    sh = synth.shape(4)
+    free_host = os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_AVPHYS_PAGES")
+    need = 2 * sh.n_leaves * sh.head_dim * 2 + (8 << 30)
+    if free_host < need:
+        pytest.skip("host memory %.0f GB below the %.0f GB the host-leaf shape needs" % (free_host / 1e9, need / 1e9))
+    w = synth.make_workload(sh, "cuda", 1004)
+    g = gpu_run(w, sh.keep)
+    check_structure(w, sh.keep, g)
+    trav = sample_traversals(sh.batch, sh.n_heads, 6, seed=4)
+    compare(w, sh.keep, g, trav)
