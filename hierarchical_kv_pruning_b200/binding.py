@@ -26,7 +26,10 @@ ATLASKV_LEAVES_DEVICE, ATLASKV_LEAVES_HOST_PINNED = 0, 1
 
 # Every symbol include/atlaskv.h declares.
 EXPORTED = ("atlaskv_create_tree", "atlaskv_workspace_size", "atlaskv_attend", "atlaskv_sync_status",
-            "atlaskv_set_profiling", "atlaskv_stage_times", "atlaskv_destroy", "atlaskv_last_error")
+            "atlaskv_set_profiling", "atlaskv_stage_times", "atlaskv_attend_static", "atlaskv_destroy",
+            "atlaskv_last_error")
+# Size of the library's static device scratch (ATLASKV_STATIC_SCRATCH_BYTES).
+ATLASKV_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class AtlaskvError(RuntimeError):
@@ -83,6 +86,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
             lib.atlaskv_workspace_size.argtypes = [V, ctypes.POINTER(atlaskv_params), I32, I32, I32, I32,
                                                    ctypes.POINTER(SZ)]
             lib.atlaskv_attend.argtypes = [V, ctypes.POINTER(atlaskv_params), ctypes.POINTER(atlaskv_io), V, SZ, V]
+            lib.atlaskv_attend_static.argtypes = [V, ctypes.POINTER(atlaskv_params), ctypes.POINTER(atlaskv_io), V]
             lib.atlaskv_sync_status.argtypes = [V, V]
             lib.atlaskv_set_profiling.argtypes = [V, I32]
             lib.atlaskv_stage_times.argtypes = [V, ctypes.POINTER(ctypes.c_float), I32]
@@ -124,6 +128,14 @@ def atlaskv_attend(tree: int, params: atlaskv_params, io: atlaskv_io, workspace:
                    stream: int = 0) -> None:
     _check(load_library().atlaskv_attend(ctypes.c_void_p(tree), ctypes.byref(params), ctypes.byref(io),
                                          ctypes.c_void_p(workspace), workspace_bytes, ctypes.c_void_p(stream)))
+
+
+def atlaskv_attend_static(tree: int, params: atlaskv_params, io: atlaskv_io, stream: int = 0) -> None:
+    """atlaskv_attend without a caller workspace: the library's static device
+    scratch (ATLASKV_STATIC_SCRATCH_BYTES) is used instead.  For callers that
+    cannot allocate device memory; calls that overlap on the GPU race."""
+    _check(load_library().atlaskv_attend_static(ctypes.c_void_p(tree), ctypes.byref(params), ctypes.byref(io),
+                                                ctypes.c_void_p(stream)))
 
 
 def atlaskv_sync_status(tree: int, stream: int = 0) -> None:

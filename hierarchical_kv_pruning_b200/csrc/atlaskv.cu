@@ -15,6 +15,7 @@
 #include "atlaskv.h"
 #include "attend.cuh"
 #include "descend.cuh"
+#include "internal.h"
 #include "staging.cuh"
 
 namespace {
@@ -51,6 +52,12 @@ constexpr int kMaxCandidates = 8192;   // per level and traversal (shared-memory
 constexpr int kNumEvents = 6;
 
 }  // namespace
+
+atlaskv_status akv_report(atlaskv_status st, const char *msg)
+{
+    g_last_error = msg;
+    return st;
+}
 
 struct atlaskv_tree {
     atlaskv_tree_desc d;

@@ -156,6 +156,31 @@ atlaskv_status atlaskv_sync_status(atlaskv_tree *tree, void *stream);
 atlaskv_status atlaskv_set_profiling(atlaskv_tree *tree, int32_t enable);
 atlaskv_status atlaskv_stage_times(atlaskv_tree *tree, float *ms, int32_t n);
 
+/* Size in bytes of the static device scratch used by atlaskv_attend_static. */
+#define ATLASKV_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* Allocation-free variant of atlaskv_attend.  The paper has no counterpart:
+ * this exists for callers that cannot give the library a device workspace --
+ * a host program using only this C ABI with no device allocator of its own, a
+ * process whose device memory is fully pre-partitioned by another runtime, or a
+ * hot loop where a device allocation (which may synchronise the device and
+ * take unbounded time) is not allowed.  Same inputs, outputs, validation and
+ * results as atlaskv_attend; the scratch comes from a static device array of
+ * ATLASKV_STATIC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.
+ * - Sizes whose atlaskv_workspace_size() exceeds ATLASKV_STATIC_SCRATCH_BYTES
+ *   are rejected with ATLASKV_ENOMEM and nothing is enqueued (host-resident
+ *   leaf trees of realistic size always are: their staging pools are large).
+ * - The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.
+ * - All calls share the one array, and it keeps the previous call's contents.
+ *   Calls whose work overlaps on the GPU (different streams, or different host
+ *   threads, without ordering between them) race on it: serialise them.
+ * - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+atlaskv_status atlaskv_attend_static(atlaskv_tree *tree, const atlaskv_params *params, const atlaskv_io *io,
+                                     void *stream);
+
 /* Release the handle and the small device buffers it owns; the caller's
  * buffers are untouched.  NULL is accepted. */
 atlaskv_status atlaskv_destroy(atlaskv_tree *tree);
