@@ -223,7 +223,7 @@ def run_ours(args):
     stage = [0.0, 0.0, 0.0]
     step_ms = []
     launches = 0
-    n_launch = 2 if not sh.leaf_on_host else 8
+    n_launch = 8 if not sh.leaf_on_host else 14   # 3 levels x (score + select) + attention (+ memset, staging)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -240,6 +240,7 @@ def run_ours(args):
             for i in range(3):
                 stage[i] += st[i]
             launches += n_launch
+        refine = tree.refine_stats()
         torch.cuda.synchronize()
     tree.set_profiling(False)
     total_ms = sum(step_ms)
@@ -309,6 +310,7 @@ def run_ours(args):
     roof["stage_ms"] = {n: round(v, 4) for n, v in zip(names, st_ms)}
     roof["algorithmic_bytes"] = {k: alg[k] for k in ("descend", "attend", "staging")}
     roof["attend_tflops"] = alg["attend_flops"] / (st_ms[2] * 1e-3) / 1e12 if st_ms[2] > 0 else None
+    roof["exact_refinement_last_step"] = refine
 
     clocks = clk.summary()
     line = {

@@ -26,8 +26,8 @@ ATLASKV_LEAVES_DEVICE, ATLASKV_LEAVES_HOST_PINNED = 0, 1
 
 # Every symbol include/atlaskv.h declares.
 EXPORTED = ("atlaskv_create_tree", "atlaskv_workspace_size", "atlaskv_attend", "atlaskv_sync_status",
-            "atlaskv_set_profiling", "atlaskv_stage_times", "atlaskv_attend_static", "atlaskv_destroy",
-            "atlaskv_last_error")
+            "atlaskv_set_profiling", "atlaskv_stage_times", "atlaskv_refine_stats", "atlaskv_attend_static",
+            "atlaskv_destroy", "atlaskv_last_error")
 # Size of the library's static device scratch (ATLASKV_STATIC_SCRATCH_BYTES).
 ATLASKV_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -90,6 +90,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
             lib.atlaskv_sync_status.argtypes = [V, V]
             lib.atlaskv_set_profiling.argtypes = [V, I32]
             lib.atlaskv_stage_times.argtypes = [V, ctypes.POINTER(ctypes.c_float), I32]
+            lib.atlaskv_refine_stats.argtypes = [V, ctypes.POINTER(ctypes.c_uint64), I32]
             lib.atlaskv_destroy.argtypes = [V]
             lib.atlaskv_last_error.argtypes = []
             lib.atlaskv_last_error.restype = ctypes.c_char_p
@@ -150,6 +151,16 @@ def atlaskv_stage_times(tree: int):
     buf = (ctypes.c_float * 3)()
     _check(load_library().atlaskv_stage_times(ctypes.c_void_p(tree), buf, 3))
     return [float(x) for x in buf]
+
+
+def atlaskv_refine_stats(tree: int):
+    """Descent counters of the last profiled call: per level [selections,
+    selections needing exact refinement, ambiguous candidates, exact scores]."""
+    buf = (ctypes.c_uint64 * 12)()
+    _check(load_library().atlaskv_refine_stats(ctypes.c_void_p(tree), buf, 12))
+    v = [int(x) for x in buf]
+    return {lvl: dict(zip(("selections", "refined", "ambiguous", "exact_scores"), v[4 * i:4 * i + 4]))
+            for i, lvl in enumerate(("root", "mid", "leaf"))}
 
 
 def atlaskv_destroy(tree: int) -> None:
@@ -267,3 +278,6 @@ class HikvpTree:
 
     def stage_times(self):
         return atlaskv_stage_times(self.handle)
+
+    def refine_stats(self):
+        return atlaskv_refine_stats(self.handle)

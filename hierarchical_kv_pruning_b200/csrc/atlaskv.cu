@@ -66,6 +66,7 @@ struct atlaskv_tree {
     const void *leaf_values_dev;
     float *norm_bound;             // device [3][H_kv]
     int *status;                   // device sticky status word
+    unsigned long long *stats;     // device [3][4] descent counters (filled while profiling)
     bool profiling;
     bool timed;                    // the last attend recorded events
     bool host_mode_last;
@@ -77,8 +78,9 @@ namespace {
 size_t esize(int dtype) { return dtype == ATLASKV_F32 ? 4 : 2; }
 
 struct Layout {
-    size_t s_ws, anorm_ws, kept[3], leaf_slot, kept_leaf_row, vslot, umid, ucount_mid, uleaf, ucount_leaf,
-        key_pool, val_pool, total;
+    size_t s_ws, s64_ws, a64_ws, anorm_ws, f_ws, queue, qcount, kept[3], leaf_slot, kept_leaf_row, vslot, umid,
+        ucount_mid, uleaf, ucount_leaf, key_pool, val_pool, total;
+    int cap, kcap, fstride;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -97,8 +99,18 @@ Layout plan(const atlaskv_tree *t, const atlaskv_params *p, int B, int N, int H,
         off = align256(off + bytes);
         return o;
     };
+    const long long cmax = std::max<long long>(t->d.fanout[0], std::max<long long>((long long)p->K_root * t->d.fanout[1],
+                                                                                  (long long)p->K_mid * t->d.fanout[2]));
+    L.cap = (int)((cmax + 3) & ~3LL);
+    L.kcap = pow2_at_least(std::max(p->K_root, std::max(p->K_mid, p->K_leaf)), 32);
+    L.fstride = L.cap + 2 * L.kcap;
     L.s_ws = take(BH * D * 4);
+    L.s64_ws = take(BH * D * 8);
+    L.a64_ws = take(BH * D * 8);
     L.anorm_ws = take(BH * 4);
+    L.f_ws = take(BH * (size_t)L.fstride * 4);
+    L.queue = take(3 * BH * 3 * 4);
+    L.qcount = take(4 * 4);
     for (int l = 0; l < 3; ++l) L.kept[l] = take(BH * (size_t)(l == 0 ? p->K_root : l == 1 ? p->K_mid : p->K_leaf) * 4);
     if (host) {
         const int G = H / t->d.n_kv_heads;
@@ -184,26 +196,96 @@ atlaskv_status check_table(const int32_t *tab, long long entries_per_head, int H
     return ATLASKV_OK;
 }
 
-// ---- descent launch -------------------------------------------------------
-template <typename T, int D>
-atlaskv_status launch_descend(const akv::DescendParams &dp, int grid, cudaStream_t s)
+// ---- descent launches -----------------------------------------------------
+// Scoring CTAs serve GP query heads of a (query, KV head) group: the largest
+// of 4, 2, 1 that divides G.  Selection runs one warp per traversal.
+int heads_per_cta(int G) { return G % 4 == 0 ? 4 : (G % 2 == 0 ? 2 : 1); }
+
+template <typename T, int D, int GP>
+atlaskv_status launch_root(const akv::DescendParams &dp, cudaStream_t s)
 {
-    const size_t smem = akv::DescendSmem<D>::bytes(dp.cap, dp.kcap);
-    static size_t configured = 0;
-    if (smem > configured) {
-        AKV_CUDA(cudaFuncSetAttribute(akv::descend_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        configured = smem;
-    }
-    akv::descend_kernel<T, D><<<grid, akv::kDescendThreads, smem, s>>>(dp);
+    const long long grid = (long long)dp.B * dp.H_kv * (dp.G / GP);
+    const size_t smem = akv::root_kernel_smem<T, D, GP>();
+    akv::root_kernel<T, D, GP><<<(unsigned)grid, akv::kScoreThreads, smem, s>>>(dp);
     AKV_CUDA(cudaGetLastError());
     return ATLASKV_OK;
 }
 
-atlaskv_status dispatch_descend(int dtype, int D, const akv::DescendParams &dp, int grid, cudaStream_t s)
+template <typename T, int D, int GP>
+atlaskv_status launch_score(const akv::DescendParams &dp, int L, cudaStream_t s)
+{
+    const int Kp = dp.K[L - 1], fo = dp.fanout[L];
+    const int ppc = std::max(1, 512 / fo);            // parents per chunk: about 512 rows
+    const int pchunks = (Kp + ppc - 1) / ppc;         // covers a union of Kp parents; larger ones loop
+    const long long grid = (long long)dp.B * dp.H_kv * (dp.G / GP) * pchunks;
+    if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "scoring grid too large");
+    const size_t smem = akv::score_kernel_smem<GP>(Kp);
+    static size_t configured = 0;
+    if (smem > 48 * 1024 && smem > configured) {
+        AKV_CUDA(cudaFuncSetAttribute(akv::score_kernel<T, D, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem));
+        configured = smem;
+    }
+    akv::score_kernel<T, D, GP><<<(unsigned)grid, akv::kScoreThreads, smem, s>>>(dp, L, ppc, pchunks);
+    AKV_CUDA(cudaGetLastError());
+    return ATLASKV_OK;
+}
+
+template <typename T, int D>
+atlaskv_status launch_select(const akv::DescendParams &dp, int L, cudaStream_t s)
+{
+    const long long BH = (long long)dp.B * dp.H;
+    const long long grid = (BH + akv::kSelectWarps - 1) / akv::kSelectWarps;
+    const size_t smem = (size_t)akv::kSelectWarps * akv::SelectScratch::bytes(dp.cap, dp.kcap, D);
+    if (smem > 227 * 1024)
+        return fail(ATLASKV_EUNSUPPORTED, "selection needs %zu bytes of shared memory per CTA", smem);
+    static size_t configured = 0;
+    if (smem > 48 * 1024 && smem > configured) {
+        AKV_CUDA(cudaFuncSetAttribute(akv::select_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem));
+        configured = smem;
+    }
+    akv::select_kernel<T, D><<<(unsigned)grid, akv::kSelectWarps * 32, smem, s>>>(dp, L);
+    AKV_CUDA(cudaGetLastError());
+    // tier 3 for whatever the bounds left undecided (usually nothing: the warps read an empty queue)
+    const size_t esmem = (size_t)akv::kSelectWarps * akv::ExactScratch::bytes(dp.kcap);
+    static size_t econfigured = 0;
+    if (esmem > 48 * 1024 && esmem > econfigured) {
+        AKV_CUDA(cudaFuncSetAttribute(akv::exact_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)esmem));
+        econfigured = esmem;
+    }
+    const long long egrid = std::min<long long>(grid, 2 * 148);
+    akv::exact_kernel<T, D><<<(unsigned)egrid, akv::kSelectWarps * 32, esmem, s>>>(dp, L);
+    AKV_CUDA(cudaGetLastError());
+    return ATLASKV_OK;
+}
+
+// Run levels [first, last] of the descent (scores then selection per level).
+template <typename T, int D>
+atlaskv_status descend_levels(const akv::DescendParams &dp, int first, int last, cudaStream_t s)
+{
+    const int gp = heads_per_cta(dp.G);
+    for (int L = first; L <= last; ++L) {
+        atlaskv_status st;
+        if (L == 0)
+            st = gp == 4 ? launch_root<T, D, 4>(dp, s) : gp == 2 ? launch_root<T, D, 2>(dp, s) : launch_root<T, D, 1>(dp, s);
+        else
+            st = gp == 4 ? launch_score<T, D, 4>(dp, L, s)
+                         : gp == 2 ? launch_score<T, D, 2>(dp, L, s) : launch_score<T, D, 1>(dp, L, s);
+        if (st != ATLASKV_OK) return st;
+        st = launch_select<T, D>(dp, L, s);
+        if (st != ATLASKV_OK) return st;
+    }
+    return ATLASKV_OK;
+}
+
+atlaskv_status dispatch_descend(int dtype, int D, const akv::DescendParams &dp, int first, int last, cudaStream_t s)
 {
     if (dtype == ATLASKV_F32)
-        return D == 64 ? launch_descend<float, 64>(dp, grid, s) : launch_descend<float, 128>(dp, grid, s);
-    return D == 64 ? launch_descend<__nv_bfloat16, 64>(dp, grid, s) : launch_descend<__nv_bfloat16, 128>(dp, grid, s);
+        return D == 64 ? descend_levels<float, 64>(dp, first, last, s) : descend_levels<float, 128>(dp, first, last, s);
+    return D == 64 ? descend_levels<__nv_bfloat16, 64>(dp, first, last, s)
+                   : descend_levels<__nv_bfloat16, 128>(dp, first, last, s);
 }
 
 // ---- attention launch -----------------------------------------------------
@@ -353,7 +435,8 @@ atlaskv_status atlaskv_create_tree(const atlaskv_tree_desc *d, void *stream, atl
         t->leaf_values_dev = pv;
     }
     if (cudaMalloc(&t->norm_bound, 3 * sizeof(float) * d->n_kv_heads) != cudaSuccess ||
-        cudaMalloc(&t->status, sizeof(int)) != cudaSuccess) {
+        cudaMalloc(&t->status, sizeof(int)) != cudaSuccess ||
+        cudaMalloc(&t->stats, 12 * sizeof(unsigned long long)) != cudaSuccess) {
         cudaGetLastError();
         return bail(fail(ATLASKV_ECUDA, "device allocation of the tree's bound/status words failed"));
     }
@@ -457,11 +540,16 @@ atlaskv_status atlaskv_attend(atlaskv_tree *t, const atlaskv_params *p, const at
     dp.K[2] = p->K_leaf;
     dp.s_ws = reinterpret_cast<float *>(ws + L.s_ws);
     dp.anorm_ws = reinterpret_cast<float *>(ws + L.anorm_ws);
-    const long long cmax = std::max<long long>(t->d.fanout[0], std::max<long long>((long long)p->K_root * t->d.fanout[1],
-                                                                                  (long long)p->K_mid * t->d.fanout[2]));
-    dp.cap = pow2_at_least(cmax, 64);
-    dp.kcap = pow2_at_least(std::max(p->K_root, std::max(p->K_mid, p->K_leaf)), 64);
+    dp.s64_ws = reinterpret_cast<double *>(ws + L.s64_ws);
+    dp.a64_ws = reinterpret_cast<double *>(ws + L.a64_ws);
+    dp.f_ws = reinterpret_cast<float *>(ws + L.f_ws);
+    dp.fstride = L.fstride;
+    dp.cap = L.cap;
+    dp.kcap = L.kcap;
+    dp.queue = reinterpret_cast<int *>(ws + L.queue);
+    dp.qcount = reinterpret_cast<int *>(ws + L.qcount);
     dp.status = t->status;
+    dp.stats = t->profiling ? t->stats : nullptr;
 
     const float scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)D);
     akv::AttnParams ap{};
@@ -491,12 +579,10 @@ atlaskv_status atlaskv_attend(atlaskv_tree *t, const atlaskv_params *p, const at
         if (st_ != ATLASKV_OK) return st_;     \
     } while (0)
 
+    if (prof) AKV_CUDA(cudaMemsetAsync(t->stats, 0, 12 * sizeof(unsigned long long), s));
     if (!host) {
         AKV_STEP(mark(0));
-        dp.first_level = 0;
-        dp.last_level = 2;
-        dp.s_ws = nullptr;   // fused: token sums stay in shared memory
-        AKV_STEP(dispatch_descend(t->d.dtype, D, dp, BH, s));
+        AKV_STEP(dispatch_descend(t->d.dtype, D, dp, 0, 2, s));
         AKV_STEP(mark(1));
         ap.lk_base = t->d.leaf_keys;
         ap.lv_base = t->d.leaf_values;
@@ -518,19 +604,15 @@ atlaskv_status atlaskv_attend(atlaskv_tree *t, const atlaskv_params *p, const at
         void *pool = ws + L.key_pool;
         void *vpool = ws + L.val_pool;
         AKV_STEP(mark(0));
-        dp.first_level = 0;
-        dp.last_level = 1;
-        AKV_STEP(dispatch_descend(t->d.dtype, D, dp, BH, s));
+        AKV_STEP(dispatch_descend(t->d.dtype, D, dp, 0, 1, s));
         AKV_STEP(mark(1));
         AKV_STEP(launch_dedupe(kept[1], n_mid, groups, umid, leaf_slot, cmid, s));
         AKV_STEP(dispatch_stage_keys(t, umid, cmid, n_mid, groups, pool, s));
         AKV_STEP(mark(2));
-        dp.first_level = 2;
-        dp.last_level = 2;
         dp.keys[2] = pool;
         dp.leaf_slot = leaf_slot;
         dp.kept_leaf_row = kept_leaf_row;
-        AKV_STEP(dispatch_descend(t->d.dtype, D, dp, BH, s));
+        AKV_STEP(dispatch_descend(t->d.dtype, D, dp, 2, 2, s));
         AKV_STEP(mark(3));
         AKV_STEP(launch_dedupe(kept[2], n_leaf, groups, uleaf, vslot, cleaf, s));
         AKV_STEP(dispatch_stage_values(t, uleaf, cleaf, n_leaf, groups, vpool, s));
@@ -596,11 +678,22 @@ atlaskv_status atlaskv_stage_times(atlaskv_tree *t, float *ms, int32_t n)
     return ATLASKV_OK;
 }
 
+atlaskv_status atlaskv_refine_stats(atlaskv_tree *t, uint64_t *counts, int32_t n)
+{
+    if (!t || !counts || n < 1) return fail(ATLASKV_EINVAL, "null tree/counts or n < 1");
+    if (!t->timed) return fail(ATLASKV_EINVAL, "no attend call was profiled (enable profiling first)");
+    unsigned long long v[12];
+    AKV_CUDA(cudaMemcpy(v, t->stats, sizeof v, cudaMemcpyDeviceToHost));
+    for (int i = 0; i < n && i < 12; ++i) counts[i] = v[i];
+    return ATLASKV_OK;
+}
+
 atlaskv_status atlaskv_destroy(atlaskv_tree *t)
 {
     if (!t) return ATLASKV_OK;
     if (t->norm_bound) cudaFree(t->norm_bound);
     if (t->status) cudaFree(t->status);
+    if (t->stats) cudaFree(t->stats);
     for (int i = 0; i < kNumEvents; ++i)
         if (t->ev[i]) cudaEventDestroy(t->ev[i]);
     delete t;

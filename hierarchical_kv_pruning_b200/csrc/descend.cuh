@@ -1,4 +1,4 @@
-// Level-by-level HiKVP descent: one CTA per traversal (query b, head h).
+// Level-by-level HiKVP descent.
 //
 // "AtlasKV: Augmenting LLMs with Billion-Scale Knowledge Graphs in 20GB VRAM",
 // section "Quick read / How it works": score the query against the resident
@@ -7,15 +7,24 @@
 // the query tokens of <q_n, k>/sqrt(D); ranking by x(k) = sum_d s[d] k[d] with
 // s[d] = sum_n q[n][d] is equivalent.
 //
+// The descent runs level-synchronously over all traversals (query b, head h):
+//   root_kernel    token sums s of GP heads per CTA, fp32 scores of all roots
+//   select_kernel  one warp per traversal: top-K of its candidates' scores
+//   score_kernel   one CTA per (query, KV head, chunk of the union of its GP
+//                  heads' kept parents): every child row is loaded once and
+//                  scored against the GP token-sum vectors
+// Scores live in a per-traversal buffer (workspace, L2-resident at the
+// benchmark sizes); each phase is a wide, short kernel.
+//
 // Ranking is exact.  Each candidate gets an fp32 score f (token sums and dot
 // products in fp32) with the rigorous bound |f - x| <= E, where
 //   E = (g_D (1 + g_N) + g_N) * ||a||_2 * max_k ||k||_2 + D 2^-148,
 //   g_n = n u / (1 - n u), u = 2^-24, a[d] = sum_n |q[n][d]|
-// (Higham's dot-product and summation bounds plus Cauchy-Schwarz; the last
-// term covers underflow).  With t the K-th largest f, every candidate with
-// f > t + 2E is certainly kept, every one with f < t - 2E certainly dropped;
-// the rest (always containing t's candidate) are ranked by their exact score
-// (exact.cuh) and then by lower row id.
+// (Higham's dot-product and summation bounds, for any evaluation order, plus
+// Cauchy-Schwarz; the last term covers underflow).  With t the K-th largest f,
+// every candidate with f > t + 2E is certainly kept, every one with
+// f < t - 2E certainly dropped; the rest (always containing t's candidate) are
+// ranked by their exact score and then by lower row id.
 #pragma once
 
 #include <float.h>
@@ -25,8 +34,9 @@
 
 namespace akv {
 
-constexpr int kDescendThreads = 256;
-constexpr int kRefineChunk = 64;
+constexpr int kScoreThreads = 256;
+constexpr int kSelectWarps = 4;
+constexpr int kRefineChunk = 16;   // exact scores per refinement chunk (a pool of two chunks fills a warp)
 
 struct DescendParams {
     const void *q_kg;            // [B][N][H][D]
@@ -38,15 +48,22 @@ struct DescendParams {
     const float *norm_bound;     // [3][H_kv] upper bounds of key row 2-norms
     int K[3];
     int32_t *kept[3];            // [B H][K_l] ascending row ids
-    float *s_ws;                 // [B H][D] fp32 token sums (split launches)
-    float *anorm_ws;             // [B H] upper bound of ||a||_2 (split launches)
-    int first_level, last_level;
-    int cap;                     // candidate capacity (power of two >= every level's C)
+    float *s_ws;                 // [B H][D] fp32 token sums (rounded from s64)
+    double *s64_ws;              // [B H][D] fp64 token sums
+    double *a64_ws;              // [B H][D] fp64 sums of |q| over the tokens
+    float *anorm_ws;             // [B H] upper bound of ||a||_2
+    float *f_ws;                 // [B H][fstride] fp32 filter scores of the current level; for a traversal
+                                 // left to the exact pass: its candidate list, then its decided entries
+    int fstride;                 // floats per traversal in f_ws: cap + 2 kcap
+    int cap;                     // per-traversal score capacity (>= every level's candidate count)
     int kcap;                    // kept capacity (power of two >= every K)
-    // host-staged leaves: kept mid k of traversal bh has its leaf block at pool slot
-    // leaf_slot[bh K_mid + k]; leaf candidate (k, j) is pool row slot * b_L + j.
+    int *queue;                  // [3][B H][3] (traversal, decided, listed) left to the exact pass
+    int *qcount;                 // [3] queue lengths (zeroed by the root kernel)
+    // host-staged leaves: kept mid k of traversal bh has its leaf block at pool
+    // slot leaf_slot[bh K_mid + k]; leaf candidate (k, j) is pool row slot * b_L + j.
     const int32_t *leaf_slot;
     int32_t *kept_leaf_row;      // [B H][K_leaf] pool row of each kept leaf (host path)
+    unsigned long long *stats;   // [3][4] optional counters: selections, refined, ambiguous, exact scores
     int *status;
 };
 
@@ -56,64 +73,346 @@ __device__ __forceinline__ double gamma_n(int n)
     return nu / (1.0 - nu);
 }
 
-// --------------------------------------------------------------------------
-// Block-wide k-th largest (1-based) of n uint32 keys, MSB-first radix select.
-template <typename KeyFn>
-__device__ uint32_t block_kth_largest(int n, int k, KeyFn key_of, uint32_t *hist, int *misc)
+__device__ __forceinline__ unsigned lanemask_lt() { return (1u << (threadIdx.x & 31)) - 1u; }
+
+// ==========================================================================
+// Scoring side (CTA-level)
+// ==========================================================================
+
+// Token sums of GP consecutive heads (a1), in float64: s64[g][d] =
+// sum_n q[n][h0+g][d] and a64[g][d] = sum_n |q[n][h0+g][d]| (relative error
+// below g_N in binary64).  The fp32 filter uses s = fl32(s64), whose error
+// |s - sum_n q| <= (u32 + g64_N) a is well inside the g32_N a of the bound.
+// Every thread issues 16-byte loads; partial sums over token slices meet in
+// `part` ([SLICES][COMBOS][2][EV] doubles).
+template <typename T, int D, int GP>
+__device__ void token_sums(const T *qb, size_t q_stride, int N, float *s, double *s64, double *a64, double *part,
+                           double *anorm)
 {
-    uint32_t prefix = 0, mask = 0;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-        __syncthreads();
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            const uint32_t key = key_of(i);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            const int lane = threadIdx.x;
-            uint32_t cnt[8], tot = 0;
+    constexpr int EV = Vec16<T>::E;
+    constexpr int VPH = D / EV;
+    constexpr int COMBOS = GP * VPH;
+    static_assert(kScoreThreads % COMBOS == 0, "columns must divide the block");
+    constexpr int SLICES = kScoreThreads / COMBOS;
+    const int combo = threadIdx.x % COMBOS, slice = threadIdx.x / COMBOS;
+    const int g = combo / VPH, v = combo % VPH;
+    double ps[EV], pa[EV];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                cnt[j] = hist[255 - 8 * lane - j];
-                tot += cnt[j];
-            }
-            uint32_t incl = tot;
+    for (int e = 0; e < EV; ++e) ps[e] = pa[e] = 0.0;
+    const T *col = qb + (size_t)g * D + v * EV;
+    int n = slice;
+    for (; n + 3 * SLICES < N; n += 4 * SLICES) {
+        uint4 w[4];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
-            }
-            const uint32_t excl = incl - tot;
-            if (excl < (uint32_t)k && (uint32_t)k <= incl) {
-                uint32_t run = excl;
+        for (int u = 0; u < 4; ++u) w[u] = ldg16(col + (size_t)(n + u * SLICES) * q_stride);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (run + cnt[j] >= (uint32_t)k) {
-                        misc[0] = 255 - 8 * lane - j;
-                        misc[1] = k - (int)run;
-                        break;
-                    }
-                    run += cnt[j];
-                }
+        for (int u = 0; u < 4; ++u) {
+            float x[EV];
+            Vec16<T>::unpack(w[u], x);
+#pragma unroll
+            for (int e = 0; e < EV; ++e) {
+                ps[e] += (double)x[e];
+                pa[e] += fabs((double)x[e]);
             }
         }
-        __syncthreads();
-        prefix |= ((uint32_t)misc[0]) << shift;
-        mask |= 255u << shift;
-        k = misc[1];
-        __syncthreads();
     }
-    return prefix;
+    for (; n < N; n += SLICES) {
+        float x[EV];
+        Vec16<T>::unpack(ldg16(col + (size_t)n * q_stride), x);
+#pragma unroll
+        for (int e = 0; e < EV; ++e) {
+            ps[e] += (double)x[e];
+            pa[e] += fabs((double)x[e]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < EV; ++e) {
+        part[((slice * COMBOS + combo) * 2 + 0) * EV + e] = ps[e];
+        part[((slice * COMBOS + combo) * 2 + 1) * EV + e] = pa[e];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < GP * D; i += blockDim.x) {
+        const int cb = i / EV, e = i % EV;   // i = (g * VPH + v) * EV + e
+        double ss = 0.0, aa = 0.0;
+        for (int sl = 0; sl < SLICES; ++sl) {
+            ss += part[((sl * COMBOS + cb) * 2 + 0) * EV + e];
+            aa += part[((sl * COMBOS + cb) * 2 + 1) * EV + e];
+        }
+        s64[i] = ss;
+        a64[i] = aa;
+        s[i] = (float)ss;
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int gg = warp; gg < GP; gg += blockDim.x >> 5) {
+        double acc = 0.0;
+        for (int d = lane; d < D; d += 32) acc = fma(a64[gg * D + d], a64[gg * D + d], acc);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) anorm[gg] = sqrt(acc) * (1.0 + 1e-9);   // covers the binary64 rounding of a64
+    }
+    __syncthreads();
 }
 
-// Ascending block bitonic sort of n (power of two) uint64 values.
-__device__ void block_sort_u64(uint64_t *a, int n)
+template <typename T, int D, int GP>
+__host__ __device__ constexpr size_t root_kernel_smem()
 {
+    return (size_t)kScoreThreads * 2 * Vec16<T>::E * 8 + (size_t)2 * GP * D * 8;
+}
+
+// Score `nrows` rows against the GP token-sum vectors s (shared).  Eight lanes
+// per row, each holding its slice of every s in registers; rows are fetched
+// with 16-byte coalesced loads, four rows per lane group in flight.
+// row_of(r) gives the row index (in units of D elements) of row r;
+// store(g, r, value) stores head g's score of row r.
+template <typename T, int D, int GP, typename RowFn, typename StoreFn>
+__device__ void score_rows(const T *__restrict__ kbase, const float *s, int nrows, RowFn row_of, StoreFn store)
+{
+    constexpr int EV = Vec16<T>::E;
+    constexpr int VPR = D / EV;
+    constexpr int LPG = 8;
+    constexpr int VPL = VPR / LPG;
+    constexpr int U = 4;
+    static_assert(VPL >= 1 && VPR % LPG == 0, "row must split over 8 lanes");
+    static_assert(GP <= LPG, "one storing lane per head");
+    const int sub = threadIdx.x & 7;
+    const int grp = threadIdx.x >> 3;
+    const int ngrp = blockDim.x >> 3;
+    float sreg[GP][VPL * EV];
+#pragma unroll
+    for (int g = 0; g < GP; ++g)
+#pragma unroll
+        for (int v = 0; v < VPL; ++v)
+#pragma unroll
+            for (int e = 0; e < EV; ++e) sreg[g][v * EV + e] = s[g * D + (sub + LPG * v) * EV + e];
+
+    for (int base_r = 0; base_r < nrows; base_r += ngrp * U) {
+        uint4 buf[U][VPL];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int r = base_r + u * ngrp + grp;
+            const T *rp = kbase + (size_t)(r < nrows ? row_of(r) : 0) * D;
+#pragma unroll
+            for (int v = 0; v < VPL; ++v)
+                buf[u][v] = r < nrows ? ldg16(rp + (sub + LPG * v) * EV) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float acc[GP];
+#pragma unroll
+            for (int g = 0; g < GP; ++g) acc[g] = 0.f;
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                float x[EV];
+                Vec16<T>::unpack(buf[u][v], x);
+#pragma unroll
+                for (int e = 0; e < EV; ++e)
+#pragma unroll
+                    for (int g = 0; g < GP; ++g) acc[g] = fmaf(sreg[g][v * EV + e], x[e], acc[g]);
+            }
+#pragma unroll
+            for (int g = 0; g < GP; ++g) {
+                acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 4);
+                acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 2);
+                acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 1);
+            }
+            float val = acc[0];
+#pragma unroll
+            for (int g = 1; g < GP; ++g)
+                if (g == sub) val = acc[g];
+            const int r = base_r + u * ngrp + grp;
+            if (sub < GP && r < nrows) store(sub, r, val);
+        }
+    }
+}
+
+// Root level (a1 + a2 scores): one CTA per GP heads of a (query, KV head).
+template <typename T, int D, int GP>
+__global__ void __launch_bounds__(kScoreThreads) root_kernel(const DescendParams p)
+{
+    constexpr int EV = Vec16<T>::E;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    double *part = reinterpret_cast<double *>(smem_raw);            // [256 * 2 * EV]
+    double *s64 = part + kScoreThreads * 2 * EV;                     // [GP * D]
+    double *a64 = s64 + GP * D;                                       // [GP * D]
+    __shared__ float s[GP * D];
+    __shared__ double anorm[GP];
+    if (blockIdx.x == 0 && threadIdx.x < 3) p.qcount[threadIdx.x] = 0;
+    const int chunks = p.G / GP;
+    const int cid = blockIdx.x % chunks;
+    const int grp_id = blockIdx.x / chunks;   // b * H_kv + hkv
+    const int b = grp_id / p.H_kv, hkv = grp_id % p.H_kv;
+    const int h0 = hkv * p.G + cid * GP;
+    const long long bh0 = (long long)b * p.H + h0;
+    const T *qb = reinterpret_cast<const T *>(p.q_kg) + ((size_t)b * p.N * p.H + h0) * D;
+    token_sums<T, D, GP>(qb, (size_t)p.H * D, p.N, s, s64, a64, part, anorm);
+    for (int i = threadIdx.x; i < GP * D; i += blockDim.x) {
+        p.s_ws[(size_t)bh0 * D + i] = s[i];
+        p.s64_ws[(size_t)bh0 * D + i] = s64[i];
+        p.a64_ws[(size_t)bh0 * D + i] = a64[i];
+    }
+    if (threadIdx.x < GP) p.anorm_ws[bh0 + threadIdx.x] = (float)anorm[threadIdx.x] * (1.0f + 1e-6f);
+    const T *kbase = reinterpret_cast<const T *>(p.keys[0]);
+    const long long base_row = (long long)hkv * p.rows[0];
+    float *f = p.f_ws;
+    const int fstride = p.fstride;
+    score_rows<T, D, GP>(
+        kbase, s, p.fanout[0], [&](int r) -> long long { return base_row + r; },
+        [&](int g, int r, float v) { f[(size_t)(bh0 + g) * fstride + r] = v; });
+    (void)EV;
+}
+
+// Dynamic shared memory of score_kernel for GP heads with Kp parents each.
+template <int GP>
+__host__ __device__ constexpr size_t score_kernel_smem(int Kp)
+{
+    return (size_t)4 * GP * Kp * 4 + (size_t)GP * GP * Kp * 2;
+}
+
+// Children of the kept parents (levels 1 and 2).  Grid: (query, KV head, GP-head
+// chunk, parent chunk).  The CTA forms the union of its GP heads' kept parent
+// lists (each ascending) in first-appearance order and scores the children of
+// parents [pc * ppc, (pc + 1) * ppc) of that union (and of every pchunks-th
+// chunk after it).
+template <typename T, int D, int GP>
+__global__ void __launch_bounds__(kScoreThreads) score_kernel(const DescendParams p, int L, int ppc, int pchunks)
+{
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ float s[GP * D];
+    __shared__ int seg[kScoreThreads];
+    __shared__ int nP_sh;
+    const int Kp = p.K[L - 1];
+    const int fo = p.fanout[L];
+    const int total = GP * Kp;
+    int32_t *lists = reinterpret_cast<int32_t *>(smem_raw);          // [GP][Kp] kept parents
+    int32_t *first = lists + total;                                   // [total] index of the first occurrence
+    int32_t *P = first + total;                                       // [total] union
+    int32_t *firstpos = P + total;                                    // [total]
+    int16_t *pidx = reinterpret_cast<int16_t *>(firstpos + total);    // [GP][total]
+
+    const int pc = blockIdx.x % pchunks;
+    const int rest = blockIdx.x / pchunks;
+    const int chunks = p.G / GP;
+    const int cid = rest % chunks;
+    const int grp_id = rest / chunks;
+    const int b = grp_id / p.H_kv, hkv = grp_id % p.H_kv;
+    const long long bh0 = (long long)b * p.H + (long long)hkv * p.G + (long long)cid * GP;
+
+    for (int i = threadIdx.x; i < GP * D; i += blockDim.x) s[i] = p.s_ws[(size_t)bh0 * D + i];
+    for (int t = threadIdx.x; t < total; t += blockDim.x) {
+        const int g = t / Kp, k = t - g * Kp;
+        lists[t] = p.kept[L - 1][(bh0 + g) * Kp + k];
+    }
+    for (int i = threadIdx.x; i < GP * total; i += blockDim.x) pidx[i] = -1;
+    __syncthreads();
+    // first occurrence of each element (binary search in the earlier heads' lists)
+    for (int t = threadIdx.x; t < total; t += blockDim.x) {
+        const int g = t / Kp;
+        const int x = lists[t];
+        int ft = t;
+        for (int g2 = 0; g2 < g && ft == t; ++g2) {
+            const int32_t *lst = lists + g2 * Kp;
+            int lo = 0, hi = Kp;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (lst[mid] < x) lo = mid + 1;
+                else hi = mid;
+            }
+            if (lo < Kp && lst[lo] == x) ft = g2 * Kp + lo;
+        }
+        first[t] = ft;
+    }
+    __syncthreads();
+    // exclusive scan of "is a first occurrence"
+    const int per = (total + blockDim.x - 1) / blockDim.x;
+    const int t0 = threadIdx.x * per, t1 = min(total, t0 + per);
+    int cnt = 0;
+    for (int t = t0; t < t1; ++t) cnt += (first[t] == t);
+    seg[threadIdx.x] = cnt;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        int run = 0;
+        for (int base = 0; base < (int)blockDim.x; base += 32) {
+            const int v = seg[base + threadIdx.x];
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int w = __shfl_up_sync(0xffffffffu, incl, o);
+                if ((int)threadIdx.x >= o) incl += w;
+            }
+            seg[base + threadIdx.x] = run + incl - v;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (threadIdx.x == 0) nP_sh = run;
+    }
+    __syncthreads();
+    {
+        int run = seg[threadIdx.x];
+        for (int t = t0; t < t1; ++t)
+            if (first[t] == t) {
+                firstpos[t] = run;
+                P[run] = lists[t];
+                ++run;
+            }
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < total; t += blockDim.x) {
+        const int g = t / Kp, k = t - g * Kp;
+        pidx[g * total + firstpos[first[t]]] = (int16_t)k;
+    }
+    __syncthreads();
+    const int nP = nP_sh;
+    const T *kbase = reinterpret_cast<const T *>(p.keys[L]);
+    const int32_t *tab = p.child[L - 1];
+    const long long prow = p.rows[L - 1], rows = p.rows[L];
+    const int32_t *slot = (L == 2) ? p.leaf_slot : nullptr;
+    float *f = p.f_ws;
+    const int fstride = p.fstride;
+    int *status = p.status;
+    // parent chunks pc, pc + pchunks, ...: pchunks covers the usual union (the
+    // heads of a group mostly agree); larger unions loop
+    for (int i0 = pc * ppc; i0 < nP; i0 += pchunks * ppc) {
+    const int i1 = min(nP, i0 + ppc);
+    score_rows<T, D, GP>(
+        kbase, s, (i1 - i0) * fo,
+        [&](int r) -> long long {
+            const int i = i0 + r / fo, j = r % fo;
+            if (slot) {
+                // the pool slot of parent P[i]: take it from the first head listing it
+                for (int g = 0; g < GP; ++g) {
+                    const int k = pidx[g * total + i];
+                    if (k >= 0) return (long long)slot[(bh0 + g) * Kp + k] * fo + j;
+                }
+                return 0;
+            }
+            const long long par = P[i];
+            long long id = tab ? (long long)tab[((size_t)hkv * prow + par) * fo + j] : par * fo + j;
+            if (id < 0 || id >= rows) {
+                set_status(status, kDevBadChild);
+                id = 0;
+            }
+            return (long long)hkv * rows + id;
+        },
+        [&](int g, int r, float v) {
+            const int i = i0 + r / fo, j = r % fo;
+            const int k = pidx[g * total + i];
+            if (k >= 0) f[(size_t)(bh0 + g) * fstride + (size_t)k * fo + j] = v;
+        });
+    }
+}
+
+// ==========================================================================
+// Selection side (warp-level)
+// ==========================================================================
+
+// Ascending warp bitonic sort of n (power of two) uint64 in shared memory.
+__device__ void warp_sort_u64(uint64_t *a, int n)
+{
+    const int lane = threadIdx.x & 31;
     for (int size = 2; size <= n; size <<= 1) {
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            __syncthreads();
-            for (int i = threadIdx.x; i < n / 2; i += blockDim.x) {
+            __syncwarp();
+            for (int i = lane; i < n / 2; i += 32) {
                 const int lo = 2 * i - (i & (stride - 1));
                 const int hi = lo + stride;
                 const bool asc = (lo & size) == 0;
@@ -125,374 +424,586 @@ __device__ void block_sort_u64(uint64_t *a, int n)
             }
         }
     }
-    __syncthreads();
+    __syncwarp();
 }
 
-// --------------------------------------------------------------------------
-// fp32 filter scores f[c] = sum_d s[d] * key[cand_row[c]][d].  Eight lanes per
-// candidate, each holding the token sums of its slice of d; every 16-byte
-// vector read is part of a 128-byte coalesced row segment.
-template <typename T, int D>
-__device__ void score_candidates(const T *__restrict__ base, const int32_t *cand_row, int C,
-                                 const float *s, float *f)
+// k-th largest (1-based) of n floats f[0..n), warp-level.  Values are
+// bucketed linearly between their min and max (a monotone map); the bucket
+// holding the k-th largest is then searched exactly: sorted when small, else
+// narrowed by MSB-first radix passes over the order-preserving bit image.
+// hist: this warp's 256 bins; tmp: 64 scratch uint64.
+__device__ float warp_kth_largest(const float *f, int n, int k, uint32_t *hist, uint64_t *tmp)
 {
-    constexpr int EV = Vec16<T>::E;
-    constexpr int VPR = D / EV;
-    constexpr int LPG = 8;
-    constexpr int VPL = VPR / LPG;
-    constexpr int U = 4;
-    static_assert(VPL >= 1 && VPR % LPG == 0, "row must split over 8 lanes");
-    const int sub = threadIdx.x & 7;
-    const int grp = threadIdx.x >> 3;
-    const int ngrp = blockDim.x >> 3;
-    float sreg[VPL * EV];
+    const int lane = threadIdx.x & 31;
+    float mn = INFINITY, mx = -INFINITY;
+    for (int i = lane; i < n; i += 32) {
+        mn = fminf(mn, f[i]);
+        mx = fmaxf(mx, f[i]);
+    }
 #pragma unroll
-    for (int v = 0; v < VPL; ++v)
+    for (int o = 16; o > 0; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (!(mx > mn) || !isfinite(mx - mn)) {
+        if (mx == mn) return mx;   // all equal
+    } else {
+        const float scale = 255.99f / (mx - mn);
+        auto bucket = [&](float v) { return min(255, max(0, (int)((v - mn) * scale))); };
 #pragma unroll
-        for (int e = 0; e < EV; ++e) sreg[v * EV + e] = s[(sub + LPG * v) * EV + e];
-
-    for (int base_c = 0; base_c < C; base_c += ngrp * U) {
-        uint4 buf[U][VPL];
+        for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
+        __syncwarp();
+        for (int i = lane; i < n; i += 32) atomicAdd(&hist[bucket(f[i])], 1u);
+        __syncwarp();
+        uint32_t cnt[8], tot = 0;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int c = base_c + u * ngrp + grp;
-            const bool ok = c < C;
-            const T *row = base + (size_t)(ok ? cand_row[c] : 0) * D;
-#pragma unroll
-            for (int v = 0; v < VPL; ++v)
-                buf[u][v] = ok ? ldg16(row + (sub + LPG * v) * EV) : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < 8; ++j) {
+            cnt[j] = hist[255 - 8 * lane - j];
+            tot += cnt[j];
         }
+        uint32_t incl = tot;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            float acc = 0.f;
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const uint32_t excl = incl - tot;
+        int bk = 0, rem = 0, bcount = 0;
+        const bool mine = excl < (uint32_t)k && (uint32_t)k <= incl;
+        if (mine) {
+            uint32_t run = excl;
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) {
-                float x[EV];
-                Vec16<T>::unpack(buf[u][v], x);
-#pragma unroll
-                for (int e = 0; e < EV; ++e) acc = fmaf(sreg[v * EV + e], x[e], acc);
+            for (int j = 0; j < 8; ++j) {
+                if (run + cnt[j] >= (uint32_t)k) {
+                    bk = 255 - 8 * lane - j;
+                    rem = k - (int)run;
+                    bcount = (int)cnt[j];
+                    break;
+                }
+                run += cnt[j];
             }
-            acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            const int c = base_c + u * ngrp + grp;
-            if (sub == 0 && c < C) f[c] = acc;
+        }
+        const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+        bk = __shfl_sync(0xffffffffu, bk, src);
+        rem = __shfl_sync(0xffffffffu, rem, src);
+        bcount = __shfl_sync(0xffffffffu, bcount, src);
+        __syncwarp();
+        if (bcount <= 64) {
+            // collect the bucket, sort it descending by value, take the rem-th
+            int m = 0;
+            for (int i0 = 0; i0 < n; i0 += 32) {
+                const int i = i0 + lane;
+                const bool in = i < n && bucket(f[i]) == bk;
+                const unsigned msk = __ballot_sync(0xffffffffu, in);
+                if (in) tmp[m + __popc(msk & lanemask_lt())] = ~(uint64_t)float_key(f[i]);
+                m += __popc(msk);
+            }
+            for (int i = m + lane; i < 64; i += 32) tmp[i] = ~0ull;
+            warp_sort_u64(tmp, 64);
+            const float t = key_float((uint32_t)~tmp[rem - 1]);
+            __syncwarp();
+            return t;
         }
     }
+    // general case: radix select on the bit image
+    uint32_t prefix = 0, mask = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
+        __syncwarp();
+        for (int i = lane; i < n; i += 32) {
+            const uint32_t key = float_key(f[i]);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        }
+        __syncwarp();
+        uint32_t cnt[8], tot = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            cnt[j] = hist[255 - 8 * lane - j];
+            tot += cnt[j];
+        }
+        uint32_t incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const uint32_t excl = incl - tot;
+        int digit = 0, rem = 0;
+        const bool mine = excl < (uint32_t)k && (uint32_t)k <= incl;
+        if (mine) {
+            uint32_t run = excl;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (run + cnt[j] >= (uint32_t)k) {
+                    digit = 255 - 8 * lane - j;
+                    rem = k - (int)run;
+                    break;
+                }
+                run += cnt[j];
+            }
+        }
+        const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+        digit = __shfl_sync(0xffffffffu, digit, src);
+        k = __shfl_sync(0xffffffffu, rem, src);
+        prefix |= ((uint32_t)digit) << shift;
+        mask |= 255u << shift;
+        __syncwarp();
+    }
+    return key_float(prefix);
 }
 
-// --------------------------------------------------------------------------
-// Shared-memory layout of one descent CTA.
-template <int D>
-struct DescendSmem {
-    float *s;          // [D] fp32 token sums
-    float *absq;       // [D] fp32 sums of |q|
-    int32_t *cand_id;  // [cap]
-    int32_t *cand_row; // [cap]
-    float *cand_f;     // [cap]   } contiguous: reused as the uint64 sort buffer
-    int32_t *alist;    // [cap]   }
-    int32_t *kept_pos; // [kcap]
-    int32_t *kept_id;  // [kcap]  parents of the next level
-    uint32_t *hist;    // [256]
-    int *misc;         // [16]
-    double *dmisc;     // [8]
-    // refinement
-    uint32_t *ex;      // [3 * kRefineChunk][kScoreDigits]
-    int32_t *ex_id;    // [3 * kRefineChunk]
-    int32_t *ex_pos;   // [3 * kRefineChunk]
-    int32_t *ex_rank;  // [4 * kRefineChunk] ranks + validity flags
-    uint32_t *smag;    // [kSumDigits * D]
-    uint8_t *sneg;     // [D]
-    int8_t *slo, *shi; // [D]
+// One traversal's candidates at one level: candidate c = (k, j) is child j of
+// its k-th kept parent; at the root level c is the root itself.
+struct LevelView {
+    int L, C, fo;
+    const int32_t *prev;      // kept parents (ascending ids), null at the root level
+    const int32_t *tab;       // child table of the parent level, or null
+    long long prow, rows;     // rows per KV head of the parent level / this level
+    int hkv;
+    const int32_t *slot;      // host pool slots of the kept parents (leaf level, host path), or null
 
-    __device__ DescendSmem(uint8_t *p, int cap, int kcap)
+    __device__ __forceinline__ int id(int c) const
     {
-        auto take = [&](size_t bytes) {
-            uint8_t *r = p;
-            p += (bytes + 15) & ~size_t(15);
-            return r;
-        };
-        dmisc = (double *)take(8 * sizeof(double));
-        s = (float *)take(D * sizeof(float));
-        absq = (float *)take(D * sizeof(float));
-        cand_id = (int32_t *)take(cap * 4);
-        cand_row = (int32_t *)take(cap * 4);
-        cand_f = (float *)take(cap * 4);
-        alist = (int32_t *)take(cap * 4);
-        kept_pos = (int32_t *)take(kcap * 4);
-        kept_id = (int32_t *)take(kcap * 4);
-        hist = (uint32_t *)take(256 * 4);
-        misc = (int *)take(16 * 4);
-        ex = (uint32_t *)take(3 * kRefineChunk * kScoreDigits * 4);
-        ex_id = (int32_t *)take(3 * kRefineChunk * 4);
-        ex_pos = (int32_t *)take(3 * kRefineChunk * 4);
-        ex_rank = (int32_t *)take(4 * kRefineChunk * 4);
-        smag = (uint32_t *)take(kSumDigits * D * 4);
-        sneg = (uint8_t *)take(D);
-        slo = (int8_t *)take(D);
-        shi = (int8_t *)take(D);
+        if (L == 0) return c;
+        const int k = c / fo, j = c - k * fo;
+        const long long par = prev[k];
+        long long v = tab ? (long long)tab[((size_t)hkv * prow + par) * fo + j] : par * fo + j;
+        return (v < 0 || v >= rows) ? 0 : (int)v;
     }
-
-    static size_t bytes(int cap, int kcap)
+    __device__ __forceinline__ long long row(int c) const
     {
-        auto r = [](size_t b) { return (b + 15) & ~size_t(15); };
-        return r(64) + 2 * r(D * 4) + 4 * r((size_t)cap * 4) + 2 * r((size_t)kcap * 4) + r(1024) + r(64) +
-               r(3 * kRefineChunk * kScoreDigits * 4) + 2 * r(3 * kRefineChunk * 4) + r(4 * kRefineChunk * 4) +
-               r(kSumDigits * D * 4) + 3 * r(D);
+        if (L == 0) return (long long)hkv * rows + c;
+        if (slot) {
+            const int k = c / fo, j = c - k * fo;
+            return (long long)slot[k] * fo + j;
+        }
+        return (long long)hkv * rows + id(c);
     }
 };
 
-// Pick the r best of the ambiguous candidates alist[0..nA) by (exact score
-// desc, row id asc) and append their positions to kept_pos[base_out..).
-// The ambiguous set is processed in chunks with a bounded best-set; passes
-// repeat (each excluding what earlier passes chose, i.e. everything not
-// strictly worse than the last chosen "pivot") until r are chosen.
-template <typename T, int D>
-__device__ void refine_exact(DescendSmem<D> &sm, const T *qbase, size_t q_stride, int N,
-                             const T *__restrict__ kbase, int nA, int r, int base_out)
+template <typename T>
+__device__ LevelView level_view(const DescendParams &p, int L, long long bh, const int32_t *prev)
 {
-    constexpr int RC = kRefineChunk;
-    static_assert(kDescendThreads >= 2 * RC, "one pool element per thread");
-    const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    exact_token_sums<T, D>(qbase, q_stride, N, nullptr, sm.smag, sm.sneg, sm.slo, sm.shi);
-    __syncthreads();
-
-    uint32_t *BEST = sm.ex;                        // [RC]
-    uint32_t *CH = sm.ex + RC * kScoreDigits;      // [RC]
-    uint32_t *TMP = sm.ex + 2 * RC * kScoreDigits; // [RC]
-    int32_t *best_id = sm.ex_id, *ch_id = sm.ex_id + RC, *tmp_id = sm.ex_id + 2 * RC;
-    int32_t *best_pos = sm.ex_pos, *ch_pos = sm.ex_pos + RC, *tmp_pos = sm.ex_pos + 2 * RC;
-    int32_t *valid = sm.ex_rank + 2 * RC;          // [2 RC]
-    int32_t *rank = sm.ex_rank;                    // [2 RC]
-
-    int chosen = 0;
-    bool have_pivot = false;
-    uint32_t pivot[kScoreDigits];
-    int pivot_id = 0;
-    while (chosen < r) {
-        const int want = min(r - chosen, RC);
-        int nbest = 0;
-        for (int b0 = 0; b0 < nA; b0 += RC) {
-            const int len = min(RC, nA - b0);
-            for (int i = warp; i < len; i += nwarps) {
-                const int pos = sm.alist[b0 + i];
-                exact_row_score<T, D>(kbase + (size_t)sm.cand_row[pos] * D, sm.smag, sm.sneg, sm.slo, sm.shi,
-                                      CH + i * kScoreDigits);
-                if ((threadIdx.x & 31) == 0) {
-                    ch_id[i] = sm.cand_id[pos];
-                    ch_pos[i] = pos;
-                }
-            }
-            __syncthreads();
-            // pool = BEST[0..nbest) + chunk members strictly worse than the pivot
-            const int npool = nbest + len;
-            const int e = threadIdx.x;
-            const uint32_t *xe = nullptr;
-            int ide = 0;
-            if (e < npool) {
-                xe = e < nbest ? BEST + e * kScoreDigits : CH + (e - nbest) * kScoreDigits;
-                ide = e < nbest ? best_id[e] : ch_id[e - nbest];
-                valid[e] = (e < nbest || !have_pivot || exact_better(pivot, pivot_id, xe, ide)) ? 1 : 0;
-            }
-            __syncthreads();
-            int my_rank = 0x7fffffff;
-            if (e < npool && valid[e]) {
-                my_rank = 0;
-                for (int f2 = 0; f2 < npool; ++f2) {
-                    if (f2 == e || !valid[f2]) continue;
-                    const uint32_t *xf = f2 < nbest ? BEST + f2 * kScoreDigits : CH + (f2 - nbest) * kScoreDigits;
-                    const int idf = f2 < nbest ? best_id[f2] : ch_id[f2 - nbest];
-                    if (exact_better(xf, idf, xe, ide)) ++my_rank;
-                }
-            }
-            const int total_valid = __syncthreads_count(e < npool && valid[e]);
-            if (my_rank < want) {
-#pragma unroll
-                for (int q = 0; q < kScoreDigits; ++q) TMP[my_rank * kScoreDigits + q] = xe[q];
-                tmp_id[my_rank] = ide;
-                tmp_pos[my_rank] = e < nbest ? best_pos[e] : ch_pos[e - nbest];
-            }
-            __syncthreads();
-            nbest = min(want, total_valid);
-            for (int i = threadIdx.x; i < nbest; i += blockDim.x) {
-#pragma unroll
-                for (int q = 0; q < kScoreDigits; ++q) BEST[i * kScoreDigits + q] = TMP[i * kScoreDigits + q];
-                best_id[i] = tmp_id[i];
-                best_pos[i] = tmp_pos[i];
-            }
-            __syncthreads();
-        }
-        for (int i = threadIdx.x; i < nbest; i += blockDim.x) sm.kept_pos[base_out + chosen + i] = best_pos[i];
-        if (nbest == 0) break;  // only if r > nA, which the caller rules out
-        chosen += nbest;
-#pragma unroll
-        for (int q = 0; q < kScoreDigits; ++q) pivot[q] = BEST[(nbest - 1) * kScoreDigits + q];
-        pivot_id = best_id[nbest - 1];
-        have_pivot = true;
-        __syncthreads();
-    }
-    (void)rank;
+    const int h = (int)(bh % p.H);
+    const int Kp = L == 0 ? 0 : p.K[L - 1];
+    LevelView lv;
+    lv.L = L;
+    lv.fo = L == 0 ? 1 : p.fanout[L];
+    lv.C = L == 0 ? p.fanout[0] : Kp * lv.fo;
+    lv.tab = L == 0 ? nullptr : p.child[L - 1];
+    lv.prow = L == 0 ? 0 : p.rows[L - 1];
+    lv.rows = p.rows[L];
+    lv.hkv = h / p.G;
+    lv.slot = (L == 2 && p.leaf_slot) ? p.leaf_slot + bh * Kp : nullptr;
+    lv.prev = prev;
+    return lv;
 }
 
-// Select the K best candidates of cand_*[0..C) and leave their positions,
-// sorted by ascending row id, in kept_pos[0..K); ids in kept_id.
-template <typename T, int D>
-__device__ void select_level(DescendSmem<D> &sm, int C, int K, double E, const T *qbase, size_t q_stride,
-                             int N, const T *__restrict__ kbase, int cap)
-{
-    if (K >= C) {
-        for (int c = threadIdx.x; c < C; c += blockDim.x) sm.kept_pos[c] = c;
-        __syncthreads();
-    } else {
-        const float *f = sm.cand_f;
-        const uint32_t tkey = block_kth_largest(C, K, [&](int i) { return float_key(f[i]); }, sm.hist, sm.misc);
-        const double t = (double)key_float(tkey);
-        // any non-finite filter score or bound: every candidate is ambiguous
-        int bad = 0;
-        for (int c = threadIdx.x; c < C; c += blockDim.x) bad |= !isfinite(f[c]);
-        bad = __syncthreads_or(bad) || !isfinite(E) || !isfinite(t);
-        const double two_e = 2.0 * E;
-        const double hi = bad ? INFINITY : __dadd_ru(t, two_e);
-        const double lo = bad ? -INFINITY : __dsub_rd(t, two_e);
-        if (threadIdx.x == 0) {
-            sm.misc[2] = 0;
-            sm.misc[3] = 0;
-        }
-        __syncthreads();
-        for (int c = threadIdx.x; c < C; c += blockDim.x) {
-            const double fd = (double)f[c];
-            if (!bad && fd > hi) {
-                sm.kept_pos[atomicAdd(&sm.misc[2], 1)] = c;
-            } else if (bad || fd >= lo) {
-                sm.alist[atomicAdd(&sm.misc[3], 1)] = c;
-            }
-        }
-        __syncthreads();
-        const int n_in = sm.misc[2], nA = sm.misc[3];
-        const int r = K - n_in;
-        __syncthreads();
-        if (nA == r) {
-            for (int i = threadIdx.x; i < nA; i += blockDim.x) sm.kept_pos[n_in + i] = sm.alist[i];
-            __syncthreads();
-        } else {
-            refine_exact<T, D>(sm, qbase, q_stride, N, kbase, nA, r, n_in);
-            __syncthreads();
-        }
+// Per-warp shared scratch of the selection.
+struct SelectScratch {
+    float *f;          // [cap] scores
+    int32_t *prev;     // [kcap] kept parents of the traversal
+    uint32_t *hist;    // [256]
+    uint64_t *sortb;   // [kcap] (id << 32 | position)
+    uint64_t *tmp;     // [64]
+    double *s64;       // [D]
+    double *a64;       // [D]
+
+    __host__ __device__ static size_t bytes(int cap, int kcap, int D)
+    {
+        auto r = [](size_t b) { return (b + 15) & ~size_t(15); };
+        return r((size_t)cap * 4) + r((size_t)kcap * 4) + r(1024) + r((size_t)kcap * 8) + r(512) +
+               2 * r((size_t)D * 8);
     }
-    // sort kept positions by row id: pack (id, pos) into uint64 in the cand_f/alist area
+    __device__ SelectScratch(uint8_t *p, int cap, int kcap, int D)
+    {
+        auto take = [&](size_t b) {
+            uint8_t *q = p;
+            p += (b + 15) & ~size_t(15);
+            return q;
+        };
+        f = (float *)take((size_t)cap * 4);
+        prev = (int32_t *)take((size_t)kcap * 4);
+        hist = (uint32_t *)take(1024);
+        sortb = (uint64_t *)take((size_t)kcap * 8);
+        tmp = (uint64_t *)take(512);
+        s64 = (double *)take((size_t)D * 8);
+        a64 = (double *)take((size_t)D * 8);
+    }
+};
+
+// Write the final kept list of a traversal from sortb[0..K) (ascending after sorting).
+__device__ void write_kept(const DescendParams &p, const LevelView &lv, int L, long long bh, uint64_t *sortb, int K)
+{
+    const int lane = threadIdx.x & 31;
     int n2 = 1;
     while (n2 < K) n2 <<= 1;
-    uint64_t *buf = reinterpret_cast<uint64_t *>(sm.cand_f);
-    for (int i = threadIdx.x; i < n2; i += blockDim.x)
-        buf[i] = i < K ? (((uint64_t)(uint32_t)sm.cand_id[sm.kept_pos[i]]) << 32) | (uint32_t)sm.kept_pos[i]
-                       : ~0ull;
-    block_sort_u64(buf, n2);
-    for (int i = threadIdx.x; i < K; i += blockDim.x) {
-        sm.kept_pos[i] = (int32_t)(uint32_t)(buf[i] & 0xffffffffull);
-        sm.kept_id[i] = (int32_t)(buf[i] >> 32);
-    }
-    __syncthreads();
-    (void)cap;
+    for (int i = K + lane; i < n2; i += 32) sortb[i] = ~0ull;
+    warp_sort_u64(sortb, n2);
+    for (int i = lane; i < K; i += 32) p.kept[L][bh * K + i] = (int32_t)(sortb[i] >> 32);
+    if (L == 2 && p.kept_leaf_row)
+        for (int i = lane; i < K; i += 32)
+            p.kept_leaf_row[bh * K + i] = (int32_t)lv.row((int)(sortb[i] & 0xffffffffu));
 }
 
+// One warp per traversal: top-K of level L's candidates.
+//   tier 1: fp32 scores with the rigorous bound E decide everything outside
+//           the band [t - 2E, t + 2E] around the K-th largest score t;
+//   tier 2: when at most 32 candidates are left in the band, each lane scores
+//           one of them in float64 from the float64 token sums, with its own
+//           rigorous bound  (g64_D (1 + g64_N) + g64_N) sum_d a64_d |k_d|,
+//           and the same band argument is repeated among them;
+//   tier 3: whatever is still undecided (true ties, or a band wider than a
+//           warp) is queued for exact_kernel.
 template <typename T, int D>
-__global__ void __launch_bounds__(kDescendThreads) descend_kernel(const DescendParams p)
+__global__ void __launch_bounds__(kSelectWarps * 32) select_kernel(const DescendParams p, int L)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    DescendSmem<D> sm(smem_raw, p.cap, p.kcap);
-    const int bh = blockIdx.x;
-    const int b = bh / p.H, h = bh % p.H;
-    const int hkv = h / p.G;
-    const T *qbase = reinterpret_cast<const T *>(p.q_kg) + ((size_t)b * p.N * p.H + h) * D;
-    const size_t q_stride = (size_t)p.H * D;
-
-    // ---- token sums (a1) ----
-    if (p.first_level == 0) {
-        for (int d = threadIdx.x; d < D; d += blockDim.x) {
-            float s = 0.f, a = 0.f;
-            const T *q = qbase + d;
-#pragma unroll 8
-            for (int n = 0; n < p.N; ++n) {
-                const float x = elem_f32(q[(size_t)n * q_stride]);
-                s += x;
-                a += fabsf(x);
-            }
-            sm.s[d] = s;
-            sm.absq[d] = a;
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            double acc = 0.0;
-            for (int d = threadIdx.x; d < D; d += 32) acc += (double)sm.absq[d] * (double)sm.absq[d];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (threadIdx.x == 0) {
-                const double an = sqrt(acc) * (1.0 + 1e-12) / (1.0 - gamma_n(p.N));
-                sm.dmisc[0] = an;
-            }
-        }
-        __syncthreads();
-        if (p.s_ws) {
-            for (int d = threadIdx.x; d < D; d += blockDim.x) p.s_ws[(size_t)bh * D + d] = sm.s[d];
-            if (threadIdx.x == 0) p.anorm_ws[bh] = (float)sm.dmisc[0] * (1.0f + 1e-6f);
-        }
-    } else {
-        for (int d = threadIdx.x; d < D; d += blockDim.x) sm.s[d] = p.s_ws[(size_t)bh * D + d];
-        if (threadIdx.x == 0) sm.dmisc[0] = (double)p.anorm_ws[bh];
-        const int prev = p.first_level - 1;
-        for (int i = threadIdx.x; i < p.K[prev]; i += blockDim.x)
-            sm.kept_id[i] = p.kept[prev][(size_t)bh * p.K[prev] + i];
-        __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long bh = (long long)blockIdx.x * kSelectWarps + warp;
+    if (bh >= (long long)p.B * p.H) return;
+    SelectScratch sc(smem_raw + (size_t)warp * SelectScratch::bytes(p.cap, p.kcap, D), p.cap, p.kcap, D);
+    const int Kp = L == 0 ? 0 : p.K[L - 1];
+    for (int k = lane; k < Kp; k += 32) sc.prev[k] = p.kept[L - 1][bh * Kp + k];
+    const LevelView lv = level_view<T>(p, L, bh, sc.prev);
+    const int C = lv.C, K = p.K[L];
+    float *fslot = p.f_ws + (size_t)bh * p.fstride;
+    for (int c = lane; c < C; c += 32) sc.f[c] = fslot[c];
+    __syncwarp();
+    if (p.stats && lane == 0) atomicAdd(p.stats + L * 4, 1ull);
+    const float *f = sc.f;
+    uint64_t *sortb = sc.sortb;
+    int nsel = 0;
+    auto emit = [&](bool pred, int c) {
+        const unsigned m = __ballot_sync(0xffffffffu, pred);
+        if (pred) sortb[nsel + __popc(m & lanemask_lt())] = ((uint64_t)(uint32_t)lv.id(c) << 32) | (uint32_t)c;
+        nsel += __popc(m);
+    };
+    if (K >= C) {
+        for (int c0 = 0; c0 < C; c0 += 32) emit(c0 + lane < C, c0 + lane);
+        write_kept(p, lv, L, bh, sortb, K);
+        return;
     }
-    const double anorm = sm.dmisc[0];
+    // ---- tier 1 ----
     const double cprime = gamma_n(D) * (1.0 + gamma_n(p.N)) + gamma_n(p.N);
-
-    for (int L = p.first_level; L <= p.last_level; ++L) {
-        const T *kbase = reinterpret_cast<const T *>(p.keys[L]);
-        int C;
-        if (L == 0) {
-            C = p.fanout[0];
-            for (int c = threadIdx.x; c < C; c += blockDim.x) {
-                sm.cand_id[c] = c;
-                sm.cand_row[c] = (int32_t)(hkv * p.rows[0] + c);
-            }
-        } else {
-            const int fo = p.fanout[L];
-            const int Kp = p.K[L - 1];
-            C = Kp * fo;
-            const long long prow = p.rows[L - 1];
-            const int32_t *tab = p.child[L - 1];
-            for (int c = threadIdx.x; c < C; c += blockDim.x) {
-                const int k = c / fo, j = c - k * fo;
-                const long long par = sm.kept_id[k];
-                long long id = tab ? (long long)tab[((size_t)hkv * prow + par) * fo + j] : par * fo + j;
-                if (id < 0 || id >= p.rows[L]) {
-                    set_status(p.status, kDevBadChild);
-                    id = 0;
+    const double E = cprime * (double)p.anorm_ws[bh] * (double)p.norm_bound[L * p.H_kv + lv.hkv] * (1.0 + 1e-6) +
+                     D * 0x1p-148;
+    const double t = (double)warp_kth_largest(f, C, K, sc.hist, sc.tmp);
+    bool bad = !isfinite(E) || !isfinite(t);
+    for (int c = lane; c < C && !bad; c += 32) bad = !isfinite(f[c]);
+    bad = __any_sync(0xffffffffu, bad);
+    const double hi = bad ? INFINITY : __dadd_ru(t, 2.0 * E);
+    const double lo = bad ? -INFINITY : __dsub_rd(t, 2.0 * E);
+    auto in_set = [&](int c) { return c < C && !bad && (double)f[c] > hi; };
+    auto amb = [&](int c) {
+        if (c >= C) return false;
+        const double fd = (double)f[c];
+        return bad || (fd >= lo && !(fd > hi));
+    };
+    int n_in = 0, nA = 0;
+    for (int c = lane; c < C; c += 32) {
+        n_in += in_set(c);
+        nA += amb(c);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        n_in += __shfl_xor_sync(0xffffffffu, n_in, o);
+        nA += __shfl_xor_sync(0xffffffffu, nA, o);
+    }
+    const int r = K - n_in;
+    for (int c0 = 0; c0 < C; c0 += 32) emit(in_set(c0 + lane), c0 + lane);
+    if (nA == r) {
+        for (int c0 = 0; c0 < C; c0 += 32) emit(amb(c0 + lane), c0 + lane);
+        write_kept(p, lv, L, bh, sortb, K);
+        return;
+    }
+    if (p.stats && lane == 0) {
+        atomicAdd(p.stats + L * 4 + 1, 1ull);
+        atomicAdd(p.stats + L * 4 + 2, (unsigned long long)nA);
+    }
+    // the ambiguous positions, in position order, one per lane (when nA <= 32)
+    int my_pos = -1, na = 0;
+    for (int c0 = 0; c0 < C && na <= 32; c0 += 32) {
+        const bool a = amb(c0 + lane);
+        const unsigned m = __ballot_sync(0xffffffffu, a);
+        const int at = na + __popc(m & lanemask_lt());
+        if (a && at < 32) my_pos = c0 + lane;
+        // lanes receive their position below
+        if (a && at < 32) sc.tmp[at] = (uint64_t)(c0 + lane);
+        na += __popc(m);
+    }
+    __syncwarp();
+    int nlist = nA;
+    int r_left = r;
+    bool listed_all = true;   // the exact pass gets every ambiguous candidate
+    if (!bad && nA <= 32) {
+        // ---- tier 2 ----
+        for (int d = lane; d < D; d += 32) {
+            sc.s64[d] = p.s64_ws[(size_t)bh * D + d];
+            sc.a64[d] = p.a64_ws[(size_t)bh * D + d];
+        }
+        __syncwarp();
+        my_pos = lane < nA ? (int)sc.tmp[lane] : -1;
+        double y = -INFINITY, e2 = 0.0;
+        if (my_pos >= 0) {
+            const T *krow = reinterpret_cast<const T *>(p.keys[L]) + (size_t)lv.row(my_pos) * D;
+            double acc = 0.0, mag = 0.0;
+            for (int d = 0; d < D; d += Vec16<T>::E) {
+                float x[Vec16<T>::E];
+                Vec16<T>::unpack(ldg16(krow + d), x);
+#pragma unroll
+                for (int e = 0; e < Vec16<T>::E; ++e) {
+                    acc = fma(sc.s64[d + e], (double)x[e], acc);
+                    mag = fma(sc.a64[d + e], fabs((double)x[e]), mag);
                 }
-                sm.cand_id[c] = (int32_t)id;
-                long long row;
-                if (L == 2 && p.leaf_slot)
-                    row = (long long)p.leaf_slot[(size_t)bh * Kp + k] * fo + j;
-                else
-                    row = hkv * p.rows[L] + id;
-                sm.cand_row[c] = (int32_t)row;
+            }
+            const double g64d = (double)D * 0x1p-53 / (1.0 - (double)D * 0x1p-53);
+            const double g64n = (double)p.N * 0x1p-53 / (1.0 - (double)p.N * 0x1p-53);
+            y = acc;
+            e2 = (g64d * (1.0 + g64n) + g64n) * mag * (1.0 + 1e-6) + 0x1p-1000;
+        }
+        double E2 = e2;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) E2 = fmax(E2, __shfl_xor_sync(0xffffffffu, E2, o));
+        // r-th largest y among the nA lanes
+        int rank = 0;
+        for (int j = 0; j < nA; ++j) {
+            const double yj = __shfl_sync(0xffffffffu, y, j);
+            rank += (yj > y) || (yj == y && j < lane);
+        }
+        const int tl = __ffs(__ballot_sync(0xffffffffu, my_pos >= 0 && rank == r - 1)) - 1;
+        const double t2 = __shfl_sync(0xffffffffu, y, tl);
+        const double hi2 = __dadd_ru(t2, 2.0 * E2), lo2 = __dsub_rd(t2, 2.0 * E2);
+        const bool in2 = my_pos >= 0 && y > hi2;
+        const bool amb2 = my_pos >= 0 && !in2 && y >= lo2;
+        const int n_in2 = __popc(__ballot_sync(0xffffffffu, in2));
+        const int nA2 = __popc(__ballot_sync(0xffffffffu, amb2));
+        emit(in2, my_pos);
+        if (nA2 == r - n_in2) {
+            emit(amb2, my_pos);
+            write_kept(p, lv, L, bh, sortb, K);
+            return;
+        }
+        // hand the still-ambiguous ones to the exact pass
+        const unsigned m2 = __ballot_sync(0xffffffffu, amb2);
+        int *list = reinterpret_cast<int *>(fslot);
+        if (amb2) list[__popc(m2 & lanemask_lt())] = my_pos;
+        nlist = nA2;
+        r_left = r - n_in2;
+        listed_all = false;
+    }
+    if (listed_all) {
+        int *list = reinterpret_cast<int *>(fslot);
+        int at = 0;
+        for (int c0 = 0; c0 < C; c0 += 32) {
+            const bool a = amb(c0 + lane);
+            const unsigned m = __ballot_sync(0xffffffffu, a);
+            if (a) list[at + __popc(m & lanemask_lt())] = c0 + lane;
+            at += __popc(m);
+        }
+    }
+    // decided entries (id << 32 | position) after the list, then the queue entry
+    uint64_t *decided = reinterpret_cast<uint64_t *>(fslot + p.cap);
+    for (int i = lane; i < nsel; i += 32) decided[i] = sortb[i];
+    if (lane == 0) {
+        const int qi = atomicAdd(p.qcount + L, 1);
+        int *e = p.queue + ((size_t)L * p.B * p.H + qi) * 3;
+        e[0] = (int)bh;
+        e[1] = nsel;
+        e[2] = nlist;
+    }
+    (void)r_left;
+}
+
+// Exact score of one key row: x = sum_n sum_d q[n][d] k[d] over the stored
+// numbers (binary32, or bfloat16 widened exactly: every value is m 2^e with an
+// integer m < 2^24 and e >= -149), accumulated without rounding in digits of
+// weight 2^(32 i - 298) (Kulisch's exact dot product), one warp, lanes over d.
+// Lane 0 writes the canonical digits to out.
+template <typename T, int D>
+__device__ void warp_exact_score(const T *q, size_t q_stride, int N, const T *krow, uint32_t *out)
+{
+    const int lane = threadIdx.x & 31;
+    int64_t acc[kScoreDigits];
+#pragma unroll
+    for (int i = 0; i < kScoreDigits; ++i) acc[i] = 0;
+    for (int d = lane; d < D; d += 32) {
+        uint32_t mk;
+        int ek;
+        const int sk = split_binary32(elem_bits(krow[d]), mk, ek);
+        if (mk == 0) continue;
+        for (int n = 0; n < N; ++n) {
+            uint32_t mq;
+            int eq;
+            const int sq = split_binary32(elem_bits(q[(size_t)n * q_stride + d]), mq, eq);
+            if (mq == 0) continue;
+            const uint64_t prod = (uint64_t)mq * (uint64_t)mk;   // < 2^48
+            const int pos = eq + ek + 298;                         // >= 0
+            const int di = pos >> 5, sh = pos & 31;
+            const uint64_t lo64 = prod << sh;
+            const uint64_t hi64 = sh ? (prod >> (64 - sh)) : 0ull;
+            const int64_t c0 = (int64_t)(lo64 & 0xffffffffull), c1 = (int64_t)(lo64 >> 32), c2 = (int64_t)hi64;
+            const bool minus = (sq != 0) != (sk != 0);
+#pragma unroll
+            for (int j = 0; j < kScoreDigits - 2; ++j) {
+                if (j == di) {
+                    acc[j] += minus ? -c0 : c0;
+                    acc[j + 1] += minus ? -c1 : c1;
+                    acc[j + 2] += minus ? -c2 : c2;
+                }
             }
         }
-        __syncthreads();
-        score_candidates<T, D>(kbase, sm.cand_row, C, sm.s, sm.cand_f);
-        __syncthreads();
-        const double E = cprime * anorm * (double)p.norm_bound[L * p.H_kv + hkv] * (1.0 + 1e-6) + D * 0x1p-148;
-        select_level<T, D>(sm, C, p.K[L], E, qbase, q_stride, p.N, kbase, p.cap);
+    }
+#pragma unroll
+    for (int i = 0; i < kScoreDigits; ++i) {
+        int64_t v = acc[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        acc[i] = v;
+    }
+    if (lane == 0) {
+        normalize_digits<kScoreDigits>(acc);
+#pragma unroll
+        for (int i = 0; i < kScoreDigits; ++i) out[i] = (uint32_t)acc[i];
+    }
+    __syncwarp();
+}
+
+struct ExactScratch {
+    int32_t *prev;     // [kcap]
+    uint64_t *sortb;   // [kcap]
+    uint32_t *ex;      // [3 RC][kScoreDigits]
+    int32_t *ids;      // [3 RC]
+    int32_t *poss;     // [3 RC]
+    __host__ __device__ static size_t bytes(int kcap)
+    {
+        auto r = [](size_t b) { return (b + 15) & ~size_t(15); };
+        return r((size_t)kcap * 4) + r((size_t)kcap * 8) + r(3 * kRefineChunk * kScoreDigits * 4) +
+               2 * r(3 * kRefineChunk * 4);
+    }
+    __device__ ExactScratch(uint8_t *p, int kcap)
+    {
+        auto take = [&](size_t b) {
+            uint8_t *q = p;
+            p += (b + 15) & ~size_t(15);
+            return q;
+        };
+        prev = (int32_t *)take((size_t)kcap * 4);
+        sortb = (uint64_t *)take((size_t)kcap * 8);
+        ex = (uint32_t *)take(3 * kRefineChunk * kScoreDigits * 4);
+        ids = (int32_t *)take(3 * kRefineChunk * 4);
+        poss = (int32_t *)take(3 * kRefineChunk * 4);
+    }
+};
+
+// Tier 3: traversals the fp32 and fp64 bounds could not settle.  For each
+// queued traversal, pick the remaining K - decided candidates of its list by
+// (exact score desc, row id asc): the list is scanned in chunks of RC with a
+// bounded best-set, and passes repeat (each excluding everything not strictly
+// worse than the last one chosen) until enough are chosen.
+template <typename T, int D>
+__global__ void __launch_bounds__(kSelectWarps * 32) exact_kernel(const DescendParams p, int L)
+{
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    constexpr int RC = kRefineChunk;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qn = p.qcount[L];
+    ExactScratch sc(smem_raw + (size_t)warp * ExactScratch::bytes(p.kcap), p.kcap);
+    uint32_t *BEST = sc.ex, *CH = sc.ex + RC * kScoreDigits, *TMP = sc.ex + 2 * RC * kScoreDigits;
+    int32_t *best_id = sc.ids, *ch_id = sc.ids + RC, *tmp_id = sc.ids + 2 * RC;
+    int32_t *best_pos = sc.poss, *ch_pos = sc.poss + RC, *tmp_pos = sc.poss + 2 * RC;
+    for (int qi = blockIdx.x * kSelectWarps + warp; qi < qn; qi += gridDim.x * kSelectWarps) {
+        const int *e = p.queue + ((size_t)L * p.B * p.H + qi) * 3;
+        const long long bh = e[0];
+        int nsel = e[1];
+        const int nlist = e[2];
         const int K = p.K[L];
-        if (p.kept[L])
-            for (int i = threadIdx.x; i < K; i += blockDim.x) p.kept[L][(size_t)bh * K + i] = sm.kept_id[i];
-        if (L == 2 && p.kept_leaf_row)
-            for (int i = threadIdx.x; i < K; i += blockDim.x)
-                p.kept_leaf_row[(size_t)bh * K + i] = sm.cand_row[sm.kept_pos[i]];
-        __syncthreads();
+        const int r = K - nsel;
+        const int Kp = L == 0 ? 0 : p.K[L - 1];
+        for (int k = lane; k < Kp; k += 32) sc.prev[k] = p.kept[L - 1][bh * Kp + k];
+        const float *fslot = p.f_ws + (size_t)bh * p.fstride;
+        const int *list = reinterpret_cast<const int *>(fslot);
+        const uint64_t *decided = reinterpret_cast<const uint64_t *>(fslot + p.cap);
+        for (int i = lane; i < nsel; i += 32) sc.sortb[i] = decided[i];
+        __syncwarp();
+        const LevelView lv = level_view<T>(p, L, bh, sc.prev);
+        const int b = (int)(bh / p.H), h = (int)(bh % p.H);
+        const T *qh = reinterpret_cast<const T *>(p.q_kg) + ((size_t)b * p.N * p.H + h) * D;
+        const size_t q_stride = (size_t)p.H * D;
+        const T *kbase = reinterpret_cast<const T *>(p.keys[L]);
+        int chosen = 0;
+        bool have_pivot = false;
+        uint32_t pivot[kScoreDigits];
+        int pivot_id = 0;
+        while (chosen < r) {
+            const int want = min(r - chosen, RC);
+            int nbest = 0;
+            for (int b0 = 0; b0 < nlist; b0 += RC) {
+                const int len = min(RC, nlist - b0);
+                for (int i = 0; i < len; ++i) {
+                    const int pos = list[b0 + i];
+                    warp_exact_score<T, D>(qh, q_stride, p.N, kbase + (size_t)lv.row(pos) * D, CH + i * kScoreDigits);
+                    if (lane == 0) {
+                        ch_id[i] = lv.id(pos);
+                        ch_pos[i] = pos;
+                    }
+                }
+                if (p.stats && lane == 0) atomicAdd(p.stats + L * 4 + 3, (unsigned long long)len);
+                __syncwarp();
+                // merge the chunk into BEST: pool element ep = lane
+                const int npool = nbest + len;
+                const int ep = lane;
+                const uint32_t *xe = ep < nbest ? BEST + ep * kScoreDigits : CH + (ep - nbest) * kScoreDigits;
+                const int ide = ep < nbest ? best_id[ep] : (ep < npool ? ch_id[ep - nbest] : 0);
+                const bool valid = ep < npool && (ep < nbest || !have_pivot || exact_better(pivot, pivot_id, xe, ide));
+                const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+                int rank = 0x7fffffff;
+                if (valid) {
+                    rank = 0;
+                    unsigned others = vmask & ~(1u << ep);
+                    while (others) {
+                        const int f2 = __ffs(others) - 1;
+                        others &= others - 1;
+                        const uint32_t *xf = f2 < nbest ? BEST + f2 * kScoreDigits : CH + (f2 - nbest) * kScoreDigits;
+                        const int idf = f2 < nbest ? best_id[f2] : ch_id[f2 - nbest];
+                        if (exact_better(xf, idf, xe, ide)) ++rank;
+                    }
+                }
+                if (rank < want) {
+#pragma unroll
+                    for (int q = 0; q < kScoreDigits; ++q) TMP[rank * kScoreDigits + q] = xe[q];
+                    tmp_id[rank] = ide;
+                    tmp_pos[rank] = ep < nbest ? best_pos[ep] : ch_pos[ep - nbest];
+                }
+                __syncwarp();
+                nbest = min(want, __popc(vmask));
+                for (int i = lane; i < nbest * kScoreDigits; i += 32) BEST[i] = TMP[i];
+                if (lane < nbest) {
+                    best_id[lane] = tmp_id[lane];
+                    best_pos[lane] = tmp_pos[lane];
+                }
+                __syncwarp();
+            }
+            if (nbest == 0) break;   // only if r exceeded the list, which cannot happen
+            if (lane < nbest)
+                sc.sortb[nsel + lane] = ((uint64_t)(uint32_t)best_id[lane] << 32) | (uint32_t)best_pos[lane];
+            nsel += nbest;
+            chosen += nbest;
+#pragma unroll
+            for (int q = 0; q < kScoreDigits; ++q) pivot[q] = BEST[(nbest - 1) * kScoreDigits + q];
+            pivot_id = best_id[nbest - 1];
+            have_pivot = true;
+            __syncwarp();
+        }
+        write_kept(p, lv, L, bh, sc.sortb, K);
+        __syncwarp();
     }
 }
+
+// ==========================================================================
+// Tree set-up kernels
+// ==========================================================================
 
 // Per-level, per-KV-head maximum of key row 2-norms (for the filter bound),
 // as float bits rounded up; grid.y = KV head, one warp per row.  atomicMax on

@@ -156,6 +156,13 @@ atlaskv_status atlaskv_sync_status(atlaskv_tree *tree, void *stream);
 atlaskv_status atlaskv_set_profiling(atlaskv_tree *tree, int32_t enable);
 atlaskv_status atlaskv_stage_times(atlaskv_tree *tree, float *ms, int32_t n);
 
+/* Descent counters of the most recent attend call made while profiling was
+ * on, per level l = 0 (roots), 1 (mids), 2 (leaves): counts[4 l + 0] traversals
+ * selected, [4 l + 1] selections the fp32 bound could not settle alone,
+ * [4 l + 2] ambiguous candidates in those, [4 l + 3] exact scores computed.
+ * Synchronises the device; n is the capacity of counts (at most 12 written). */
+atlaskv_status atlaskv_refine_stats(atlaskv_tree *tree, uint64_t *counts, int32_t n);
+
 /* Size in bytes of the static device scratch used by atlaskv_attend_static. */
 #define ATLASKV_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 
