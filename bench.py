@@ -37,7 +37,21 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fanout", default=None, help="override the tree fan-outs, e.g. 100,100,100 (smaller cases)")
+    ap.add_argument("--batch", type=int, default=None, help="override the number of queries B")
     return ap.parse_args()
+
+
+def workload_shape(args):
+    import dataclasses
+    from hierarchical_kv_pruning_b200 import synth
+    sh = synth.shape(args.config)
+    if args.fanout:
+        fo = tuple(int(x) for x in args.fanout.split(","))
+        sh = dataclasses.replace(sh, fanout=fo, name="%s@%s" % (sh.name, "x".join(map(str, fo))))
+    if args.batch:
+        sh = dataclasses.replace(sh, batch=args.batch, name="%s@B%d" % (sh.name, args.batch))
+    return sh
 
 
 def measured_peaks():
@@ -198,7 +212,7 @@ def run_ours(args):
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    sh = synth.shape(args.config)
+    sh = workload_shape(args)
     w = synth.make_workload(sh, "cuda", 1000 + args.config + 100 * rank)
     stream = torch.cuda.current_stream()
     tree = HikvpTree.from_workload(w)
@@ -347,7 +361,7 @@ def run_reference(args):
     import torch
 
     from hierarchical_kv_pruning_b200 import synth
-    sh = synth.shape(args.config)
+    sh = workload_shape(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     w = synth.make_workload(sh, dev, 1000 + args.config)
     per_step = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))

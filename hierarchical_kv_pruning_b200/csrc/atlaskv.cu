@@ -109,7 +109,7 @@ Layout plan(const atlaskv_tree *t, const atlaskv_params *p, int B, int N, int H,
     L.a64_ws = take(BH * D * 8);
     L.anorm_ws = take(BH * 4);
     L.f_ws = take(BH * (size_t)L.fstride * 4);
-    L.queue = take(3 * BH * 3 * 4);
+    L.queue = take(3 * BH * 4 * 4);
     L.qcount = take(4 * 4);
     for (int l = 0; l < 3; ++l) L.kept[l] = take(BH * (size_t)(l == 0 ? p->K_root : l == 1 ? p->K_mid : p->K_leaf) * 4);
     if (host) {
@@ -211,24 +211,41 @@ atlaskv_status launch_root(const akv::DescendParams &dp, cudaStream_t s)
     return ATLASKV_OK;
 }
 
-template <typename T, int D, int GP>
-atlaskv_status launch_score(const akv::DescendParams &dp, int L, cudaStream_t s)
+// Children scoring: one CTA per (query, KV head, chunk of GC <= 32 heads,
+// parent chunk); HPT heads per thread.
+template <typename T, int D, int HPT>
+atlaskv_status launch_score_hpt(const akv::DescendParams &dp, int L, int GC, cudaStream_t s)
 {
     const int Kp = dp.K[L - 1], fo = dp.fanout[L];
     const int ppc = std::max(1, 512 / fo);            // parents per chunk: about 512 rows
     const int pchunks = (Kp + ppc - 1) / ppc;         // covers a union of Kp parents; larger ones loop
-    const long long grid = (long long)dp.B * dp.H_kv * (dp.G / GP) * pchunks;
+    const long long grid = (long long)dp.B * dp.H_kv * (dp.G / GC) * pchunks;
     if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "scoring grid too large");
-    const size_t smem = akv::score_kernel_smem<GP>(Kp);
+    const size_t smem = akv::score_kernel_smem<T, D>(GC, Kp);
+    if (smem > 227 * 1024) return fail(ATLASKV_EUNSUPPORTED, "scoring needs %zu bytes of shared memory", smem);
     static size_t configured = 0;
     if (smem > 48 * 1024 && smem > configured) {
-        AKV_CUDA(cudaFuncSetAttribute(akv::score_kernel<T, D, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        AKV_CUDA(cudaFuncSetAttribute(akv::score_kernel<T, D, HPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem));
         configured = smem;
     }
-    akv::score_kernel<T, D, GP><<<(unsigned)grid, akv::kScoreThreads, smem, s>>>(dp, L, ppc, pchunks);
+    akv::score_kernel<T, D, HPT><<<(unsigned)grid, akv::kScoreThreads, smem, s>>>(dp, L, GC, ppc, pchunks);
     AKV_CUDA(cudaGetLastError());
     return ATLASKV_OK;
+}
+
+template <typename T, int D>
+atlaskv_status launch_score(const akv::DescendParams &dp, int L, cudaStream_t s)
+{
+    int GC = 1;
+    for (int c = std::min(dp.G, 32); c >= 1; --c)
+        if (dp.G % c == 0) {
+            GC = c;
+            break;
+        }
+    if (GC % 4 == 0) return launch_score_hpt<T, D, 4>(dp, L, GC, s);
+    if (GC % 2 == 0) return launch_score_hpt<T, D, 2>(dp, L, GC, s);
+    return launch_score_hpt<T, D, 1>(dp, L, GC, s);
 }
 
 template <typename T, int D>
@@ -248,7 +265,7 @@ atlaskv_status launch_select(const akv::DescendParams &dp, int L, cudaStream_t s
     akv::select_kernel<T, D><<<(unsigned)grid, akv::kSelectWarps * 32, smem, s>>>(dp, L);
     AKV_CUDA(cudaGetLastError());
     // tier 3 for whatever the bounds left undecided (usually nothing: the warps read an empty queue)
-    const size_t esmem = (size_t)akv::kSelectWarps * akv::ExactScratch::bytes(dp.kcap);
+    const size_t esmem = (size_t)akv::kSelectWarps * akv::ExactScratch::bytes(dp.kcap, D);
     static size_t econfigured = 0;
     if (esmem > 48 * 1024 && esmem > econfigured) {
         AKV_CUDA(cudaFuncSetAttribute(akv::exact_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -271,8 +288,7 @@ atlaskv_status descend_levels(const akv::DescendParams &dp, int first, int last,
         if (L == 0)
             st = gp == 4 ? launch_root<T, D, 4>(dp, s) : gp == 2 ? launch_root<T, D, 2>(dp, s) : launch_root<T, D, 1>(dp, s);
         else
-            st = gp == 4 ? launch_score<T, D, 4>(dp, L, s)
-                         : gp == 2 ? launch_score<T, D, 2>(dp, L, s) : launch_score<T, D, 1>(dp, L, s);
+            st = launch_score<T, D>(dp, L, s);
         if (st != ATLASKV_OK) return st;
         st = launch_select<T, D>(dp, L, s);
         if (st != ATLASKV_OK) return st;

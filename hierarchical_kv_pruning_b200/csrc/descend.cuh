@@ -57,7 +57,7 @@ struct DescendParams {
     int fstride;                 // floats per traversal in f_ws: cap + 2 kcap
     int cap;                     // per-traversal score capacity (>= every level's candidate count)
     int kcap;                    // kept capacity (power of two >= every K)
-    int *queue;                  // [3][B H][3] (traversal, decided, listed) left to the exact pass
+    int *queue;                  // [3][B H][4] (traversal, decided, listed, non-finite) left to the exact pass
     int *qcount;                 // [3] queue lengths (zeroed by the root kernel)
     // host-staged leaves: kept mid k of traversal bh has its leaf block at pool
     // slot leaf_slot[bh K_mid + k]; leaf candidate (k, j) is pool row slot * b_L + j.
@@ -262,50 +262,106 @@ __global__ void __launch_bounds__(kScoreThreads) root_kernel(const DescendParams
     (void)EV;
 }
 
-// Dynamic shared memory of score_kernel for GP heads with Kp parents each.
-template <int GP>
-__host__ __device__ constexpr size_t score_kernel_smem(int Kp)
+// --------------------------------------------------------------------------
+// Children of the kept parents (levels 1 and 2).
+//
+// Grid: (query b, KV head, head chunk of GC heads, parent chunk).  The CTA forms
+// the union of its GC heads' kept parent lists (each ascending) in
+// first-appearance order, then scores every child row of union parents
+// [pc ppc, (pc + 1) ppc) (and of every pchunks-th chunk after it) against all
+// GC token-sum vectors: each row crosses from L2/HBM once per CTA.  Rows are
+// staged in shared memory in tiles of kTileRows by cp.async (kStages deep);
+// thread (row stream, head group, d-slice) keeps HPT heads x D/8 token sums in
+// registers, and the eight d-slice partial sums meet through a 4-shuffle
+// reduce-scatter.  Head g's score of child j of union parent P[i] lands at its
+// own candidate slot k fo + j, k = position of P[i] in g's sorted list.
+constexpr int kTileRows = 64;
+constexpr int kStages = 3;
+
+template <typename T, int D>
+__host__ __device__ constexpr size_t score_kernel_smem(int GC, int Kp)
 {
-    return (size_t)4 * GP * Kp * 4 + (size_t)GP * GP * Kp * 2;
+    return (size_t)kStages * kTileRows * D * sizeof(T) + (size_t)2 * kStages * kTileRows * 4 + (size_t)4 * GC * Kp * 4;
 }
 
-// Children of the kept parents (levels 1 and 2).  Grid: (query, KV head, GP-head
-// chunk, parent chunk).  The CTA forms the union of its GP heads' kept parent
-// lists (each ascending) in first-appearance order and scores the children of
-// parents [pc * ppc, (pc + 1) * ppc) of that union (and of every pchunks-th
-// chunk after it).
-template <typename T, int D, int GP>
-__global__ void __launch_bounds__(kScoreThreads) score_kernel(const DescendParams p, int L, int ppc, int pchunks)
+__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, bool valid)
 {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    const int sz = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "r"(sz));
+}
+
+// Reduce HPT per-lane partial sums over the 8 lanes of a d-slice group; lane
+// ds ends with the total of head (ds / (8 / HPT)).
+template <int HPT>
+__device__ __forceinline__ float reduce_scatter8(const float (&acc)[HPT], int ds)
+{
+    if constexpr (HPT == 4) {
+        const bool up = ds & 4;
+        float a0 = up ? acc[2] : acc[0], a1 = up ? acc[3] : acc[1];
+        const float b0 = up ? acc[0] : acc[2], b1 = up ? acc[1] : acc[3];
+        a0 += __shfl_xor_sync(0xffffffffu, b0, 4);
+        a1 += __shfl_xor_sync(0xffffffffu, b1, 4);
+        const bool mid = ds & 2;
+        float c = mid ? a1 : a0;
+        const float d2 = mid ? a0 : a1;
+        c += __shfl_xor_sync(0xffffffffu, d2, 2);
+        c += __shfl_xor_sync(0xffffffffu, c, 1);
+        return c;
+    } else if constexpr (HPT == 2) {
+        const bool up = ds & 4;
+        float c = up ? acc[1] : acc[0];
+        const float d2 = up ? acc[0] : acc[1];
+        c += __shfl_xor_sync(0xffffffffu, d2, 4);
+        c += __shfl_xor_sync(0xffffffffu, c, 2);
+        c += __shfl_xor_sync(0xffffffffu, c, 1);
+        return c;
+    } else {
+        float c = acc[0];
+        c += __shfl_xor_sync(0xffffffffu, c, 4);
+        c += __shfl_xor_sync(0xffffffffu, c, 2);
+        c += __shfl_xor_sync(0xffffffffu, c, 1);
+        return c;
+    }
+}
+
+template <typename T, int D, int HPT>
+__global__ void __launch_bounds__(kScoreThreads) score_kernel(const DescendParams p, int L, int GC, int ppc,
+                                                               int pchunks)
+{
+    constexpr int EV = Vec16<T>::E;          // elements per 16-byte vector
+    constexpr int CPR = D / EV;              // 16-byte chunks per row
+    constexpr int VPS = CPR / 8;             // chunks per d-slice: slice ds owns chunks ds, ds + 8, ...
+    static_assert(VPS >= 1 && CPR % 8 == 0, "a row splits into 8 d-slices of whole chunks");
+    static_assert(kScoreThreads % CPR == 0, "loader mapping");
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    __shared__ float s[GP * D];
-    __shared__ int seg[kScoreThreads];
-    __shared__ int nP_sh;
+    T *tiles = reinterpret_cast<T *>(smem_raw);                                        // [kStages][kTileRows][D]
+    int *meta_i = reinterpret_cast<int *>(tiles + (size_t)kStages * kTileRows * D);   // [kStages][kTileRows]
+    int *meta_j = meta_i + kStages * kTileRows;                                        // [kStages][kTileRows]
     const int Kp = p.K[L - 1];
     const int fo = p.fanout[L];
-    const int total = GP * Kp;
-    int32_t *lists = reinterpret_cast<int32_t *>(smem_raw);          // [GP][Kp] kept parents
-    int32_t *first = lists + total;                                   // [total] index of the first occurrence
-    int32_t *P = first + total;                                       // [total] union
-    int32_t *firstpos = P + total;                                    // [total]
-    int16_t *pidx = reinterpret_cast<int16_t *>(firstpos + total);    // [GP][total]
+    const int total = GC * Kp;
+    int32_t *lists = meta_j + kStages * kTileRows;   // [GC][Kp]
+    int32_t *first = lists + total;                  // [total]
+    int32_t *P = first + total;                      // [total]
+    int32_t *firstpos = P + total;                   // [total]
+    __shared__ int seg[kScoreThreads];
+    __shared__ int nP_sh;
 
     const int pc = blockIdx.x % pchunks;
     const int rest = blockIdx.x / pchunks;
-    const int chunks = p.G / GP;
-    const int cid = rest % chunks;
-    const int grp_id = rest / chunks;
+    const int hchunks = p.G / GC;
+    const int hc = rest % hchunks;
+    const int grp_id = rest / hchunks;
     const int b = grp_id / p.H_kv, hkv = grp_id % p.H_kv;
-    const long long bh0 = (long long)b * p.H + (long long)hkv * p.G + (long long)cid * GP;
+    const long long bh0 = (long long)b * p.H + (long long)hkv * p.G + (long long)hc * GC;
 
-    for (int i = threadIdx.x; i < GP * D; i += blockDim.x) s[i] = p.s_ws[(size_t)bh0 * D + i];
+    // ---- union of the GC heads' kept parents ----
     for (int t = threadIdx.x; t < total; t += blockDim.x) {
         const int g = t / Kp, k = t - g * Kp;
         lists[t] = p.kept[L - 1][(bh0 + g) * Kp + k];
     }
-    for (int i = threadIdx.x; i < GP * total; i += blockDim.x) pidx[i] = -1;
     __syncthreads();
-    // first occurrence of each element (binary search in the earlier heads' lists)
     for (int t = threadIdx.x; t < total; t += blockDim.x) {
         const int g = t / Kp;
         const int x = lists[t];
@@ -323,30 +379,29 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const DescendParam
         first[t] = ft;
     }
     __syncthreads();
-    // exclusive scan of "is a first occurrence"
-    const int per = (total + blockDim.x - 1) / blockDim.x;
-    const int t0 = threadIdx.x * per, t1 = min(total, t0 + per);
-    int cnt = 0;
-    for (int t = t0; t < t1; ++t) cnt += (first[t] == t);
-    seg[threadIdx.x] = cnt;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        int run = 0;
-        for (int base = 0; base < (int)blockDim.x; base += 32) {
-            const int v = seg[base + threadIdx.x];
-            int incl = v;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int w = __shfl_up_sync(0xffffffffu, incl, o);
-                if ((int)threadIdx.x >= o) incl += w;
-            }
-            seg[base + threadIdx.x] = run + incl - v;
-            run += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (threadIdx.x == 0) nP_sh = run;
-    }
-    __syncthreads();
     {
+        const int per = (total + blockDim.x - 1) / blockDim.x;
+        const int t0 = threadIdx.x * per, t1 = min(total, t0 + per);
+        int cnt = 0;
+        for (int t = t0; t < t1; ++t) cnt += (first[t] == t);
+        seg[threadIdx.x] = cnt;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            int run = 0;
+            for (int base = 0; base < (int)blockDim.x; base += 32) {
+                const int v = seg[base + threadIdx.x];
+                int incl = v;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int w = __shfl_up_sync(0xffffffffu, incl, o);
+                    if ((int)threadIdx.x >= o) incl += w;
+                }
+                seg[base + threadIdx.x] = run + incl - v;
+                run += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (threadIdx.x == 0) nP_sh = run;
+        }
+        __syncthreads();
         int run = seg[threadIdx.x];
         for (int t = t0; t < t1; ++t)
             if (first[t] == t) {
@@ -356,48 +411,145 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const DescendParam
             }
     }
     __syncthreads();
-    for (int t = threadIdx.x; t < total; t += blockDim.x) {
-        const int g = t / Kp, k = t - g * Kp;
-        pidx[g * total + firstpos[first[t]]] = (int16_t)k;
-    }
-    __syncthreads();
     const int nP = nP_sh;
+    if (pc * ppc >= nP) return;
+    // rows of this CTA: chunks c = pc, pc + pchunks, ... of ppc parents each
+    const int nchunks_mine = (nP - pc * ppc + pchunks * ppc - 1) / (pchunks * ppc);
+    const int full_rows = ppc * fo;
+    const int last_i0 = (pc + (nchunks_mine - 1) * pchunks) * ppc;
+    const int nR = (nchunks_mine - 1) * full_rows + min(ppc, nP - last_i0) * fo;
+    const int ntiles = (nR + kTileRows - 1) / kTileRows;
+
     const T *kbase = reinterpret_cast<const T *>(p.keys[L]);
     const int32_t *tab = p.child[L - 1];
     const long long prow = p.rows[L - 1], rows = p.rows[L];
     const int32_t *slot = (L == 2) ? p.leaf_slot : nullptr;
-    float *f = p.f_ws;
-    const int fstride = p.fstride;
-    int *status = p.status;
-    // parent chunks pc, pc + pchunks, ...: pchunks covers the usual union (the
-    // heads of a group mostly agree); larger unions loop
-    for (int i0 = pc * ppc; i0 < nP; i0 += pchunks * ppc) {
-    const int i1 = min(nP, i0 + ppc);
-    score_rows<T, D, GP>(
-        kbase, s, (i1 - i0) * fo,
-        [&](int r) -> long long {
-            const int i = i0 + r / fo, j = r % fo;
-            if (slot) {
-                // the pool slot of parent P[i]: take it from the first head listing it
-                for (int g = 0; g < GP; ++g) {
-                    const int k = pidx[g * total + i];
-                    if (k >= 0) return (long long)slot[(bh0 + g) * Kp + k] * fo + j;
+
+    // ---- tile loader: thread t copies chunk t % CPR of rows t / CPR + q (256 / CPR) ----
+    auto load_tile = [&](int tile, int stage) {
+        constexpr int RPP = kScoreThreads / CPR;   // rows per pass
+        const int c = threadIdx.x % CPR;
+#pragma unroll
+        for (int q = 0; q < kTileRows / RPP; ++q) {
+            const int rr = threadIdx.x / CPR + q * RPP;
+            const int rho = tile * kTileRows + rr;
+            const bool ok = rho < nR;
+            long long row = 0;
+            int i = -1, j = 0;
+            if (ok) {
+                const int cc = rho / full_rows, r = rho - cc * full_rows;
+                i = (pc + cc * pchunks) * ppc + r / fo;
+                j = r % fo;
+                if (slot) {
+                    // pool slot of parent P[i] from the first head listing it
+                    const int x = P[i];
+                    int k = -1, g = 0;
+                    for (; g < GC; ++g) {
+                        const int32_t *lst = lists + g * Kp;
+                        int lo = 0, hi = Kp;
+                        while (lo < hi) {
+                            const int mid = (lo + hi) >> 1;
+                            if (lst[mid] < x) lo = mid + 1;
+                            else hi = mid;
+                        }
+                        if (lo < Kp && lst[lo] == x) {
+                            k = lo;
+                            break;
+                        }
+                    }
+                    row = (long long)slot[(bh0 + g) * Kp + k] * fo + j;
+                } else {
+                    const long long par = P[i];
+                    long long id = tab ? (long long)tab[((size_t)hkv * prow + par) * fo + j] : par * fo + j;
+                    if (id < 0 || id >= rows) {
+                        set_status(p.status, kDevBadChild);
+                        id = 0;
+                    }
+                    row = (long long)hkv * rows + id;
                 }
-                return 0;
             }
-            const long long par = P[i];
-            long long id = tab ? (long long)tab[((size_t)hkv * prow + par) * fo + j] : par * fo + j;
-            if (id < 0 || id >= rows) {
-                set_status(status, kDevBadChild);
-                id = 0;
+            if (c == 0) {
+                meta_i[stage * kTileRows + rr] = i;
+                meta_j[stage * kTileRows + rr] = j;
             }
-            return (long long)hkv * rows + id;
-        },
-        [&](int g, int r, float v) {
-            const int i = i0 + r / fo, j = r % fo;
-            const int k = pidx[g * total + i];
-            if (k >= 0) f[(size_t)(bh0 + g) * fstride + (size_t)k * fo + j] = v;
-        });
+            cp_async16_zfill(tiles + ((size_t)stage * kTileRows + rr) * D + c * EV, kbase + (size_t)row * D + c * EV,
+                             ok);
+        }
+        asm volatile("cp.async.commit_group;\n" ::);
+    };
+
+    // ---- thread roles for the dot products ----
+    const int HGC = GC / HPT;            // head groups
+    const int TPR = HGC * 8;             // threads per row stream
+    const int NRS = kScoreThreads / TPR; // row streams
+    const int rs = threadIdx.x / TPR;
+    const int hg = (threadIdx.x % TPR) >> 3;
+    const int ds = threadIdx.x & 7;
+    const bool worker = rs < NRS;
+    float sreg[HPT][VPS * EV];
+#pragma unroll
+    for (int e = 0; e < HPT; ++e)
+#pragma unroll
+        for (int v = 0; v < VPS; ++v)
+#pragma unroll
+            for (int q = 0; q < EV; ++q)
+                sreg[e][v * EV + q] =
+                    worker ? p.s_ws[(size_t)(bh0 + hg * HPT + e) * D + (ds + 8 * v) * EV + q] : 0.f;
+    const int hsel = ds / (8 / HPT);
+    const bool storer = worker && (ds % (8 / HPT)) == 0;
+    const int gstore = hg * HPT + hsel;
+    const int32_t *mylist = lists + gstore * Kp;
+    float *fout = p.f_ws + (size_t)(bh0 + gstore) * p.fstride;
+
+    auto dot_row = [&](const T *rowp, float (&acc)[HPT]) {
+#pragma unroll
+        for (int e = 0; e < HPT; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int v = 0; v < VPS; ++v) {
+            float x[EV];
+            Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(rowp + (ds + 8 * v) * EV), x);
+#pragma unroll
+            for (int q = 0; q < EV; ++q)
+#pragma unroll
+                for (int e = 0; e < HPT; ++e) acc[e] = fmaf(sreg[e][v * EV + q], x[q], acc[e]);
+        }
+    };
+    auto store = [&](int stage, int rr, float val) {
+        const int i = meta_i[stage * kTileRows + rr];
+        if (i < 0) return;
+        const int x = P[i];
+        int lo = 0, hi = Kp;
+        while (lo < hi) {
+            const int m = (lo + hi) >> 1;
+            if (mylist[m] < x) lo = m + 1;
+            else hi = m;
+        }
+        if (lo < Kp && mylist[lo] == x) fout[(size_t)lo * fo + meta_j[stage * kTileRows + rr]] = val;
+    };
+
+    load_tile(0, 0);
+    if (ntiles > 1) load_tile(1, 1);
+    for (int tile = 0; tile < ntiles; ++tile) {
+        if (tile + 1 < ntiles) asm volatile("cp.async.wait_group 1;\n" ::);
+        else asm volatile("cp.async.wait_group 0;\n" ::);
+        __syncthreads();
+        if (tile + 2 < ntiles) load_tile(tile + 2, (tile + 2) % kStages);
+        const int stage = tile % kStages;
+        const T *trows = tiles + (size_t)stage * kTileRows * D;
+        // two rows per step for independent FMA chains (all lanes of a warp step together)
+        for (int rr0 = 0; rr0 < kTileRows; rr0 += 2 * NRS) {
+            const int ra = rr0 + rs, rb = rr0 + NRS + rs;
+            const bool la = worker && ra < kTileRows, lb = worker && rb < kTileRows;
+            float acca[HPT], accb[HPT];
+            dot_row(trows + (size_t)(la ? ra : 0) * D, acca);
+            dot_row(trows + (size_t)(lb ? rb : 0) * D, accb);
+            const float va = reduce_scatter8<HPT>(acca, ds);
+            const float vb = reduce_scatter8<HPT>(accb, ds);
+            if (storer) {
+                if (la) store(stage, ra, va);
+                if (lb) store(stage, rb, vb);
+            }
+        }
     }
 }
 
@@ -427,27 +579,17 @@ __device__ void warp_sort_u64(uint64_t *a, int n)
     __syncwarp();
 }
 
-// k-th largest (1-based) of n floats f[0..n), warp-level.  Values are
-// bucketed linearly between their min and max (a monotone map); the bucket
+// k-th largest (1-based) of n floats f[0..n) (n a multiple of 4 in storage,
+// entries past n ignored), warp-level, given their min mn and max mx.  Values
+// are bucketed linearly between min and max (a monotone map); the bucket
 // holding the k-th largest is then searched exactly: sorted when small, else
 // narrowed by MSB-first radix passes over the order-preserving bit image.
 // hist: this warp's 256 bins; tmp: 64 scratch uint64.
-__device__ float warp_kth_largest(const float *f, int n, int k, uint32_t *hist, uint64_t *tmp)
+__device__ float warp_kth_largest(const float *f, int n, int k, float mn, float mx, uint32_t *hist, uint64_t *tmp)
 {
     const int lane = threadIdx.x & 31;
-    float mn = INFINITY, mx = -INFINITY;
-    for (int i = lane; i < n; i += 32) {
-        mn = fminf(mn, f[i]);
-        mx = fmaxf(mx, f[i]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    }
-    if (!(mx > mn) || !isfinite(mx - mn)) {
-        if (mx == mn) return mx;   // all equal
-    } else {
+    if (mx == mn) return mx;   // all equal
+    if (mx > mn && isfinite(mx - mn)) {
         const float scale = 255.99f / (mx - mn);
         auto bucket = [&](float v) { return min(255, max(0, (int)((v - mn) * scale))); };
 #pragma unroll
@@ -647,15 +789,25 @@ __device__ void write_kept(const DescendParams &p, const LevelView &lv, int L, l
             p.kept_leaf_row[bh * K + i] = (int32_t)lv.row((int)(sortb[i] & 0xffffffffu));
 }
 
-// One warp per traversal: top-K of level L's candidates.
-//   tier 1: fp32 scores with the rigorous bound E decide everything outside
-//           the band [t - 2E, t + 2E] around the K-th largest score t;
-//   tier 2: when at most 32 candidates are left in the band, each lane scores
-//           one of them in float64 from the float64 token sums, with its own
-//           rigorous bound  (g64_D (1 + g64_N) + g64_N) sum_d a64_d |k_d|,
-//           and the same band argument is repeated among them;
-//   tier 3: whatever is still undecided (true ties, or a band wider than a
-//           warp) is queued for exact_kernel.
+// Warp exclusive prefix sum.
+__device__ __forceinline__ int warp_excl_scan(int v, int &total)
+{
+    const int lane = threadIdx.x & 31;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int w = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += w;
+    }
+    total = __shfl_sync(0xffffffffu, incl, 31);
+    return incl - v;
+}
+
+// One warp per traversal: top-K of level L's candidates, tier 1.  The fp32
+// scores and their rigorous bound E settle every candidate outside the band
+// [t - 2E, t + 2E] around the K-th largest score t.  When the band holds more
+// candidates than places left, the traversal is queued for exact_kernel with
+// its decided entries and the band's positions.
 template <typename T, int D>
 __global__ void __launch_bounds__(kSelectWarps * 32) select_kernel(const DescendParams p, int L)
 {
@@ -669,52 +821,104 @@ __global__ void __launch_bounds__(kSelectWarps * 32) select_kernel(const Descend
     const LevelView lv = level_view<T>(p, L, bh, sc.prev);
     const int C = lv.C, K = p.K[L];
     float *fslot = p.f_ws + (size_t)bh * p.fstride;
-    for (int c = lane; c < C; c += 32) sc.f[c] = fslot[c];
+    const int nv = (C + 3) >> 2;
+    float mn = INFINITY, mx = -INFINITY;
+    bool bad = false;
+    {
+        // 16-byte loads, several in flight per lane; min / max / finiteness on the way
+        const float4 *src = reinterpret_cast<const float4 *>(fslot);
+        float4 *dst = reinterpret_cast<float4 *>(sc.f);
+        auto take = [&](float4 t, int v) {
+            dst[v] = t;
+            const float e[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (4 * v + q < C) {
+                    mn = fminf(mn, e[q]);
+                    mx = fmaxf(mx, e[q]);
+                    bad |= !isfinite(e[q]);
+                }
+        };
+        int v = lane;
+        for (; v + 3 * 32 < nv; v += 4 * 32) {
+            float4 t[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) t[u] = __ldcg(src + v + u * 32);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) take(t[u], v + u * 32);
+        }
+        for (; v < nv; v += 32) take(__ldcg(src + v), v);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+    }
     __syncwarp();
     if (p.stats && lane == 0) atomicAdd(p.stats + L * 4, 1ull);
     const float *f = sc.f;
     uint64_t *sortb = sc.sortb;
-    int nsel = 0;
-    auto emit = [&](bool pred, int c) {
-        const unsigned m = __ballot_sync(0xffffffffu, pred);
-        if (pred) sortb[nsel + __popc(m & lanemask_lt())] = ((uint64_t)(uint32_t)lv.id(c) << 32) | (uint32_t)c;
-        nsel += __popc(m);
-    };
     if (K >= C) {
-        for (int c0 = 0; c0 < C; c0 += 32) emit(c0 + lane < C, c0 + lane);
+        for (int c = lane; c < C; c += 32) sortb[c] = ((uint64_t)(uint32_t)lv.id(c) << 32) | (uint32_t)c;
+        __syncwarp();
         write_kept(p, lv, L, bh, sortb, K);
         return;
     }
-    // ---- tier 1 ----
     const double cprime = gamma_n(D) * (1.0 + gamma_n(p.N)) + gamma_n(p.N);
     const double E = cprime * (double)p.anorm_ws[bh] * (double)p.norm_bound[L * p.H_kv + lv.hkv] * (1.0 + 1e-6) +
                      D * 0x1p-148;
-    const double t = (double)warp_kth_largest(f, C, K, sc.hist, sc.tmp);
-    bool bad = !isfinite(E) || !isfinite(t);
-    for (int c = lane; c < C && !bad; c += 32) bad = !isfinite(f[c]);
     bad = __any_sync(0xffffffffu, bad);
+    const double t = bad ? 0.0 : (double)warp_kth_largest(f, C, K, mn, mx, sc.hist, sc.tmp);
+    bad = bad || !isfinite(E) || !isfinite(t);
     const double hi = bad ? INFINITY : __dadd_ru(t, 2.0 * E);
     const double lo = bad ? -INFINITY : __dsub_rd(t, 2.0 * E);
-    auto in_set = [&](int c) { return c < C && !bad && (double)f[c] > hi; };
-    auto amb = [&](int c) {
-        if (c >= C) return false;
+    // class of candidate c: 1 kept for sure, 2 ambiguous, 0 dropped
+    auto cls = [&](int c) -> int {
+        if (c >= C) return 0;
+        if (bad) return 2;
         const double fd = (double)f[c];
-        return bad || (fd >= lo && !(fd > hi));
+        return fd > hi ? 1 : (fd >= lo ? 2 : 0);
     };
     int n_in = 0, nA = 0;
-    for (int c = lane; c < C; c += 32) {
-        n_in += in_set(c);
-        nA += amb(c);
-    }
+    for (int v = lane; v < nv; v += 32)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int k = cls(4 * v + q);
+            n_in += k == 1;
+            nA += k == 2;
+        }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         n_in += __shfl_xor_sync(0xffffffffu, n_in, o);
         nA += __shfl_xor_sync(0xffffffffu, nA, o);
     }
     const int r = K - n_in;
-    for (int c0 = 0; c0 < C; c0 += 32) emit(in_set(c0 + lane), c0 + lane);
-    if (nA == r) {
-        for (int c0 = 0; c0 < C; c0 += 32) emit(amb(c0 + lane), c0 + lane);
+    const bool settle = nA == r;   // every ambiguous candidate is kept
+    int *list = reinterpret_cast<int *>(fslot);
+    int base_in = 0, base_a = 0;
+    for (int v0 = 0; v0 < nv; v0 += 32) {
+        const int v = v0 + lane;
+        int ci[4], nin = 0, na = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            ci[q] = v < nv ? cls(4 * v + q) : 0;
+            nin += ci[q] == 1 || (settle && ci[q] == 2);
+            na += !settle && ci[q] == 2;
+        }
+        int tin, ta;
+        int oin = base_in + warp_excl_scan(nin, tin);
+        int oa = base_a + warp_excl_scan(na, ta);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int c = 4 * v + q;
+            if (ci[q] == 1 || (settle && ci[q] == 2)) sortb[oin++] = ((uint64_t)(uint32_t)lv.id(c) << 32) | (uint32_t)c;
+            else if (ci[q] == 2) list[oa++] = c;
+        }
+        base_in += tin;
+        base_a += ta;
+    }
+    __syncwarp();
+    if (settle) {
         write_kept(p, lv, L, bh, sortb, K);
         return;
     }
@@ -722,98 +926,16 @@ __global__ void __launch_bounds__(kSelectWarps * 32) select_kernel(const Descend
         atomicAdd(p.stats + L * 4 + 1, 1ull);
         atomicAdd(p.stats + L * 4 + 2, (unsigned long long)nA);
     }
-    // the ambiguous positions, in position order, one per lane (when nA <= 32)
-    int my_pos = -1, na = 0;
-    for (int c0 = 0; c0 < C && na <= 32; c0 += 32) {
-        const bool a = amb(c0 + lane);
-        const unsigned m = __ballot_sync(0xffffffffu, a);
-        const int at = na + __popc(m & lanemask_lt());
-        if (a && at < 32) my_pos = c0 + lane;
-        // lanes receive their position below
-        if (a && at < 32) sc.tmp[at] = (uint64_t)(c0 + lane);
-        na += __popc(m);
-    }
-    __syncwarp();
-    int nlist = nA;
-    int r_left = r;
-    bool listed_all = true;   // the exact pass gets every ambiguous candidate
-    if (!bad && nA <= 32) {
-        // ---- tier 2 ----
-        for (int d = lane; d < D; d += 32) {
-            sc.s64[d] = p.s64_ws[(size_t)bh * D + d];
-            sc.a64[d] = p.a64_ws[(size_t)bh * D + d];
-        }
-        __syncwarp();
-        my_pos = lane < nA ? (int)sc.tmp[lane] : -1;
-        double y = -INFINITY, e2 = 0.0;
-        if (my_pos >= 0) {
-            const T *krow = reinterpret_cast<const T *>(p.keys[L]) + (size_t)lv.row(my_pos) * D;
-            double acc = 0.0, mag = 0.0;
-            for (int d = 0; d < D; d += Vec16<T>::E) {
-                float x[Vec16<T>::E];
-                Vec16<T>::unpack(ldg16(krow + d), x);
-#pragma unroll
-                for (int e = 0; e < Vec16<T>::E; ++e) {
-                    acc = fma(sc.s64[d + e], (double)x[e], acc);
-                    mag = fma(sc.a64[d + e], fabs((double)x[e]), mag);
-                }
-            }
-            const double g64d = (double)D * 0x1p-53 / (1.0 - (double)D * 0x1p-53);
-            const double g64n = (double)p.N * 0x1p-53 / (1.0 - (double)p.N * 0x1p-53);
-            y = acc;
-            e2 = (g64d * (1.0 + g64n) + g64n) * mag * (1.0 + 1e-6) + 0x1p-1000;
-        }
-        double E2 = e2;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) E2 = fmax(E2, __shfl_xor_sync(0xffffffffu, E2, o));
-        // r-th largest y among the nA lanes
-        int rank = 0;
-        for (int j = 0; j < nA; ++j) {
-            const double yj = __shfl_sync(0xffffffffu, y, j);
-            rank += (yj > y) || (yj == y && j < lane);
-        }
-        const int tl = __ffs(__ballot_sync(0xffffffffu, my_pos >= 0 && rank == r - 1)) - 1;
-        const double t2 = __shfl_sync(0xffffffffu, y, tl);
-        const double hi2 = __dadd_ru(t2, 2.0 * E2), lo2 = __dsub_rd(t2, 2.0 * E2);
-        const bool in2 = my_pos >= 0 && y > hi2;
-        const bool amb2 = my_pos >= 0 && !in2 && y >= lo2;
-        const int n_in2 = __popc(__ballot_sync(0xffffffffu, in2));
-        const int nA2 = __popc(__ballot_sync(0xffffffffu, amb2));
-        emit(in2, my_pos);
-        if (nA2 == r - n_in2) {
-            emit(amb2, my_pos);
-            write_kept(p, lv, L, bh, sortb, K);
-            return;
-        }
-        // hand the still-ambiguous ones to the exact pass
-        const unsigned m2 = __ballot_sync(0xffffffffu, amb2);
-        int *list = reinterpret_cast<int *>(fslot);
-        if (amb2) list[__popc(m2 & lanemask_lt())] = my_pos;
-        nlist = nA2;
-        r_left = r - n_in2;
-        listed_all = false;
-    }
-    if (listed_all) {
-        int *list = reinterpret_cast<int *>(fslot);
-        int at = 0;
-        for (int c0 = 0; c0 < C; c0 += 32) {
-            const bool a = amb(c0 + lane);
-            const unsigned m = __ballot_sync(0xffffffffu, a);
-            if (a) list[at + __popc(m & lanemask_lt())] = c0 + lane;
-            at += __popc(m);
-        }
-    }
-    // decided entries (id << 32 | position) after the list, then the queue entry
     uint64_t *decided = reinterpret_cast<uint64_t *>(fslot + p.cap);
-    for (int i = lane; i < nsel; i += 32) decided[i] = sortb[i];
+    for (int i = lane; i < n_in; i += 32) decided[i] = sortb[i];
     if (lane == 0) {
         const int qi = atomicAdd(p.qcount + L, 1);
-        int *e = p.queue + ((size_t)L * p.B * p.H + qi) * 3;
+        int *e = p.queue + ((size_t)L * p.B * p.H + qi) * 4;
         e[0] = (int)bh;
-        e[1] = nsel;
-        e[2] = nlist;
+        e[1] = n_in;
+        e[2] = nA;
+        e[3] = bad ? 1 : 0;
     }
-    (void)r_left;
 }
 
 // Exact score of one key row: x = sum_n sum_d q[n][d] k[d] over the stored
@@ -876,13 +998,16 @@ struct ExactScratch {
     uint32_t *ex;      // [3 RC][kScoreDigits]
     int32_t *ids;      // [3 RC]
     int32_t *poss;     // [3 RC]
-    __host__ __device__ static size_t bytes(int kcap)
+    int32_t *list2;    // [32] positions still ambiguous after tier 2
+    double *s64;       // [D]
+    double *a64;       // [D]
+    __host__ __device__ static size_t bytes(int kcap, int D)
     {
         auto r = [](size_t b) { return (b + 15) & ~size_t(15); };
         return r((size_t)kcap * 4) + r((size_t)kcap * 8) + r(3 * kRefineChunk * kScoreDigits * 4) +
-               2 * r(3 * kRefineChunk * 4);
+               2 * r(3 * kRefineChunk * 4) + r(128) + 2 * r((size_t)D * 8);
     }
-    __device__ ExactScratch(uint8_t *p, int kcap)
+    __device__ ExactScratch(uint8_t *p, int kcap, int D)
     {
         auto take = [&](size_t b) {
             uint8_t *q = p;
@@ -894,32 +1019,42 @@ struct ExactScratch {
         ex = (uint32_t *)take(3 * kRefineChunk * kScoreDigits * 4);
         ids = (int32_t *)take(3 * kRefineChunk * 4);
         poss = (int32_t *)take(3 * kRefineChunk * 4);
+        list2 = (int32_t *)take(128);
+        s64 = (double *)take((size_t)D * 8);
+        a64 = (double *)take((size_t)D * 8);
     }
 };
 
-// Tier 3: traversals the fp32 and fp64 bounds could not settle.  For each
-// queued traversal, pick the remaining K - decided candidates of its list by
-// (exact score desc, row id asc): the list is scanned in chunks of RC with a
-// bounded best-set, and passes repeat (each excluding everything not strictly
-// worse than the last one chosen) until enough are chosen.
+// Traversals tier 1 left open.  For each, with `decided` entries already kept
+// and r = K - decided places left among the listed band candidates:
+//   tier 2: when at most 32 are listed (and all scores were finite), each lane
+//           scores one of them in float64 from the float64 token sums, with its
+//           own rigorous bound  (g64_D (1 + g64_N) + g64_N) sum_d a64_d |k_d|,
+//           and the band argument is repeated among them;
+//   tier 3: whatever is still open is ranked by exact score, then row id: the
+//           candidates are scanned in chunks of RC with a bounded best-set, and
+//           passes repeat (each excluding everything not strictly worse than
+//           the last one chosen) until r are chosen.
 template <typename T, int D>
 __global__ void __launch_bounds__(kSelectWarps * 32) exact_kernel(const DescendParams p, int L)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     constexpr int RC = kRefineChunk;
+    constexpr int EV = Vec16<T>::E;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qn = p.qcount[L];
-    ExactScratch sc(smem_raw + (size_t)warp * ExactScratch::bytes(p.kcap), p.kcap);
+    ExactScratch sc(smem_raw + (size_t)warp * ExactScratch::bytes(p.kcap, D), p.kcap, D);
     uint32_t *BEST = sc.ex, *CH = sc.ex + RC * kScoreDigits, *TMP = sc.ex + 2 * RC * kScoreDigits;
     int32_t *best_id = sc.ids, *ch_id = sc.ids + RC, *tmp_id = sc.ids + 2 * RC;
     int32_t *best_pos = sc.poss, *ch_pos = sc.poss + RC, *tmp_pos = sc.poss + 2 * RC;
     for (int qi = blockIdx.x * kSelectWarps + warp; qi < qn; qi += gridDim.x * kSelectWarps) {
-        const int *e = p.queue + ((size_t)L * p.B * p.H + qi) * 3;
+        const int *e = p.queue + ((size_t)L * p.B * p.H + qi) * 4;
         const long long bh = e[0];
         int nsel = e[1];
-        const int nlist = e[2];
+        int nlist = e[2];
+        const bool bad = e[3] != 0;
         const int K = p.K[L];
-        const int r = K - nsel;
+        int r = K - nsel;
         const int Kp = L == 0 ? 0 : p.K[L - 1];
         for (int k = lane; k < Kp; k += 32) sc.prev[k] = p.kept[L - 1][bh * Kp + k];
         const float *fslot = p.f_ws + (size_t)bh * p.fstride;
@@ -932,6 +1067,72 @@ __global__ void __launch_bounds__(kSelectWarps * 32) exact_kernel(const DescendP
         const T *qh = reinterpret_cast<const T *>(p.q_kg) + ((size_t)b * p.N * p.H + h) * D;
         const size_t q_stride = (size_t)p.H * D;
         const T *kbase = reinterpret_cast<const T *>(p.keys[L]);
+
+        if (!bad && nlist <= 32) {
+            // ---- tier 2 ----
+            if (p.stats && lane == 0) atomicAdd(p.stats + L * 4 + 3, 0ull);
+            for (int d = lane; d < D; d += 32) {
+                sc.s64[d] = p.s64_ws[(size_t)bh * D + d];
+                sc.a64[d] = p.a64_ws[(size_t)bh * D + d];
+            }
+            __syncwarp();
+            const int my_pos = lane < nlist ? list[lane] : -1;
+            double y = -INFINITY, e2 = 0.0;
+            if (my_pos >= 0) {
+                const T *krow = kbase + (size_t)lv.row(my_pos) * D;
+                uint4 w[D / EV];
+#pragma unroll
+                for (int v = 0; v < D / EV; ++v) w[v] = ldg16(krow + v * EV);
+                double acc = 0.0, mag = 0.0;
+#pragma unroll
+                for (int v = 0; v < D / EV; ++v) {
+                    float x[EV];
+                    Vec16<T>::unpack(w[v], x);
+#pragma unroll
+                    for (int q = 0; q < EV; ++q) {
+                        acc = fma(sc.s64[v * EV + q], (double)x[q], acc);
+                        mag = fma(sc.a64[v * EV + q], fabs((double)x[q]), mag);
+                    }
+                }
+                const double g64d = (double)D * 0x1p-53 / (1.0 - (double)D * 0x1p-53);
+                const double g64n = (double)p.N * 0x1p-53 / (1.0 - (double)p.N * 0x1p-53);
+                y = acc;
+                e2 = (g64d * (1.0 + g64n) + g64n) * mag * (1.0 + 1e-6) + 0x1p-1000;
+            }
+            double E2 = e2;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) E2 = fmax(E2, __shfl_xor_sync(0xffffffffu, E2, o));
+            int rank = 0;
+            for (int j = 0; j < nlist; ++j) {
+                const double yj = __shfl_sync(0xffffffffu, y, j);
+                rank += (yj > y) || (yj == y && j < lane);
+            }
+            const int tl = __ffs(__ballot_sync(0xffffffffu, my_pos >= 0 && rank == r - 1)) - 1;
+            const double t2 = __shfl_sync(0xffffffffu, y, tl);
+            const double hi2 = __dadd_ru(t2, 2.0 * E2), lo2 = __dsub_rd(t2, 2.0 * E2);
+            const bool in2 = my_pos >= 0 && y > hi2;
+            const bool amb2 = my_pos >= 0 && !in2 && y >= lo2;
+            const unsigned min2 = __ballot_sync(0xffffffffu, in2);
+            const unsigned ma2 = __ballot_sync(0xffffffffu, amb2);
+            const int n_in2 = __popc(min2), nA2 = __popc(ma2);
+            const bool settle = nA2 == r - n_in2;
+            if (in2 || (settle && amb2)) {
+                const unsigned m = settle ? (min2 | ma2) : min2;
+                sc.sortb[nsel + __popc(m & lanemask_lt())] = ((uint64_t)(uint32_t)lv.id(my_pos) << 32) | (uint32_t)my_pos;
+            }
+            if (!settle && amb2) sc.list2[__popc(ma2 & lanemask_lt())] = my_pos;
+            __syncwarp();
+            if (settle) {
+                write_kept(p, lv, L, bh, sc.sortb, K);
+                __syncwarp();
+                continue;
+            }
+            nsel += n_in2;
+            r -= n_in2;
+            nlist = nA2;
+            list = sc.list2;
+        }
+        // ---- tier 3 ----
         int chosen = 0;
         bool have_pivot = false;
         uint32_t pivot[kScoreDigits];
@@ -958,23 +1159,23 @@ __global__ void __launch_bounds__(kSelectWarps * 32) exact_kernel(const DescendP
                 const int ide = ep < nbest ? best_id[ep] : (ep < npool ? ch_id[ep - nbest] : 0);
                 const bool valid = ep < npool && (ep < nbest || !have_pivot || exact_better(pivot, pivot_id, xe, ide));
                 const unsigned vmask = __ballot_sync(0xffffffffu, valid);
-                int rank = 0x7fffffff;
+                int rk = 0x7fffffff;
                 if (valid) {
-                    rank = 0;
+                    rk = 0;
                     unsigned others = vmask & ~(1u << ep);
                     while (others) {
                         const int f2 = __ffs(others) - 1;
                         others &= others - 1;
                         const uint32_t *xf = f2 < nbest ? BEST + f2 * kScoreDigits : CH + (f2 - nbest) * kScoreDigits;
                         const int idf = f2 < nbest ? best_id[f2] : ch_id[f2 - nbest];
-                        if (exact_better(xf, idf, xe, ide)) ++rank;
+                        if (exact_better(xf, idf, xe, ide)) ++rk;
                     }
                 }
-                if (rank < want) {
+                if (rk < want) {
 #pragma unroll
-                    for (int q = 0; q < kScoreDigits; ++q) TMP[rank * kScoreDigits + q] = xe[q];
-                    tmp_id[rank] = ide;
-                    tmp_pos[rank] = ep < nbest ? best_pos[ep] : ch_pos[ep - nbest];
+                    for (int q = 0; q < kScoreDigits; ++q) TMP[rk * kScoreDigits + q] = xe[q];
+                    tmp_id[rk] = ide;
+                    tmp_pos[rk] = ep < nbest ? best_pos[ep] : ch_pos[ep - nbest];
                 }
                 __syncwarp();
                 nbest = min(want, __popc(vmask));
