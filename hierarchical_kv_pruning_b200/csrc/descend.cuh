@@ -275,76 +275,41 @@ __global__ void __launch_bounds__(kScoreThreads) root_kernel(const DescendParams
 // registers, and the eight d-slice partial sums meet through a 4-shuffle
 // reduce-scatter.  Head g's score of child j of union parent P[i] lands at its
 // own candidate slot k fo + j, k = position of P[i] in g's sorted list.
-constexpr int kTileRows = 64;
-constexpr int kStages = 3;
-
-template <typename T, int D>
+// Dynamic shared memory of score_kernel: token sums [D][GPB] + union
+// bookkeeping (4 GC Kp ints) + the (head, union parent) -> slot table.
+template <int D, int GPB>
 __host__ __device__ constexpr size_t score_kernel_smem(int GC, int Kp)
 {
-    return (size_t)kStages * kTileRows * D * sizeof(T) + (size_t)2 * kStages * kTileRows * 4 + (size_t)4 * GC * Kp * 4;
+    return (size_t)D * GPB * 4 + (size_t)4 * GC * Kp * 4 + (size_t)GPB * GC * Kp * 2 + 16;
 }
 
-__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, bool valid)
-{
-    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
-    const int sz = valid ? 16 : 0;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "r"(sz));
-}
-
-// Reduce HPT per-lane partial sums over the 8 lanes of a d-slice group; lane
-// ds ends with the total of head (ds / (8 / HPT)).
-template <int HPT>
-__device__ __forceinline__ float reduce_scatter8(const float (&acc)[HPT], int ds)
-{
-    if constexpr (HPT == 4) {
-        const bool up = ds & 4;
-        float a0 = up ? acc[2] : acc[0], a1 = up ? acc[3] : acc[1];
-        const float b0 = up ? acc[0] : acc[2], b1 = up ? acc[1] : acc[3];
-        a0 += __shfl_xor_sync(0xffffffffu, b0, 4);
-        a1 += __shfl_xor_sync(0xffffffffu, b1, 4);
-        const bool mid = ds & 2;
-        float c = mid ? a1 : a0;
-        const float d2 = mid ? a0 : a1;
-        c += __shfl_xor_sync(0xffffffffu, d2, 2);
-        c += __shfl_xor_sync(0xffffffffu, c, 1);
-        return c;
-    } else if constexpr (HPT == 2) {
-        const bool up = ds & 4;
-        float c = up ? acc[1] : acc[0];
-        const float d2 = up ? acc[0] : acc[1];
-        c += __shfl_xor_sync(0xffffffffu, d2, 4);
-        c += __shfl_xor_sync(0xffffffffu, c, 2);
-        c += __shfl_xor_sync(0xffffffffu, c, 1);
-        return c;
-    } else {
-        float c = acc[0];
-        c += __shfl_xor_sync(0xffffffffu, c, 4);
-        c += __shfl_xor_sync(0xffffffffu, c, 2);
-        c += __shfl_xor_sync(0xffffffffu, c, 1);
-        return c;
-    }
-}
-
-template <typename T, int D, int HPT>
+// Children of the kept parents (levels 1 and 2).
+//
+// Grid: (query b, KV head, head chunk of GC <= GPB heads, parent chunk).  The
+// CTA forms the union of its GC heads' kept parent lists (each ascending) in
+// first-appearance order and scores every child row of union parents
+// [pc ppc, (pc + 1) ppc) (and of every pchunks-th chunk after it) against all
+// GC token-sum vectors, one row per thread: the thread fetches the whole row
+// with independent 16-byte loads and runs GC accumulation chains, reading the
+// token sums (stored [d][head]) as shared-memory broadcasts.  Each row leaves
+// L2/HBM once per CTA; no cross-lane reduction is needed.  Head g's score of
+// child j of union parent P[i] lands at its candidate slot kidx[g][i] fo + j.
+template <typename T, int D, int GPB>
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(const DescendParams p, int L, int GC, int ppc,
                                                                int pchunks)
 {
-    constexpr int EV = Vec16<T>::E;          // elements per 16-byte vector
-    constexpr int CPR = D / EV;              // 16-byte chunks per row
-    constexpr int VPS = CPR / 8;             // chunks per d-slice: slice ds owns chunks ds, ds + 8, ...
-    static_assert(VPS >= 1 && CPR % 8 == 0, "a row splits into 8 d-slices of whole chunks");
-    static_assert(kScoreThreads % CPR == 0, "loader mapping");
+    constexpr int EV = Vec16<T>::E;
+    constexpr int VPR = D / EV;              // 16-byte vectors per row
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    T *tiles = reinterpret_cast<T *>(smem_raw);                                        // [kStages][kTileRows][D]
-    int *meta_i = reinterpret_cast<int *>(tiles + (size_t)kStages * kTileRows * D);   // [kStages][kTileRows]
-    int *meta_j = meta_i + kStages * kTileRows;                                        // [kStages][kTileRows]
+    float *st = reinterpret_cast<float *>(smem_raw);      // [D][GPB]
     const int Kp = p.K[L - 1];
     const int fo = p.fanout[L];
     const int total = GC * Kp;
-    int32_t *lists = meta_j + kStages * kTileRows;   // [GC][Kp]
-    int32_t *first = lists + total;                  // [total]
-    int32_t *P = first + total;                      // [total]
-    int32_t *firstpos = P + total;                   // [total]
+    int32_t *lists = reinterpret_cast<int32_t *>(st + D * GPB);   // [GC][Kp]
+    int32_t *first = lists + total;                               // [total]
+    int32_t *P = first + total;                                   // [total]
+    int32_t *firstpos = P + total;                                // [total]
+    int16_t *kidx = reinterpret_cast<int16_t *>(firstpos + total);   // [GPB][total]
     __shared__ int seg[kScoreThreads];
     __shared__ int nP_sh;
 
@@ -356,12 +321,17 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const DescendParam
     const int b = grp_id / p.H_kv, hkv = grp_id % p.H_kv;
     const long long bh0 = (long long)b * p.H + (long long)hkv * p.G + (long long)hc * GC;
 
-    // ---- union of the GC heads' kept parents ----
+    for (int i = threadIdx.x; i < D * GPB; i += blockDim.x) {
+        const int d = i / GPB, g = i % GPB;
+        st[i] = g < GC ? p.s_ws[(size_t)(bh0 + g) * D + d] : 0.f;
+    }
     for (int t = threadIdx.x; t < total; t += blockDim.x) {
         const int g = t / Kp, k = t - g * Kp;
         lists[t] = p.kept[L - 1][(bh0 + g) * Kp + k];
     }
+    for (int i = threadIdx.x; i < GPB * total; i += blockDim.x) kidx[i] = -1;
     __syncthreads();
+    // ---- union of the GC heads' kept parents, first-appearance order ----
     for (int t = threadIdx.x; t < total; t += blockDim.x) {
         const int g = t / Kp;
         const int x = lists[t];
@@ -411,143 +381,119 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const DescendParam
             }
     }
     __syncthreads();
+    for (int t = threadIdx.x; t < total; t += blockDim.x) {
+        const int g = t / Kp, k = t - g * Kp;
+        kidx[g * total + firstpos[first[t]]] = (int16_t)k;
+    }
+    __syncthreads();
     const int nP = nP_sh;
     if (pc * ppc >= nP) return;
-    // rows of this CTA: chunks c = pc, pc + pchunks, ... of ppc parents each
     const int nchunks_mine = (nP - pc * ppc + pchunks * ppc - 1) / (pchunks * ppc);
     const int full_rows = ppc * fo;
     const int last_i0 = (pc + (nchunks_mine - 1) * pchunks) * ppc;
     const int nR = (nchunks_mine - 1) * full_rows + min(ppc, nP - last_i0) * fo;
-    const int ntiles = (nR + kTileRows - 1) / kTileRows;
 
     const T *kbase = reinterpret_cast<const T *>(p.keys[L]);
     const int32_t *tab = p.child[L - 1];
     const long long prow = p.rows[L - 1], rows = p.rows[L];
     const int32_t *slot = (L == 2) ? p.leaf_slot : nullptr;
+    float *f = p.f_ws;
+    const int fstride = p.fstride;
 
-    // ---- tile loader: thread t copies chunk t % CPR of rows t / CPR + q (256 / CPR) ----
-    auto load_tile = [&](int tile, int stage) {
-        constexpr int RPP = kScoreThreads / CPR;   // rows per pass
-        const int c = threadIdx.x % CPR;
+    // Register tile: RT rows x HT heads per thread.  Per element of the rows,
+    // one read of HT token sums (HT/4 broadcast 16-byte shared loads) feeds
+    // HT x RT FMAs, which balances the FMA and shared-memory pipes.
+    constexpr int HT = GPB < 8 ? GPB : 8;
+    constexpr int HGN = GPB / HT;            // head groups sharing a row group
+    constexpr int RT = 4;
+    const int hgi = threadIdx.x % HGN;
+    const int rgi = threadIdx.x / HGN;
+    const int rows_per_pass = (kScoreThreads / HGN) * RT;
+    const float *sh = st + hgi * HT;
+
+    auto row_of = [&](int rho, int &i, int &j) -> long long {
+        const int cc = rho / full_rows, r = rho - cc * full_rows;
+        i = (pc + cc * pchunks) * ppc + r / fo;
+        j = r % fo;
+        if (slot) {
+            // pool slot of parent P[i] from the first head listing it
+            int g = 0;
+            while (g < GC - 1 && kidx[g * total + i] < 0) ++g;
+            return (long long)slot[(bh0 + g) * Kp + kidx[g * total + i]] * fo + j;
+        }
+        const long long par = P[i];
+        long long id = tab ? (long long)tab[((size_t)hkv * prow + par) * fo + j] : par * fo + j;
+        if (id < 0 || id >= rows) {
+            set_status(p.status, kDevBadChild);
+            id = 0;
+        }
+        return (long long)hkv * rows + id;
+    };
+
+    for (int base = 0; base < nR; base += rows_per_pass) {
+        const T *rp[RT];
+        int ii[RT], jj[RT];
+        bool ok[RT];
 #pragma unroll
-        for (int q = 0; q < kTileRows / RPP; ++q) {
-            const int rr = threadIdx.x / CPR + q * RPP;
-            const int rho = tile * kTileRows + rr;
-            const bool ok = rho < nR;
-            long long row = 0;
-            int i = -1, j = 0;
-            if (ok) {
-                const int cc = rho / full_rows, r = rho - cc * full_rows;
-                i = (pc + cc * pchunks) * ppc + r / fo;
-                j = r % fo;
-                if (slot) {
-                    // pool slot of parent P[i] from the first head listing it
-                    const int x = P[i];
-                    int k = -1, g = 0;
-                    for (; g < GC; ++g) {
-                        const int32_t *lst = lists + g * Kp;
-                        int lo = 0, hi = Kp;
-                        while (lo < hi) {
-                            const int mid = (lo + hi) >> 1;
-                            if (lst[mid] < x) lo = mid + 1;
-                            else hi = mid;
-                        }
-                        if (lo < Kp && lst[lo] == x) {
-                            k = lo;
-                            break;
-                        }
+        for (int k = 0; k < RT; ++k) {
+            const int rho = base + rgi * RT + k;
+            ok[k] = rho < nR;
+            ii[k] = 0;
+            jj[k] = 0;
+            rp[k] = kbase + (size_t)(ok[k] ? row_of(rho, ii[k], jj[k]) : 0) * D;
+        }
+        float acc[HT][RT];
+#pragma unroll
+        for (int h = 0; h < HT; ++h)
+#pragma unroll
+            for (int k = 0; k < RT; ++k) acc[h][k] = 0.f;
+        uint4 cur[RT], nxt[RT];
+#pragma unroll
+        for (int k = 0; k < RT; ++k) cur[k] = ok[k] ? ldg16(rp[k]) : make_uint4(0, 0, 0, 0);
+#pragma unroll 2
+        for (int v = 0; v < VPR; ++v) {
+            if (v + 1 < VPR) {
+#pragma unroll
+                for (int k = 0; k < RT; ++k) nxt[k] = ok[k] ? ldg16(rp[k] + (v + 1) * EV) : make_uint4(0, 0, 0, 0);
+            }
+            float x[RT][EV];
+#pragma unroll
+            for (int k = 0; k < RT; ++k) Vec16<T>::unpack(cur[k], x[k]);
+#pragma unroll
+            for (int q = 0; q < EV; ++q) {
+                const float *sd = sh + (v * EV + q) * GPB;
+                float sv[HT];
+                if constexpr (HT % 4 == 0) {
+#pragma unroll
+                    for (int h4 = 0; h4 < HT; h4 += 4) {
+                        const float4 t4 = *reinterpret_cast<const float4 *>(sd + h4);
+                        sv[h4] = t4.x;
+                        sv[h4 + 1] = t4.y;
+                        sv[h4 + 2] = t4.z;
+                        sv[h4 + 3] = t4.w;
                     }
-                    row = (long long)slot[(bh0 + g) * Kp + k] * fo + j;
                 } else {
-                    const long long par = P[i];
-                    long long id = tab ? (long long)tab[((size_t)hkv * prow + par) * fo + j] : par * fo + j;
-                    if (id < 0 || id >= rows) {
-                        set_status(p.status, kDevBadChild);
-                        id = 0;
-                    }
-                    row = (long long)hkv * rows + id;
+#pragma unroll
+                    for (int h = 0; h < HT; ++h) sv[h] = sd[h];
                 }
+#pragma unroll
+                for (int h = 0; h < HT; ++h)
+#pragma unroll
+                    for (int k = 0; k < RT; ++k) acc[h][k] = fmaf(sv[h], x[k][q], acc[h][k]);
             }
-            if (c == 0) {
-                meta_i[stage * kTileRows + rr] = i;
-                meta_j[stage * kTileRows + rr] = j;
-            }
-            cp_async16_zfill(tiles + ((size_t)stage * kTileRows + rr) * D + c * EV, kbase + (size_t)row * D + c * EV,
-                             ok);
+#pragma unroll
+            for (int k = 0; k < RT; ++k) cur[k] = nxt[k];
         }
-        asm volatile("cp.async.commit_group;\n" ::);
-    };
-
-    // ---- thread roles for the dot products ----
-    const int HGC = GC / HPT;            // head groups
-    const int TPR = HGC * 8;             // threads per row stream
-    const int NRS = kScoreThreads / TPR; // row streams
-    const int rs = threadIdx.x / TPR;
-    const int hg = (threadIdx.x % TPR) >> 3;
-    const int ds = threadIdx.x & 7;
-    const bool worker = rs < NRS;
-    float sreg[HPT][VPS * EV];
 #pragma unroll
-    for (int e = 0; e < HPT; ++e)
+        for (int k = 0; k < RT; ++k) {
+            if (!ok[k]) continue;
 #pragma unroll
-        for (int v = 0; v < VPS; ++v)
-#pragma unroll
-            for (int q = 0; q < EV; ++q)
-                sreg[e][v * EV + q] =
-                    worker ? p.s_ws[(size_t)(bh0 + hg * HPT + e) * D + (ds + 8 * v) * EV + q] : 0.f;
-    const int hsel = ds / (8 / HPT);
-    const bool storer = worker && (ds % (8 / HPT)) == 0;
-    const int gstore = hg * HPT + hsel;
-    const int32_t *mylist = lists + gstore * Kp;
-    float *fout = p.f_ws + (size_t)(bh0 + gstore) * p.fstride;
-
-    auto dot_row = [&](const T *rowp, float (&acc)[HPT]) {
-#pragma unroll
-        for (int e = 0; e < HPT; ++e) acc[e] = 0.f;
-#pragma unroll
-        for (int v = 0; v < VPS; ++v) {
-            float x[EV];
-            Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(rowp + (ds + 8 * v) * EV), x);
-#pragma unroll
-            for (int q = 0; q < EV; ++q)
-#pragma unroll
-                for (int e = 0; e < HPT; ++e) acc[e] = fmaf(sreg[e][v * EV + q], x[q], acc[e]);
-        }
-    };
-    auto store = [&](int stage, int rr, float val) {
-        const int i = meta_i[stage * kTileRows + rr];
-        if (i < 0) return;
-        const int x = P[i];
-        int lo = 0, hi = Kp;
-        while (lo < hi) {
-            const int m = (lo + hi) >> 1;
-            if (mylist[m] < x) lo = m + 1;
-            else hi = m;
-        }
-        if (lo < Kp && mylist[lo] == x) fout[(size_t)lo * fo + meta_j[stage * kTileRows + rr]] = val;
-    };
-
-    load_tile(0, 0);
-    if (ntiles > 1) load_tile(1, 1);
-    for (int tile = 0; tile < ntiles; ++tile) {
-        if (tile + 1 < ntiles) asm volatile("cp.async.wait_group 1;\n" ::);
-        else asm volatile("cp.async.wait_group 0;\n" ::);
-        __syncthreads();
-        if (tile + 2 < ntiles) load_tile(tile + 2, (tile + 2) % kStages);
-        const int stage = tile % kStages;
-        const T *trows = tiles + (size_t)stage * kTileRows * D;
-        // two rows per step for independent FMA chains (all lanes of a warp step together)
-        for (int rr0 = 0; rr0 < kTileRows; rr0 += 2 * NRS) {
-            const int ra = rr0 + rs, rb = rr0 + NRS + rs;
-            const bool la = worker && ra < kTileRows, lb = worker && rb < kTileRows;
-            float acca[HPT], accb[HPT];
-            dot_row(trows + (size_t)(la ? ra : 0) * D, acca);
-            dot_row(trows + (size_t)(lb ? rb : 0) * D, accb);
-            const float va = reduce_scatter8<HPT>(acca, ds);
-            const float vb = reduce_scatter8<HPT>(accb, ds);
-            if (storer) {
-                if (la) store(stage, ra, va);
-                if (lb) store(stage, rb, vb);
+            for (int h = 0; h < HT; ++h) {
+                const int g = hgi * HT + h;
+                if (g < GC) {
+                    const int kk = kidx[g * total + ii[k]];
+                    if (kk >= 0) f[(size_t)(bh0 + g) * fstride + (size_t)kk * fo + jj[k]] = acc[h][k];
+                }
             }
         }
     }
@@ -870,52 +816,47 @@ __global__ void __launch_bounds__(kSelectWarps * 32) select_kernel(const Descend
     bad = __any_sync(0xffffffffu, bad);
     const double t = bad ? 0.0 : (double)warp_kth_largest(f, C, K, mn, mx, sc.hist, sc.tmp);
     bad = bad || !isfinite(E) || !isfinite(t);
-    const double hi = bad ? INFINITY : __dadd_ru(t, 2.0 * E);
-    const double lo = bad ? -INFINITY : __dsub_rd(t, 2.0 * E);
+    // band edges rounded outward to fp32: the sure-kept and sure-dropped sets can
+    // only shrink, so the classification stays rigorous
+    const float hi32 = bad ? INFINITY : __double2float_ru(__dadd_ru(t, 2.0 * E));
+    const float lo32 = bad ? -INFINITY : __double2float_rd(__dsub_rd(t, 2.0 * E));
     // class of candidate c: 1 kept for sure, 2 ambiguous, 0 dropped
-    auto cls = [&](int c) -> int {
-        if (c >= C) return 0;
+    auto cls = [&](float fv) -> int {
         if (bad) return 2;
-        const double fd = (double)f[c];
-        return fd > hi ? 1 : (fd >= lo ? 2 : 0);
+        return fv > hi32 ? 1 : (fv >= lo32 ? 2 : 0);
     };
-    int n_in = 0, nA = 0;
-    for (int v = lane; v < nv; v += 32)
+    const float4 *f4 = reinterpret_cast<const float4 *>(f);
+    int my_in = 0, my_a = 0;
+    for (int v = lane; v < nv; v += 32) {
+        const float4 x = f4[v];
+        const float e[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int k = cls(4 * v + q);
-            n_in += k == 1;
-            nA += k == 2;
+            const int k = 4 * v + q < C ? cls(e[q]) : 0;
+            my_in += k == 1;
+            my_a += k == 2;
         }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        n_in += __shfl_xor_sync(0xffffffffu, n_in, o);
-        nA += __shfl_xor_sync(0xffffffffu, nA, o);
     }
+    int n_in, nA;
+    int off_in = warp_excl_scan(my_in, n_in);
+    int off_a = warp_excl_scan(my_a, nA);
     const int r = K - n_in;
     const bool settle = nA == r;   // every ambiguous candidate is kept
     int *list = reinterpret_cast<int *>(fslot);
-    int base_in = 0, base_a = 0;
-    for (int v0 = 0; v0 < nv; v0 += 32) {
-        const int v = v0 + lane;
-        int ci[4], nin = 0, na = 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            ci[q] = v < nv ? cls(4 * v + q) : 0;
-            nin += ci[q] == 1 || (settle && ci[q] == 2);
-            na += !settle && ci[q] == 2;
-        }
-        int tin, ta;
-        int oin = base_in + warp_excl_scan(nin, tin);
-        int oa = base_a + warp_excl_scan(na, ta);
+    if (settle) off_a += n_in;
+    for (int v = lane; v < nv; v += 32) {
+        const float4 x = f4[v];
+        const float e[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const int c = 4 * v + q;
-            if (ci[q] == 1 || (settle && ci[q] == 2)) sortb[oin++] = ((uint64_t)(uint32_t)lv.id(c) << 32) | (uint32_t)c;
-            else if (ci[q] == 2) list[oa++] = c;
+            const int k = c < C ? cls(e[q]) : 0;
+            if (k == 1) sortb[off_in++] = ((uint64_t)(uint32_t)lv.id(c) << 32) | (uint32_t)c;
+            else if (k == 2) {
+                if (settle) sortb[off_a++] = ((uint64_t)(uint32_t)lv.id(c) << 32) | (uint32_t)c;
+                else list[off_a++] = c;
+            }
         }
-        base_in += tin;
-        base_a += ta;
     }
     __syncwarp();
     if (settle) {
