@@ -14,6 +14,7 @@
 
 #include "atlaskv.h"
 #include "attend.cuh"
+#include "attend_tc.cuh"
 #include "descend.cuh"
 #include "internal.h"
 #include "staging.cuh"
@@ -337,10 +338,29 @@ atlaskv_status launch_attend_f32(const akv::AttnParams &ap, cudaStream_t s)
     return ATLASKV_OK;
 }
 
+// bf16, D = 128: tcgen05 tensor cores, one CTA per 128 query rows of a
+// (query, KV head) group.
+atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
+{
+    const int rows = ap.G * ap.N;
+    const int bpg = (rows + akv::tc::kRows - 1) / akv::tc::kRows;
+    const long long grid = (long long)ap.B * ap.H_kv * bpg;
+    if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "attention grid too large");
+    static bool configured = false;
+    if (!configured) {
+        AKV_CUDA(cudaFuncSetAttribute(akv::attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      akv::tc::kSmemBytes));
+        configured = true;
+    }
+    akv::attend_tc_kernel<<<(unsigned)grid, akv::tc::kThreads, akv::tc::kSmemBytes, s>>>(ap, bpg);
+    AKV_CUDA(cudaGetLastError());
+    return ATLASKV_OK;
+}
+
 atlaskv_status dispatch_attend(int dtype, int D, const akv::AttnParams &ap, cudaStream_t s)
 {
     if (dtype == ATLASKV_F32) return D == 64 ? launch_attend_f32<64>(ap, s) : launch_attend_f32<128>(ap, s);
-    return D == 64 ? launch_attend_bf16<64>(ap, s) : launch_attend_bf16<128>(ap, s);
+    return D == 64 ? launch_attend_bf16<64>(ap, s) : launch_attend_tc(ap, s);
 }
 
 // ---- staging launches -----------------------------------------------------
@@ -586,6 +606,7 @@ atlaskv_status atlaskv_attend(atlaskv_tree *t, const atlaskv_params *p, const at
     ap.T = io->T;
     ap.K_L = p->K_leaf;
     ap.scale_log2 = scale * 1.4426950408889634f;
+    ap.status = t->status;
 
     const bool prof = t->profiling;
     auto mark = [&](int i) -> atlaskv_status {

@@ -24,6 +24,7 @@ struct AttnParams {
     float *lse;                      // [B][N][H] or null
     int B, N, H, H_kv, G, T, K_L;
     float scale_log2;                // scale * log2(e)
+    int *status;                     // sticky device status word (bounded waits report here)
 };
 
 // ---------------------------------------------------------------------------

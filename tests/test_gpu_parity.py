@@ -131,6 +131,8 @@ SMALL = [
     (torch.bfloat16, 2, 1, 128, (5, 4, 3), (5, 20, 60), 2, 3, 70, False),      # full K: nothing pruned
     (torch.bfloat16, 32, 8, 128, (20, 20, 20), (8, 8, 32), 2, 128, 130, False),
     (torch.bfloat16, 32, 1, 128, (16, 16, 17), (16, 16, 64), 3, 32, 96, True),
+    (torch.bfloat16, 4, 2, 128, (8, 8, 10), (3, 4, 20), 2, 200, 300, False),   # one head's rows in two row blocks
+    (torch.bfloat16, 6, 2, 128, (10, 10, 12), (4, 9, 100), 2, 48, 50, True),   # row blocks cut heads; ragged leaf tile
     (torch.float32, 2, 2, 64, (30, 30, 9), (16, 200, 1000), 1, 1, 1, False),    # K above 128 and 1000 leaves
 ]
 
