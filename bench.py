@@ -54,6 +54,72 @@ def workload_shape(args):
     return sh
 
 
+def config_of(sh, world):
+    """The workload description both arms print."""
+    return {"workload": sh.name, "M": sh.n_leaves, "fanout": list(sh.fanout), "K": list(sh.keep),
+            "B": sh.batch, "N": sh.n_tokens, "T": sh.seq_len, "H": sh.n_heads, "H_kv": sh.n_kv_heads,
+            "D": sh.head_dim, "leaves": "pinned host" if sh.leaf_on_host else "HBM",
+            "l2": "inputs larger than L2 and 256 MB flush before each timed step",
+            "parallelism": "replicas x%d" % world}
+
+
+def kernels_per_step(sh):
+    """Kernels one atlaskv_attend call launches: per level (root or children
+    scoring, selection, exact pass) x 3, attention, and for host-resident
+    leaves two de-duplications and two staging copies."""
+    return 3 * 3 + 1 + (4 if sh.leaf_on_host else 0)
+
+
+def max_over_ranks(x, world, device):
+    """The largest value of x over all ranks (x itself on one rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, batch, total_ms, steps):
+    """Queries per second of all ranks together: every rank processes `batch`
+    queries per step and the slowest rank's time counts."""
+    return world * batch / (total_ms / steps * 1e-3)
+
+
+def attend_kernel_name(sh):
+    import torch
+    if sh.dtype == torch.float32:
+        return "attend_f32_kernel"
+    return "attend_tc_kernel" if sh.head_dim == 128 else "attend_bf16_kernel"
+
+
+KERNEL_SOURCES = {"attend_tc_kernel": "attend_tc.cuh", "attend_bf16_kernel": "attend.cuh",
+                  "attend_f32_kernel": "attend.cuh"}
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch (read + write) from the committed ncu summary of
+    this kernel on this workload, if the kernel source still hashes to the one
+    profiled; otherwise None."""
+    import hashlib
+    summ = os.path.join(ROOT, "profiles", "%s__%s.md" % (kernel, workload))
+    src = os.path.join(ROOT, "hierarchical_kv_pruning_b200", "csrc", KERNEL_SOURCES.get(kernel, ""))
+    if not (os.path.exists(summ) and os.path.isfile(src)):
+        return None
+    fields = {}
+    with open(summ) as f:
+        for line in f:
+            if line.startswith("- ") and ": " in line:
+                k, v = line[2:].split(": ", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    if fields.get("source_sha256") != digest or "dram_bytes_per_launch" not in fields:
+        return None
+    return int(fields["dram_bytes_per_launch"])
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -237,7 +303,7 @@ def run_ours(args):
     stage = [0.0, 0.0, 0.0]
     step_ms = []
     launches = 0
-    n_launch = 8 if not sh.leaf_on_host else 14   # 3 levels x (score + select) + attention (+ memset, staging)
+    n_launch = kernels_per_step(sh)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -257,13 +323,9 @@ def run_ours(args):
         refine = tree.refine_stats()
         torch.cuda.synchronize()
     tree.set_profiling(False)
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * sh.batch / (total_ms / args.steps * 1e-3)
+    value = whole_job_rate(world, sh.batch, total_ms, args.steps)
     tree.sync_status()
 
     # ---- end to end: pinned host inputs in, result out, through the public API ----
@@ -294,12 +356,8 @@ def run_ours(args):
         b.record(stream)
         b.synchronize()
         e2e_ms.append(a.elapsed_time(b))
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
-    e2e_value = world * sh.batch / (e2e_total / len(e2e_ms) * 1e-3)
+    e2e_total = max_over_ranks(sum(e2e_ms), world, dev)
+    e2e_value = whole_job_rate(world, sh.batch, e2e_total, len(e2e_ms))
 
     # ---- roofline of the dominant kernel ----
     res = {"kept_root": kept[0], "kept_mid": kept[1], "kept_leaf": kept[2]}
@@ -314,15 +372,29 @@ def run_ours(args):
         roof = {"bound": "host_link", "achieved": achieved, "peak": link, "unit": "GB/s", "frac": achieved / link,
                 "traffic": None, "kernel": "stage_leaf_blocks_kernel + stage_value_rows_kernel",
                 "peak_source": "pinned cudaMemcpyAsync H2D measured in this run"}
+    elif names[dom] == "attend":
+        kname = attend_kernel_name(sh)
+        t_hbm = alg["attend"] / (peaks["hbm_gbs"] * 1e9)
+        t_tc = alg["attend_flops"] / (peaks["bf16_tflops"] * 1e12)
+        if sh.dtype == torch.bfloat16 and t_tc > t_hbm:
+            achieved = alg["attend_flops"] / (st_ms[2] * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_tflops"]}
+        else:
+            achieved = alg["attend"] / (st_ms[2] * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"]}
+        roof.update({"traffic": profiled_traffic(kname, sh.name), "kernel": kname,
+                     "peak_source": peak_src + " (burst)"})
     else:
-        nbytes_k = alg[names[dom]]
-        achieved = nbytes_k / (st_ms[dom] * 1e-3) / 1e9
+        achieved = alg["descend"] / (st_ms[0] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                "kernel": "descend_kernel" if names[dom] == "descend" else "attend_bf16_kernel",
+                "kernel": "descent: root_kernel, score_kernel x2, select_kernel x3, exact_kernel x3",
                 "peak_source": peak_src}
     roof["stage_ms"] = {n: round(v, 4) for n, v in zip(names, st_ms)}
     roof["algorithmic_bytes"] = {k: alg[k] for k in ("descend", "attend", "staging")}
+    roof["attend_flops"] = alg["attend_flops"]
     roof["attend_tflops"] = alg["attend_flops"] / (st_ms[2] * 1e-3) / 1e12 if st_ms[2] > 0 else None
     roof["exact_refinement_last_step"] = refine
 
@@ -332,11 +404,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32" if sh.dtype == torch.float32 else "bf16",
         "data": "synthetic (seeded hierarchical-Gaussian tree and queries)",
-        "config": {"workload": sh.name, "M": sh.n_leaves, "fanout": list(sh.fanout), "K": list(K),
-                   "B": sh.batch, "N": sh.n_tokens, "T": sh.seq_len, "H": sh.n_heads, "H_kv": sh.n_kv_heads,
-                   "D": sh.head_dim, "leaves": "pinned host" if sh.leaf_on_host else "HBM",
-                   "l2": "inputs larger than L2 and 256 MB flush before each timed step",
-                   "parallelism": "replicas x%d" % world},
+        "config": config_of(sh, world),
         "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "roofline": roof,
@@ -378,7 +446,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded hierarchical-Gaussian tree and queries)",
-        "config": {"workload": sh.name, "M": sh.n_leaves, "B": sh.batch},
+        "config": config_of(sh, 1),
         "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "cpu_baseline": {"value": value, "unit": "queries/s", "kind": "oracle",
                          "cores": int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)),

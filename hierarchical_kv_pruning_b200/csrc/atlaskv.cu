@@ -213,24 +213,25 @@ atlaskv_status launch_root(const akv::DescendParams &dp, cudaStream_t s)
 }
 
 // Children scoring: one CTA per (query, KV head, chunk of GC <= 32 heads,
-// parent chunk); GPB = GC rounded up to a power of two.
-template <typename T, int D, int GPB>
-atlaskv_status launch_score_gpb(const akv::DescendParams &dp, int L, int GC, cudaStream_t s)
+// parent chunk); a warp serves HT heads (HT = GC rounded up to a power of two,
+// at most 8).
+template <typename T, int D, int HT>
+atlaskv_status launch_score_ht(const akv::DescendParams &dp, int L, int GC, cudaStream_t s)
 {
     const int Kp = dp.K[L - 1], fo = dp.fanout[L];
     const int ppc = std::max(1, 1024 / fo);           // parents per chunk: about 1024 rows per CTA
     const int pchunks = (Kp + ppc - 1) / ppc;         // covers a union of Kp parents; larger ones loop
     const long long grid = (long long)dp.B * dp.H_kv * (dp.G / GC) * pchunks;
     if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "scoring grid too large");
-    const size_t smem = akv::score_kernel_smem<D, GPB>(GC, Kp);
+    const size_t smem = akv::score_kernel_smem<D, (int)sizeof(T)>(GC, Kp);
     if (smem > 227 * 1024) return fail(ATLASKV_EUNSUPPORTED, "scoring needs %zu bytes of shared memory", smem);
     static size_t configured = 0;
     if (smem > 48 * 1024 && smem > configured) {
-        AKV_CUDA(cudaFuncSetAttribute(akv::score_kernel<T, D, GPB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        AKV_CUDA(cudaFuncSetAttribute(akv::score_kernel<T, D, HT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem));
         configured = smem;
     }
-    akv::score_kernel<T, D, GPB><<<(unsigned)grid, akv::kScoreThreads, smem, s>>>(dp, L, GC, ppc, pchunks);
+    akv::score_kernel<T, D, HT><<<(unsigned)grid, akv::kScoreThreads, smem, s>>>(dp, L, GC, ppc, pchunks);
     AKV_CUDA(cudaGetLastError());
     return ATLASKV_OK;
 }
@@ -244,12 +245,10 @@ atlaskv_status launch_score(const akv::DescendParams &dp, int L, cudaStream_t s)
             GC = c;
             break;
         }
-    if (GC <= 1) return launch_score_gpb<T, D, 1>(dp, L, GC, s);
-    if (GC <= 2) return launch_score_gpb<T, D, 2>(dp, L, GC, s);
-    if (GC <= 4) return launch_score_gpb<T, D, 4>(dp, L, GC, s);
-    if (GC <= 8) return launch_score_gpb<T, D, 8>(dp, L, GC, s);
-    if (GC <= 16) return launch_score_gpb<T, D, 16>(dp, L, GC, s);
-    return launch_score_gpb<T, D, 32>(dp, L, GC, s);
+    if (GC <= 1) return launch_score_ht<T, D, 1>(dp, L, GC, s);
+    if (GC <= 2) return launch_score_ht<T, D, 2>(dp, L, GC, s);
+    if (GC <= 4) return launch_score_ht<T, D, 4>(dp, L, GC, s);
+    return launch_score_ht<T, D, 8>(dp, L, GC, s);
 }
 
 template <typename T, int D>

@@ -265,51 +265,92 @@ __global__ void __launch_bounds__(kScoreThreads) root_kernel(const DescendParams
 // --------------------------------------------------------------------------
 // Children of the kept parents (levels 1 and 2).
 //
-// Grid: (query b, KV head, head chunk of GC heads, parent chunk).  The CTA forms
-// the union of its GC heads' kept parent lists (each ascending) in
-// first-appearance order, then scores every child row of union parents
-// [pc ppc, (pc + 1) ppc) (and of every pchunks-th chunk after it) against all
-// GC token-sum vectors: each row crosses from L2/HBM once per CTA.  Rows are
-// staged in shared memory in tiles of kTileRows by cp.async (kStages deep);
-// thread (row stream, head group, d-slice) keeps HPT heads x D/8 token sums in
-// registers, and the eight d-slice partial sums meet through a 4-shuffle
-// reduce-scatter.  Head g's score of child j of union parent P[i] lands at its
-// own candidate slot k fo + j, k = position of P[i] in g's sorted list.
-// Dynamic shared memory of score_kernel: token sums [D][GPB] + union
-// bookkeeping (4 GC Kp ints) + the (head, union parent) -> slot table.
-template <int D, int GPB>
-__host__ __device__ constexpr size_t score_kernel_smem(int GC, int Kp)
+// Grid: (query b, KV head, head chunk of GC <= 32 heads, parent chunk).  The
+// CTA forms the union of its GC heads' kept parent lists (a shared-memory hash
+// set: O(GC Kp) work) and scores every child row of the union parents
+// [pc ppc, (pc + 1) ppc), [(pc + pchunks) ppc, ...) against all GC token-sum
+// vectors, so each row crosses from L2/HBM once per head group.
+//
+// Rows reach the CTA in tiles of kScoreTile rows, copied by cp.async (LPG
+// consecutive threads per row, kScoreStages - 1 tiles in flight ahead of the
+// one being scored) into shared memory.  Each tile's row table (key row,
+// union parent, child index) is built one tile ahead, one thread per row, so
+// the copy and store loops do no index arithmetic.  For the dot products a
+// row is split over LPG = D / EV lanes, one 16-byte vector each, so a warp's
+// shared-memory read covers 32 / LPG whole rows without bank conflicts.  A
+// warp serves HT heads and keeps their token-sum slices in registers; a lane
+// group takes R = LPG / HT rows at a time, forms R x HT partial dot products
+// per lane and reduces them over the group by recursive halving, after which
+// lane `sub` of the group holds the full score of value index
+// sub = (row k, head h) = (sub / HT, sub % HT).  Head g's score of child j of
+// union parent P[i] lands at its own candidate slot kidx[g][i] fo + j.  The
+// fp32 sum of D products, in whatever order, stays within the g_D bound of
+// the filter.
+constexpr int kScoreTile = 64;
+constexpr int kScoreStages = 4;
+
+__host__ __device__ constexpr int score_hash_size(int total)
 {
-    return (size_t)D * GPB * 4 + (size_t)4 * GC * Kp * 4 + (size_t)GPB * GC * Kp * 2 + 16;
+    int hs = 64;
+    while (hs < 2 * total) hs <<= 1;
+    return hs;
 }
 
-// Children of the kept parents (levels 1 and 2).
-//
-// Grid: (query b, KV head, head chunk of GC <= GPB heads, parent chunk).  The
-// CTA forms the union of its GC heads' kept parent lists (each ascending) in
-// first-appearance order and scores every child row of union parents
-// [pc ppc, (pc + 1) ppc) (and of every pchunks-th chunk after it) against all
-// GC token-sum vectors, one row per thread: the thread fetches the whole row
-// with independent 16-byte loads and runs GC accumulation chains, reading the
-// token sums (stored [d][head]) as shared-memory broadcasts.  Each row leaves
-// L2/HBM once per CTA; no cross-lane reduction is needed.  Head g's score of
-// child j of union parent P[i] lands at its candidate slot kidx[g][i] fo + j.
-template <typename T, int D, int GPB>
-__global__ void __launch_bounds__(kScoreThreads) score_kernel(const DescendParams p, int L, int GC, int ppc,
-                                                               int pchunks)
+struct ScoreRow {
+    long long row;   // key row (units of D elements), -1: none
+    int i, j;        // union parent, child index
+};
+
+// Region A holds the row tiles; before the first tile it holds the union's
+// hash set (keys, inserting entry, union index: 3 hs ints) and each entry's
+// slot (total ints).  Then the row tables, lists / P / owner (3 total ints)
+// and kidx ([GC][total] int16).
+template <int D, int E>
+__host__ __device__ constexpr size_t score_region_a(int GC, int Kp)
 {
-    constexpr int EV = Vec16<T>::E;
-    constexpr int VPR = D / EV;              // 16-byte vectors per row
+    return (size_t)kScoreStages * kScoreTile * D * E > (size_t)(3 * score_hash_size(GC * Kp) + GC * Kp) * 4
+               ? (size_t)kScoreStages * kScoreTile * D * E
+               : ((size_t)(3 * score_hash_size(GC * Kp) + GC * Kp) * 4 + 15) / 16 * 16;
+}
+
+template <int D, int E>
+__host__ __device__ constexpr size_t score_kernel_smem(int GC, int Kp)
+{
+    return score_region_a<D, E>(GC, Kp) + (size_t)(kScoreStages + 1) * kScoreTile * sizeof(ScoreRow) +
+           (size_t)3 * GC * Kp * 4 + (size_t)GC * GC * Kp * 2 + 16;
+}
+
+template <typename T, int D, int HT>
+__global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const DescendParams p, int L, int GC, int ppc,
+                                                                  int pchunks)
+{
+    constexpr int EV = Vec16<T>::E;          // elements per 16-byte vector
+    constexpr int LPG = D / EV;              // lanes per row = 16-byte vectors per row
+    constexpr int GPW = 32 / LPG;            // rows per warp read
+    constexpr int R = LPG / HT;              // rows per lane group per reduction
+    static_assert(LPG >= 8 && LPG <= 32 && R >= 1 && R * HT == LPG, "one score per lane");
+    constexpr int NW = kScoreThreads / 32;
+    constexpr int ROWB = D * (int)sizeof(T);
+    constexpr int TILEB = kScoreTile * ROWB;
+    constexpr int NINFO = kScoreStages + 1;
+    constexpr int CPR = kScoreThreads / LPG;               // rows one copy round of the CTA covers
+    static_assert(kScoreTile % CPR == 0 && kScoreTile <= kScoreThreads, "tile shape");
+
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    float *st = reinterpret_cast<float *>(smem_raw);      // [D][GPB]
     const int Kp = p.K[L - 1];
     const int fo = p.fanout[L];
     const int total = GC * Kp;
-    int32_t *lists = reinterpret_cast<int32_t *>(st + D * GPB);   // [GC][Kp]
-    int32_t *first = lists + total;                               // [total]
-    int32_t *P = first + total;                                   // [total]
-    int32_t *firstpos = P + total;                                // [total]
-    int16_t *kidx = reinterpret_cast<int16_t *>(firstpos + total);   // [GPB][total]
+    const int hs = score_hash_size(total);
+    uint8_t *tiles = smem_raw;                                // [stages][rows][D]
+    int32_t *hkey = reinterpret_cast<int32_t *>(smem_raw);    // setup only: [hs] parent id or -1
+    int32_t *hown = hkey + hs;                                // [hs] inserting entry
+    int32_t *huid = hown + hs;                                // [hs] union index of the slot
+    int32_t *eslot = huid + hs;                               // [total] hash slot of entry t
+    ScoreRow *info = reinterpret_cast<ScoreRow *>(smem_raw + score_region_a<D, sizeof(T)>(GC, Kp));
+    int32_t *lists = reinterpret_cast<int32_t *>(info + NINFO * kScoreTile);   // [GC][Kp] ascending
+    int32_t *P = lists + total;                               // union parents
+    int32_t *Pown = P + total;                                // an entry (g Kp + k) listing P[i]
+    int16_t *kidx = reinterpret_cast<int16_t *>(Pown + total);   // [GC][total] slot of union parent i in g's list
     __shared__ int seg[kScoreThreads];
     __shared__ int nP_sh;
 
@@ -321,39 +362,32 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const DescendParam
     const int b = grp_id / p.H_kv, hkv = grp_id % p.H_kv;
     const long long bh0 = (long long)b * p.H + (long long)hkv * p.G + (long long)hc * GC;
 
-    for (int i = threadIdx.x; i < D * GPB; i += blockDim.x) {
-        const int d = i / GPB, g = i % GPB;
-        st[i] = g < GC ? p.s_ws[(size_t)(bh0 + g) * D + d] : 0.f;
-    }
+    for (int i = threadIdx.x; i < hs; i += blockDim.x) hkey[i] = -1;
+    for (int i = threadIdx.x; i < GC * total; i += blockDim.x) kidx[i] = -1;
     for (int t = threadIdx.x; t < total; t += blockDim.x) {
         const int g = t / Kp, k = t - g * Kp;
         lists[t] = p.kept[L - 1][(bh0 + g) * Kp + k];
     }
-    for (int i = threadIdx.x; i < GPB * total; i += blockDim.x) kidx[i] = -1;
     __syncthreads();
-    // ---- union of the GC heads' kept parents, first-appearance order ----
+    // ---- union of the GC heads' kept parents: insert into the hash set ----
     for (int t = threadIdx.x; t < total; t += blockDim.x) {
-        const int g = t / Kp;
         const int x = lists[t];
-        int ft = t;
-        for (int g2 = 0; g2 < g && ft == t; ++g2) {
-            const int32_t *lst = lists + g2 * Kp;
-            int lo = 0, hi = Kp;
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (lst[mid] < x) lo = mid + 1;
-                else hi = mid;
-            }
-            if (lo < Kp && lst[lo] == x) ft = g2 * Kp + lo;
+        unsigned h = ((unsigned)x * 2654435761u) & (unsigned)(hs - 1);
+        for (int probe = 0; probe < hs; ++probe) {
+            const int prev = atomicCAS(&hkey[h], -1, x);
+            if (prev == -1) hown[h] = t;
+            if (prev == -1 || prev == x) break;
+            h = (h + 1) & (unsigned)(hs - 1);
         }
-        first[t] = ft;
+        eslot[t] = (int)h;
     }
     __syncthreads();
+    // ---- number the occupied slots (table order): union index, P ----
     {
-        const int per = (total + blockDim.x - 1) / blockDim.x;
-        const int t0 = threadIdx.x * per, t1 = min(total, t0 + per);
+        const int per = (hs + (int)blockDim.x - 1) / (int)blockDim.x;
+        const int t0 = min(hs, (int)threadIdx.x * per), t1 = min(hs, t0 + per);
         int cnt = 0;
-        for (int t = t0; t < t1; ++t) cnt += (first[t] == t);
+        for (int t = t0; t < t1; ++t) cnt += (hkey[t] >= 0);
         seg[threadIdx.x] = cnt;
         __syncthreads();
         if (threadIdx.x < 32) {
@@ -374,24 +408,25 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const DescendParam
         __syncthreads();
         int run = seg[threadIdx.x];
         for (int t = t0; t < t1; ++t)
-            if (first[t] == t) {
-                firstpos[t] = run;
-                P[run] = lists[t];
+            if (hkey[t] >= 0) {
+                P[run] = hkey[t];
+                Pown[run] = hown[t];
+                huid[t] = run;
                 ++run;
             }
     }
     __syncthreads();
     for (int t = threadIdx.x; t < total; t += blockDim.x) {
         const int g = t / Kp, k = t - g * Kp;
-        kidx[g * total + firstpos[first[t]]] = (int16_t)k;
+        kidx[g * total + huid[eslot[t]]] = (int16_t)k;
     }
-    __syncthreads();
     const int nP = nP_sh;
     if (pc * ppc >= nP) return;
     const int nchunks_mine = (nP - pc * ppc + pchunks * ppc - 1) / (pchunks * ppc);
     const int full_rows = ppc * fo;
     const int last_i0 = (pc + (nchunks_mine - 1) * pchunks) * ppc;
     const int nR = (nchunks_mine - 1) * full_rows + min(ppc, nP - last_i0) * fo;
+    const int ntiles = (nR + kScoreTile - 1) / kScoreTile;
 
     const T *kbase = reinterpret_cast<const T *>(p.keys[L]);
     const int32_t *tab = p.child[L - 1];
@@ -400,103 +435,132 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const DescendParam
     float *f = p.f_ws;
     const int fstride = p.fstride;
 
-    // Register tile: RT rows x HT heads per thread.  Per element of the rows,
-    // one read of HT token sums (HT/4 broadcast 16-byte shared loads) feeds
-    // HT x RT FMAs, which balances the FMA and shared-memory pipes.
-    constexpr int HT = GPB < 8 ? GPB : 8;
-    constexpr int HGN = GPB / HT;            // head groups sharing a row group
-    constexpr int RT = 4;
-    const int hgi = threadIdx.x % HGN;
-    const int rgi = threadIdx.x / HGN;
-    const int rows_per_pass = (kScoreThreads / HGN) * RT;
-    const float *sh = st + hgi * HT;
-
-    auto row_of = [&](int rho, int &i, int &j) -> long long {
-        const int cc = rho / full_rows, r = rho - cc * full_rows;
-        i = (pc + cc * pchunks) * ppc + r / fo;
-        j = r % fo;
-        if (slot) {
-            // pool slot of parent P[i] from the first head listing it
-            int g = 0;
-            while (g < GC - 1 && kidx[g * total + i] < 0) ++g;
-            return (long long)slot[(bh0 + g) * Kp + kidx[g * total + i]] * fo + j;
+    // row table of tile tl (threads 0 .. kScoreTile-1, one row each)
+    auto build_info = [&](int tl) {
+        if (threadIdx.x >= kScoreTile) return;
+        ScoreRow sr;
+        const int rho = tl * kScoreTile + (int)threadIdx.x;
+        sr.row = -1;
+        sr.i = 0;
+        sr.j = 0;
+        if (rho < nR) {
+            const int cc = rho / full_rows, r = rho - cc * full_rows;
+            const int i = (pc + cc * pchunks) * ppc + r / fo;
+            const int j = r - (r / fo) * fo;
+            long long row;
+            if (slot) {
+                const int own = Pown[i];
+                row = (long long)slot[(bh0 + own / Kp) * Kp + own % Kp] * fo + j;
+            } else {
+                const long long par = P[i];
+                long long id = tab ? (long long)tab[((size_t)hkv * prow + par) * fo + j] : par * fo + j;
+                if (id < 0 || id >= rows) {
+                    set_status(p.status, kDevBadChild);
+                    id = 0;
+                }
+                row = (long long)hkv * rows + id;
+            }
+            sr.row = row;
+            sr.i = i;
+            sr.j = j;
         }
-        const long long par = P[i];
-        long long id = tab ? (long long)tab[((size_t)hkv * prow + par) * fo + j] : par * fo + j;
-        if (id < 0 || id >= rows) {
-            set_status(p.status, kDevBadChild);
-            id = 0;
+        info[(tl % NINFO) * kScoreTile + threadIdx.x] = sr;
+    };
+    // copy tile tl into stage tl % S: thread (row lr, vector lc), rows lr + CPR i
+    const int lc = threadIdx.x % LPG, lr = threadIdx.x / LPG;
+    auto load_tile = [&](int tl) {
+        const ScoreRow *ti = info + (tl % NINFO) * kScoreTile;
+        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(tiles + (tl % kScoreStages) * TILEB) + lc * 16;
+#pragma unroll
+        for (int i = 0; i < kScoreTile / CPR; ++i) {
+            const int r = lr + CPR * i;
+            const long long row = ti[r].row;
+            const T *src = row >= 0 ? kbase + (size_t)row * D + lc * EV : kbase;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst + r * ROWB), "l"(src),
+                         "r"(row >= 0 ? 16 : 0));
         }
-        return (long long)hkv * rows + id;
+        asm volatile("cp.async.commit_group;\n" ::);
     };
 
-    for (int base = 0; base < nR; base += rows_per_pass) {
-        const T *rp[RT];
-        int ii[RT], jj[RT];
-        bool ok[RT];
+    // warp -> (head group, row stream); lane -> (row group, vector of the row)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int hgn = (GC + HT - 1) / HT;
+    const int streams = NW / hgn;
+    const bool computes = warp < streams * hgn;
+    const int hg = warp % hgn, rs = warp / hgn;
+    const int lg = lane / LPG, sub = lane % LPG;
+    float sreg[HT][EV];
 #pragma unroll
-        for (int k = 0; k < RT; ++k) {
-            const int rho = base + rgi * RT + k;
-            ok[k] = rho < nR;
-            ii[k] = 0;
-            jj[k] = 0;
-            rp[k] = kbase + (size_t)(ok[k] ? row_of(rho, ii[k], jj[k]) : 0) * D;
+    for (int h = 0; h < HT; ++h) {
+        const int g = hg * HT + h;
+        const float *sp = p.s_ws + (size_t)(bh0 + (g < GC ? g : 0)) * D + sub * EV;
+#pragma unroll
+        for (int e = 0; e < EV; e += 4) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(sp + e);
+            sreg[h][e] = g < GC ? t4.x : 0.f;
+            sreg[h][e + 1] = g < GC ? t4.y : 0.f;
+            sreg[h][e + 2] = g < GC ? t4.z : 0.f;
+            sreg[h][e + 3] = g < GC ? t4.w : 0.f;
         }
-        float acc[HT][RT];
+    }
+    const int k_mine = sub / HT, g_mine = hg * HT + (sub - (sub / HT) * HT);
+    const bool stores = g_mine < GC;
+    const int16_t *kid_mine = kidx + (stores ? g_mine : 0) * total;
+    float *f_mine = f + (size_t)(bh0 + (stores ? g_mine : 0)) * fstride;
+
+    for (int tl = 0; tl < kScoreStages; ++tl)
+        if (tl < ntiles) build_info(tl);
+    __syncthreads();   // kidx and the first row tables are complete
 #pragma unroll
-        for (int h = 0; h < HT; ++h)
+    for (int st = 0; st < kScoreStages - 1; ++st) {
+        if (st < ntiles) load_tile(st);
+        else asm volatile("cp.async.commit_group;\n" ::);
+    }
+    for (int tl = 0; tl < ntiles; ++tl) {
+        asm volatile("cp.async.wait_group %0;\n" ::"n"(kScoreStages - 2));
+        __syncthreads();   // tile tl landed for every warp; tile tl-1's stage and row table are free
+        const int nx = tl + kScoreStages - 1;
+        if (nx < ntiles) load_tile(nx);
+        else asm volatile("cp.async.commit_group;\n" ::);
+        if (nx + 1 < ntiles) build_info(nx + 1);
+        if (!computes) continue;
+        const uint8_t *tb = tiles + (tl % kScoreStages) * TILEB;
+        const ScoreRow *ti = info + (tl % NINFO) * kScoreTile;
+        const int tile_rows = min(kScoreTile, nR - tl * kScoreTile);
+        for (int r0 = (rs * GPW + lg) * R; r0 < tile_rows; r0 += streams * GPW * R) {
+            float v[LPG];
 #pragma unroll
-            for (int k = 0; k < RT; ++k) acc[h][k] = 0.f;
-        uint4 cur[RT], nxt[RT];
+            for (int k = 0; k < R; ++k) {
+                float xf[EV];
+                Vec16<T>::unpack(*reinterpret_cast<const uint4 *>(tb + (r0 + k) * ROWB + sub * 16), xf);
 #pragma unroll
-        for (int k = 0; k < RT; ++k) cur[k] = ok[k] ? ldg16(rp[k]) : make_uint4(0, 0, 0, 0);
-#pragma unroll 2
-        for (int v = 0; v < VPR; ++v) {
-            if (v + 1 < VPR) {
+                for (int h = 0; h < HT; ++h) {
+                    float acc = 0.f;
 #pragma unroll
-                for (int k = 0; k < RT; ++k) nxt[k] = ok[k] ? ldg16(rp[k] + (v + 1) * EV) : make_uint4(0, 0, 0, 0);
-            }
-            float x[RT][EV];
-#pragma unroll
-            for (int k = 0; k < RT; ++k) Vec16<T>::unpack(cur[k], x[k]);
-#pragma unroll
-            for (int q = 0; q < EV; ++q) {
-                const float *sd = sh + (v * EV + q) * GPB;
-                float sv[HT];
-                if constexpr (HT % 4 == 0) {
-#pragma unroll
-                    for (int h4 = 0; h4 < HT; h4 += 4) {
-                        const float4 t4 = *reinterpret_cast<const float4 *>(sd + h4);
-                        sv[h4] = t4.x;
-                        sv[h4 + 1] = t4.y;
-                        sv[h4 + 2] = t4.z;
-                        sv[h4 + 3] = t4.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int h = 0; h < HT; ++h) sv[h] = sd[h];
+                    for (int e = 0; e < EV; ++e) acc = fmaf(sreg[h][e], xf[e], acc);
+                    v[k * HT + h] = acc;
                 }
-#pragma unroll
-                for (int h = 0; h < HT; ++h)
-#pragma unroll
-                    for (int k = 0; k < RT; ++k) acc[h][k] = fmaf(sv[h], x[k][q], acc[h][k]);
             }
+            // recursive halving over the LPG lanes of the group
 #pragma unroll
-            for (int k = 0; k < RT; ++k) cur[k] = nxt[k];
-        }
+            for (int m = LPG / 2; m >= 1; m >>= 1) {
+                const bool upper = (sub & m) != 0;
 #pragma unroll
-        for (int k = 0; k < RT; ++k) {
-            if (!ok[k]) continue;
-#pragma unroll
-            for (int h = 0; h < HT; ++h) {
-                const int g = hgi * HT + h;
-                if (g < GC) {
-                    const int kk = kidx[g * total + ii[k]];
-                    if (kk >= 0) f[(size_t)(bh0 + g) * fstride + (size_t)kk * fo + jj[k]] = acc[h][k];
+                for (int q = 0; q < m; ++q) {
+                    const float send = upper ? v[q] : v[q + m];
+                    const float keep = upper ? v[q + m] : v[q];
+                    v[q] = keep + __shfl_xor_sync(0xffffffffu, send, m);
                 }
+            }
+            const int rr = r0 + k_mine;
+            if (stores && rr < tile_rows) {
+                const ScoreRow sr = ti[rr];
+                const int kk = kid_mine[sr.i];
+                if (kk >= 0) f_mine[(size_t)kk * fo + sr.j] = v[0];
             }
         }
     }
+    asm volatile("cp.async.wait_group 0;\n" ::);
 }
 
 // ==========================================================================
