@@ -3,6 +3,8 @@
 // Host side: argument validation, workspace planning and kernel launches.  All
 // device work of atlaskv_attend runs in the kernels of descend.cuh,
 // staging.cuh and attend.cuh; nothing here computes on the host.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -337,21 +339,56 @@ atlaskv_status launch_attend_f32(const akv::AttnParams &ap, cudaStream_t s)
     return ATLASKV_OK;
 }
 
-// bf16, D = 128: tcgen05 tensor cores, one CTA per 128 query rows of a
-// (query, KV head) group.
+// Tensor map of a sequence K or V tensor [B][T][H_kv][D] (bf16, D = 128) for
+// the attention kernel: dims (D, H_kv, T, B), box (64, 1, 64, 1), 128-byte
+// swizzle, zero fill outside.  cuTensorMapEncodeTiled is a host-only call,
+// reached through the runtime's driver entry point.
+atlaskv_status encode_seq_map(CUtensorMap *map, const void *base, int B, int T, int H_kv)
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        cudaDriverEntryPointQueryResult q;
+        void *fn = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return fail(ATLASKV_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if (reinterpret_cast<uintptr_t>(base) & 15u) return fail(ATLASKV_EINVAL, "sequence K/V must be 16-byte aligned");
+    const int D = akv::tc::kD;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H_kv, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H_kv * D * 2, (cuuint64_t)T * H_kv * D * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)akv::tc::kKeys, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ATLASKV_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return ATLASKV_OK;
+}
+
+// bf16, D = 128: tcgen05 tensor cores, one CTA per 256 query rows of a
+// (query, KV head) group, sequence tiles by TMA.
 atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
 {
     const int rows = ap.G * ap.N;
-    const int bpg = (rows + akv::tc::kRows - 1) / akv::tc::kRows;
-    const long long grid = (long long)ap.B * ap.H_kv * bpg;
+    const int cpg = (rows + akv::tc::kCtaRows - 1) / akv::tc::kCtaRows;
+    const long long grid = (long long)ap.B * ap.H_kv * cpg;
     if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "attention grid too large");
+    if (ap.lk_rows >= (1LL << 31) || ap.lv_rows >= (1LL << 31))
+        return fail(ATLASKV_EUNSUPPORTED, "more than 2^31 leaf rows");
+    CUtensorMap mk, mv;
+    atlaskv_status st = encode_seq_map(&mk, ap.k_seq, ap.B, ap.T, ap.H_kv);
+    if (st != ATLASKV_OK) return st;
+    st = encode_seq_map(&mv, ap.v_seq, ap.B, ap.T, ap.H_kv);
+    if (st != ATLASKV_OK) return st;
     static bool configured = false;
     if (!configured) {
         AKV_CUDA(cudaFuncSetAttribute(akv::attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       akv::tc::kSmemBytes));
         configured = true;
     }
-    akv::attend_tc_kernel<<<(unsigned)grid, akv::tc::kThreads, akv::tc::kSmemBytes, s>>>(ap, bpg);
+    akv::attend_tc_kernel<<<(unsigned)grid, akv::tc::kThreads, akv::tc::kSmemBytes, s>>>(ap, cpg, mk, mv);
     AKV_CUDA(cudaGetLastError());
     return ATLASKV_OK;
 }
@@ -628,6 +665,7 @@ atlaskv_status atlaskv_attend(atlaskv_tree *t, const atlaskv_params *p, const at
         ap.lk_idx = kept[2];
         ap.lv_idx = kept[2];
         ap.leaf_head_stride = t->rows[2];
+        ap.lk_rows = ap.lv_rows = (long long)H_kv * t->rows[2];
         AKV_STEP(dispatch_attend(t->d.dtype, D, ap, s));
         AKV_STEP(mark(2));
     } else {
@@ -661,6 +699,8 @@ atlaskv_status atlaskv_attend(atlaskv_tree *t, const atlaskv_params *p, const at
         ap.lk_idx = kept_leaf_row;
         ap.lv_idx = vslot;
         ap.leaf_head_stride = 0;
+        ap.lk_rows = (long long)groups * n_mid * t->d.fanout[2];
+        ap.lv_rows = (long long)groups * n_leaf;
         AKV_STEP(dispatch_attend(t->d.dtype, D, ap, s));
         AKV_STEP(mark(5));
     }

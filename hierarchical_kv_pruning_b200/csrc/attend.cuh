@@ -20,6 +20,7 @@ struct AttnParams {
     const void *lk_base, *lv_base;   // leaf key / value row bases
     const int32_t *lk_idx, *lv_idx;  // [B H][K_L] row of each kept leaf
     long long leaf_head_stride;      // rows per KV head added to the index (0 when indices are absolute)
+    long long lk_rows, lv_rows;      // rows in the leaf key / value arrays
     void *out;                       // [B][N][H][D]
     float *lse;                      // [B][N][H] or null
     int B, N, H, H_kv, G, T, K_L;

@@ -4,21 +4,36 @@
 // Same computation as attend.cuh ("AtlasKV: Augmenting LLMs with Billion-Scale
 // Knowledge Graphs in 20GB VRAM": the lambda-weighted merge of the knowledge and
 // sequence softmaxes equals one softmax over both key sets), organised for
-// sm_100a:
-//   * a CTA of 4 warps owns 128 query rows of one (query b, KV head): row
-//     r = g N + n is token n of head g of the group, so the G heads of a KV head
-//     share every sequence K/V tile;
-//   * key tiles of 64 rows (first the CTA's heads' kept leaves, each visible
-//     only to its own head's rows, then the causal sequence tiles) are copied by
-//     cp.async into 128-byte-swizzled shared memory, double buffered;
-//   * one thread issues S = Q K^T (M 128, N 64, K 128) into TMEM, every thread
-//     reads back its own row of S (tcgen05.ld 32x32b), runs the online softmax
-//     and writes its row of P (bf16, swizzled) to shared memory; then one
-//     thread issues O_t = P V (M 128, N 128, K 64) into TMEM and every thread
-//     folds its row of O_t into its register accumulator;
-//   * tcgen05.commit arrives on an mbarrier when the issuing thread's MMAs are
-//     done; every wait is bounded and reports ETIMEOUT through the tree status.
+// sm_100a as a warp-specialised pipeline.  A CTA owns 256 query rows of one
+// (query b, KV head) group (row r = g N + n is token n of head g), in two
+// 128-row tiles, one per softmax warpgroup, and streams 64-key tiles shared by
+// both: first the causal sequence, then the kept leaves of the CTA's heads (each
+// visible only to its own head's rows); the online softmax is order-free.
+//
+//   producer warp   sequence K/V tiles by TMA (4-D tensor maps, 128-byte
+//                   swizzle) and gathered leaf rows by cp.async, into a K ring
+//                   (a stage is released as soon as S has read it) and a V
+//                   ring, each guarded by full / empty mbarriers;
+//   MMA warp        one thread issues S(w, t) = Q_w K_t^T (M 128, N 64,
+//                   K 128, both operands in shared memory) into a double-
+//                   buffered S in TMEM for both warpgroups, then
+//                   O_w += P_w V_{t-1} (M 128, N 128, K 64) with P_w read from
+//                   TMEM, so S(t) runs under softmax(t - 1); tcgen05.commit
+//                   arrives on the mbarriers;
+//   2 warpgroups    one thread per query row: read its S row (tcgen05.ld),
+//                   mask, online softmax with a lazily rescaled running max
+//                   (O in TMEM is rescaled only when the row max grows by more
+//                   than 2^8), P (bf16 pairs) written back over the first half
+//                   of the same S buffer (tcgen05.st), so P never touches
+//                   shared memory; finally O / l and the log-sum-exp.
+// Shared-memory bandwidth is what the tensor core waits on here (the MMA
+// operands plus the K/V copies); P in TMEM removes its store and its reread.
+//
+// Every mbarrier wait is bounded; a wait that gives up sets ETIMEOUT in the
+// tree's status word and the roles drain without further waits.
 #pragma once
+
+#include <cuda.h>
 
 #include "attend.cuh"
 #include "common.cuh"
@@ -26,31 +41,45 @@
 namespace akv {
 namespace tc {
 
-constexpr int kRows = 128;       // query rows per CTA (UMMA M)
-constexpr int kKeys = 64;        // keys per tile (UMMA N of QK^T, K of PV)
-constexpr int kD = 128;          // head dim
-constexpr int kThreads = 128;
+constexpr int kRows = 128;                 // query rows per warpgroup (UMMA M)
+constexpr int kKeys = 64;                  // keys per tile
+constexpr int kD = 128;                    // head dim
+constexpr int kWG = 2;                     // softmax warpgroups per CTA
+constexpr int kKStages = 4;                // K ring depth (a stage is freed when S = Q K^T completes)
+constexpr int kVStages = 3;                // V ring depth (freed when P V completes)
+constexpr int kProducerWarp = 4 * kWG;
+constexpr int kMmaWarp = 4 * kWG + 1;
+constexpr int kThreads = 32 * (4 * kWG + 2);
+constexpr int kCtaRows = kWG * kRows;
 constexpr long long kSpinLimit = 1ll << 22;   // bounded mbarrier waits (seconds at most)
+constexpr float kRescaleLog2 = 8.f;            // rescale O only when the row max grows by more than this
 
-// shared-memory layout (byte offsets; every operand region 1024-byte aligned).
-// P (the bf16 probabilities of the current tile) is written over the K tile of
-// the same stage once S = Q K^T has completed: that K tile is dead by then and
-// the next copy into the stage starts only after P V has completed.
-constexpr int kQBytes = kRows * kD * 2;            // 32 KB: 2 K-blocks of [128 rows][64]
-constexpr int kKVBytes = kKeys * kD * 2;           // 16 KB: 2 blocks of [64 keys][64]
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;             // 2 stages (P aliases the current one)
-constexpr int kOffV = kOffK + 2 * kKVBytes;        // 2 stages
-constexpr int kOffMeta = kOffV + 2 * kKVBytes;     // mbarriers, TMEM base
-constexpr int kMetaBytes = 1024;
-constexpr int kSmemBytes = kOffMeta + kMetaBytes + 1024;   // + slack to align the base to 1024
-constexpr int kTmemCols = 256;                     // S: columns [0, 64), O tile: [64, 192)
+// shared memory (byte offsets from a 1024-aligned base; operand tiles in the
+// canonical 128-byte-swizzled UMMA layouts)
+constexpr int kQBytes = kRows * kD * 2;       // 32 KB: 2 K-blocks of [128 rows][64]
+constexpr int kKVBytes = kKeys * kD * 2;      // 16 KB: 2 blocks of [64 keys][64]
+constexpr int kOffQ = 0;                                  // [kWG]
+constexpr int kOffK = kOffQ + kWG * kQBytes;              // [kKStages]
+constexpr int kOffV = kOffK + kKStages * kKVBytes;        // [kVStages]
+constexpr int kOffBar = kOffV + kVStages * kKVBytes;
+// mbarriers (8 bytes each); [kWG][2] arrays are indexed by warpgroup and tile parity
+constexpr int kBarFullK = 0;                        // [kKStages] K tile landed
+constexpr int kBarEmptyK = kBarFullK + kKStages;    // [kKStages] S of the tile done
+constexpr int kBarFullV = kBarEmptyK + kKStages;    // [kVStages] V tile landed
+constexpr int kBarEmptyV = kBarFullV + kVStages;    // [kVStages] P V of the tile done
+constexpr int kBarSFull = kBarEmptyV + kVStages;    // [kWG][2] S(w, t) in TMEM buffer t & 1
+constexpr int kBarPReady = kBarSFull + 2 * kWG;     // [kWG][2] P(w, t) written over it, O_w rescaled (4 warps)
+constexpr int kBarODone = kBarPReady + 2 * kWG;     // [kWG][2] O_w += P V from that buffer done
+constexpr int kBarQReady = kBarODone + 2 * kWG;     // [kWG] Q_w loaded (4 warps)
+constexpr int kNumBars = kBarQReady + kWG;
+constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024;   // + slack to align the base to 1024
+constexpr int kTmemCols = 512;                 // warpgroup w: S / P buffers [256 w, 256 w + 128), O [256 w + 128, 256 w + 256)
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
 // Byte offset of 16-byte chunk c (0..7) of row r inside a 128-byte-swizzled
-// block of rows that are 128 bytes long (the canonical SWIZZLE_128B atom:
-// chunk index XOR (row mod 8)).
+// block of 128-byte rows (the SWIZZLE_128B atom: chunk index XOR (row mod 8)).
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
 // UMMA shared-memory descriptor: SWIZZLE_128B, version 1 (sm_100).
@@ -86,6 +115,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t da, uint64_t 
         "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
 }
 
+// Same with the A operand (M x 16, K-major, 16-bit values packed in pairs
+// per 32-bit column: 8 columns per K step) read from TMEM.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+
 __device__ __forceinline__ void mma_commit(uint32_t mbar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar) : "memory");
@@ -96,7 +137,17 @@ __device__ __forceinline__ void mbar_init(uint32_t mbar, int count)
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count));
 }
 
-// Bounded wait for the given phase parity; returns false on timeout.
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
+}
+
+// Bounded wait for the phase with the given parity; false on timeout.
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity)
 {
     for (long long i = 0; i < kSpinLimit; ++i) {
@@ -132,7 +183,37 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
+// 2^x with the MUFU approximation (ex2.approx.ftz: relative error about
+// 2^-22, 2^-inf = 0); the probabilities are rounded to bf16 afterwards.
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void cp16(uint32_t dst, const void *src, bool valid)
 {
@@ -140,43 +221,61 @@ __device__ __forceinline__ void cp16(uint32_t dst, const void *src, bool valid)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(sz));
 }
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::); }
-__device__ __forceinline__ void cp_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::); }
+__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
+
+// TMA tile load of a 4-D box into shared memory, completion counted in bytes
+// on the mbarrier.  No multicast.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
+                                            uint32_t mbar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5}], [%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(mbar)
+        : "memory");
+}
 
 }  // namespace tc
 
-// One CTA per (query b, KV head, 128-row block of the group's G N rows).
-__global__ void __launch_bounds__(tc::kThreads, 2) attend_tc_kernel(const AttnParams p, int blocks_per_group)
+// One CTA per (query b, KV head, 256-row block of the group's G N rows).
+// tm_k / tm_v: the sequence keys / values [B][T][H_kv][D] as 4-D tensor maps
+// (D, H_kv, T, B) with a (64, 1, 64, 1) box and 128-byte swizzle.
+__global__ void __launch_bounds__(tc::kThreads, 1)
+    attend_tc_kernel(const AttnParams p, int ctas_per_group, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v)
 {
     using namespace tc;
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t sbase = smem_addr(smem);
-    // meta: mbarriers at +0 (S done) and +8 (O tile done), TMEM base at +64
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMeta + 64);
+    const uint32_t sb = smem_addr(smem);
+    auto bar = [&](int i) -> uint32_t { return sb + kOffBar + 8 * i; };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffTmemSlot);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int grp_id = blockIdx.x / blocks_per_group;
-    const int blk = blockIdx.x - grp_id * blocks_per_group;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp_id = blockIdx.x / ctas_per_group;
+    const int cta = blockIdx.x - grp_id * ctas_per_group;
     const int b = grp_id / p.H_kv, hkv = grp_id - b * p.H_kv;
     const int GN = p.G * p.N;
-    const int r0 = blk * kRows;
-    const int row = r0 + tid;                 // this thread's query row in the group
-    const bool row_ok = row < GN;
-    const int g = row_ok ? row / p.N : 0;
-    const int n = row_ok ? row - g * p.N : 0;
-    const int h = hkv * p.G + g;
-    const int last_key = p.T - p.N + n;       // causal limit of this row
-    const int g_first = r0 / p.N;
-    const int g_last = min(GN - 1, r0 + kRows - 1) / p.N;   // heads g_first..g_last own the rows
-    const int nheads = g_last - g_first + 1;
+    const int r0 = cta * kCtaRows;                       // first group row of the CTA
+    const int r_end = min(GN, r0 + kCtaRows) - 1;        // last valid one
+    const int g_first = r0 / p.N, g_last = r_end / p.N;  // heads g_first..g_last own the rows
+    const int n_leaf = (g_last - g_first + 1) * p.K_L;   // their kept leaves, head by head
+    const int n_leaf_tiles = (n_leaf + kKeys - 1) / kKeys;
+    // causal extent: the largest token index of the CTA is N - 1 when its rows
+    // span two heads, else that of its last row
+    const int cta_last = p.T - p.N + (r_end / p.N != r0 / p.N ? p.N - 1 : r_end % p.N);
+    const int n_seq_tiles = (cta_last + kKeys) / kKeys;
+    const int n_tiles = n_leaf_tiles + n_seq_tiles;
 
     if (tid == 0) {
-        mbar_init(sbase + kOffMeta, 1);
-        mbar_init(sbase + kOffMeta + 8, 1);
+        for (int i = 0; i < kNumBars; ++i) {
+            const bool per_warp = (i >= kBarPReady && i < kBarPReady + 2 * kWG) || (i >= kBarQReady);
+            mbar_init(bar(i), per_warp ? 4 : 1);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) {
+    if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
                      "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
@@ -185,225 +284,324 @@ __global__ void __launch_bounds__(tc::kThreads, 2) attend_tc_kernel(const AttnPa
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem;          // columns [0, 64): S
-    const uint32_t tO = tmem + 64;     // columns [64, 192): O tile
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
-    // Loads are mapped so that 16 consecutive threads copy the 16 chunks of
-    // one 256-byte row: a warp instruction reads two whole rows.
-    const int lc = tid & 15, lr = tid >> 4;   // chunk, first row of this thread
+    if (warp < 4 * kWG) {
+        // ================= softmax warpgroup w: one thread per query row =================
+        const int w = warp >> 2;
+        const int lrow = tid & (kRows - 1);                    // row of the Q tile = TMEM lane
+        const int row = r0 + w * kRows + lrow;
+        const bool row_ok = row < GN;
+        const int g = row_ok ? row / p.N : g_first;
+        const int n = row_ok ? row - g * p.N : 0;
+        const int h = hkv * p.G + g;
+        const int last_key = p.T - p.N + n;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + 256 * w, tO = tmem + 256 * w + 128;
+        const uint32_t qa = sb + kOffQ + w * kQBytes;
+        bool failed = false;
 
-    // ---- Q rows into the swizzled A tile ----
-    auto load_q = [&](const void *qptr) {
-        const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(qptr);
-        const uint32_t dst0 = sbase + kOffQ + (lc >> 3) * (kRows * 128);
+        // Q_w rows into the swizzled A tile: 16 consecutive threads per 256-byte row
+        auto load_q = [&](const void *qptr) {
+            const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(qptr);
+            const int lc = lrow & 15, lr = lrow >> 4;
+            const uint32_t dst0 = qa + (lc >> 3) * (kRows * 128);
 #pragma unroll 4
-        for (int i = 0; i < kRows / 8; ++i) {
-            const int r = lr + 8 * i, rr = r0 + r;
-            const bool ok = rr < GN;
-            const int gg = ok ? rr / p.N : 0, nn = ok ? rr - gg * p.N : 0;
-            const __nv_bfloat16 *src = q + (((size_t)b * p.N + nn) * p.H + hkv * p.G + gg) * kD + lc * 8;
-            cp16(dst0 + sw128(r, lc & 7), src, ok);
-        }
-        cp_commit();
-    };
-
-    // ---- key tile loaders (K and V rows into the swizzled tiles of a stage) ----
-    const __nv_bfloat16 *kseq = reinterpret_cast<const __nv_bfloat16 *>(p.k_seq);
-    const __nv_bfloat16 *vseq = reinterpret_cast<const __nv_bfloat16 *>(p.v_seq);
-    // row_src(key) -> (K row, V row) pointers or nullptr for a zero row
-    auto load_kv_rows = [&](int stage, auto row_src) {
-        const uint32_t off0 = (lc >> 3) * (kKeys * 128);
-        const uint32_t kb = sbase + kOffK + stage * kKVBytes + off0, vb = sbase + kOffV + stage * kKVBytes + off0;
-#pragma unroll
-        for (int i = 0; i < kKeys / 8; ++i) {
-            const int key = lr + 8 * i;
-            const __nv_bfloat16 *ks, *vs;
-            row_src(key, ks, vs);
-            const bool ok = ks != nullptr;
-            const uint32_t off = sw128(key, lc & 7);
-            cp16(kb + off, ok ? ks + lc * 8 : kseq, ok);
-            cp16(vb + off, ok ? vs + lc * 8 : vseq, ok);
-        }
-        cp_commit();
-    };
-
-    // leaf keys of the CTA's heads: nheads * K_L of them, head-major
-    const int n_leaf = nheads * p.K_L;
-    const int n_leaf_tiles = (n_leaf + kKeys - 1) / kKeys;
-    const __nv_bfloat16 *lkb = reinterpret_cast<const __nv_bfloat16 *>(p.lk_base);
-    const __nv_bfloat16 *lvb = reinterpret_cast<const __nv_bfloat16 *>(p.lv_base);
-    auto leaf_src = [&](int tile, int key, const __nv_bfloat16 *&ks, const __nv_bfloat16 *&vs) {
-        const int j = tile * kKeys + key;
-        if (j >= n_leaf) {
-            ks = vs = nullptr;
-            return;
-        }
-        const int gg = g_first + j / p.K_L, jj = j - (j / p.K_L) * p.K_L;
-        const long long e = ((long long)b * p.H + hkv * p.G + gg) * p.K_L + jj;
-        ks = lkb + (size_t)(p.leaf_head_stride * hkv + p.lk_idx[e]) * kD;
-        vs = lvb + (size_t)(p.leaf_head_stride * hkv + p.lv_idx[e]) * kD;
-    };
-    // causal extent of the CTA's rows
-    // causal extent of the CTA: its largest token index is N - 1 when its rows
-    // span two heads, else that of its last row
-    const int r_end = min(GN - 1, r0 + kRows - 1);
-    const int cta_last = p.T - p.N + (r_end / p.N != r0 / p.N ? p.N - 1 : r_end % p.N);
-    const int n_seq_tiles = (cta_last + kKeys) / kKeys;
-    const size_t seq_stride = (size_t)p.H_kv * kD;
-    const __nv_bfloat16 *kseq_b = kseq + ((size_t)b * p.T * p.H_kv + hkv) * kD;
-    const __nv_bfloat16 *vseq_b = vseq + ((size_t)b * p.T * p.H_kv + hkv) * kD;
-    auto issue_tile = [&](int t, int stage) {   // t < n_leaf_tiles: leaf tile; else sequence tile
-        if (t < n_leaf_tiles) {
-            load_kv_rows(stage, [&](int key, const __nv_bfloat16 *&ks, const __nv_bfloat16 *&vs) {
-                leaf_src(t, key, ks, vs);
-            });
-        } else {
-            const int t0 = (t - n_leaf_tiles) * kKeys;
-            load_kv_rows(stage, [&](int key, const __nv_bfloat16 *&ks, const __nv_bfloat16 *&vs) {
-                const bool ok = t0 + key < p.T;
-                ks = ok ? kseq_b + (size_t)(t0 + key) * seq_stride : nullptr;
-                vs = ok ? vseq_b + (size_t)(t0 + key) * seq_stride : nullptr;
-            });
-        }
-    };
-
-    const int n_tiles = n_leaf_tiles + n_seq_tiles;
-    const uint32_t idesc_s = make_idesc(kRows, kKeys, 0, 0);   // Q (K-major) x K^T (K-major)
-    const uint32_t idesc_o = make_idesc(kRows, kD, 0, 1);      // P (K-major) x V (MN-major)
-
-    float o[kD];
-#pragma unroll
-    for (int i = 0; i < kD; ++i) o[i] = 0.f;
-    float m = -INFINITY, l = 0.f;
-    const float sl2 = p.scale_log2;
-    bool failed = false;
-
-    load_q(p.q_kg);
-    issue_tile(0, 0);
-    for (int t = 0; t < n_tiles && !failed; ++t) {
-        const int stage = t & 1;
-        const bool leaf = t < n_leaf_tiles;
-        if (t == n_leaf_tiles) {
-            // switch A to the sequence queries (the previous MMAs finished: O waited below)
-            load_q(p.q_seq);
-        }
-        if (t + 1 < n_tiles) {
-            issue_tile(t + 1, stage ^ 1);
-            cp_wait_1();   // everything but the newest group: Q and tile t have landed
-        } else {
+            for (int i = 0; i < kRows / 8; ++i) {
+                const int rl = lr + 8 * i, rr = r0 + w * kRows + rl;
+                const bool ok = rr < GN;
+                const int gg = ok ? rr / p.N : 0, nn = ok ? rr - gg * p.N : 0;
+                const __nv_bfloat16 *src = q + (((size_t)b * p.N + nn) * p.H + hkv * p.G + gg) * kD + lc * 8;
+                cp16(dst0 + sw128(rl, lc & 7), src, ok);
+            }
+            cp_commit();
             cp_wait_all();
-        }
-        fence_async_smem();   // make this thread's cp.async data visible to the tensor cores
-        fence_before_sync();
-        __syncthreads();
-        fence_after_sync();
-        // ---- S = Q K^T ----
-        if (tid == 0) {
-            const uint32_t qa = sbase + kOffQ, kbase = sbase + kOffK + stage * kKVBytes;
-#pragma unroll
-            for (int s = 0; s < kD / 16; ++s) {
-                const uint64_t da = make_desc(qa + (s >> 2) * (kRows * 128) + (s & 3) * 32, 16, 1024);
-                const uint64_t db = make_desc(kbase + (s >> 2) * (kKeys * 128) + (s & 3) * 32, 16, 1024);
-                mma_bf16(tS, da, db, idesc_s, s > 0 ? 1u : 0u);
-            }
-            mma_commit(sbase + kOffMeta);
-        }
-        if (!mbar_wait(sbase + kOffMeta, (uint32_t)(t & 1))) failed = true;
-        fence_after_sync();
-        // ---- online softmax on this thread's row ----
-        float sc[kKeys];
-        tmem_ld32(tS + lane_off, sc);
-        tmem_ld32(tS + lane_off + 32, sc + 32);
-        tmem_wait_ld();
-        float mx = m;
-        // visible keys of this tile: [lo, hi) in tile-local index.  The leaves
-        // are stored head by head, K_L per head, so a row sees one contiguous
-        // run of them; a sequence tile is cut by the causal limit.
-        int lo, hi;
-        if (leaf) {
-            lo = (g - g_first) * p.K_L - t * kKeys;
-            hi = lo + p.K_L;
-        } else {
-            lo = 0;
-            hi = last_key + 1 - (t - n_leaf_tiles) * kKeys;
-        }
-        if (!row_ok) hi = lo;
-#pragma unroll
-        for (int j = 0; j < kKeys; ++j) {
-            sc[j] = (j >= lo && j < hi) ? sc[j] * sl2 : -INFINITY;
-            mx = fmaxf(mx, sc[j]);
-        }
-        const float base = mx == -INFINITY ? 0.f : mx;
-        const float alpha = exp2f(m - base);
-        m = mx;
-        float psum = 0.f;
-        uint32_t pk[kKeys / 2];
-#pragma unroll
-        for (int j = 0; j < kKeys; j += 2) {
-            const float e0 = exp2f(sc[j] - base), e1 = exp2f(sc[j + 1] - base);
-            psum += e0 + e1;
-            __nv_bfloat162 v2 = __floats2bfloat162_rn(e0, e1);
-            pk[j / 2] = *reinterpret_cast<uint32_t *>(&v2);
-        }
-        l = l * alpha + psum;
-        // row tid of P: 8 chunks of 16 bytes, swizzled
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            *reinterpret_cast<uint4 *>(smem + kOffK + stage * kKVBytes + sw128(tid, c)) = v;
-        }
-        fence_async_smem();
-        fence_before_sync();
-        __syncthreads();
-        fence_after_sync();
-        // ---- O_t = P V ----
-        if (tid == 0) {
-            const uint32_t pa = sbase + kOffK + stage * kKVBytes, vbase = sbase + kOffV + stage * kKVBytes;
-#pragma unroll
-            for (int s = 0; s < kKeys / 16; ++s) {
-                const uint64_t da = make_desc(pa + s * 32, 16, 1024);
-                const uint64_t db = make_desc(vbase + s * 16 * 128, kKeys * 128, 1024);
-                mma_bf16(tO, da, db, idesc_o, s > 0 ? 1u : 0u);
-            }
-            mma_commit(sbase + kOffMeta + 8);
-        }
-        if (!mbar_wait(sbase + kOffMeta + 8, (uint32_t)(t & 1))) failed = true;
-        fence_after_sync();
-#pragma unroll
-        for (int c = 0; c < kD; c += 32) {
-            float ot[32];
-            tmem_ld32(tO + lane_off + c, ot);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[c + i] = fmaf(o[c + i], alpha, ot[i]);
-        }
-        fence_before_sync();
-        failed = __syncthreads_or(failed);
-    }
-    if (failed && tid == 0) set_status(p.status, kDevTimeout);
-    cp_wait_all();
+            fence_async_smem();   // visible to the tensor cores once the barrier is passed
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarQReady + w));
+        };
+        load_q(p.q_seq);
 
-    // ---- epilogue: this thread's row ----
-    if (row_ok && !failed) {
-        const float inv = 1.f / l;
-        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.out) + (((size_t)b * p.N + n) * p.H + h) * kD;
+        const float sl2 = p.scale_log2;
+        float m_used = -INFINITY, l = 0.f;
+        for (int t = 0; t < n_tiles; ++t) {
+            const int bs = t & 1;
+            failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarSFull + 2 * w + bs), (t >> 1) & 1));
+            if (failed) break;
+            fence_after_sync();
+            float sc[kKeys];
+            tmem_ld32(tS + 64 * bs + lane_off, sc);
+            tmem_ld32(tS + 64 * bs + 32 + lane_off, sc + 32);
+            tmem_wait_ld();
+            // S(w, last sequence tile) has completed: Q_w may now be replaced by q_kg
+            if (t == n_seq_tiles - 1 && n_leaf_tiles > 0) load_q(p.q_kg);
+
+            // visible keys of this tile, [lo, hi) in tile-local index: the leaves
+            // are stored head by head, K_L per head; a sequence tile is cut by
+            // the causal limit
+            int lo, hi;
+            if (t >= n_seq_tiles) {
+                lo = (g - g_first) * p.K_L - (t - n_seq_tiles) * kKeys;
+                hi = lo + p.K_L;
+            } else {
+                lo = 0;
+                hi = last_key + 1 - t * kKeys;
+            }
+            if (!row_ok) hi = lo;
+            if (!(lo <= 0 && hi >= kKeys)) {
 #pragma unroll
-        for (int c = 0; c < kD; c += 8) {
-            __nv_bfloat162 a0 = __floats2bfloat162_rn(o[c] * inv, o[c + 1] * inv);
-            __nv_bfloat162 a1 = __floats2bfloat162_rn(o[c + 2] * inv, o[c + 3] * inv);
-            __nv_bfloat162 a2 = __floats2bfloat162_rn(o[c + 4] * inv, o[c + 5] * inv);
-            __nv_bfloat162 a3 = __floats2bfloat162_rn(o[c + 6] * inv, o[c + 7] * inv);
-            uint4 v = make_uint4(*reinterpret_cast<uint32_t *>(&a0), *reinterpret_cast<uint32_t *>(&a1),
-                                 *reinterpret_cast<uint32_t *>(&a2), *reinterpret_cast<uint32_t *>(&a3));
-            *reinterpret_cast<uint4 *>(dst + c) = v;
+                for (int j = 0; j < kKeys; ++j) sc[j] = (j >= lo && j < hi) ? sc[j] : -INFINITY;
+            }
+            // row max with 8 independent chains
+            float mx8[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mx8[k] = sc[k];
+#pragma unroll
+            for (int j = 8; j < kKeys; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], sc[j]);
+            const float tmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            const float m_new = fmaxf(m_used, tmax * sl2);   // scores in log2 units (sl2 > 0)
+            if (t == 0) {
+                m_used = m_new;   // O_w is initialised by the first P V
+            } else {
+                const bool need = m_new > m_used + kRescaleLog2;   // also when m_used is still -inf
+                if (__any_sync(0xffffffffu, need)) {
+                    // O_w may be rescaled only once the previous P V has landed in it
+                    failed = __any_sync(0xffffffffu,
+                                        !mbar_wait(bar(kBarODone + 2 * w + ((t - 1) & 1)), ((t - 1) >> 1) & 1));
+                    if (failed) break;
+                    fence_after_sync();
+                    const float f = need ? fast_exp2(m_used - m_new) : 1.f;
+#pragma unroll
+                    for (int c = 0; c < kD; c += 32) {
+                        float ov[32];
+                        tmem_ld32(tO + lane_off + c, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) ov[i] *= f;
+                        tmem_st32(tO + lane_off + c, ov);
+                    }
+                    tmem_wait_st();
+                    if (need) {
+                        l *= f;
+                        m_used = m_new;
+                    }
+                }
+            }
+            float psum = 0.f;
+            uint32_t pk[kKeys / 2];
+            if (m_used != -INFINITY) {
+                const float neg = -m_used;
+                float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int j = 0; j < kKeys; j += 2) {
+                    const float e0 = fast_exp2(fmaf(sc[j], sl2, neg));
+                    const float e1 = fast_exp2(fmaf(sc[j + 1], sl2, neg));
+                    ps8[(j >> 1) & 7] += e0 + e1;
+                    __nv_bfloat162 v2 = __floats2bfloat162_rn(e0, e1);
+                    pk[j / 2] = *reinterpret_cast<uint32_t *>(&v2);
+                }
+                psum = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+            } else {
+#pragma unroll
+                for (int j = 0; j < kKeys / 2; ++j) pk[j] = 0u;
+            }
+            l += psum;
+            // P(t) over the first 32 columns of S buffer bs (bf16 pairs: key 2c in
+            // the low half of column c), the A operand of P V
+            tmem_st32(tS + 64 * bs + lane_off, reinterpret_cast<const float *>(pk));
+            tmem_wait_st();
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarPReady + 2 * w + bs));
         }
-        if (p.lse) p.lse[((size_t)b * p.N + n) * p.H + h] = (m + log2f(l)) * 0.69314718055994530942f;
+        if (!failed) {
+            failed = __any_sync(0xffffffffu,
+                                !mbar_wait(bar(kBarODone + 2 * w + ((n_tiles - 1) & 1)), ((n_tiles - 1) >> 1) & 1));
+            fence_after_sync();
+        }
+        if (!failed) {
+            const float inv = 1.f / l;
+            __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.out) + (((size_t)b * p.N + n) * p.H + h) * kD;
+#pragma unroll
+            for (int c = 0; c < kD; c += 32) {
+                float ov[32];
+                tmem_ld32(tO + lane_off + c, ov);
+                tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        __nv_bfloat162 a0 = __floats2bfloat162_rn(ov[i] * inv, ov[i + 1] * inv);
+                        __nv_bfloat162 a1 = __floats2bfloat162_rn(ov[i + 2] * inv, ov[i + 3] * inv);
+                        __nv_bfloat162 a2 = __floats2bfloat162_rn(ov[i + 4] * inv, ov[i + 5] * inv);
+                        __nv_bfloat162 a3 = __floats2bfloat162_rn(ov[i + 6] * inv, ov[i + 7] * inv);
+                        *reinterpret_cast<uint4 *>(dst + c + i) =
+                            make_uint4(*reinterpret_cast<uint32_t *>(&a0), *reinterpret_cast<uint32_t *>(&a1),
+                                       *reinterpret_cast<uint32_t *>(&a2), *reinterpret_cast<uint32_t *>(&a3));
+                    }
+                }
+            }
+            if (row_ok && p.lse) p.lse[((size_t)b * p.N + n) * p.H + h] = (m_used + log2f(l)) * 0.69314718055994530942f;
+        }
+        if (failed && lane == 0) set_status(p.status, kDevTimeout);
+    } else if (warp == kProducerWarp) {
+        // ================= producer: K and V tiles into their rings =================
+        const __nv_bfloat16 *lkb = reinterpret_cast<const __nv_bfloat16 *>(p.lk_base);
+        const __nv_bfloat16 *lvb = reinterpret_cast<const __nv_bfloat16 *>(p.lv_base);
+        bool failed = false;
+        int pending = -1;   // leaf tile whose cp.async copies are in flight, not yet announced
+        // leaf rows of keys `lane` and `lane + 32` of leaf tile lt (-1: none), fetched one tile ahead
+        auto fetch_rows = [&](int lt, int *rk, int *rv) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int j = lt * kKeys + lane + 32 * u;
+                rk[u] = rv[u] = -1;
+                if (j < n_leaf) {
+                    const int gg = g_first + j / p.K_L, jj = j - (j / p.K_L) * p.K_L;
+                    const long long e = ((long long)b * p.H + hkv * p.G + gg) * p.K_L + jj;
+                    rk[u] = (int)(p.leaf_head_stride * hkv + p.lk_idx[e]);
+                    rv[u] = (int)(p.leaf_head_stride * hkv + p.lv_idx[e]);
+                }
+            }
+        };
+        // cp.async of 64 gathered rows (two per warp instruction, 16 lanes per 256-byte row)
+        auto gather = [&](uint32_t dst, const __nv_bfloat16 *base, const int *rows2) {
+            const int c = lane & 15;
+#pragma unroll 4
+            for (int i = 0; i < kKeys / 2; ++i) {
+                const int r = 2 * i + (lane >> 4);
+                const int x = __shfl_sync(0xffffffffu, i < 16 ? rows2[0] : rows2[1], r & 31);
+                cp16(dst + (c >> 3) * (kKeys * 128) + sw128(r, c & 7), x >= 0 ? base + (size_t)x * kD + c * 8 : base,
+                     x >= 0);
+            }
+            cp_commit();
+        };
+        // announce the pending leaf tile once its copies have landed (newer: groups committed after it)
+        auto announce = [&](int newer) {
+            if (newer) cp_wait_1();
+            else cp_wait_all();
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(kBarFullK + pending % kKStages));
+                mbar_arrive(bar(kBarFullV + pending % kVStages));
+            }
+            pending = -1;
+        };
+        int nk[2] = {-1, -1}, nv[2] = {-1, -1};
+        if (n_leaf_tiles > 0) fetch_rows(0, nk, nv);
+        for (int t = 0; t < n_tiles; ++t) {
+            const int sk = t % kKStages, sv = t % kVStages;
+            const bool leaf = t >= n_seq_tiles;
+            const uint32_t kd = sb + kOffK + sk * kKVBytes, vd = sb + kOffV + sv * kKVBytes;
+            if (t >= kKStages) {
+                failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarEmptyK + sk), ((t / kKStages) + 1) & 1));
+                if (failed) break;
+            }
+            int rk[2] = {-1, -1}, rv[2] = {-1, -1};
+            if (leaf) {
+                rk[0] = nk[0];
+                rk[1] = nk[1];
+                rv[0] = nv[0];
+                rv[1] = nv[1];
+                const int lt = t - n_seq_tiles;
+                if (lt + 1 < n_leaf_tiles) fetch_rows(lt + 1, nk, nv);
+                gather(kd, lkb, rk);
+            } else {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(kBarFullK + sk), kKVBytes);
+#pragma unroll
+                    for (int half = 0; half < 2; ++half)
+                        tma_load_4d(kd + half * (kKeys * 128), &tm_k, half * 64, hkv, t * kKeys, b, bar(kBarFullK + sk));
+                }
+                __syncwarp();
+            }
+            // the previous leaf tile goes out before any wait on a V stage
+            if (pending >= 0) announce(leaf ? 1 : 0);
+            if (t >= kVStages) {
+                failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarEmptyV + sv), ((t / kVStages) + 1) & 1));
+                if (failed) break;
+            }
+            if (leaf) {
+                gather(vd, lvb, rv);
+                pending = t;
+            } else {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(kBarFullV + sv), kKVBytes);
+#pragma unroll
+                    for (int half = 0; half < 2; ++half)
+                        tma_load_4d(vd + half * (kKeys * 128), &tm_v, half * 64, hkv, t * kKeys, b, bar(kBarFullV + sv));
+                }
+                __syncwarp();
+            }
+        }
+        if (!failed && pending >= 0) announce(0);
+        // the CTA must not exit with copies in flight: wait until the last tile of each stage has landed
+        if (!failed) {
+            for (int t = max(0, n_tiles - kKStages); t < n_tiles; ++t)
+                failed |= !mbar_wait(bar(kBarFullK + t % kKStages), (t / kKStages) & 1);
+            for (int t = max(0, n_tiles - kVStages); t < n_tiles; ++t)
+                failed |= !mbar_wait(bar(kBarFullV + t % kVStages), (t / kVStages) & 1);
+        }
+        cp_wait_all();
+        if (failed && lane == 0) set_status(p.status, kDevTimeout);
+    } else {
+        // ================= MMA issue: one thread =================
+        if (lane == 0) {
+            const uint32_t idesc_s = make_idesc(kRows, kKeys, 0, 0);   // Q (K-major) x K^T (K-major)
+            const uint32_t idesc_o = make_idesc(kRows, kD, 0, 1);      // P (K-major) x V (MN-major)
+            auto issue_s = [&](int t) -> bool {
+                const int sk = t % kKStages, bs = t & 1;
+                if (!mbar_wait(bar(kBarFullK + sk), (t / kKStages) & 1)) return false;
+                for (int w = 0; w < kWG; ++w) {
+                    if (t == 0 && !mbar_wait(bar(kBarQReady + w), 0)) return false;
+                    if (t == n_seq_tiles && n_leaf_tiles > 0 && !mbar_wait(bar(kBarQReady + w), 1)) return false;
+                    // buffer bs still holds P(t - 2) until its P V has completed
+                    if (t >= 2 && !mbar_wait(bar(kBarODone + 2 * w + bs), ((t - 2) >> 1) & 1)) return false;
+                    fence_after_sync();
+                    const uint32_t qa = sb + kOffQ + w * kQBytes, kb = sb + kOffK + sk * kKVBytes;
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const uint64_t da = make_desc(qa + (ks >> 2) * (kRows * 128) + (ks & 3) * 32, 16, 1024);
+                        const uint64_t db = make_desc(kb + (ks >> 2) * (kKeys * 128) + (ks & 3) * 32, 16, 1024);
+                        mma_bf16(tmem + 256 * w + 64 * bs, da, db, idesc_s, ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(kBarSFull + 2 * w + bs));
+                }
+                mma_commit(bar(kBarEmptyK + sk));
+                return true;
+            };
+            auto issue_pv = [&](int u) -> bool {
+                const int sv = u % kVStages, bs = u & 1;
+                if (!mbar_wait(bar(kBarFullV + sv), (u / kVStages) & 1)) return false;
+                for (int w = 0; w < kWG; ++w) {
+                    if (!mbar_wait(bar(kBarPReady + 2 * w + bs), (u >> 1) & 1)) return false;
+                    fence_after_sync();
+                    const uint32_t ta = tmem + 256 * w + 64 * bs, vb = sb + kOffV + sv * kKVBytes;
+#pragma unroll
+                    for (int ks = 0; ks < kKeys / 16; ++ks) {
+                        const uint64_t db = make_desc(vb + ks * 16 * 128, kKeys * 128, 1024);
+                        mma_bf16_ts(tmem + 256 * w + 128, ta + 8 * ks, db, idesc_o, (u > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bar(kBarODone + 2 * w + bs));
+                }
+                mma_commit(bar(kBarEmptyV + sv));
+                return true;
+            };
+            bool ok = true;
+            for (int t = 0; t < n_tiles && ok; ++t) {
+                ok = issue_s(t);
+                if (ok && t > 0) ok = issue_pv(t - 1);
+            }
+            if (ok) ok = issue_pv(n_tiles - 1);
+            if (!ok) set_status(p.status, kDevTimeout);
+        }
+        __syncwarp();
     }
+
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    if (warp == kMmaWarp) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
 }  // namespace akv
