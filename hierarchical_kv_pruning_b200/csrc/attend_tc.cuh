@@ -549,6 +549,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         if (lane == 0) {
             const uint32_t idesc_s = make_idesc(kRows, kKeys, 0, 0);   // Q (K-major) x K^T (K-major)
             const uint32_t idesc_o = make_idesc(kRows, kD, 0, 1);      // P (K-major) x V (MN-major)
+            // descriptors of the first tile of each operand region; a tile or
+            // K-step offset is added to the start-address field (the low 14 bits,
+            // in 16-byte units: shared addresses stay below 256 KB, so no carry)
+            const uint64_t dq0 = make_desc(sb + kOffQ, 16, 1024);
+            const uint64_t dk0 = make_desc(sb + kOffK, 16, 1024);
+            const uint64_t dv0 = make_desc(sb + kOffV, kKeys * 128, 1024);
             auto issue_s = [&](int t) -> bool {
                 const int sk = t % kKStages, bs = t & 1;
                 if (!mbar_wait(bar(kBarFullK + sk), (t / kKStages) & 1)) return false;
@@ -558,12 +564,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                     // buffer bs still holds P(t - 2) until its P V has completed
                     if (t >= 2 && !mbar_wait(bar(kBarODone + 2 * w + bs), ((t - 2) >> 1) & 1)) return false;
                     fence_after_sync();
-                    const uint32_t qa = sb + kOffQ + w * kQBytes, kb = sb + kOffK + sk * kKVBytes;
+                    const uint64_t qd = dq0 + (uint64_t)((w * kQBytes) >> 4);
+                    const uint64_t kdsc = dk0 + (uint64_t)((sk * kKVBytes) >> 4);
+                    const uint32_t td = tmem + 256 * w + 64 * bs;
 #pragma unroll
                     for (int ks = 0; ks < kD / 16; ++ks) {
-                        const uint64_t da = make_desc(qa + (ks >> 2) * (kRows * 128) + (ks & 3) * 32, 16, 1024);
-                        const uint64_t db = make_desc(kb + (ks >> 2) * (kKeys * 128) + (ks & 3) * 32, 16, 1024);
-                        mma_bf16(tmem + 256 * w + 64 * bs, da, db, idesc_s, ks > 0 ? 1u : 0u);
+                        mma_bf16(td, qd + (uint64_t)(((ks >> 2) * (kRows * 128) + (ks & 3) * 32) >> 4),
+                                 kdsc + (uint64_t)(((ks >> 2) * (kKeys * 128) + (ks & 3) * 32) >> 4), idesc_s,
+                                 ks > 0 ? 1u : 0u);
                     }
                     mma_commit(bar(kBarSFull + 2 * w + bs));
                 }
@@ -576,12 +584,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                 for (int w = 0; w < kWG; ++w) {
                     if (!mbar_wait(bar(kBarPReady + 2 * w + bs), (u >> 1) & 1)) return false;
                     fence_after_sync();
-                    const uint32_t ta = tmem + 256 * w + 64 * bs, vb = sb + kOffV + sv * kKVBytes;
+                    const uint32_t ta = tmem + 256 * w + 64 * bs, td = tmem + 256 * w + 128;
+                    const uint64_t vdsc = dv0 + (uint64_t)((sv * kKVBytes) >> 4);
 #pragma unroll
-                    for (int ks = 0; ks < kKeys / 16; ++ks) {
-                        const uint64_t db = make_desc(vb + ks * 16 * 128, kKeys * 128, 1024);
-                        mma_bf16_ts(tmem + 256 * w + 128, ta + 8 * ks, db, idesc_o, (u > 0 || ks > 0) ? 1u : 0u);
-                    }
+                    for (int ks = 0; ks < kKeys / 16; ++ks)
+                        mma_bf16_ts(td, ta + 8 * ks, vdsc + (uint64_t)((ks * 16 * 128) >> 4), idesc_o,
+                                    (u > 0 || ks > 0) ? 1u : 0u);
                     mma_commit(bar(kBarODone + 2 * w + bs));
                 }
                 mma_commit(bar(kBarEmptyV + sv));
