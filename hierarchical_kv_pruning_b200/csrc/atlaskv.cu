@@ -53,6 +53,12 @@ int pow2_at_least(long long x, int floor_)
 
 constexpr int kMaxCandidates = 8192;   // per level and traversal (shared-memory bound of the descent CTA)
 constexpr int kNumEvents = 6;
+// Host-resident leaves: the batch is split into up to kMaxChunks query chunks
+// so that staging one chunk's leaf blocks over the host link overlaps the
+// scoring and attention of the others (a second stream owned by the tree).
+constexpr int kMaxChunks = 4;
+constexpr int kChunkEvents = 4;          // per chunk: mids kept, keys staged, leaves kept, values staged
+constexpr int kTimingEvents = 10;        // per chunk: begin / end of 5 segments
 
 }  // namespace
 
@@ -73,7 +79,11 @@ struct atlaskv_tree {
     bool profiling;
     bool timed;                    // the last attend recorded events
     bool host_mode_last;
+    int chunks_last;
     cudaEvent_t ev[kNumEvents];
+    cudaStream_t stage_stream;                        // host leaves: staging copies
+    cudaEvent_t cev[kMaxChunks * kChunkEvents + 1];   // cross-stream ordering (+1: start)
+    cudaEvent_t tev[kMaxChunks * kTimingEvents];      // segment timing while profiling
 };
 
 namespace {
@@ -113,7 +123,7 @@ Layout plan(const atlaskv_tree *t, const atlaskv_params *p, int B, int N, int H,
     L.anorm_ws = take(BH * 4);
     L.f_ws = take(BH * (size_t)L.fstride * 4);
     L.queue = take(3 * BH * 4 * 4);
-    L.qcount = take(4 * 4);
+    L.qcount = take(kMaxChunks * 4 * 4);   // per query chunk: [3] exact-pass queue lengths
     for (int l = 0; l < 3; ++l) L.kept[l] = take(BH * (size_t)(l == 0 ? p->K_root : l == 1 ? p->K_mid : p->K_leaf) * 4);
     if (host) {
         const int G = H / t->d.n_kv_heads;
@@ -400,6 +410,18 @@ atlaskv_status dispatch_attend(int dtype, int D, const akv::AttnParams &ap, cuda
 }
 
 // ---- staging launches -----------------------------------------------------
+int num_sms()
+{
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
 atlaskv_status launch_dedupe(const int32_t *ids, int n, int groups, int32_t *uniq, int32_t *slot, int32_t *count,
                              cudaStream_t s)
 {
@@ -419,7 +441,7 @@ template <typename T, int D>
 atlaskv_status stage_keys(const atlaskv_tree *t, const int32_t *umid, const int32_t *cnt, int n, int groups,
                           void *pool, cudaStream_t s)
 {
-    akv::stage_leaf_blocks_kernel<T, D><<<592, 256, 0, s>>>(
+    akv::stage_leaf_blocks_kernel<T, D><<<akv::kStageCtasPerSm * num_sms(), 256, 0, s>>>(
         reinterpret_cast<const T *>(t->leaf_keys_dev), t->d.mid_child, t->rows[1], t->rows[2], t->d.fanout[2],
         t->d.n_kv_heads, umid, cnt, n, groups, reinterpret_cast<T *>(pool), t->status);
     AKV_CUDA(cudaGetLastError());
@@ -430,7 +452,7 @@ template <typename T, int D>
 atlaskv_status stage_values(const atlaskv_tree *t, const int32_t *uleaf, const int32_t *cnt, int n, int groups,
                             void *vpool, cudaStream_t s)
 {
-    akv::stage_value_rows_kernel<T, D><<<592, 256, 0, s>>>(reinterpret_cast<const T *>(t->leaf_values_dev), t->rows[2],
+    akv::stage_value_rows_kernel<T, D><<<akv::kStageCtasPerSm * num_sms(), 256, 0, s>>>(reinterpret_cast<const T *>(t->leaf_values_dev), t->rows[2],
                                                           t->d.n_kv_heads, uleaf, cnt, n, groups,
                                                           reinterpret_cast<T *>(vpool));
     AKV_CUDA(cudaGetLastError());
@@ -669,40 +691,121 @@ atlaskv_status atlaskv_attend(atlaskv_tree *t, const atlaskv_params *p, const at
         AKV_STEP(dispatch_attend(t->d.dtype, D, ap, s));
         AKV_STEP(mark(2));
     } else {
-        const int groups = io->B * H_kv;
+        // Query chunks: chunk c covers queries [b0, b0 + Bc).  The caller's
+        // stream runs the descent and the attention of each chunk; the staging
+        // stream copies the chunk's leaf-key blocks once its mids are kept and
+        // its value rows once its leaves are kept, so the host link works while
+        // the other chunks compute.
+        const int nc = io->B >= 2 * kMaxChunks ? kMaxChunks : 1;
+        if (!t->stage_stream) {
+            // highest priority: the copies are bound by the host link, so the
+            // block scheduler should keep them resident and let the compute fill in
+            int lo_prio = 0, hi_prio = 0;
+            AKV_CUDA(cudaDeviceGetStreamPriorityRange(&lo_prio, &hi_prio));
+            AKV_CUDA(cudaStreamCreateWithPriority(&t->stage_stream, cudaStreamNonBlocking, hi_prio));
+            for (cudaEvent_t &e : t->cev) AKV_CUDA(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+        }
+        if (prof && !t->tev[0])
+            for (cudaEvent_t &e : t->tev) AKV_CUDA(cudaEventCreate(&e));
+        cudaStream_t s1 = t->stage_stream;
         const int n_mid = G * p->K_mid, n_leaf = G * p->K_leaf;
-        int32_t *leaf_slot = reinterpret_cast<int32_t *>(ws + L.leaf_slot);
-        int32_t *kept_leaf_row = reinterpret_cast<int32_t *>(ws + L.kept_leaf_row);
-        int32_t *vslot = reinterpret_cast<int32_t *>(ws + L.vslot);
-        int32_t *umid = reinterpret_cast<int32_t *>(ws + L.umid);
-        int32_t *cmid = reinterpret_cast<int32_t *>(ws + L.ucount_mid);
-        int32_t *uleaf = reinterpret_cast<int32_t *>(ws + L.uleaf);
-        int32_t *cleaf = reinterpret_cast<int32_t *>(ws + L.ucount_leaf);
-        void *pool = ws + L.key_pool;
-        void *vpool = ws + L.val_pool;
-        AKV_STEP(mark(0));
-        AKV_STEP(dispatch_descend(t->d.dtype, D, dp, 0, 1, s));
-        AKV_STEP(mark(1));
-        AKV_STEP(launch_dedupe(kept[1], n_mid, groups, umid, leaf_slot, cmid, s));
-        AKV_STEP(dispatch_stage_keys(t, umid, cmid, n_mid, groups, pool, s));
-        AKV_STEP(mark(2));
-        dp.keys[2] = pool;
-        dp.leaf_slot = leaf_slot;
-        dp.kept_leaf_row = kept_leaf_row;
-        AKV_STEP(dispatch_descend(t->d.dtype, D, dp, 2, 2, s));
-        AKV_STEP(mark(3));
-        AKV_STEP(launch_dedupe(kept[2], n_leaf, groups, uleaf, vslot, cleaf, s));
-        AKV_STEP(dispatch_stage_values(t, uleaf, cleaf, n_leaf, groups, vpool, s));
-        AKV_STEP(mark(4));
-        ap.lk_base = pool;
-        ap.lv_base = vpool;
-        ap.lk_idx = kept_leaf_row;
-        ap.lv_idx = vslot;
-        ap.leaf_head_stride = 0;
-        ap.lk_rows = (long long)groups * n_mid * t->d.fanout[2];
-        ap.lv_rows = (long long)groups * n_leaf;
-        AKV_STEP(dispatch_attend(t->d.dtype, D, ap, s));
-        AKV_STEP(mark(5));
+        const size_t esz = esize(t->d.dtype);
+        auto cev = [&](int c, int k) { return t->cev[c * kChunkEvents + k]; };
+        auto tmark = [&](int c, int k, cudaStream_t st) -> atlaskv_status {
+            if (prof) AKV_CUDA(cudaEventRecord(t->tev[c * kTimingEvents + k], st));
+            return ATLASKV_OK;
+        };
+        akv::DescendParams dpc[kMaxChunks];
+        akv::AttnParams apc[kMaxChunks];
+        int32_t *umid[kMaxChunks], *cmid[kMaxChunks], *uleaf[kMaxChunks], *cleaf[kMaxChunks];
+        int32_t *leaf_slot[kMaxChunks], *vslot[kMaxChunks];
+        int groups[kMaxChunks];
+        for (int c = 0; c < nc; ++c) {
+            const int b0 = (int)((long long)io->B * c / nc), b1 = (int)((long long)io->B * (c + 1) / nc);
+            const int Bc = b1 - b0;
+            const size_t bh0 = (size_t)b0 * io->H, g0 = (size_t)b0 * H_kv;
+            groups[c] = Bc * H_kv;
+            akv::DescendParams d = dp;
+            d.B = Bc;
+            d.q_kg = reinterpret_cast<const uint8_t *>(io->q_kg) + (size_t)b0 * io->N * io->H * D * esz;
+            for (int l = 0; l < 3; ++l) d.kept[l] = kept[l] + bh0 * dp.K[l];
+            d.s_ws = dp.s_ws + bh0 * D;
+            d.s64_ws = dp.s64_ws + bh0 * D;
+            d.a64_ws = dp.a64_ws + bh0 * D;
+            d.anorm_ws = dp.anorm_ws + bh0;
+            d.f_ws = dp.f_ws + bh0 * (size_t)L.fstride;
+            d.qcount = dp.qcount + 4 * c;
+            leaf_slot[c] = reinterpret_cast<int32_t *>(ws + L.leaf_slot) + bh0 * p->K_mid;
+            vslot[c] = reinterpret_cast<int32_t *>(ws + L.vslot) + bh0 * p->K_leaf;
+            umid[c] = reinterpret_cast<int32_t *>(ws + L.umid) + g0 * n_mid;
+            cmid[c] = reinterpret_cast<int32_t *>(ws + L.ucount_mid) + g0;
+            uleaf[c] = reinterpret_cast<int32_t *>(ws + L.uleaf) + g0 * n_leaf;
+            cleaf[c] = reinterpret_cast<int32_t *>(ws + L.ucount_leaf) + g0;
+            uint8_t *pool = ws + L.key_pool + g0 * n_mid * (size_t)t->d.fanout[2] * D * esz;
+            uint8_t *vpool = ws + L.val_pool + g0 * n_leaf * (size_t)D * esz;
+            int32_t *kept_leaf_row = reinterpret_cast<int32_t *>(ws + L.kept_leaf_row) + bh0 * p->K_leaf;
+            d.keys[2] = pool;
+            d.leaf_slot = leaf_slot[c];
+            d.kept_leaf_row = kept_leaf_row;
+            dpc[c] = d;
+            akv::AttnParams a = ap;
+            a.B = Bc;
+            const size_t qoff = (size_t)b0 * io->N * io->H * D * esz, kvoff = (size_t)b0 * io->T * H_kv * D * esz;
+            a.q_kg = reinterpret_cast<const uint8_t *>(io->q_kg) + qoff;
+            a.q_seq = reinterpret_cast<const uint8_t *>(io->q_seq) + qoff;
+            a.out = reinterpret_cast<uint8_t *>(io->out) + qoff;
+            a.lse = io->lse ? io->lse + (size_t)b0 * io->N * io->H : nullptr;
+            a.k_seq = reinterpret_cast<const uint8_t *>(io->k_seq) + kvoff;
+            a.v_seq = reinterpret_cast<const uint8_t *>(io->v_seq) + kvoff;
+            a.lk_base = pool;
+            a.lv_base = vpool;
+            a.lk_idx = kept_leaf_row;
+            a.lv_idx = vslot[c];
+            a.leaf_head_stride = 0;
+            a.lk_rows = (long long)groups[c] * n_mid * t->d.fanout[2];
+            a.lv_rows = (long long)groups[c] * n_leaf;
+            apc[c] = a;
+        }
+        // the staging stream starts after everything already queued on the caller's stream
+        AKV_CUDA(cudaEventRecord(t->cev[kMaxChunks * kChunkEvents], s));
+        AKV_CUDA(cudaStreamWaitEvent(s1, t->cev[kMaxChunks * kChunkEvents], 0));
+        for (int c = 0; c < nc; ++c) {   // levels 0-1
+            AKV_STEP(tmark(c, 0, s));
+            AKV_STEP(dispatch_descend(t->d.dtype, D, dpc[c], 0, 1, s));
+            AKV_STEP(tmark(c, 1, s));
+            AKV_CUDA(cudaEventRecord(cev(c, 0), s));
+        }
+        for (int c = 0; c < nc; ++c) {   // leaf-key blocks of the kept mids
+            AKV_CUDA(cudaStreamWaitEvent(s1, cev(c, 0), 0));
+            AKV_STEP(tmark(c, 2, s1));
+            AKV_STEP(launch_dedupe(dpc[c].kept[1], n_mid, groups[c], umid[c], leaf_slot[c], cmid[c], s1));
+            AKV_STEP(dispatch_stage_keys(t, umid[c], cmid[c], n_mid, groups[c], const_cast<void *>(dpc[c].keys[2]), s1));
+            AKV_STEP(tmark(c, 3, s1));
+            AKV_CUDA(cudaEventRecord(cev(c, 1), s1));
+        }
+        for (int c = 0; c < nc; ++c) {   // level 2 on the staged blocks
+            AKV_CUDA(cudaStreamWaitEvent(s, cev(c, 1), 0));
+            AKV_STEP(tmark(c, 4, s));
+            AKV_STEP(dispatch_descend(t->d.dtype, D, dpc[c], 2, 2, s));
+            AKV_STEP(tmark(c, 5, s));
+            AKV_CUDA(cudaEventRecord(cev(c, 2), s));
+        }
+        for (int c = 0; c < nc; ++c) {   // value rows of the kept leaves
+            AKV_CUDA(cudaStreamWaitEvent(s1, cev(c, 2), 0));
+            AKV_STEP(tmark(c, 6, s1));
+            AKV_STEP(launch_dedupe(dpc[c].kept[2], n_leaf, groups[c], uleaf[c], vslot[c], cleaf[c], s1));
+            AKV_STEP(dispatch_stage_values(t, uleaf[c], cleaf[c], n_leaf, groups[c], const_cast<void *>(apc[c].lv_base),
+                                           s1));
+            AKV_STEP(tmark(c, 7, s1));
+            AKV_CUDA(cudaEventRecord(cev(c, 3), s1));
+        }
+        for (int c = 0; c < nc; ++c) {   // attention; the caller's stream joins the staging stream here
+            AKV_CUDA(cudaStreamWaitEvent(s, cev(c, 3), 0));
+            AKV_STEP(tmark(c, 8, s));
+            AKV_STEP(dispatch_attend(t->d.dtype, D, apc[c], s));
+            AKV_STEP(tmark(c, 9, s));
+        }
+        t->chunks_last = nc;
     }
 #undef AKV_STEP
     t->timed = prof;
@@ -742,16 +845,19 @@ atlaskv_status atlaskv_stage_times(atlaskv_tree *t, float *ms, int32_t n)
         AKV_CUDA(cudaEventElapsedTime(&v[0], t->ev[0], t->ev[1]));
         AKV_CUDA(cudaEventElapsedTime(&v[2], t->ev[1], t->ev[2]));
     } else {
-        float a, b2, c, d2, e;
-        AKV_CUDA(cudaEventSynchronize(t->ev[5]));
-        AKV_CUDA(cudaEventElapsedTime(&a, t->ev[0], t->ev[1]));
-        AKV_CUDA(cudaEventElapsedTime(&b2, t->ev[1], t->ev[2]));
-        AKV_CUDA(cudaEventElapsedTime(&c, t->ev[2], t->ev[3]));
-        AKV_CUDA(cudaEventElapsedTime(&d2, t->ev[3], t->ev[4]));
-        AKV_CUDA(cudaEventElapsedTime(&e, t->ev[4], t->ev[5]));
-        v[0] = a + c;
-        v[1] = b2 + d2;
-        v[2] = e;
+        // busy time of each kind of segment, summed over the query chunks
+        // (segments of different kinds overlap on the two streams)
+        const int nc = t->chunks_last;
+        AKV_CUDA(cudaEventSynchronize(t->tev[(nc - 1) * kTimingEvents + 9]));
+        for (int c = 0; c < nc; ++c) {
+            float seg[5];
+            for (int k = 0; k < 5; ++k)
+                AKV_CUDA(cudaEventElapsedTime(&seg[k], t->tev[c * kTimingEvents + 2 * k],
+                                              t->tev[c * kTimingEvents + 2 * k + 1]));
+            v[0] += seg[0] + seg[2];
+            v[1] += seg[1] + seg[3];
+            v[2] += seg[4];
+        }
     }
     for (int i = 0; i < n && i < 3; ++i) ms[i] = v[i];
     return ATLASKV_OK;
@@ -775,6 +881,11 @@ atlaskv_status atlaskv_destroy(atlaskv_tree *t)
     if (t->stats) cudaFree(t->stats);
     for (int i = 0; i < kNumEvents; ++i)
         if (t->ev[i]) cudaEventDestroy(t->ev[i]);
+    for (cudaEvent_t e : t->cev)
+        if (e) cudaEventDestroy(e);
+    for (cudaEvent_t e : t->tev)
+        if (e) cudaEventDestroy(e);
+    if (t->stage_stream) cudaStreamDestroy(t->stage_stream);
     delete t;
     return ATLASKV_OK;
 }

@@ -83,60 +83,97 @@ __global__ void __launch_bounds__(kDedupeThreads) dedupe_kernel(const int32_t *_
     if (threadIdx.x == 0) count[b] = flag[n - 1];
 }
 
+// Copies from mapped host memory cross the host link with long latency, so
+// every warp keeps kStageUnroll row groups in flight: a row is D e / 16
+// lanes' 16-byte vectors and a warp instruction covers 32 / that rows; all
+// loads of an iteration are issued before its stores.  A small grid (two CTAs
+// per SM) then fills the link while leaving the SMs to the descent and the
+// attention of the other query chunks running beside it.
+constexpr int kStageUnroll = 4;
+constexpr int kStageCtasPerSm = 2;
+
 // Copy the b_L leaf-key rows of every unique kept mid of every group into the
 // key pool: pool row (q*n + u) * b_L + j <- host leaf row child(mid, j) of KV
-// head q % H_kv.  One warp per (block, row); 16-byte loads from mapped host
-// memory.
+// head q % H_kv.
 template <typename T, int D>
-__global__ void stage_leaf_blocks_kernel(const T *__restrict__ host_leaf_keys, const int32_t *__restrict__ mid_child,
-                                         long long n_mid, long long n_leaf, int b_leaf, int H_kv,
-                                         const int32_t *__restrict__ uniq, const int32_t *__restrict__ count,
-                                         int n, int n_groups, T *pool, int *status)
+__global__ void __launch_bounds__(256) stage_leaf_blocks_kernel(
+    const T *__restrict__ host_leaf_keys, const int32_t *__restrict__ mid_child, long long n_mid, long long n_leaf,
+    int b_leaf, int H_kv, const int32_t *__restrict__ uniq, const int32_t *__restrict__ count, int n, int n_groups,
+    T *pool, int *status)
 {
-    constexpr int VPR = D * (int)sizeof(T) / 16;   // 16-byte vectors per row
-    const int lane = threadIdx.x & 31;
+    constexpr int VPR = D * (int)sizeof(T) / 16;   // 16-byte vectors per row = lanes per row
+    constexpr int RPI = 32 / VPR;                  // rows per warp instruction
+    const int lane = threadIdx.x & 31, sub = lane % VPR, rsel = lane / VPR;
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
     const long long total = (long long)n_groups * n * b_leaf;
-    for (long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
-        const long long blk = w / b_leaf;
-        const int j = (int)(w - blk * b_leaf);
-        const int b = (int)(blk / n);
-        const int u = (int)(blk - (long long)b * n);
-        if (u >= count[b]) continue;
-        const int hkv = b % H_kv;   // group b = query * H_kv + hkv
-        const long long mid = uniq[blk];
-        const long long leaf = mid_child ? (long long)mid_child[((size_t)hkv * n_mid + mid) * b_leaf + j]
-                                         : mid * b_leaf + j;
-        if (leaf < 0 || leaf >= n_leaf) {
-            if (lane == 0) set_status(status, kDevBadChild);
-            continue;
+    for (long long r0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * (RPI * kStageUnroll);
+         r0 < total; r0 += warps * RPI * kStageUnroll) {
+        uint4 buf[kStageUnroll];
+        uint4 *dst[kStageUnroll];
+#pragma unroll
+        for (int k = 0; k < kStageUnroll; ++k) {
+            const long long w = r0 + (long long)k * RPI + rsel;
+            dst[k] = nullptr;
+            if (w < total) {
+                const long long blk = w / b_leaf;
+                const int j = (int)(w - blk * b_leaf);
+                const int b = (int)(blk / n);
+                const int u = (int)(blk - (long long)b * n);
+                if (u < count[b]) {
+                    const int hkv = b % H_kv;   // group b = query * H_kv + hkv
+                    const long long mid = uniq[blk];
+                    const long long leaf = mid_child ? (long long)mid_child[((size_t)hkv * n_mid + mid) * b_leaf + j]
+                                                     : mid * b_leaf + j;
+                    if (leaf < 0 || leaf >= n_leaf) {
+                        set_status(status, kDevBadChild);
+                    } else {
+                        buf[k] = reinterpret_cast<const uint4 *>(host_leaf_keys + ((size_t)hkv * n_leaf + leaf) * D)[sub];
+                        dst[k] = reinterpret_cast<uint4 *>(pool + ((size_t)blk * b_leaf + j) * D) + sub;
+                    }
+                }
+            }
         }
-        const uint4 *src = reinterpret_cast<const uint4 *>(host_leaf_keys + ((size_t)hkv * n_leaf + leaf) * D);
-        uint4 *dst = reinterpret_cast<uint4 *>(pool + ((size_t)blk * b_leaf + j) * D);
-        for (int v = lane; v < VPR; v += 32) dst[v] = src[v];
+#pragma unroll
+        for (int k = 0; k < kStageUnroll; ++k)
+            if (dst[k]) *dst[k] = buf[k];
     }
 }
 
 // Copy value rows: vpool row (q*n + u) <- host leaf value row uniq[q*n + u]
 // of KV head q % H_kv.
 template <typename T, int D>
-__global__ void stage_value_rows_kernel(const T *__restrict__ host_leaf_values, long long n_leaf, int H_kv,
-                                        const int32_t *__restrict__ uniq, const int32_t *__restrict__ count, int n,
-                                        int n_groups, T *vpool)
+__global__ void __launch_bounds__(256) stage_value_rows_kernel(const T *__restrict__ host_leaf_values, long long n_leaf,
+                                                               int H_kv, const int32_t *__restrict__ uniq,
+                                                               const int32_t *__restrict__ count, int n, int n_groups,
+                                                               T *vpool)
 {
     constexpr int VPR = D * (int)sizeof(T) / 16;
-    const int lane = threadIdx.x & 31;
+    constexpr int RPI = 32 / VPR;
+    const int lane = threadIdx.x & 31, sub = lane % VPR, rsel = lane / VPR;
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
     const long long total = (long long)n_groups * n;
-    for (long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
-        const int b = (int)(w / n);
-        const int u = (int)(w - (long long)b * n);
-        if (u >= count[b]) continue;
-        const int hkv = b % H_kv;
-        const long long leaf = uniq[w];
-        const uint4 *src = reinterpret_cast<const uint4 *>(host_leaf_values + ((size_t)hkv * n_leaf + leaf) * D);
-        uint4 *dst = reinterpret_cast<uint4 *>(vpool + (size_t)w * D);
-        for (int v = lane; v < VPR; v += 32) dst[v] = src[v];
+    for (long long r0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * (RPI * kStageUnroll);
+         r0 < total; r0 += warps * RPI * kStageUnroll) {
+        uint4 buf[kStageUnroll];
+        uint4 *dst[kStageUnroll];
+#pragma unroll
+        for (int k = 0; k < kStageUnroll; ++k) {
+            const long long w = r0 + (long long)k * RPI + rsel;
+            dst[k] = nullptr;
+            if (w < total) {
+                const int b = (int)(w / n);
+                const int u = (int)(w - (long long)b * n);
+                if (u < count[b]) {
+                    const int hkv = b % H_kv;
+                    const long long leaf = uniq[w];
+                    buf[k] = reinterpret_cast<const uint4 *>(host_leaf_values + ((size_t)hkv * n_leaf + leaf) * D)[sub];
+                    dst[k] = reinterpret_cast<uint4 *>(vpool + (size_t)w * D) + sub;
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kStageUnroll; ++k)
+            if (dst[k]) *dst[k] = buf[k];
     }
 }
 

@@ -140,8 +140,12 @@ atlaskv_status atlaskv_workspace_size(const atlaskv_tree *tree, const atlaskv_pa
  * leaves when the tree's leaves are in host memory), knowledge + sequence
  * attention and merge.  `workspace` is device memory of at least
  * atlaskv_workspace_size() bytes, 256-byte aligned, not shared with a
- * concurrent call.  Returns EINVAL / ENOMEM (workspace too small) /
- * EUNSUPPORTED without enqueuing anything. */
+ * concurrent call.  With host-resident leaves the batch is processed in query
+ * chunks and the leaf blocks are staged on a second stream owned by the tree
+ * (joined back into `stream` before the call's last kernel), so the host link
+ * works while other chunks compute; calls on one such tree must therefore not
+ * overlap.  Returns EINVAL / ENOMEM (workspace too small) / EUNSUPPORTED
+ * without enqueuing anything. */
 atlaskv_status atlaskv_attend(atlaskv_tree *tree, const atlaskv_params *params, const atlaskv_io *io,
                               void *workspace, size_t workspace_bytes, void *stream);
 
