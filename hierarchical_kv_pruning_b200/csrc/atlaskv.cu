@@ -267,8 +267,9 @@ template <typename T, int D>
 atlaskv_status launch_select(const akv::DescendParams &dp, int L, cudaStream_t s)
 {
     const long long BH = (long long)dp.B * dp.H;
-    const long long grid = (BH + akv::kSelectWarps - 1) / akv::kSelectWarps;
-    const size_t smem = (size_t)akv::kSelectWarps * akv::SelectScratch::bytes(dp.cap, dp.kcap, D);
+    const long long grid = BH;   // one CTA per traversal
+    if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "selection grid too large");
+    const size_t smem = akv::SelectScratch::bytes(dp.cap, dp.kcap, D);
     if (smem > 227 * 1024)
         return fail(ATLASKV_EUNSUPPORTED, "selection needs %zu bytes of shared memory per CTA", smem);
     static size_t configured = 0;
@@ -277,7 +278,7 @@ atlaskv_status launch_select(const akv::DescendParams &dp, int L, cudaStream_t s
                                       (int)smem));
         configured = smem;
     }
-    akv::select_kernel<T, D><<<(unsigned)grid, akv::kSelectWarps * 32, smem, s>>>(dp, L);
+    akv::select_kernel<T, D><<<(unsigned)grid, akv::kSelThreads, smem, s>>>(dp, L);
     AKV_CUDA(cudaGetLastError());
     // tier 3 for whatever the bounds left undecided (usually nothing: the warps read an empty queue)
     const size_t esmem = (size_t)akv::kSelectWarps * akv::ExactScratch::bytes(dp.kcap, D);
@@ -287,7 +288,7 @@ atlaskv_status launch_select(const akv::DescendParams &dp, int L, cudaStream_t s
                                       (int)esmem));
         econfigured = esmem;
     }
-    const long long egrid = std::min<long long>(grid, 2 * 148);
+    const long long egrid = std::min<long long>((BH + akv::kSelectWarps - 1) / akv::kSelectWarps, 2 * 148);
     akv::exact_kernel<T, D><<<(unsigned)egrid, akv::kSelectWarps * 32, esmem, s>>>(dp, L);
     AKV_CUDA(cudaGetLastError());
     return ATLASKV_OK;

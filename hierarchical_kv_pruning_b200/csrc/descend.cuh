@@ -589,122 +589,6 @@ __device__ void warp_sort_u64(uint64_t *a, int n)
     __syncwarp();
 }
 
-// k-th largest (1-based) of n floats f[0..n) (n a multiple of 4 in storage,
-// entries past n ignored), warp-level, given their min mn and max mx.  Values
-// are bucketed linearly between min and max (a monotone map); the bucket
-// holding the k-th largest is then searched exactly: sorted when small, else
-// narrowed by MSB-first radix passes over the order-preserving bit image.
-// hist: this warp's 256 bins; tmp: 64 scratch uint64.
-__device__ float warp_kth_largest(const float *f, int n, int k, float mn, float mx, uint32_t *hist, uint64_t *tmp)
-{
-    const int lane = threadIdx.x & 31;
-    if (mx == mn) return mx;   // all equal
-    if (mx > mn && isfinite(mx - mn)) {
-        const float scale = 255.99f / (mx - mn);
-        auto bucket = [&](float v) { return min(255, max(0, (int)((v - mn) * scale))); };
-#pragma unroll
-        for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
-        __syncwarp();
-        for (int i = lane; i < n; i += 32) atomicAdd(&hist[bucket(f[i])], 1u);
-        __syncwarp();
-        uint32_t cnt[8], tot = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            cnt[j] = hist[255 - 8 * lane - j];
-            tot += cnt[j];
-        }
-        uint32_t incl = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        const uint32_t excl = incl - tot;
-        int bk = 0, rem = 0, bcount = 0;
-        const bool mine = excl < (uint32_t)k && (uint32_t)k <= incl;
-        if (mine) {
-            uint32_t run = excl;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if (run + cnt[j] >= (uint32_t)k) {
-                    bk = 255 - 8 * lane - j;
-                    rem = k - (int)run;
-                    bcount = (int)cnt[j];
-                    break;
-                }
-                run += cnt[j];
-            }
-        }
-        const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-        bk = __shfl_sync(0xffffffffu, bk, src);
-        rem = __shfl_sync(0xffffffffu, rem, src);
-        bcount = __shfl_sync(0xffffffffu, bcount, src);
-        __syncwarp();
-        if (bcount <= 64) {
-            // collect the bucket, sort it descending by value, take the rem-th
-            int m = 0;
-            for (int i0 = 0; i0 < n; i0 += 32) {
-                const int i = i0 + lane;
-                const bool in = i < n && bucket(f[i]) == bk;
-                const unsigned msk = __ballot_sync(0xffffffffu, in);
-                if (in) tmp[m + __popc(msk & lanemask_lt())] = ~(uint64_t)float_key(f[i]);
-                m += __popc(msk);
-            }
-            for (int i = m + lane; i < 64; i += 32) tmp[i] = ~0ull;
-            warp_sort_u64(tmp, 64);
-            const float t = key_float((uint32_t)~tmp[rem - 1]);
-            __syncwarp();
-            return t;
-        }
-    }
-    // general case: radix select on the bit image
-    uint32_t prefix = 0, mask = 0;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
-        __syncwarp();
-        for (int i = lane; i < n; i += 32) {
-            const uint32_t key = float_key(f[i]);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-        }
-        __syncwarp();
-        uint32_t cnt[8], tot = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            cnt[j] = hist[255 - 8 * lane - j];
-            tot += cnt[j];
-        }
-        uint32_t incl = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        const uint32_t excl = incl - tot;
-        int digit = 0, rem = 0;
-        const bool mine = excl < (uint32_t)k && (uint32_t)k <= incl;
-        if (mine) {
-            uint32_t run = excl;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if (run + cnt[j] >= (uint32_t)k) {
-                    digit = 255 - 8 * lane - j;
-                    rem = k - (int)run;
-                    break;
-                }
-                run += cnt[j];
-            }
-        }
-        const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-        digit = __shfl_sync(0xffffffffu, digit, src);
-        k = __shfl_sync(0xffffffffu, rem, src);
-        prefix |= ((uint32_t)digit) << shift;
-        mask |= 255u << shift;
-        __syncwarp();
-    }
-    return key_float(prefix);
-}
-
 // One traversal's candidates at one level: candidate c = (k, j) is child j of
 // its k-th kept parent; at the root level c is the root itself.
 struct LevelView {
@@ -813,29 +697,165 @@ __device__ __forceinline__ int warp_excl_scan(int v, int &total)
     return incl - v;
 }
 
-// One warp per traversal: top-K of level L's candidates, tier 1.  The fp32
+// CTA-wide exclusive scan of one int per thread (kSelThreads threads): this
+// thread's exclusive prefix; the total in `total`.  red: kSelThreads / 32 ints.
+constexpr int kSelThreads = 128;
+
+__device__ __forceinline__ int cta_excl_scan(int v, int &total, int *red)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int wt;
+    const int ex = warp_excl_scan(v, wt);
+    if (lane == 0) red[warp] = wt;
+    __syncthreads();
+    int base = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+        const int x = red[w];
+        base += w < warp ? x : 0;
+        tot += x;
+    }
+    __syncthreads();
+    total = tot;
+    return base + ex;
+}
+
+// k-th largest (1-based) of the n floats f[0..n), by all kSelThreads threads,
+// given their min mn and max mx.  Values are bucketed linearly between min and
+// max (a monotone map); the bucket holding the k-th largest is then searched
+// exactly: sorted when it holds at most 64, else narrowed by MSB-first radix
+// passes over the order-preserving bit image.  hist: 256 bins; tmp: 64 scratch
+// uint64; sh: 8 ints of shared scratch.
+__device__ float cta_kth_largest(const float *f, int n, int k, float mn, float mx, uint32_t *hist, uint64_t *tmp,
+                                 int *sh)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (mx == mn) return mx;   // all equal
+    // warp 0: find the bin holding the k-th largest from the 256 counts
+    auto pick = [&](int kk, int &bin, int &rem, int &bcount) {
+        uint32_t cnt[8], tot = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            cnt[j] = hist[255 - 8 * lane - j];
+            tot += cnt[j];
+        }
+        uint32_t incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const uint32_t excl = incl - tot;
+        bin = rem = bcount = 0;
+        const bool mine = excl < (uint32_t)kk && (uint32_t)kk <= incl;
+        if (mine) {
+            uint32_t run = excl;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (run + cnt[j] >= (uint32_t)kk) {
+                    bin = 255 - 8 * lane - j;
+                    rem = kk - (int)run;
+                    bcount = (int)cnt[j];
+                    break;
+                }
+                run += cnt[j];
+            }
+        }
+        const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+        bin = __shfl_sync(0xffffffffu, bin, src);
+        rem = __shfl_sync(0xffffffffu, rem, src);
+        bcount = __shfl_sync(0xffffffffu, bcount, src);
+    };
+    if (mx > mn && isfinite(mx - mn)) {
+        const float scale = 255.99f / (mx - mn);
+        auto bucket = [&](float v) { return min(255, max(0, (int)((v - mn) * scale))); };
+        for (int j = tid; j < 256; j += kSelThreads) hist[j] = 0;
+        __syncthreads();
+        for (int i = tid; i < n; i += kSelThreads) atomicAdd(&hist[bucket(f[i])], 1u);
+        __syncthreads();
+        if (warp == 0) {
+            int bk, rem, bcount;
+            pick(k, bk, rem, bcount);
+            if (lane == 0) {
+                sh[0] = bk;
+                sh[1] = rem;
+                sh[2] = bcount;
+                sh[3] = 0;
+            }
+        }
+        __syncthreads();
+        const int bk = sh[0], rem = sh[1], bcount = sh[2];
+        if (bcount <= 64) {
+            // the bucket's members (order is irrelevant: they are sorted next)
+            for (int i = tid; i < n; i += kSelThreads)
+                if (bucket(f[i]) == bk) tmp[atomicAdd(&sh[3], 1)] = ~(uint64_t)float_key(f[i]);
+            __syncthreads();
+            if (warp == 0) {
+                for (int i = sh[3] + lane; i < 64; i += 32) tmp[i] = ~0ull;
+                warp_sort_u64(tmp, 64);
+                if (lane == 0) sh[4] = (int)(uint32_t)~tmp[rem - 1];
+            }
+            __syncthreads();
+            const float t = key_float((uint32_t)sh[4]);
+            __syncthreads();
+            return t;
+        }
+        __syncthreads();
+    }
+    // general case: radix select on the bit image
+    uint32_t prefix = 0, mask = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int j = tid; j < 256; j += kSelThreads) hist[j] = 0;
+        __syncthreads();
+        for (int i = tid; i < n; i += kSelThreads) {
+            const uint32_t key = float_key(f[i]);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int digit, rem, unused;
+            pick(k, digit, rem, unused);
+            if (lane == 0) {
+                sh[0] = digit;
+                sh[1] = rem;
+            }
+        }
+        __syncthreads();
+        prefix |= ((uint32_t)sh[0]) << shift;
+        mask |= 255u << shift;
+        k = sh[1];
+        __syncthreads();
+    }
+    return key_float(prefix);
+}
+
+// One CTA per traversal: top-K of level L's candidates, tier 1.  The fp32
 // scores and their rigorous bound E settle every candidate outside the band
 // [t - 2E, t + 2E] around the K-th largest score t.  When the band holds more
 // candidates than places left, the traversal is queued for exact_kernel with
-// its decided entries and the band's positions.
+// its decided entries and the band's positions.  Every pass over the
+// candidates is spread over the CTA's threads; the small sorts run on warp 0.
 template <typename T, int D>
-__global__ void __launch_bounds__(kSelectWarps * 32) select_kernel(const DescendParams p, int L)
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const DescendParams p, int L)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long bh = (long long)blockIdx.x * kSelectWarps + warp;
+    __shared__ int sh[8];
+    __shared__ int red[kSelThreads / 32];
+    __shared__ float redf[2][kSelThreads / 32];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long bh = blockIdx.x;
     if (bh >= (long long)p.B * p.H) return;
-    SelectScratch sc(smem_raw + (size_t)warp * SelectScratch::bytes(p.cap, p.kcap, D), p.cap, p.kcap, D);
+    SelectScratch sc(smem_raw, p.cap, p.kcap, D);
     const int Kp = L == 0 ? 0 : p.K[L - 1];
-    for (int k = lane; k < Kp; k += 32) sc.prev[k] = p.kept[L - 1][bh * Kp + k];
+    for (int k = tid; k < Kp; k += kSelThreads) sc.prev[k] = p.kept[L - 1][bh * Kp + k];
     const LevelView lv = level_view<T>(p, L, bh, sc.prev);
     const int C = lv.C, K = p.K[L];
     float *fslot = p.f_ws + (size_t)bh * p.fstride;
     const int nv = (C + 3) >> 2;
     float mn = INFINITY, mx = -INFINITY;
-    bool bad = false;
+    int bad = 0;
     {
-        // 16-byte loads, several in flight per lane; min / max / finiteness on the way
+        // 16-byte loads, several in flight per thread; min / max / finiteness on the way
         const float4 *src = reinterpret_cast<const float4 *>(fslot);
         float4 *dst = reinterpret_cast<float4 *>(sc.f);
         auto take = [&](float4 t, int v) {
@@ -849,49 +869,61 @@ __global__ void __launch_bounds__(kSelectWarps * 32) select_kernel(const Descend
                     bad |= !isfinite(e[q]);
                 }
         };
-        int v = lane;
-        for (; v + 3 * 32 < nv; v += 4 * 32) {
+        int v = tid;
+        for (; v + 3 * kSelThreads < nv; v += 4 * kSelThreads) {
             float4 t[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) t[u] = __ldcg(src + v + u * 32);
+            for (int u = 0; u < 4; ++u) t[u] = __ldcg(src + v + u * kSelThreads);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) take(t[u], v + u * 32);
+            for (int u = 0; u < 4; ++u) take(t[u], v + u * kSelThreads);
         }
-        for (; v < nv; v += 32) take(__ldcg(src + v), v);
+        for (; v < nv; v += kSelThreads) take(__ldcg(src + v), v);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         }
+        bad = __any_sync(0xffffffffu, bad);
+        if (lane == 0) {
+            redf[0][warp] = mn;
+            redf[1][warp] = mx;
+            red[warp] = bad;
+        }
+        __syncthreads();   // scores, kept parents and the partial reductions are visible
+#pragma unroll
+        for (int w = 0; w < kSelThreads / 32; ++w) {
+            mn = fminf(mn, redf[0][w]);
+            mx = fmaxf(mx, redf[1][w]);
+            bad |= red[w];
+        }
+        __syncthreads();
     }
-    __syncwarp();
-    if (p.stats && lane == 0) atomicAdd(p.stats + L * 4, 1ull);
+    if (p.stats && tid == 0) atomicAdd(p.stats + L * 4, 1ull);
     const float *f = sc.f;
     uint64_t *sortb = sc.sortb;
     if (K >= C) {
-        for (int c = lane; c < C; c += 32) sortb[c] = ((uint64_t)(uint32_t)lv.id(c) << 32) | (uint32_t)c;
-        __syncwarp();
-        write_kept(p, lv, L, bh, sortb, K);
+        for (int c = tid; c < C; c += kSelThreads) sortb[c] = ((uint64_t)(uint32_t)lv.id(c) << 32) | (uint32_t)c;
+        __syncthreads();
+        if (warp == 0) write_kept(p, lv, L, bh, sortb, K);
         return;
     }
     const double cprime = gamma_n(D) * (1.0 + gamma_n(p.N)) + gamma_n(p.N);
     const double E = cprime * (double)p.anorm_ws[bh] * (double)p.norm_bound[L * p.H_kv + lv.hkv] * (1.0 + 1e-6) +
                      D * 0x1p-148;
-    bad = __any_sync(0xffffffffu, bad);
-    const double t = bad ? 0.0 : (double)warp_kth_largest(f, C, K, mn, mx, sc.hist, sc.tmp);
-    bad = bad || !isfinite(E) || !isfinite(t);
+    const double t = bad ? 0.0 : (double)cta_kth_largest(f, C, K, mn, mx, sc.hist, sc.tmp, sh);
+    const bool bad2 = bad || !isfinite(E) || !isfinite(t);
     // band edges rounded outward to fp32: the sure-kept and sure-dropped sets can
     // only shrink, so the classification stays rigorous
-    const float hi32 = bad ? INFINITY : __double2float_ru(__dadd_ru(t, 2.0 * E));
-    const float lo32 = bad ? -INFINITY : __double2float_rd(__dsub_rd(t, 2.0 * E));
+    const float hi32 = bad2 ? INFINITY : __double2float_ru(__dadd_ru(t, 2.0 * E));
+    const float lo32 = bad2 ? -INFINITY : __double2float_rd(__dsub_rd(t, 2.0 * E));
     // class of candidate c: 1 kept for sure, 2 ambiguous, 0 dropped
     auto cls = [&](float fv) -> int {
-        if (bad) return 2;
+        if (bad2) return 2;
         return fv > hi32 ? 1 : (fv >= lo32 ? 2 : 0);
     };
     const float4 *f4 = reinterpret_cast<const float4 *>(f);
     int my_in = 0, my_a = 0;
-    for (int v = lane; v < nv; v += 32) {
+    for (int v = tid; v < nv; v += kSelThreads) {
         const float4 x = f4[v];
         const float e[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -902,13 +934,13 @@ __global__ void __launch_bounds__(kSelectWarps * 32) select_kernel(const Descend
         }
     }
     int n_in, nA;
-    int off_in = warp_excl_scan(my_in, n_in);
-    int off_a = warp_excl_scan(my_a, nA);
+    int off_in = cta_excl_scan(my_in, n_in, red);
+    int off_a = cta_excl_scan(my_a, nA, red);
     const int r = K - n_in;
     const bool settle = nA == r;   // every ambiguous candidate is kept
     int *list = reinterpret_cast<int *>(fslot);
     if (settle) off_a += n_in;
-    for (int v = lane; v < nv; v += 32) {
+    for (int v = tid; v < nv; v += kSelThreads) {
         const float4 x = f4[v];
         const float e[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -922,24 +954,24 @@ __global__ void __launch_bounds__(kSelectWarps * 32) select_kernel(const Descend
             }
         }
     }
-    __syncwarp();
+    __syncthreads();
     if (settle) {
-        write_kept(p, lv, L, bh, sortb, K);
+        if (warp == 0) write_kept(p, lv, L, bh, sortb, K);
         return;
     }
-    if (p.stats && lane == 0) {
+    if (p.stats && tid == 0) {
         atomicAdd(p.stats + L * 4 + 1, 1ull);
         atomicAdd(p.stats + L * 4 + 2, (unsigned long long)nA);
     }
     uint64_t *decided = reinterpret_cast<uint64_t *>(fslot + p.cap);
-    for (int i = lane; i < n_in; i += 32) decided[i] = sortb[i];
-    if (lane == 0) {
+    for (int i = tid; i < n_in; i += kSelThreads) decided[i] = sortb[i];
+    if (tid == 0) {
         const int qi = atomicAdd(p.qcount + L, 1);
         int *e = p.queue + ((size_t)L * p.B * p.H + qi) * 4;
         e[0] = (int)bh;
         e[1] = n_in;
         e[2] = nA;
-        e[3] = bad ? 1 : 0;
+        e[3] = bad2 ? 1 : 0;
     }
 }
 
