@@ -231,7 +231,7 @@ template <typename T, int D, int HT>
 atlaskv_status launch_score_ht(const akv::DescendParams &dp, int L, int GC, cudaStream_t s)
 {
     const int Kp = dp.K[L - 1], fo = dp.fanout[L];
-    const int ppc = std::max(1, 1024 / fo);           // parents per chunk: about 1024 rows per CTA
+    const int ppc = std::max(1, 2048 / fo);           // parents per chunk: about 2048 rows per CTA
     const int pchunks = (Kp + ppc - 1) / ppc;         // covers a union of Kp parents; larger ones loop
     const long long grid = (long long)dp.B * dp.H_kv * (dp.G / GC) * pchunks;
     if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "scoring grid too large");
