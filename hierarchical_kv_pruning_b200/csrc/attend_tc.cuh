@@ -67,7 +67,7 @@ constexpr int kBarFullK = 0;                        // [kKStages] K tile landed
 constexpr int kBarEmptyK = kBarFullK + kKStages;    // [kKStages] S of the tile done
 constexpr int kBarFullV = kBarEmptyK + kKStages;    // [kVStages] V tile landed
 constexpr int kBarEmptyV = kBarFullV + kVStages;    // [kVStages] P V of the tile done
-constexpr int kBarSFull = kBarEmptyV + kVStages;    // [kWG][2] S(w, t) in TMEM buffer t & 1
+constexpr int kBarSFull = kBarEmptyV + kVStages;    // [kWG][2] S in TMEM buffer (tiles taken by w so far) & 1
 constexpr int kBarPReady = kBarSFull + 2 * kWG;     // [kWG][2] P(w, t) written over it, O_w rescaled (4 warps)
 constexpr int kBarODone = kBarPReady + 2 * kWG;     // [kWG][2] O_w += P V from that buffer done
 constexpr int kBarQReady = kBarODone + 2 * kWG;     // [kWG] Q_w loaded (4 warps)
@@ -267,6 +267,30 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     const int cta_last = p.T - p.N + (r_end / p.N != r0 / p.N ? p.N - 1 : r_end % p.N);
     const int n_seq_tiles = (cta_last + kKeys) / kKeys;
     const int n_tiles = n_leaf_tiles + n_seq_tiles;
+    // Warpgroup w takes every sequence tile (if it has rows at all) and the
+    // leaf tiles holding its heads' leaves: its heads are contiguous and the
+    // leaves are stored head by head, so those are the leaf tiles
+    // [wlo[w], whi[w]] (empty when wlo > whi).  It skips the others, and so do
+    // its MMAs; its count of taken tiles drives its S / P buffers and phases.
+    int wlo[kWG], whi[kWG];
+    bool wvalid[kWG];
+#pragma unroll
+    for (int w = 0; w < kWG; ++w) {
+        const int wr0 = r0 + w * kRows;
+        wvalid[w] = wr0 < GN;
+        wlo[w] = 1;
+        whi[w] = 0;
+        if (wvalid[w] && n_leaf_tiles > 0) {
+            const int wr1 = min(GN, wr0 + kRows) - 1;
+            wlo[w] = ((wr0 / p.N - g_first) * p.K_L) / kKeys;
+            whi[w] = min(n_leaf_tiles - 1, ((wr1 / p.N - g_first + 1) * p.K_L - 1) / kKeys);
+        }
+    }
+    auto wg_takes = [&](int w, int t) -> bool {
+        return wvalid[w] && (t < n_seq_tiles || (t - n_seq_tiles >= wlo[w] && t - n_seq_tiles <= whi[w]));
+    };
+    // position of a taken tile t among warpgroup w's tiles
+    auto wg_count = [&](int w, int t) -> int { return t < n_seq_tiles ? t : n_seq_tiles + (t - n_seq_tiles - wlo[w]); };
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) {
@@ -320,12 +344,15 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             if (lane == 0) mbar_arrive(bar(kBarQReady + w));
         };
         load_q(p.q_seq);
+        const bool any_leaf = wvalid[w] && wlo[w] <= whi[w];
 
         const float sl2 = p.scale_log2;
         float m_used = -INFINITY, l = 0.f;
+        int c_w = 0;   // tiles this warpgroup has taken so far
         for (int t = 0; t < n_tiles; ++t) {
-            const int bs = t & 1;
-            failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarSFull + 2 * w + bs), (t >> 1) & 1));
+            if (!wg_takes(w, t)) continue;
+            const int bs = c_w & 1;
+            failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarSFull + 2 * w + bs), (c_w >> 1) & 1));
             if (failed) break;
             fence_after_sync();
             float sc[kKeys];
@@ -333,7 +360,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             tmem_ld32(tS + 64 * bs + 32 + lane_off, sc + 32);
             tmem_wait_ld();
             // S(w, last sequence tile) has completed: Q_w may now be replaced by q_kg
-            if (t == n_seq_tiles - 1 && n_leaf_tiles > 0) load_q(p.q_kg);
+            if (t == n_seq_tiles - 1 && any_leaf) load_q(p.q_kg);
 
             // visible keys of this tile, [lo, hi) in tile-local index: the leaves
             // are stored head by head, K_L per head; a sequence tile is cut by
@@ -360,14 +387,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             const float tmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                      fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             const float m_new = fmaxf(m_used, tmax * sl2);   // scores in log2 units (sl2 > 0)
-            if (t == 0) {
+            if (c_w == 0) {
                 m_used = m_new;   // O_w is initialised by the first P V
             } else {
                 const bool need = m_new > m_used + kRescaleLog2;   // also when m_used is still -inf
                 if (__any_sync(0xffffffffu, need)) {
                     // O_w may be rescaled only once the previous P V has landed in it
                     failed = __any_sync(0xffffffffu,
-                                        !mbar_wait(bar(kBarODone + 2 * w + ((t - 1) & 1)), ((t - 1) >> 1) & 1));
+                                        !mbar_wait(bar(kBarODone + 2 * w + ((c_w - 1) & 1)), ((c_w - 1) >> 1) & 1));
                     if (failed) break;
                     fence_after_sync();
                     const float f = need ? fast_exp2(m_used - m_new) : 1.f;
@@ -413,13 +440,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kBarPReady + 2 * w + bs));
+            ++c_w;
         }
-        if (!failed) {
+        if (!failed && c_w > 0) {
             failed = __any_sync(0xffffffffu,
-                                !mbar_wait(bar(kBarODone + 2 * w + ((n_tiles - 1) & 1)), ((n_tiles - 1) >> 1) & 1));
+                                !mbar_wait(bar(kBarODone + 2 * w + ((c_w - 1) & 1)), ((c_w - 1) >> 1) & 1));
             fence_after_sync();
         }
-        if (!failed) {
+        if (!failed && c_w > 0) {
             const float inv = 1.f / l;
             __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.out) + (((size_t)b * p.N + n) * p.H + h) * kD;
 #pragma unroll
@@ -556,13 +584,18 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
             const uint64_t dk0 = make_desc(sb + kOffK, 16, 1024);
             const uint64_t dv0 = make_desc(sb + kOffV, kKeys * 128, 1024);
             auto issue_s = [&](int t) -> bool {
-                const int sk = t % kKStages, bs = t & 1;
+                const int sk = t % kKStages;
                 if (!mbar_wait(bar(kBarFullK + sk), (t / kKStages) & 1)) return false;
+#pragma unroll
                 for (int w = 0; w < kWG; ++w) {
-                    if (t == 0 && !mbar_wait(bar(kBarQReady + w), 0)) return false;
-                    if (t == n_seq_tiles && n_leaf_tiles > 0 && !mbar_wait(bar(kBarQReady + w), 1)) return false;
-                    // buffer bs still holds P(t - 2) until its P V has completed
-                    if (t >= 2 && !mbar_wait(bar(kBarODone + 2 * w + bs), ((t - 2) >> 1) & 1)) return false;
+                    if (!wg_takes(w, t)) continue;
+                    const int cs = wg_count(w, t), bs = cs & 1;
+                    if (cs == 0 && !mbar_wait(bar(kBarQReady + w), 0)) return false;
+                    // the warpgroup's first leaf tile: Q_w has been replaced by q_kg
+                    if (t >= n_seq_tiles && t - n_seq_tiles == wlo[w] && !mbar_wait(bar(kBarQReady + w), 1))
+                        return false;
+                    // buffer bs still holds the P of this warpgroup's tile two back until its P V has completed
+                    if (cs >= 2 && !mbar_wait(bar(kBarODone + 2 * w + bs), ((cs - 2) >> 1) & 1)) return false;
                     fence_after_sync();
                     const uint64_t qd = dq0 + (uint64_t)((w * kQBytes) >> 4);
                     const uint64_t kdsc = dk0 + (uint64_t)((sk * kKVBytes) >> 4);
@@ -579,17 +612,20 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                 return true;
             };
             auto issue_pv = [&](int u) -> bool {
-                const int sv = u % kVStages, bs = u & 1;
+                const int sv = u % kVStages;
                 if (!mbar_wait(bar(kBarFullV + sv), (u / kVStages) & 1)) return false;
+#pragma unroll
                 for (int w = 0; w < kWG; ++w) {
-                    if (!mbar_wait(bar(kBarPReady + 2 * w + bs), (u >> 1) & 1)) return false;
+                    if (!wg_takes(w, u)) continue;
+                    const int lc = wg_count(w, u), bs = lc & 1;
+                    if (!mbar_wait(bar(kBarPReady + 2 * w + bs), (lc >> 1) & 1)) return false;
                     fence_after_sync();
                     const uint32_t ta = tmem + 256 * w + 64 * bs, td = tmem + 256 * w + 128;
                     const uint64_t vdsc = dv0 + (uint64_t)((sv * kKVBytes) >> 4);
 #pragma unroll
                     for (int ks = 0; ks < kKeys / 16; ++ks)
                         mma_bf16_ts(td, ta + 8 * ks, vdsc + (uint64_t)((ks * 16 * 128) >> 4), idesc_o,
-                                    (u > 0 || ks > 0) ? 1u : 0u);
+                                    (lc > 0 || ks > 0) ? 1u : 0u);
                     mma_commit(bar(kBarODone + 2 * w + bs));
                 }
                 mma_commit(bar(kBarEmptyV + sv));
