@@ -272,14 +272,17 @@ atlaskv_status launch_select(const akv::DescendParams &dp, int L, cudaStream_t s
     const size_t smem = akv::SelectScratch::bytes(dp.cap, dp.kcap, D);
     if (smem > 227 * 1024)
         return fail(ATLASKV_EUNSUPPORTED, "selection needs %zu bytes of shared memory per CTA", smem);
-    static size_t configured = 0;
-    if (smem > 48 * 1024 && smem > configured) {
-        AKV_CUDA(cudaFuncSetAttribute(akv::select_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)smem));
-        configured = smem;
-    }
-    akv::select_kernel<T, D><<<(unsigned)grid, akv::kSelThreads, smem, s>>>(dp, L);
-    AKV_CUDA(cudaGetLastError());
+    // few traversals: 64 threads each (shorter barriers); many: 128 (shorter chains)
+    auto run = [&](auto kern, int nt) -> atlaskv_status {
+        if (smem > 48 * 1024)
+            AKV_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        kern<<<(unsigned)grid, nt, smem, s>>>(dp, L);
+        AKV_CUDA(cudaGetLastError());
+        return ATLASKV_OK;
+    };
+    const atlaskv_status st =
+        BH <= 4096 ? run(akv::select_kernel<T, D, 64>, 64) : run(akv::select_kernel<T, D, 128>, 128);
+    if (st != ATLASKV_OK) return st;
     // tier 3 for whatever the bounds left undecided (usually nothing: the warps read an empty queue)
     const size_t esmem = (size_t)akv::kSelectWarps * akv::ExactScratch::bytes(dp.kcap, D);
     static size_t econfigured = 0;

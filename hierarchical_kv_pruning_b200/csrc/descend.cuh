@@ -697,10 +697,9 @@ __device__ __forceinline__ int warp_excl_scan(int v, int &total)
     return incl - v;
 }
 
-// CTA-wide exclusive scan of one int per thread (kSelThreads threads): this
-// thread's exclusive prefix; the total in `total`.  red: kSelThreads / 32 ints.
-constexpr int kSelThreads = 128;
-
+// CTA-wide exclusive scan of one int per thread (NT threads): this thread's
+// exclusive prefix; the total in `total`.  red: NT / 32 ints.
+template <int NT>
 __device__ __forceinline__ int cta_excl_scan(int v, int &total, int *red)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -710,7 +709,7 @@ __device__ __forceinline__ int cta_excl_scan(int v, int &total, int *red)
     __syncthreads();
     int base = 0, tot = 0;
 #pragma unroll
-    for (int w = 0; w < kSelThreads / 32; ++w) {
+    for (int w = 0; w < NT / 32; ++w) {
         const int x = red[w];
         base += w < warp ? x : 0;
         tot += x;
@@ -720,12 +719,13 @@ __device__ __forceinline__ int cta_excl_scan(int v, int &total, int *red)
     return base + ex;
 }
 
-// k-th largest (1-based) of the n floats f[0..n), by all kSelThreads threads,
+// k-th largest (1-based) of the n floats f[0..n), by all NT threads of the CTA,
 // given their min mn and max mx.  Values are bucketed linearly between min and
 // max (a monotone map); the bucket holding the k-th largest is then searched
 // exactly: sorted when it holds at most 64, else narrowed by MSB-first radix
 // passes over the order-preserving bit image.  hist: 256 bins; tmp: 64 scratch
 // uint64; sh: 8 ints of shared scratch.
+template <int NT>
 __device__ float cta_kth_largest(const float *f, int n, int k, float mn, float mx, uint32_t *hist, uint64_t *tmp,
                                  int *sh)
 {
@@ -769,9 +769,9 @@ __device__ float cta_kth_largest(const float *f, int n, int k, float mn, float m
     if (mx > mn && isfinite(mx - mn)) {
         const float scale = 255.99f / (mx - mn);
         auto bucket = [&](float v) { return min(255, max(0, (int)((v - mn) * scale))); };
-        for (int j = tid; j < 256; j += kSelThreads) hist[j] = 0;
+        for (int j = tid; j < 256; j += NT) hist[j] = 0;
         __syncthreads();
-        for (int i = tid; i < n; i += kSelThreads) atomicAdd(&hist[bucket(f[i])], 1u);
+        for (int i = tid; i < n; i += NT) atomicAdd(&hist[bucket(f[i])], 1u);
         __syncthreads();
         if (warp == 0) {
             int bk, rem, bcount;
@@ -787,7 +787,7 @@ __device__ float cta_kth_largest(const float *f, int n, int k, float mn, float m
         const int bk = sh[0], rem = sh[1], bcount = sh[2];
         if (bcount <= 64) {
             // the bucket's members (order is irrelevant: they are sorted next)
-            for (int i = tid; i < n; i += kSelThreads)
+            for (int i = tid; i < n; i += NT)
                 if (bucket(f[i]) == bk) tmp[atomicAdd(&sh[3], 1)] = ~(uint64_t)float_key(f[i]);
             __syncthreads();
             if (warp == 0) {
@@ -805,9 +805,9 @@ __device__ float cta_kth_largest(const float *f, int n, int k, float mn, float m
     // general case: radix select on the bit image
     uint32_t prefix = 0, mask = 0;
     for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int j = tid; j < 256; j += kSelThreads) hist[j] = 0;
+        for (int j = tid; j < 256; j += NT) hist[j] = 0;
         __syncthreads();
-        for (int i = tid; i < n; i += kSelThreads) {
+        for (int i = tid; i < n; i += NT) {
             const uint32_t key = float_key(f[i]);
             if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
         }
@@ -834,20 +834,22 @@ __device__ float cta_kth_largest(const float *f, int n, int k, float mn, float m
 // [t - 2E, t + 2E] around the K-th largest score t.  When the band holds more
 // candidates than places left, the traversal is queued for exact_kernel with
 // its decided entries and the band's positions.  Every pass over the
-// candidates is spread over the CTA's threads; the small sorts run on warp 0.
-template <typename T, int D>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const DescendParams p, int L)
+// candidates is spread over the CTA's NT threads (64 or 128: the host picks
+// the smaller when few traversals fill the GPU anyway); the small sorts run on
+// warp 0.
+template <typename T, int D, int NT>
+__global__ void __launch_bounds__(NT) select_kernel(const DescendParams p, int L)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ int sh[8];
-    __shared__ int red[kSelThreads / 32];
-    __shared__ float redf[2][kSelThreads / 32];
+    __shared__ int red[NT / 32];
+    __shared__ float redf[2][NT / 32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long bh = blockIdx.x;
     if (bh >= (long long)p.B * p.H) return;
     SelectScratch sc(smem_raw, p.cap, p.kcap, D);
     const int Kp = L == 0 ? 0 : p.K[L - 1];
-    for (int k = tid; k < Kp; k += kSelThreads) sc.prev[k] = p.kept[L - 1][bh * Kp + k];
+    for (int k = tid; k < Kp; k += NT) sc.prev[k] = p.kept[L - 1][bh * Kp + k];
     const LevelView lv = level_view<T>(p, L, bh, sc.prev);
     const int C = lv.C, K = p.K[L];
     float *fslot = p.f_ws + (size_t)bh * p.fstride;
@@ -870,14 +872,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const DescendParams
                 }
         };
         int v = tid;
-        for (; v + 3 * kSelThreads < nv; v += 4 * kSelThreads) {
+        for (; v + 3 * NT < nv; v += 4 * NT) {
             float4 t[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) t[u] = __ldcg(src + v + u * kSelThreads);
+            for (int u = 0; u < 4; ++u) t[u] = __ldcg(src + v + u * NT);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) take(t[u], v + u * kSelThreads);
+            for (int u = 0; u < 4; ++u) take(t[u], v + u * NT);
         }
-        for (; v < nv; v += kSelThreads) take(__ldcg(src + v), v);
+        for (; v < nv; v += NT) take(__ldcg(src + v), v);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
@@ -891,7 +893,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const DescendParams
         }
         __syncthreads();   // scores, kept parents and the partial reductions are visible
 #pragma unroll
-        for (int w = 0; w < kSelThreads / 32; ++w) {
+        for (int w = 0; w < NT / 32; ++w) {
             mn = fminf(mn, redf[0][w]);
             mx = fmaxf(mx, redf[1][w]);
             bad |= red[w];
@@ -902,7 +904,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const DescendParams
     const float *f = sc.f;
     uint64_t *sortb = sc.sortb;
     if (K >= C) {
-        for (int c = tid; c < C; c += kSelThreads) sortb[c] = ((uint64_t)(uint32_t)lv.id(c) << 32) | (uint32_t)c;
+        for (int c = tid; c < C; c += NT) sortb[c] = ((uint64_t)(uint32_t)lv.id(c) << 32) | (uint32_t)c;
         __syncthreads();
         if (warp == 0) write_kept(p, lv, L, bh, sortb, K);
         return;
@@ -910,7 +912,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const DescendParams
     const double cprime = gamma_n(D) * (1.0 + gamma_n(p.N)) + gamma_n(p.N);
     const double E = cprime * (double)p.anorm_ws[bh] * (double)p.norm_bound[L * p.H_kv + lv.hkv] * (1.0 + 1e-6) +
                      D * 0x1p-148;
-    const double t = bad ? 0.0 : (double)cta_kth_largest(f, C, K, mn, mx, sc.hist, sc.tmp, sh);
+    const double t = bad ? 0.0 : (double)cta_kth_largest<NT>(f, C, K, mn, mx, sc.hist, sc.tmp, sh);
     const bool bad2 = bad || !isfinite(E) || !isfinite(t);
     // band edges rounded outward to fp32: the sure-kept and sure-dropped sets can
     // only shrink, so the classification stays rigorous
@@ -923,7 +925,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const DescendParams
     };
     const float4 *f4 = reinterpret_cast<const float4 *>(f);
     int my_in = 0, my_a = 0;
-    for (int v = tid; v < nv; v += kSelThreads) {
+    for (int v = tid; v < nv; v += NT) {
         const float4 x = f4[v];
         const float e[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -934,13 +936,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const DescendParams
         }
     }
     int n_in, nA;
-    int off_in = cta_excl_scan(my_in, n_in, red);
-    int off_a = cta_excl_scan(my_a, nA, red);
+    int off_in = cta_excl_scan<NT>(my_in, n_in, red);
+    int off_a = cta_excl_scan<NT>(my_a, nA, red);
     const int r = K - n_in;
     const bool settle = nA == r;   // every ambiguous candidate is kept
     int *list = reinterpret_cast<int *>(fslot);
     if (settle) off_a += n_in;
-    for (int v = tid; v < nv; v += kSelThreads) {
+    for (int v = tid; v < nv; v += NT) {
         const float4 x = f4[v];
         const float e[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -964,7 +966,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const DescendParams
         atomicAdd(p.stats + L * 4 + 2, (unsigned long long)nA);
     }
     uint64_t *decided = reinterpret_cast<uint64_t *>(fslot + p.cap);
-    for (int i = tid; i < n_in; i += kSelThreads) decided[i] = sortb[i];
+    for (int i = tid; i < n_in; i += NT) decided[i] = sortb[i];
     if (tid == 0) {
         const int qi = atomicAdd(p.qcount + L, 1);
         int *e = p.queue + ((size_t)L * p.B * p.H + qi) * 4;
