@@ -381,7 +381,7 @@ atlaskv_status encode_seq_map(CUtensorMap *map, const void *base, int B, int T, 
     return ATLASKV_OK;
 }
 
-// bf16, D = 128: tcgen05 tensor cores, one CTA per 256 query rows of a
+// bf16, D = 128: tcgen05 tensor cores, one CTA per kWG x 128 query rows of a
 // (query, KV head) group, sequence tiles by TMA.
 atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
 {

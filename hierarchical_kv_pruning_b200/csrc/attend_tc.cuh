@@ -4,11 +4,14 @@
 // Same computation as attend.cuh ("AtlasKV: Augmenting LLMs with Billion-Scale
 // Knowledge Graphs in 20GB VRAM": the lambda-weighted merge of the knowledge and
 // sequence softmaxes equals one softmax over both key sets), organised for
-// sm_100a as a warp-specialised pipeline.  A CTA owns 256 query rows of one
-// (query b, KV head) group (row r = g N + n is token n of head g), in two
-// 128-row tiles, one per softmax warpgroup, and streams 64-key tiles shared by
-// both: first the causal sequence, then the kept leaves of the CTA's heads (each
-// visible only to its own head's rows); the online softmax is order-free.
+// sm_100a as a warp-specialised pipeline.  A CTA owns kWG 128-row tiles of
+// one (query b, KV head) group (row r = g N + n is token n of head g), one per
+// softmax warpgroup, and streams 64-key tiles shared by them: first the causal
+// sequence, then the kept leaves of the CTA's heads (each visible only to its
+// own head's rows); the online softmax is order-free.  kWG = 1 (TMEM 256
+// columns, 96 KB of shared memory) runs two CTAs per SM, so one CTA's MMA,
+// copy and softmax bubbles overlap the other's work; this measured faster than
+// two warpgroups sharing the key tiles in one CTA per SM.
 //
 //   producer warp   sequence K/V tiles by TMA (4-D tensor maps, 128-byte
 //                   swizzle) and gathered leaf rows by cp.async, into a K ring
@@ -44,9 +47,10 @@ namespace tc {
 constexpr int kRows = 128;                 // query rows per warpgroup (UMMA M)
 constexpr int kKeys = 64;                  // keys per tile
 constexpr int kD = 128;                    // head dim
-constexpr int kWG = 2;                     // softmax warpgroups per CTA
-constexpr int kKStages = 4;                // K ring depth (a stage is freed when S = Q K^T completes)
-constexpr int kVStages = 3;                // V ring depth (freed when P V completes)
+constexpr int kWG = 1;                     // softmax warpgroups per CTA (1: two CTAs per SM)
+constexpr int kKStages = kWG == 2 ? 4 : 2; // K ring depth (a stage is freed when S = Q K^T completes)
+constexpr int kVStages = kWG == 2 ? 3 : 2; // V ring depth (freed when P V completes)
+constexpr int kMinCtasPerSm = kWG == 2 ? 1 : 2;
 constexpr int kProducerWarp = 4 * kWG;
 constexpr int kMmaWarp = 4 * kWG + 1;
 constexpr int kThreads = 32 * (4 * kWG + 2);
@@ -74,7 +78,7 @@ constexpr int kBarQReady = kBarODone + 2 * kWG;     // [kWG] Q_w loaded (4 warps
 constexpr int kNumBars = kBarQReady + kWG;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024;   // + slack to align the base to 1024
-constexpr int kTmemCols = 512;                 // warpgroup w: S / P buffers [256 w, 256 w + 128), O [256 w + 128, 256 w + 256)
+constexpr int kTmemCols = 256 * kWG;           // warpgroup w: S / P buffers [256 w, 256 w + 128), O [256 w + 128, 256 w + 256)
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -238,10 +242,10 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
 
 }  // namespace tc
 
-// One CTA per (query b, KV head, 256-row block of the group's G N rows).
+// One CTA per (query b, KV head, kWG x 128-row block of the group's G N rows).
 // tm_k / tm_v: the sequence keys / values [B][T][H_kv][D] as 4-D tensor maps
 // (D, H_kv, T, B) with a (64, 1, 64, 1) box and 128-byte swizzle.
-__global__ void __launch_bounds__(tc::kThreads, 1)
+__global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
     attend_tc_kernel(const AttnParams p, int ctas_per_group, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v)
 {

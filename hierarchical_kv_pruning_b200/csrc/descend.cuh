@@ -636,24 +636,23 @@ __device__ LevelView level_view(const DescendParams &p, int L, long long bh, con
     return lv;
 }
 
-// Per-warp shared scratch of the selection.
+// Shared scratch of one traversal's selection.
 struct SelectScratch {
     float *f;          // [cap] scores
     int32_t *prev;     // [kcap] kept parents of the traversal
     uint32_t *hist;    // [256]
     uint64_t *sortb;   // [kcap] (id << 32 | position)
     uint64_t *tmp;     // [64]
-    double *s64;       // [D]
-    double *a64;       // [D]
 
     __host__ __device__ static size_t bytes(int cap, int kcap, int D)
     {
+        (void)D;
         auto r = [](size_t b) { return (b + 15) & ~size_t(15); };
-        return r((size_t)cap * 4) + r((size_t)kcap * 4) + r(1024) + r((size_t)kcap * 8) + r(512) +
-               2 * r((size_t)D * 8);
+        return r((size_t)cap * 4) + r((size_t)kcap * 4) + r(1024) + r((size_t)kcap * 8) + r(512);
     }
     __device__ SelectScratch(uint8_t *p, int cap, int kcap, int D)
     {
+        (void)D;
         auto take = [&](size_t b) {
             uint8_t *q = p;
             p += (b + 15) & ~size_t(15);
@@ -664,8 +663,6 @@ struct SelectScratch {
         hist = (uint32_t *)take(1024);
         sortb = (uint64_t *)take((size_t)kcap * 8);
         tmp = (uint64_t *)take(512);
-        s64 = (double *)take((size_t)D * 8);
-        a64 = (double *)take((size_t)D * 8);
     }
 };
 
