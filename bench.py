@@ -162,13 +162,20 @@ class ClockSampler:
             getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
         return int(fn(self._h))
 
+    def sample(self):
+        """One reading now (also called by the timing loop after every step:
+        the polling thread can be starved of the interpreter lock)."""
+        if self._thread is None:
+            return
+        try:
+            self.samples.append((float(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM)),
+                                 self._reasons()))
+        except Exception:
+            pass
+
     def _poll(self):
-        nv = self._nv
         while not self._stop.is_set():
-            try:
-                self.samples.append((float(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)), self._reasons()))
-            except Exception:
-                pass
+            self.sample()
             time.sleep(0.001)
 
     def __exit__(self, *exc):
@@ -185,7 +192,8 @@ class ClockSampler:
             mask |= r
         reasons = sorted(n for n, bit in self.REASONS.items() if mask & bit)
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(mhz), "source": "NVML, 1 ms polling during the timed steps"}
+                "samples": len(mhz), "source": "NVML: 1 ms polling thread during the timed steps plus one reading "
+                "as each step completes"}
 
 
 # ---------------------------------------------------------------------------
@@ -315,6 +323,7 @@ def run_ours(args):
             step()
             b.record(stream)
             b.synchronize()
+            clk.sample()
             step_ms.append(a.elapsed_time(b))
             st = tree.stage_times()
             for i in range(3):
