@@ -237,11 +237,10 @@ atlaskv_status launch_score_ht(const akv::DescendParams &dp, int L, int GC, cuda
     if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "scoring grid too large");
     const size_t smem = akv::score_kernel_smem<D, (int)sizeof(T)>(GC, Kp);
     if (smem > 227 * 1024) return fail(ATLASKV_EUNSUPPORTED, "scoring needs %zu bytes of shared memory", smem);
-    static size_t configured = 0;
-    if (smem > 48 * 1024 && smem > configured) {
+    // per device and cheap: set whenever the launch needs more than the default 48 KB
+    if (smem > 48 * 1024) {
         AKV_CUDA(cudaFuncSetAttribute(akv::score_kernel<T, D, HT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem));
-        configured = smem;
     }
     akv::score_kernel<T, D, HT><<<(unsigned)grid, akv::kScoreThreads, smem, s>>>(dp, L, GC, ppc, pchunks);
     AKV_CUDA(cudaGetLastError());
@@ -285,11 +284,9 @@ atlaskv_status launch_select(const akv::DescendParams &dp, int L, cudaStream_t s
     if (st != ATLASKV_OK) return st;
     // tier 3 for whatever the bounds left undecided (usually nothing: the warps read an empty queue)
     const size_t esmem = (size_t)akv::kSelectWarps * akv::ExactScratch::bytes(dp.kcap, D);
-    static size_t econfigured = 0;
-    if (esmem > 48 * 1024 && esmem > econfigured) {
+    if (esmem > 48 * 1024) {
         AKV_CUDA(cudaFuncSetAttribute(akv::exact_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)esmem));
-        econfigured = esmem;
     }
     const long long egrid = std::min<long long>((BH + akv::kSelectWarps - 1) / akv::kSelectWarps, 2 * 148);
     akv::exact_kernel<T, D><<<(unsigned)egrid, akv::kSelectWarps * 32, esmem, s>>>(dp, L);
@@ -332,11 +329,8 @@ atlaskv_status launch_attend_bf16(const akv::AttnParams &ap, cudaStream_t s)
     const long long grid = (long long)ap.B * ap.H_kv * bpg;
     if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "attention grid too large");
     const int smem = akv::AttnSmem<D>::BYTES;
-    static bool configured = false;
-    if (!configured) {
-        AKV_CUDA(cudaFuncSetAttribute(akv::attend_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-        configured = true;
-    }
+    // the attribute is per device: set it on every launch (a cheap host call)
+    AKV_CUDA(cudaFuncSetAttribute(akv::attend_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     akv::attend_bf16_kernel<D><<<(unsigned)grid, akv::kAttnWarps * 32, smem, s>>>(ap, bpg);
     AKV_CUDA(cudaGetLastError());
     return ATLASKV_OK;
@@ -396,12 +390,9 @@ atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
     if (st != ATLASKV_OK) return st;
     st = encode_seq_map(&mv, ap.v_seq, ap.B, ap.T, ap.H_kv);
     if (st != ATLASKV_OK) return st;
-    static bool configured = false;
-    if (!configured) {
-        AKV_CUDA(cudaFuncSetAttribute(akv::attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      akv::tc::kSmemBytes));
-        configured = true;
-    }
+    // the attribute is per device: set it on every launch (a cheap host call)
+    AKV_CUDA(cudaFuncSetAttribute(akv::attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  akv::tc::kSmemBytes));
     akv::attend_tc_kernel<<<(unsigned)grid, akv::tc::kThreads, akv::tc::kSmemBytes, s>>>(ap, cpg, mk, mv);
     AKV_CUDA(cudaGetLastError());
     return ATLASKV_OK;
@@ -431,10 +422,9 @@ atlaskv_status launch_dedupe(const int32_t *ids, int n, int groups, int32_t *uni
 {
     const int n2 = pow2_at_least(n, 2);
     const size_t smem = (size_t)n2 * 12;
-    static size_t configured = 0;
-    if (smem > 48 * 1024 && smem > configured) {
+    // per device and cheap: set whenever the launch needs more than the default 48 KB
+    if (smem > 48 * 1024) {
         AKV_CUDA(cudaFuncSetAttribute(akv::dedupe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        configured = smem;
     }
     akv::dedupe_kernel<<<groups, akv::kDedupeThreads, smem, s>>>(ids, n, n2, uniq, slot, count);
     AKV_CUDA(cudaGetLastError());

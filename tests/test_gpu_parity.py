@@ -224,6 +224,22 @@ def test_leaves_in_pinned_host_memory_small():
     compare(w, sh.keep, g_host)
 
 
+def test_leaves_in_pinned_host_memory_chunked():
+    # B = 9 splits into four query chunks (2, 2, 2, 3) staged on a second stream
+    # while the other chunks compute; results equal the HBM-resident path.
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(12, 10, 9),
+                      keep=(3, 4, 16), batch=9, n_tokens=16, seq_len=48, permuted=True)
+    w = synth.make_workload(sh, "cuda", 15)
+    g_dev = gpu_run(w, sh.keep)
+    hw = synth.Workload(sh, w.root_keys, w.mid_keys, w.leaf_keys.cpu().pin_memory(),
+                        w.leaf_values.cpu().pin_memory(), w.root_child, w.mid_child, w.q_kg, w.q_seq, w.k_seq,
+                        w.v_seq, w.targets)
+    g_host = gpu_run(hw, sh.keep)
+    for k in ("kept_root", "kept_mid", "kept_leaf", "out", "lse"):
+        assert torch.equal(g_dev[k], g_host[k]), k
+    compare(w, sh.keep, g_host)
+
+
 def test_deterministic_and_b0():
     sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(10, 10, 10),
                       keep=(3, 4, 16), batch=4, n_tokens=32, seq_len=64)
