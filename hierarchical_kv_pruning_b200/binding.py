@@ -27,7 +27,7 @@ ATLASKV_LEAVES_DEVICE, ATLASKV_LEAVES_HOST_PINNED = 0, 1
 # Every symbol include/atlaskv.h declares.
 EXPORTED = ("atlaskv_create_tree", "atlaskv_workspace_size", "atlaskv_attend", "atlaskv_sync_status",
             "atlaskv_set_profiling", "atlaskv_stage_times", "atlaskv_refine_stats", "atlaskv_attend_static",
-            "atlaskv_destroy", "atlaskv_last_error")
+            "atlaskv_probe_wait_timeout", "atlaskv_destroy", "atlaskv_last_error")
 # Size of the library's static device scratch (ATLASKV_STATIC_SCRATCH_BYTES).
 ATLASKV_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -91,6 +91,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
             lib.atlaskv_set_profiling.argtypes = [V, I32]
             lib.atlaskv_stage_times.argtypes = [V, ctypes.POINTER(ctypes.c_float), I32]
             lib.atlaskv_refine_stats.argtypes = [V, ctypes.POINTER(ctypes.c_uint64), I32]
+            lib.atlaskv_probe_wait_timeout.argtypes = [V, V]
             lib.atlaskv_destroy.argtypes = [V]
             lib.atlaskv_last_error.argtypes = []
             lib.atlaskv_last_error.restype = ctypes.c_char_p
@@ -161,6 +162,10 @@ def atlaskv_refine_stats(tree: int):
     v = [int(x) for x in buf]
     return {lvl: dict(zip(("selections", "refined", "ambiguous", "exact_scores"), v[4 * i:4 * i + 4]))
             for i, lvl in enumerate(("root", "mid", "leaf"))}
+
+
+def atlaskv_probe_wait_timeout(tree: int, stream: int = 0) -> None:
+    _check(load_library().atlaskv_probe_wait_timeout(ctypes.c_void_p(tree), ctypes.c_void_p(stream)))
 
 
 def atlaskv_destroy(tree: int) -> None:
@@ -272,6 +277,9 @@ class HikvpTree:
 
     def sync_status(self, stream=None):
         atlaskv_sync_status(self.handle, _stream(stream))
+
+    def probe_wait_timeout(self, stream=None):
+        atlaskv_probe_wait_timeout(self.handle, _stream(stream))
 
     def set_profiling(self, enable: bool):
         atlaskv_set_profiling(self.handle, enable)

@@ -353,15 +353,16 @@ atlaskv_status launch_attend_f32(const akv::AttnParams &ap, cudaStream_t s)
 // reached through the runtime's driver entry point.
 atlaskv_status encode_seq_map(CUtensorMap *map, const void *base, int B, int T, int H_kv)
 {
-    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-    if (!encode) {
+    // looked up once per process (thread-safe static initialisation)
+    static const PFN_cuTensorMapEncodeTiled_v12000 encode = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         cudaDriverEntryPointQueryResult q;
         void *fn = nullptr;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess || !fn)
-            return fail(ATLASKV_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
-        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    }
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }();
+    if (!encode) return fail(ATLASKV_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
     if (reinterpret_cast<uintptr_t>(base) & 15u) return fail(ATLASKV_EINVAL, "sequence K/V must be 16-byte aligned");
     const int D = akv::tc::kD;
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H_kv, (cuuint64_t)T, (cuuint64_t)B};
@@ -405,15 +406,13 @@ atlaskv_status dispatch_attend(int dtype, int D, const akv::AttnParams &ap, cuda
 }
 
 // ---- staging launches -----------------------------------------------------
+// SM count of the current device (a grid size, not a correctness matter).
 int num_sms()
 {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            n <= 0)
-            n = 148;
-    }
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        n <= 0)
+        n = 148;
     return n;
 }
 
@@ -864,6 +863,14 @@ atlaskv_status atlaskv_refine_stats(atlaskv_tree *t, uint64_t *counts, int32_t n
     unsigned long long v[12];
     AKV_CUDA(cudaMemcpy(v, t->stats, sizeof v, cudaMemcpyDeviceToHost));
     for (int i = 0; i < n && i < 12; ++i) counts[i] = v[i];
+    return ATLASKV_OK;
+}
+
+atlaskv_status atlaskv_probe_wait_timeout(atlaskv_tree *t, void *stream)
+{
+    if (!t) return fail(ATLASKV_EINVAL, "null tree");
+    akv::wait_timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(t->status);
+    AKV_CUDA(cudaGetLastError());
     return ATLASKV_OK;
 }
 

@@ -55,7 +55,7 @@ constexpr int kProducerWarp = 4 * kWG;
 constexpr int kMmaWarp = 4 * kWG + 1;
 constexpr int kThreads = 32 * (4 * kWG + 2);
 constexpr int kCtaRows = kWG * kRows;
-constexpr long long kSpinLimit = 1ll << 22;   // bounded mbarrier waits (seconds at most)
+constexpr long long kSpinLimit = 1ll << 18;   // bounded mbarrier waits (about a second on B200)
 constexpr float kRescaleLog2 = 8.f;            // rescale O only when the row max grows by more than this
 
 // shared memory (byte offsets from a 1024-aligned base; operand tiles in the
@@ -241,6 +241,21 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
 }
 
 }  // namespace tc
+
+// A wait that cannot complete: one mbarrier with an expected arrival that
+// never comes, waited on with the attention kernel's bounded wait, which gives
+// up and reports ETIMEOUT through the status word.
+__global__ void wait_timeout_probe_kernel(int *status)
+{
+    __shared__ __align__(8) uint64_t never;
+    const uint32_t b = tc::smem_addr(&never);
+    if (threadIdx.x == 0) {
+        tc::mbar_init(b, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !tc::mbar_wait(b, 0)) set_status(status, kDevTimeout);
+}
 
 // One CTA per (query b, KV head, kWG x 128-row block of the group's G N rows).
 // tm_k / tm_v: the sequence keys / values [B][T][H_kv][D] as 4-D tensor maps

@@ -192,6 +192,16 @@ atlaskv_status atlaskv_refine_stats(atlaskv_tree *tree, uint64_t *counts, int32_
 atlaskv_status atlaskv_attend_static(atlaskv_tree *tree, const atlaskv_params *params, const atlaskv_io *io,
                                      void *stream);
 
+/* Diagnostic; the paper has no counterpart.  Enqueues on `stream` one CTA
+ * that waits, with the same bounded mbarrier wait the attention kernel uses,
+ * on a barrier that nothing ever arrives on.  The wait gives up after its
+ * iteration limit and sets ATLASKV_ETIMEOUT in the tree's sticky status word,
+ * which the next atlaskv_sync_status returns; the CUDA context stays usable.
+ * It shows that a stalled device wait is reported instead of hanging.  It
+ * takes about a second, and it leaves the tree's status at ETIMEOUT, so run
+ * it on a tree made for the purpose.  Returns ECUDA if the launch fails. */
+atlaskv_status atlaskv_probe_wait_timeout(atlaskv_tree *tree, void *stream);
+
 /* Release the handle and the small device buffers it owns; the caller's
  * buffers are untouched.  NULL is accepted. */
 atlaskv_status atlaskv_destroy(atlaskv_tree *tree);

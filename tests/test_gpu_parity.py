@@ -307,3 +307,22 @@ def test_full_size_host_leaves():
     check_structure(w, sh.keep, g)
     trav = sample_traversals(sh.batch, sh.n_heads, 6, seed=4)
     compare(w, sh.keep, g, trav)
+
+
+def test_bounded_device_wait_reports_timeout():
+    # A device wait that can never complete gives up after its iteration limit
+    # and the host reads ETIMEOUT from the tree's status word; the context
+    # stays usable (a fresh tree still attends correctly afterwards).
+    import time
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=2, n_kv_heads=1, head_dim=128, fanout=(4, 4, 4),
+                      keep=(2, 2, 2), batch=1, n_tokens=2, seq_len=2)
+    w = synth.make_workload(sh, "cuda", 16)
+    with HikvpTree.from_workload(w) as tree:
+        t0 = time.time()
+        tree.probe_wait_timeout()
+        with pytest.raises(AtlaskvError) as ei:
+            tree.sync_status()
+        assert ei.value.status == 5           # ATLASKV_ETIMEOUT
+        assert time.time() - t0 < 60
+    g = gpu_run(w, sh.keep)
+    compare(w, sh.keep, g)
