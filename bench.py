@@ -406,6 +406,9 @@ def run_ours(args):
     roof["algorithmic_bytes"] = {k: alg[k] for k in ("descend", "attend", "staging")}
     roof["attend_flops"] = alg["attend_flops"]
     roof["attend_tflops"] = alg["attend_flops"] / (st_ms[2] * 1e-3) / 1e12 if st_ms[2] > 0 else None
+    # the attention's tensor-pipe share: achieved dense bf16 rate / measured burst peak
+    roof["attend_tensor_frac"] = (roof["attend_tflops"] / peaks["bf16_tflops"]
+                                  if roof["attend_tflops"] and sh.dtype == torch.bfloat16 else None)
     roof["exact_refinement_last_step"] = refine
 
     clocks = clk.summary()

@@ -1092,11 +1092,21 @@ __global__ void __launch_bounds__(kSelectWarps * 32) exact_kernel(const DescendP
         const int K = p.K[L];
         int r = K - nsel;
         const int Kp = L == 0 ? 0 : p.K[L - 1];
-        for (int k = lane; k < Kp; k += 32) sc.prev[k] = p.kept[L - 1][bh * Kp + k];
+        // every load that depends only on the queue entry goes out together:
+        // kept parents, decided entries, the fp64 token sums for tier 2 and
+        // this lane's listed candidate
+        const bool tier2 = !bad && nlist <= 32;
         const float *fslot = p.f_ws + (size_t)bh * p.fstride;
         const int *list = reinterpret_cast<const int *>(fslot);
         const uint64_t *decided = reinterpret_cast<const uint64_t *>(fslot + p.cap);
+        for (int k = lane; k < Kp; k += 32) sc.prev[k] = p.kept[L - 1][bh * Kp + k];
         for (int i = lane; i < nsel; i += 32) sc.sortb[i] = decided[i];
+        if (tier2)
+            for (int d = lane; d < D; d += 32) {
+                sc.s64[d] = p.s64_ws[(size_t)bh * D + d];
+                sc.a64[d] = p.a64_ws[(size_t)bh * D + d];
+            }
+        const int my_pos = tier2 && lane < nlist ? list[lane] : -1;
         __syncwarp();
         const LevelView lv = level_view<T>(p, L, bh, sc.prev);
         const int b = (int)(bh / p.H), h = (int)(bh % p.H);
@@ -1104,15 +1114,8 @@ __global__ void __launch_bounds__(kSelectWarps * 32) exact_kernel(const DescendP
         const size_t q_stride = (size_t)p.H * D;
         const T *kbase = reinterpret_cast<const T *>(p.keys[L]);
 
-        if (!bad && nlist <= 32) {
+        if (tier2) {
             // ---- tier 2 ----
-            if (p.stats && lane == 0) atomicAdd(p.stats + L * 4 + 3, 0ull);
-            for (int d = lane; d < D; d += 32) {
-                sc.s64[d] = p.s64_ws[(size_t)bh * D + d];
-                sc.a64[d] = p.a64_ws[(size_t)bh * D + d];
-            }
-            __syncwarp();
-            const int my_pos = lane < nlist ? list[lane] : -1;
             double y = -INFINITY, e2 = 0.0;
             if (my_pos >= 0) {
                 const T *krow = kbase + (size_t)lv.row(my_pos) * D;
