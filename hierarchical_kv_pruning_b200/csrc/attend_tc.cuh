@@ -55,7 +55,7 @@ constexpr int kProducerWarp = 4 * kWG;
 constexpr int kMmaWarp = 4 * kWG + 1;
 constexpr int kThreads = 32 * (4 * kWG + 2);
 constexpr int kCtaRows = kWG * kRows;
-constexpr long long kSpinLimit = 1ll << 18;   // bounded mbarrier waits (about a second on B200)
+constexpr long long kSpinLimit = 1ll << 18;   // bounded mbarrier waits: try_wait iterations, not a fixed time
 constexpr float kRescaleLog2 = 8.f;            // rescale O only when the row max grows by more than this
 
 // shared memory (byte offsets from a 1024-aligned base; operand tiles in the

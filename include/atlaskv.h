@@ -198,8 +198,9 @@ atlaskv_status atlaskv_attend_static(atlaskv_tree *tree, const atlaskv_params *p
  * iteration limit and sets ATLASKV_ETIMEOUT in the tree's sticky status word,
  * which the next atlaskv_sync_status returns; the CUDA context stays usable.
  * It shows that a stalled device wait is reported instead of hanging.  It
- * takes about a second, and it leaves the tree's status at ETIMEOUT, so run
- * it on a tree made for the purpose.  Returns ECUDA if the launch fails. */
+ * takes milliseconds or more (the hardware sets each try_wait's suspend
+ * time), and it leaves the tree's status at ETIMEOUT, so run it on a tree
+ * made for the purpose.  Returns ECUDA if the launch fails. */
 atlaskv_status atlaskv_probe_wait_timeout(atlaskv_tree *tree, void *stream);
 
 /* Release the handle and the small device buffers it owns; the caller's
