@@ -277,6 +277,49 @@ def test_device_errors_are_reported():
         assert ei.value.status == 1
 
 
+
+def test_attend_rejects_invalid_calls_without_side_effects():
+    # Every host-side reject of the attend boundary returns EINVAL before
+    # anything is enqueued; the caller's output buffers keep their contents and
+    # the tree stays usable.
+    from hierarchical_kv_pruning_b200.binding import ATLASKV_EINVAL
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=4, n_kv_heads=2, head_dim=128, fanout=(4, 4, 4),
+                      keep=(2, 2, 2), batch=1, n_tokens=2, seq_len=3)
+    w = synth.make_workload(sh, "cuda", 17)
+    q, qs, k, v = w.q_kg, w.q_seq, w.k_seq, w.v_seq
+
+    def misaligned(t):
+        flat = torch.full((t.numel() + 8,), 7.0, dtype=t.dtype, device=t.device)
+        m = flat[1:1 + t.numel()].view(t.shape)   # 2 bytes past a 16-byte boundary
+        m.copy_(t)
+        return m
+
+    out = torch.full_like(q, 7.0)
+    cases = [
+        dict(K=(5, 2, 2)),                      # K_root > b_R
+        dict(K=(0, 2, 2)),                      # K_root < 1
+        dict(K=(2, 9, 2)),                      # K_mid > K_root b_I
+        dict(K=(2, 2, 9)),                      # K_leaf > K_mid b_L
+        dict(scale=-1.0),
+        dict(scale=float("inf")),
+        dict(q=q[:, :, :3].contiguous(), qs=qs[:, :, :3].contiguous()),   # H = 3 not a multiple of H_kv = 2
+        dict(q=torch.cat([q, q], 1), qs=torch.cat([qs, qs], 1)),          # N = 4 > T = 3
+        dict(q=misaligned(q)),
+        dict(out=misaligned(torch.full_like(q, 7.0))),
+    ]
+    with HikvpTree.from_workload(w) as tree:
+        for c in cases:
+            qq, qqs = c.get("q", q), c.get("qs", qs)
+            o = c.get("out", out if qq.shape == q.shape else torch.full_like(qq, 7.0))
+            with pytest.raises(AtlaskvError) as ei:
+                tree.attend(qq, qqs, k, v, c.get("K", sh.keep), scale=c.get("scale", 0.0), out=o)
+            assert ei.value.status == ATLASKV_EINVAL, c
+            torch.cuda.synchronize()
+            assert bool((o.float() == 7.0).all()), c
+        g = gpu_run(w, sh.keep, tree=tree)
+    compare(w, sh.keep, g)
+
+
 # ---- benchmark shapes at full size ----------------------------------------
 
 @pytest.fixture(scope="module")
