@@ -8,6 +8,7 @@ kept sets must come back in ascending row order.  Scores here are recomputed
 with Python fractions, independently of the oracle's C accumulator.
 """
 import itertools
+import random
 from fractions import Fraction
 
 import pytest
@@ -165,3 +166,57 @@ def test_rejects_k_above_candidates():
         oracle.descend(oracle_tree(w), storage(w.q_kg), (1, 4, 1))
     with pytest.raises(ValueError):
         oracle.descend(oracle_tree(w), storage(w.q_kg), (1, 1, 4))
+
+
+# ---- randomized sweep, checked against the definition written out directly ----
+
+def _children_from_tables(w, level, hkv, p):
+    """Children of node p of `level`, read straight off the workload's child
+    tables (or the implicit layout p * fan-out + j), not through the oracle."""
+    fo = w.shape.fanout[level + 1]
+    tab = w.root_child if level == 0 else w.mid_child
+    if tab is None:
+        return [p * fo + j for j in range(fo)]
+    return [int(x) for x in tab[hkv, p].tolist()]
+
+
+def _greedy_by_definition(w, K, b, h):
+    """Kept sets of one traversal: at each level sort the candidates by exact
+    score (descending) then row id, keep the first K, report them ascending.
+    The exact score is (sum over tokens of q) . k, in rationals."""
+    sh = w.shape
+    hkv = h // (sh.n_heads // sh.n_kv_heads)
+    q = w.q_kg[b, :, h, :].double()
+    s = [sum(Fraction(float(q[n, d])) for n in range(q.shape[0])) for d in range(q.shape[1])]
+    kept, cands = [], list(range(sh.fanout[0]))
+    for level, keys in enumerate((w.root_keys, w.mid_keys, w.leaf_keys)):
+        if level > 0:
+            cands = [c for p in kept[-1] for c in _children_from_tables(w, level - 1, hkv, p)]
+        k = keys[hkv].double()
+        score = {r: sum(s[d] * Fraction(float(k[r, d])) for d in range(len(s))) for r in cands}
+        ranked = sorted(cands, key=lambda r: (-score[r], r))
+        kept.append(sorted(ranked[:K[level]]))
+    return kept
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_random_trees_match_the_greedy_definition(seed):
+    rng = random.Random(seed)
+    fanout = tuple(rng.randint(2, 5) for _ in range(3))
+    H_kv, G = rng.choice([1, 2, 2]), rng.choice([1, 2, 3])
+    K_R = rng.randint(1, fanout[0])
+    K_I = rng.randint(1, K_R * fanout[1])
+    K_L = rng.randint(1, K_I * fanout[2])
+    sh = synth.custom(dtype=rng.choice([torch.float32, torch.bfloat16]), n_heads=G * H_kv, n_kv_heads=H_kv,
+                      head_dim=rng.choice([4, 8]), fanout=fanout, keep=(K_R, K_I, K_L), batch=2,
+                      n_tokens=rng.randint(1, 3), seq_len=3, permuted=rng.random() < 0.7)
+    w = synth.make_workload(sh, "cpu", 100 + seed)
+    # exact ties: copy a few key rows onto others at every level
+    for keys in (w.root_keys, w.mid_keys, w.leaf_keys):
+        for _ in range(2):
+            a, c = rng.randrange(keys.shape[1]), rng.randrange(keys.shape[1])
+            keys[:, c] = keys[:, a]
+    kr, km, kl = oracle.descend(oracle_tree(w), storage(w.q_kg), sh.keep)
+    for i, (b, h) in enumerate(itertools.product(range(2), range(sh.n_heads))):
+        got = [kr[i].tolist(), km[i].tolist(), kl[i].tolist()]
+        assert got == _greedy_by_definition(w, sh.keep, b, h), (seed, b, h)
