@@ -220,3 +220,22 @@ def test_random_trees_match_the_greedy_definition(seed):
     for i, (b, h) in enumerate(itertools.product(range(2), range(sh.n_heads))):
         got = [kr[i].tolist(), km[i].tolist(), kl[i].tolist()]
         assert got == _greedy_by_definition(w, sh.keep, b, h), (seed, b, h)
+
+
+def test_ranking_across_a_borrow():
+    # x0 = 2^a - 20 u comes from two products of opposite sign in two digits of
+    # the exact accumulator (2^a at bit 0 of a digit, -20 u = -5 u 2^2 in the
+    # digit below); x1 = 2^a - 16 u is one product inside the lower digit.  The
+    # ranking must put x1 above x0 (u = 2^(a - 22)).
+    a = (-oracle.exact_origin()) % 32
+    while a < 22:
+        a += 32
+    u = 2.0 ** (a - 22)
+    sh = synth.custom(dtype=torch.float32, n_heads=1, n_kv_heads=1, head_dim=4, fanout=(3, 1, 1),
+                      batch=1, n_tokens=1, seq_len=1)
+    w = synth.make_workload(sh, "cpu", 2)
+    w.root_keys[0] = torch.tensor([[2.0 ** a, -20 * u, 0, 0], [2.0 ** a - 16 * u, 0, 0, 0], [0, 0, 0, 0]])
+    w.q_kg[0, 0, 0] = torch.tensor([1.0, 1.0, 0, 0])
+    tree, q = oracle_tree(w), storage(w.q_kg)
+    assert oracle.descend(tree, q, (1, 1, 1))[0].tolist() == [[1]]
+    assert oracle.descend(tree, q, (2, 1, 1))[0].tolist() == [[0, 1]]

@@ -134,3 +134,17 @@ def test_identities(seed):
     ref = float(np.sum(q.astype(np.float64) * k.astype(np.float64)))
     bound = N * D * 2.0 ** -52 * float(np.sum(np.abs(q.astype(np.float64)) * np.abs(k.astype(np.float64))))
     assert abs(x / 2.0 ** oracle.exact_origin() - ref) <= bound
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_digits_are_canonical(seed):
+    # The ranking compares digit strings from the top down, which orders the
+    # values only when every digit below the top one lies in [0, 2^32) (the
+    # top one carries the sign).  Mixed signs exercise the borrows.
+    rng = np.random.default_rng(100 + seed)
+    for _ in range(50):
+        N, D = int(rng.integers(1, 4)), int(rng.integers(1, 9))
+        q = _bits_f32(_special_values(rng, N * D).reshape(N, D))
+        k = _bits_f32(_special_values(rng, D))
+        dig = oracle.exact_digits(q, k)
+        assert all(0 <= int(d) < 1 << 32 for d in dig[:-1]), dig
