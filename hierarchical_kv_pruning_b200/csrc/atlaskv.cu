@@ -211,7 +211,7 @@ atlaskv_status check_table(const int32_t *tab, long long entries_per_head, int H
 
 // ---- descent launches -----------------------------------------------------
 // Scoring CTAs serve GP query heads of a (query, KV head) group: the largest
-// of 4, 2, 1 that divides G.  Selection runs one warp per traversal.
+// of 4, 2, 1 that divides G.  Selection runs one CTA per traversal.
 int heads_per_cta(int G) { return G % 4 == 0 ? 4 : (G % 2 == 0 ? 2 : 1); }
 
 template <typename T, int D, int GP>

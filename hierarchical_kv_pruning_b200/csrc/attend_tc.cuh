@@ -19,11 +19,11 @@
 //                   ring, each guarded by full / empty mbarriers;
 //   MMA warp        one thread issues S(w, t) = Q_w K_t^T (M 128, N 64,
 //                   K 128, both operands in shared memory) into a double-
-//                   buffered S in TMEM for both warpgroups, then
+//                   buffered S in TMEM for each warpgroup, then
 //                   O_w += P_w V_{t-1} (M 128, N 128, K 64) with P_w read from
 //                   TMEM, so S(t) runs under softmax(t - 1); tcgen05.commit
 //                   arrives on the mbarriers;
-//   2 warpgroups    one thread per query row: read its S row (tcgen05.ld),
+//   kWG warpgroups  one thread per query row: read its S row (tcgen05.ld),
 //                   mask, online softmax with a lazily rescaled running max
 //                   (O in TMEM is rescaled only when the row max grows by more
 //                   than 2^8), P (bf16 pairs) written back over the first half

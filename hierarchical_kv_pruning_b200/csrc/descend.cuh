@@ -9,10 +9,13 @@
 //
 // The descent runs level-synchronously over all traversals (query b, head h):
 //   root_kernel    token sums s of GP heads per CTA, fp32 scores of all roots
-//   select_kernel  one warp per traversal: top-K of its candidates' scores
-//   score_kernel   one CTA per (query, KV head, chunk of the union of its GP
-//                  heads' kept parents): every child row is loaded once and
-//                  scored against the GP token-sum vectors
+//   select_kernel  one CTA (64 or 128 threads) per traversal: top-K of its
+//                  candidates' fp32 scores, with a rigorous error band
+//   exact_kernel   one warp per queued traversal: the band's candidates in
+//                  fp64, then in exact arithmetic
+//   score_kernel   one CTA per (query, KV head, chunk of GC <= 32 heads, chunk
+//                  of the union of their kept parents): every child row is
+//                  loaded once and scored against the GC token-sum vectors
 // Scores live in a per-traversal buffer (workspace, L2-resident at the
 // benchmark sizes); each phase is a wide, short kernel.
 //
