@@ -65,9 +65,12 @@ def config_of(sh, world):
 
 def kernels_per_step(sh):
     """Kernels one atlaskv_attend call launches: per level (root or children
-    scoring, selection, exact pass) x 3, attention, and for host-resident
-    leaves two de-duplications and two staging copies."""
-    return 3 * 3 + 1 + (4 if sh.leaf_on_host else 0)
+    scoring, selection, exact pass) x 3 and the attention.  With host-resident
+    leaves add two de-duplications and two staging copies, and the call runs
+    all of them once per query chunk (four chunks when B >= 8, else one)."""
+    if not sh.leaf_on_host:
+        return 3 * 3 + 1
+    return (3 * 3 + 1 + 4) * (4 if sh.batch >= 8 else 1)
 
 
 def max_over_ranks(x, world, device):

@@ -141,7 +141,8 @@ atlaskv_status atlaskv_workspace_size(const atlaskv_tree *tree, const atlaskv_pa
  * attention and merge.  `workspace` is device memory of at least
  * atlaskv_workspace_size() bytes, 256-byte aligned, not shared with a
  * concurrent call.  With host-resident leaves the batch is processed in query
- * chunks and the leaf blocks are staged on a second stream owned by the tree
+ * chunks (four when B >= 8, else one; each chunk launches every kernel of the
+ * path) and the leaf blocks are staged on a second stream owned by the tree
  * (joined back into `stream` before the call's last kernel), so the host link
  * works while other chunks compute; calls on one such tree must therefore not
  * overlap.  Returns EINVAL / ENOMEM (workspace too small) / EUNSUPPORTED

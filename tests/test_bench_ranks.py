@@ -68,7 +68,9 @@ def test_kernels_per_step_and_config():
     dev = synth.shape(2)
     host = synth.shape(4)
     assert bench.kernels_per_step(dev) == 10
-    assert bench.kernels_per_step(host) == 14
+    assert host.batch >= 8 and bench.kernels_per_step(host) == 4 * 14   # four query chunks
+    import dataclasses
+    assert bench.kernels_per_step(dataclasses.replace(host, batch=7)) == 14
     c = bench.config_of(dev, 4)
     assert c["workload"] == dev.name and c["parallelism"] == "replicas x4"
     assert c["B"] == dev.batch and c["K"] == list(dev.keep)
