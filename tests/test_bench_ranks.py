@@ -74,3 +74,39 @@ def test_kernels_per_step_and_config():
     c = bench.config_of(dev, 4)
     assert c["workload"] == dev.name and c["parallelism"] == "replicas x4"
     assert c["B"] == dev.batch and c["K"] == list(dev.keep)
+
+
+def test_algorithmic_bytes_worked_example():
+    # B = 1, N = 2, H = 2 heads on H_kv = 1, D = 4, bf16 (2 bytes), fan-outs
+    # (3, 2, 2), K = (2, 2, 2), T = 3.  Kept sets of the two heads overlap, so
+    # the unique rows of the batch are roots {0,1,2}, mids {0,1,3}, leaves
+    # {0,5,7}: 3 each.  By hand:
+    #   descent: q_kg 2*1*2*2*4 = 32; key rows read (roots 1*3, mid candidates
+    #            3*2, leaf candidates 3*2) * 4 * 2 = 120; kept ids
+    #            4*1*2*(2+2+2) = 48; total 200 (plus 4 B per child-table
+    #            entry read, 4*(6+6) = 48, when the tree has tables)
+    #   attention: q_kg, q_seq, out 3*1*2*2*4*2 = 96; k_seq, v_seq
+    #            2*1*3*1*4*2 = 48; lse 4*1*2*2 = 16; leaf ids 4*1*2*2 = 16;
+    #            leaf K and V rows 2*2*4*3 = 48; total 224
+    #   flops: 4 * B*H*D * (visible sequence keys 2 + 3, plus N*K_L = 4) = 288
+    import dataclasses
+    import types
+
+    import torch
+
+    from hierarchical_kv_pruning_b200 import synth
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=2, n_kv_heads=1, head_dim=4, fanout=(3, 2, 2),
+                      keep=(2, 2, 2), batch=1, n_tokens=2, seq_len=3)
+    res = {"kept_root": torch.tensor([[[0, 1], [1, 2]]]),
+           "kept_mid": torch.tensor([[[0, 1], [1, 3]]]),
+           "kept_leaf": torch.tensor([[[0, 5], [5, 7]]])}
+    a = bench.algorithmic_bytes(sh, res, types.SimpleNamespace(root_child=None))
+    assert (a["u_root"], a["u_mid"], a["u_leaf"]) == (3, 3, 3)
+    assert a["descend"] == 200 and a["attend"] == 224 and a["attend_flops"] == 288 and a["staging"] == 0
+    a = bench.algorithmic_bytes(sh, res, types.SimpleNamespace(root_child=torch.zeros(1)))
+    assert a["descend"] == 200 + 48
+    # host-resident leaves: the staged bytes are the leaf-key blocks of the
+    # unique kept mids (6 rows) and the unique kept leaves' value rows (3)
+    host = dataclasses.replace(sh, leaf_on_host=True)
+    a = bench.algorithmic_bytes(host, res, types.SimpleNamespace(root_child=None))
+    assert a["staging"] == 2 * 4 * (6 + 3)
