@@ -110,3 +110,23 @@ def test_algorithmic_bytes_worked_example():
     host = dataclasses.replace(sh, leaf_on_host=True)
     a = bench.algorithmic_bytes(host, res, types.SimpleNamespace(root_child=None))
     assert a["staging"] == 2 * 4 * (6 + 3)
+
+
+def test_profiled_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
+    # The bench line's `traffic` comes from a committed summary only while the
+    # kernel's source still hashes to the one that was captured.
+    import hashlib
+    csrc = tmp_path / "hierarchical_kv_pruning_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    src = csrc / "attend_tc.cuh"
+    src.write_bytes(b"// kernel v1\n")
+    digest = hashlib.sha256(b"// kernel v1\n").hexdigest()
+    (tmp_path / "profiles" / "attend_tc_kernel__w.md").write_text(
+        "# summary\n\n- kernel: `attend_tc_kernel`\n- source_sha256: `%s`\n  (note)\n"
+        "- dram_bytes_per_launch: 12345\n" % digest)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("attend_tc_kernel", "w") == 12345
+    assert bench.profiled_traffic("attend_tc_kernel", "other") is None     # no summary for that workload
+    src.write_bytes(b"// kernel v2\n")
+    assert bench.profiled_traffic("attend_tc_kernel", "w") is None         # source changed since the capture
