@@ -130,3 +130,26 @@ def test_profiled_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic("attend_tc_kernel", "other") is None     # no summary for that workload
     src.write_bytes(b"// kernel v2\n")
     assert bench.profiled_traffic("attend_tc_kernel", "w") is None         # source changed since the capture
+
+
+def test_peaks_fall_back_when_unmeasured(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, source = bench.measured_peaks()
+    assert source == "fallback" and peaks["hbm_gbs"] == 6650.0 and peaks["bf16_tflops"] == 1590.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6000.0, "bf16_tflops": 1500.0}')
+    peaks, source = bench.measured_peaks()
+    assert source == "measured" and peaks["hbm_gbs"] == 6000.0
+
+
+def test_clock_summary_decodes_throttle_reasons():
+    # NVML clock-event bits: 0x4 software power cap, 0x8 hardware slowdown,
+    # 0x20 software thermal, 0x40 hardware thermal; others (0x1 idle) ignored.
+    c = bench.ClockSampler(0)
+    c.max_mhz = 1965.0
+    c.samples = [(1965.0, 0x0), (1320.0, 0x4), (1900.0, 0x1)]
+    s = c.summary()
+    assert s["sm_mhz"] == 1900.0 and s["samples"] == 3 and s["reasons"] == ["sw_power_cap"]
+    c.samples.append((900.0, 0x8 | 0x40 | 0x20))
+    assert bench.ClockSampler.summary(c)["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap",
+                                                        "sw_thermal_slowdown"]
+    assert bench.ClockSampler(0).summary()["samples"] == 0
