@@ -153,3 +153,26 @@ def test_clock_summary_decodes_throttle_reasons():
     assert bench.ClockSampler.summary(c)["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap",
                                                         "sw_thermal_slowdown"]
     assert bench.ClockSampler(0).summary()["samples"] == 0
+
+
+def test_reference_arm_contract():
+    # `--impl reference` times the oracle on the host cores: rank 0 prints one
+    # JSON line with the contract's keys, any other rank exits without work.
+    import json
+    import subprocess
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "0", "--steps", "2",
+           "--warmup", "1", "--cpu-seconds", "0.5"]
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "e2e", "cpu_baseline"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["config"]["workload"] == "tiny_fp32_10x10x10"
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, env=dict(env, RANK="1"), cwd=ROOT)
+    assert r.returncode == 0 and r.stdout.strip() == ""
