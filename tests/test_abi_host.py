@@ -98,3 +98,23 @@ def test_missing_library_fails_loudly(tmp_path):
             binding.load_library(str(tmp_path / "nope.so"))
     finally:
         binding._lib = saved
+
+
+def test_product_path_never_reaches_the_oracle():
+    # The library and its binding compute everything in CUDA; no file of the
+    # package imports, loads or links the oracle (test infrastructure only).
+    import ast
+    import glob
+    pkg = os.path.join(ROOT, "hierarchical_kv_pruning_b200")
+    for path in glob.glob(os.path.join(pkg, "*.py")):
+        tree = ast.parse(open(path).read())
+        for node in ast.walk(tree):
+            if isinstance(node, ast.Import):
+                assert not any(a.name.split(".")[0] == "oracle" for a in node.names), path
+            if isinstance(node, ast.ImportFrom):
+                assert (node.module or "").split(".")[0] != "oracle", path
+            if isinstance(node, ast.Constant) and isinstance(node.value, str):
+                assert "hikvp_oracle" not in node.value, path
+    for path in glob.glob(os.path.join(pkg, "csrc", "*")) + glob.glob(os.path.join(ROOT, "include", "*")):
+        text = open(path).read()
+        assert "hikvp_oracle" not in text and "oracle/" not in text, path
