@@ -69,6 +69,19 @@ class _Tree(ctypes.Structure):
     ]
 
 
+class _CsrTree(ctypes.Structure):
+    _fields_ = [
+        ("is_bf16", ctypes.c_int),
+        ("n_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int),
+        ("n_levels", ctypes.c_int),
+        ("rows", ctypes.c_void_p),
+        ("keys", ctypes.c_void_p),
+        ("child_off", ctypes.c_void_p),
+        ("child_id", ctypes.c_void_p),
+    ]
+
+
 def _load():
     global _lib
     with _lock:
@@ -84,6 +97,8 @@ def _load():
             lib.oracle_level_scores.restype = None
             lib.oracle_exact_digits.restype = I
             lib.oracle_exact_origin.restype = I
+            lib.oracle_descend_csr.argtypes = [ctypes.POINTER(_CsrTree), P, I, I, P, I, P, P, P]
+            lib.oracle_descend_csr.restype = I
             _lib = lib
     return _lib
 
@@ -316,3 +331,88 @@ def hikvp(tree: Tree, q_kg, q_seq, k_seq, v_seq, K, traversals=None, scale=None)
     y, lse = attend_traversals(tree, q_kg, q_seq, k_seq, v_seq, kl, traversals, scale)
     return {"kept_root": kr, "kept_mid": km, "kept_leaf": kl, "y": y, "lse": lse,
             "traversals": np.asarray(traversals).reshape(-1, 2)}
+
+
+# ---------------------------------------------------------------------------
+# Trees of any depth with variable numbers of children ("Method details /
+# Hierarchical clustering of KGKVs": clusters of unequal size; the depth can be
+# set larger).
+# ---------------------------------------------------------------------------
+
+class CsrTree:
+    """Levels 0 (roots) .. L-1 (leaves), keys [H_kv][rows_l][D] per level (stored
+    numbers), leaf values [H_kv][rows_{L-1}][D].  child_off[l]: [H_kv][rows_l + 1]
+    int32 offsets into level l's child list; child_id[l]: [H_kv][rows_{l+1}]
+    int32 row ids of level l + 1, or None (the child list positions are the row
+    ids: children stored contiguously)."""
+
+    def __init__(self, keys, leaf_values, child_off, child_id=None):
+        self.keys = [_as_storage(k) for k in keys]
+        self.leaf_values = leaf_values
+        self.n_levels = len(self.keys)
+        self.child_off = [np.ascontiguousarray(o, dtype=np.int32) for o in child_off]
+        ids = child_id if child_id is not None else [None] * (self.n_levels - 1)
+        self.child_id = [None if c is None else np.ascontiguousarray(c, dtype=np.int32) for c in ids]
+        assert len(self.child_off) == self.n_levels - 1 == len(self.child_id)
+        self.n_kv_heads, _, self.head_dim = self.keys[0].shape
+        self.rows = [k.shape[1] for k in self.keys]
+        self.is_bf16 = self.keys[0].dtype == np.uint16
+        for l in range(self.n_levels - 1):
+            assert self.child_off[l].shape == (self.n_kv_heads, self.rows[l] + 1)
+
+    @property
+    def leaf_keys(self):
+        return self.keys[-1]
+
+    def children(self, level: int, hkv: int, parent: int) -> np.ndarray:
+        o = self.child_off[level][hkv]
+        pos = np.arange(o[parent], o[parent + 1])
+        ids = self.child_id[level]
+        return (pos if ids is None else ids[hkv][pos]).astype(np.int32)
+
+
+def descend_csr(tree: CsrTree, q_kg: np.ndarray, K, traversals=None):
+    """Kept node sets per level of the greedy descent on a CSR tree: a list of
+    [T][K_l] int32 arrays (ascending row ids), one per level."""
+    lib = _load()
+    q = _as_storage(q_kg)
+    assert q.dtype == tree.keys[0].dtype
+    B, N, H, D = q.shape
+    assert len(K) == tree.n_levels
+    if traversals is None:
+        bb, hh = np.meshgrid(np.arange(B), np.arange(H), indexing="ij")
+        trav = np.stack([bb.ravel(), hh.ravel()], 1)
+    else:
+        trav = np.asarray(traversals, dtype=np.int64).reshape(-1, 2)
+    tb = np.ascontiguousarray(trav[:, 0], dtype=np.int32)
+    th = np.ascontiguousarray(trav[:, 1], dtype=np.int32)
+    n = len(tb)
+    kk = np.ascontiguousarray(K, dtype=np.int32)
+    kept = [np.zeros((n, int(k)), np.int32) for k in K]
+    L = tree.n_levels
+    rows = np.ascontiguousarray(tree.rows, dtype=np.int64)
+    keys = (ctypes.c_void_p * L)(*[k.ctypes.data for k in tree.keys])
+    offs = (ctypes.c_void_p * (L - 1))(*[o.ctypes.data for o in tree.child_off])
+    ids = (ctypes.c_void_p * (L - 1))(*[None if c is None else c.ctypes.data for c in tree.child_id])
+    outs = (ctypes.c_void_p * L)(*[k.ctypes.data for k in kept])
+    ct = _CsrTree(int(tree.is_bf16), tree.n_kv_heads, tree.head_dim, L, rows.ctypes.data,
+                  ctypes.cast(keys, ctypes.c_void_p), ctypes.cast(offs, ctypes.c_void_p),
+                  ctypes.cast(ids, ctypes.c_void_p))
+    rc = lib.oracle_descend_csr(ctypes.byref(ct), q.ctypes.data, N, H, kk.ctypes.data, n, tb.ctypes.data,
+                                th.ctypes.data, ctypes.cast(outs, ctypes.c_void_p))
+    if rc != 0:
+        raise ValueError("oracle_descend_csr rejected the arguments (a level with fewer candidates than K, or a "
+                         "child id out of range)")
+    return kept
+
+
+def hikvp_csr(tree: CsrTree, q_kg, q_seq, k_seq, v_seq, K, traversals=None, scale=None):
+    """Whole hot path on a CSR tree: descent, then the merged attention over the
+    kept leaves (the last level) and the causal sequence."""
+    B, N, H, D = q_kg.shape
+    if traversals is None:
+        bb, hh = np.meshgrid(np.arange(B), np.arange(H), indexing="ij")
+        traversals = np.stack([bb.ravel(), hh.ravel()], 1)
+    kept = descend_csr(tree, q_kg, K, traversals)
+    y, lse = attend_traversals(tree, q_kg, q_seq, k_seq, v_seq, kept[-1], traversals, scale)
+    return {"kept": kept, "y": y, "lse": lse, "traversals": np.asarray(traversals).reshape(-1, 2)}

@@ -299,3 +299,101 @@ void oracle_level_scores(const oracle_tree *t, int level, const void *q_kg, int 
         memcpy(digits_out + (size_t)c * EX_DIGITS, x.dig, sizeof(x.dig));
     }
 }
+
+/* ---------------------------------------------------------------------------
+ * Trees of any depth with a variable number of children per node ("Method
+ * details / Hierarchical clustering of KGKVs": the clustering gives clusters
+ * of unequal size, and the depth can be set larger).  Level 0 holds the roots,
+ * level n_levels - 1 the leaves.  The children of node p of level l (l <
+ * n_levels - 1) are given in compressed-sparse-row form per KV head:
+ * positions child_off[l][hkv * (rows[l] + 1) + p] .. (p + 1) - 1 of level l's
+ * child list, whose entries are row ids of level l + 1 (child_id[l], laid out
+ * [H_kv][rows[l + 1]]) or, when child_id[l] is NULL, the positions themselves.
+ * The descent is the same greedy one: all roots are candidates; at each next
+ * level the candidates are the children of the kept nodes of the level above,
+ * ranked by exact score, ties to the lower row id; K[l] are kept per level.
+ * ------------------------------------------------------------------------- */
+#define ORACLE_MAX_LEVELS 8
+
+typedef struct {
+    int is_bf16;
+    int n_kv_heads, head_dim, n_levels;
+    const int64_t *rows;                       /* [n_levels] rows per KV head */
+    const void *const *keys;                   /* [n_levels] keys [H_kv][rows[l]][D] */
+    const int32_t *const *child_off;           /* [n_levels - 1] [H_kv][rows[l] + 1] */
+    const int32_t *const *child_id;            /* [n_levels - 1] [H_kv][rows[l + 1]] or NULL entries */
+} oracle_csr_tree;
+
+/* kept: n_levels arrays, kept[l] is [n_trav][K[l]] (ascending row ids).
+ * Returns 0, or -1 on a bad argument (a level with fewer candidates than K,
+ * an id out of range). */
+int oracle_descend_csr(const oracle_csr_tree *t, const void *q_kg, int N, int H, const int32_t *K,
+                       int n_trav, const int32_t *trav_b, const int32_t *trav_h, int32_t *const *kept)
+{
+    const int D = t->head_dim;
+    const int nl = t->n_levels;
+    if (nl < 2 || nl > ORACLE_MAX_LEVELS || H % t->n_kv_heads != 0)
+        return -1;
+    const int G = H / t->n_kv_heads;
+    /* the largest candidate list: all roots, or the children of K[l-1] parents */
+    int64_t max_cand = t->rows[0];
+    for (int l = 1; l < nl; ++l) {
+        if (K[l - 1] < 1 || K[l - 1] > t->rows[l - 1])
+            return -1;
+        if ((int64_t)K[l - 1] * t->rows[l] > max_cand)   /* a safe upper bound */
+            max_cand = (int64_t)K[l - 1] * t->rows[l];
+    }
+    if (K[nl - 1] < 1 || max_cand > (1 << 26))
+        return -1;
+    int failed = 0;
+
+#pragma omp parallel
+    {
+        cand_t *work = (cand_t *)malloc(sizeof(cand_t) * (size_t)max_cand);
+        int32_t *rows = (int32_t *)malloc(sizeof(int32_t) * (size_t)max_cand);
+#pragma omp for schedule(dynamic, 1)
+        for (int i = 0; i < n_trav; ++i) {
+            int b = trav_b[i], h = trav_h[i];
+            int hkv = h / G;
+            size_t q_off = (((size_t)b * N) * H + h) * (size_t)D;
+            size_t q_stride = (size_t)H * D;
+            const int32_t *prev = NULL;
+            int n_prev = 0;
+            for (int l = 0; l < nl && !failed; ++l) {
+                int nc = 0;
+                if (l == 0) {
+                    for (int64_t r = 0; r < t->rows[0]; ++r)
+                        rows[nc++] = (int32_t)r;
+                } else {
+                    const int32_t *off = t->child_off[l - 1] + (size_t)hkv * (size_t)(t->rows[l - 1] + 1);
+                    const int32_t *ids = t->child_id[l - 1]
+                        ? t->child_id[l - 1] + (size_t)hkv * (size_t)t->rows[l] : NULL;
+                    for (int k = 0; k < n_prev; ++k) {
+                        int32_t p = prev[k];
+                        for (int32_t e = off[p]; e < off[p + 1]; ++e) {
+                            int32_t c = ids ? ids[e] : e;
+                            if (c < 0 || (int64_t)c >= t->rows[l]) { failed = 1; c = 0; }
+                            rows[nc++] = c;
+                        }
+                    }
+                }
+                if (nc < K[l]) { failed = 1; break; }
+                int32_t *out = kept[l] + (size_t)i * K[l];
+                for (int c = 0; c < nc; ++c) {
+                    size_t k_off = ((size_t)hkv * (size_t)t->rows[l] + (size_t)rows[c]) * (size_t)D;
+                    exact_node_score(q_kg, q_off, q_stride, N, t->keys[l], k_off, D, t->is_bf16, &work[c].score);
+                    work[c].row = rows[c];
+                }
+                qsort(work, (size_t)nc, sizeof(cand_t), cand_order);
+                for (int k = 0; k < K[l]; ++k)
+                    out[k] = work[k].row;
+                qsort(out, (size_t)K[l], sizeof(int32_t), int32_order);
+                prev = out;
+                n_prev = K[l];
+            }
+        }
+        free(work);
+        free(rows);
+    }
+    return failed ? -1 : 0;
+}
