@@ -11,6 +11,13 @@ H_kv = 8, D = 128, B = 64 queries of N = 64 tokens, T = 1024, K = 16/16/64),
 fully HBM resident.  Inputs are larger than the 126 MB L2 and L2 is also
 flushed (256 MB write) before every timed step.  Under torchrun every rank runs
 an independent replica on its own GPU (weak scaling, no data-path collective).
+
+Per workload: the headline steps are timed clean (no library instrumentation);
+a second pass of as many steps records the library's per-stage CUDA events
+(each kernel timed on its own stream), from which the per-kernel rooflines
+come; one more call reads the descent's refinement counters.  On one GPU the
+line also carries `per_config`, the same measurement for the other four
+benchmark shapes (the tiny one replayed as a CUDA graph).  --only skips it.
 """
 from __future__ import annotations
 
@@ -39,6 +46,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fanout", default=None, help="override the tree fan-outs, e.g. 100,100,100 (smaller cases)")
     ap.add_argument("--batch", type=int, default=None, help="override the number of queries B")
+    ap.add_argument("--only", action="store_true", help="time the --config workload only (no per_config block)")
+    ap.add_argument("--descent", default="auto", choices=["auto", "fused", "parent_major"],
+                    help="how the descent runs (the results are the same)")
     return ap.parse_args()
 
 
@@ -63,14 +73,26 @@ def config_of(sh, world):
             "parallelism": "replicas x%d" % world}
 
 
+def splits_attention(sh):
+    """bf16, D = 128: the sequence part is its own launch beside the descent
+    and the knowledge part merges with it (tensor-core attention)."""
+    import torch
+    return sh.dtype == torch.bfloat16 and sh.head_dim == 128
+
+
 def kernels_per_step(sh):
-    """Kernels one atlaskv_attend call launches: per level (root or children
-    scoring, selection, exact pass) x 3 and the attention.  With host-resident
-    leaves add two de-duplications and two staging copies, and the call runs
-    all of them once per query chunk (four chunks when B >= 8, else one)."""
+    """Kernels one atlaskv_attend call launches.  Leaves in HBM: the fused
+    descent, then the attention as one launch, or as two (sequence part,
+    knowledge part) when it is split.  Host-resident leaves: per query chunk
+    (four chunks when B >= 8, else one) the descent of levels 0-1, a
+    de-duplication and a staging copy of the leaf-key blocks, the descent of
+    level 2, a de-duplication and a staging copy of the value rows, and the
+    knowledge part; plus one sequence-part launch for the whole batch."""
+    split = splits_attention(sh)
     if not sh.leaf_on_host:
-        return 3 * 3 + 1
-    return (3 * 3 + 1 + 4) * (4 if sh.batch >= 8 else 1)
+        return 3 if split else 2
+    chunks = 4 if sh.batch >= 8 else 1
+    return 7 * chunks + (1 if split else 0)
 
 
 def max_over_ranks(x, world, device):
@@ -98,7 +120,8 @@ def attend_kernel_name(sh):
 
 
 KERNEL_SOURCES = {"attend_tc_kernel": "attend_tc.cuh", "attend_bf16_kernel": "attend.cuh",
-                  "attend_f32_kernel": "attend.cuh"}
+                  "attend_f32_kernel": "attend.cuh", "descend_kernel": "descend.cuh",
+                  "stage_leaf_blocks_kernel": "staging.cuh"}
 
 
 def profiled_traffic(kernel, workload):
@@ -224,12 +247,16 @@ def algorithmic_bytes(sh, res, w):
     table = 4 * (mid_cand_rows + leaf_cand_rows) if w.root_child is not None else 0
     descend = (e * B * N * H * D + e * D * (Hkv * bR + mid_cand_rows + leaf_cand_rows) + table
                + 4 * B * H * (K_R + K_I + K_L))
-    attend = (e * (3 * B * N * H * D + 2 * B * T * Hkv * D) + 4 * B * N * H + 4 * B * H * K_L
-              + 2 * e * D * u_leaf)
+    # the attention's bytes, split by part: the sequence part reads q_seq and
+    # the sequence K/V; the knowledge part reads q_kg, the kept ids and the
+    # kept leaves' K/V rows and writes out and the LSE
+    attend_seq = e * (B * N * H * D + 2 * B * T * Hkv * D)
+    attend_leaf = e * 2 * B * N * H * D + 4 * B * N * H + 4 * B * H * K_L + 2 * e * D * u_leaf
     vis = sum(T - N + n + 1 for n in range(N))
     attend_flops = 4 * B * H * D * (vis + N * K_L)
     staging = e * D * (leaf_cand_rows + u_leaf) if sh.leaf_on_host else 0
-    return {"descend": descend, "attend": attend, "attend_flops": attend_flops, "staging": staging,
+    return {"descend": descend, "attend": attend_seq + attend_leaf, "attend_seq": attend_seq,
+            "attend_leaf": attend_leaf, "attend_flops": attend_flops, "staging": staging,
             "u_root": u_root, "u_mid": u_mid, "u_leaf": u_leaf}
 
 
@@ -275,26 +302,83 @@ def pinned_h2d_gbs(torch):
     return best
 
 
-def run_ours(args):
+def host_memory_ok(sh):
+    """Enough free host memory to pin a host-leaf shape's leaf keys and values."""
+    if not sh.leaf_on_host:
+        return True
+    free_host = os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_AVPHYS_PAGES")
+    return free_host >= 2 * sh.n_leaves * sh.n_kv_heads * sh.head_dim * 2 + (8 << 30)
+
+
+def roofline_of(sh, alg, st, ms_per_step, peaks, peak_src, link_gbs):
+    """Rooflines from the algorithmic bytes and the per-launch stage times
+    (CUDA events on each kernel's own stream, averaged over the stage pass).
+    The headline is the kernel with the largest time; `kernels` lists each
+    launch kind; `step` is the whole step against HBM (and, with host leaves,
+    the staged bytes against the host link)."""
     import torch
-    import torch.distributed as dist
+    hbm = peaks["hbm_gbs"]
+    kernels = {}
+
+    def entry(name, nbytes, ms, kernel):
+        if not ms or ms <= 0:
+            return
+        ach = nbytes / (ms * 1e-3) / 1e9
+        kernels[name] = {"kernel": kernel, "ms": round(ms, 5), "algorithmic_bytes": nbytes, "achieved": ach,
+                         "unit": "GB/s", "frac": ach / hbm, "bound": "hbm"}
+
+    entry("descend", alg["descend"], st["descend"], "descend_kernel")
+    if splits_attention(sh):
+        entry("attend_seq", alg["attend_seq"], st["attend_seq"], "attend_tc_kernel (sequence part)")
+        entry("attend_leaf", alg["attend_leaf"], st["attend_leaf"], "attend_tc_kernel (knowledge part + merge)")
+    else:
+        entry("attend", alg["attend"], st["attend"], attend_kernel_name(sh))
+    if sh.leaf_on_host:
+        ach = alg["staging"] / (st["staging"] * 1e-3) / 1e9 if st["staging"] > 0 else 0.0
+        kernels["staging"] = {"kernel": "stage_leaf_blocks_kernel + stage_value_rows_kernel",
+                              "ms": round(st["staging"], 5), "algorithmic_bytes": alg["staging"], "achieved": ach,
+                              "unit": "GB/s", "frac": ach / link_gbs, "bound": "host_link",
+                              "peak": link_gbs, "peak_source": "pinned cudaMemcpyAsync H2D measured in this run"}
+    step_bytes = alg["descend"] + alg["attend"]
+    step = {"algorithmic_bytes": step_bytes, "ms": ms_per_step,
+            "achieved": step_bytes / (ms_per_step * 1e-3) / 1e9, "unit": "GB/s", "peak": hbm}
+    step["frac"] = step["achieved"] / hbm
+    if sh.leaf_on_host:
+        # the two streams overlap: the step is bound by the host link
+        link_ach = alg["staging"] / (ms_per_step * 1e-3) / 1e9
+        step["host_link"] = {"algorithmic_bytes": alg["staging"], "achieved": link_ach, "peak": link_gbs,
+                             "frac": link_ach / link_gbs}
+        top = dict(kernels["staging"])
+        top["bound"] = "host_link"
+    else:
+        name = max(kernels, key=lambda k: kernels[k]["ms"])
+        top = dict(kernels[name])
+        top["peak"] = hbm
+        top["peak_source"] = peak_src + " (burst)"
+    kname = top["kernel"].split(" ")[0]
+    top["traffic"] = profiled_traffic(kname, sh.name)
+    attend_ms = st["attend"]
+    tflops = alg["attend_flops"] / (attend_ms * 1e-3) / 1e12 if attend_ms > 0 else None
+    top.update({"kernels": kernels, "step": step, "stage_ms": {k: round(v, 5) for k, v in st.items()},
+                "attend_flops": alg["attend_flops"], "attend_tflops": tflops,
+                "attend_tensor_frac": (tflops / peaks["bf16_tflops"]
+                                       if tflops and sh.dtype == torch.bfloat16 and sh.head_dim == 128 else None)})
+    return top
+
+
+def measure(sh, seed, args, world, rank, local, cpu_seconds, use_graph=False):
+    """Benchmark one workload: returns the fields of its JSON entry."""
+    import torch
 
     from hierarchical_kv_pruning_b200 import synth
-    from hierarchical_kv_pruning_b200.binding import HikvpTree
+    from hierarchical_kv_pruning_b200.binding import STAGE_NAMES, HikvpTree
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    sh = workload_shape(args)
-    w = synth.make_workload(sh, "cuda", 1000 + args.config + 100 * rank)
+    dev = torch.device("cuda", local)
+    w = synth.make_workload(sh, "cuda", seed)
     stream = torch.cuda.current_stream()
     tree = HikvpTree.from_workload(w)
+    tree.set_descent({"auto": 0, "fused": 1, "parent_major": 2}[args.descent])
     K = sh.keep
-    dev = torch.device("cuda", local)
     out = torch.empty_like(w.q_kg)
     lse = torch.empty((sh.batch, sh.n_tokens, sh.n_heads), dtype=torch.float32, device=dev)
     kept = tuple(torch.empty((sh.batch, sh.n_heads, k), dtype=torch.int32, device=dev) for k in K)
@@ -308,37 +392,68 @@ def run_ours(args):
     for _ in range(args.warmup):
         step()
     tree.sync_status()
+    run = step
+    graph = None
+    if use_graph:
+        # a launch-latency-bound step: capture it once and replay the graph
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            step()
+        stream.wait_stream(cap)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap, capture_error_mode="thread_local"):
+            step()
+        torch.cuda.synchronize()
+        run = graph.replay
+        for _ in range(args.warmup):
+            run()
 
-    # ---- timed region: per-step CUDA events, L2 flushed before each step ----
-    tree.set_profiling(True)
-    stage = [0.0, 0.0, 0.0]
-    step_ms = []
-    launches = 0
-    n_launch = kernels_per_step(sh)
+    def timed(fn, n, label_flush):
+        ms = []
+        for _ in range(n):
+            flush.fill_(label_flush)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ms.append(a.elapsed_time(b))
+        return ms
+
+    # ---- timed region: clean steps (no library instrumentation), L2 flushed before each ----
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        step_ms = []
         for _ in range(args.steps):
-            flush.fill_(1.0)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            step()
-            b.record(stream)
-            b.synchronize()
+            step_ms.extend(timed(run, 1, 1.0))
             clk.sample()
-            step_ms.append(a.elapsed_time(b))
-            st = tree.stage_times()
-            for i in range(3):
-                stage[i] += st[i]
-            launches += n_launch
-        refine = tree.refine_stats()
         torch.cuda.synchronize()
-    tree.set_profiling(False)
     total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
     value = whole_job_rate(world, sh.batch, total_ms, args.steps)
     tree.sync_status()
+
+    # ---- stage pass: the same steps with the library's stage events on ----
+    tree.set_profiling(times=True, counters=False)
+    stage = [0.0] * len(STAGE_NAMES)
+    n_stage = max(3, args.steps)
+    for _ in range(n_stage):
+        flush.fill_(3.0)
+        step()
+        for i, v in enumerate(tree.stage_times()):
+            stage[i] += v
+    # ---- one call with the descent counters ----
+    tree.set_profiling(times=False, counters=True)
+    step()
+    refine = tree.refine_stats()
+    tree.set_profiling(times=False, counters=False)
+    tree.sync_status()
+    st = {n: v / n_stage for n, v in zip(STAGE_NAMES, stage)}
 
     # ---- end to end: pinned host inputs in, result out, through the public API ----
     host = {k: getattr(w, k).cpu().pin_memory() for k in ("q_kg", "q_seq", "k_seq", "v_seq")}
@@ -359,76 +474,72 @@ def run_ours(args):
     for _ in range(2):
         e2e_step()
     torch.cuda.synchronize()
-    e2e_ms = []
-    for _ in range(max(3, args.steps // 2)):
-        flush.fill_(2.0)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        e2e_step()
-        b.record(stream)
-        b.synchronize()
-        e2e_ms.append(a.elapsed_time(b))
+    e2e_ms = timed(e2e_step, max(3, args.steps // 2), 2.0)
     e2e_total = max_over_ranks(sum(e2e_ms), world, dev)
     e2e_value = whole_job_rate(world, sh.batch, e2e_total, len(e2e_ms))
 
-    # ---- roofline of the dominant kernel ----
     res = {"kept_root": kept[0], "kept_mid": kept[1], "kept_leaf": kept[2]}
     alg = algorithmic_bytes(sh, res, w)
     peaks, peak_src = measured_peaks()
-    st_ms = [s / args.steps for s in stage]
-    names = ["descend", "staging", "attend"]
-    # The dominant kernel: with leaves in HBM, the attention kernel is the
-    # largest single kernel of a step (the descent stage is nine shorter
-    # launches); with host-resident leaves the stages overlap on two streams
-    # and the path is bound by the host link.
-    if sh.leaf_on_host:
-        link = pinned_h2d_gbs(torch)
-        achieved = alg["staging"] / (st_ms[1] * 1e-3) / 1e9
-        roof = {"bound": "host_link", "achieved": achieved, "peak": link, "unit": "GB/s", "frac": achieved / link,
-                "traffic": None, "kernel": "stage_leaf_blocks_kernel + stage_value_rows_kernel",
-                "peak_source": "pinned cudaMemcpyAsync H2D measured in this run"}
-    else:
-        kname = attend_kernel_name(sh)
-        t_hbm = alg["attend"] / (peaks["hbm_gbs"] * 1e9)
-        t_tc = alg["attend_flops"] / (peaks["bf16_tflops"] * 1e12)
-        if sh.dtype == torch.bfloat16 and t_tc > t_hbm:
-            achieved = alg["attend_flops"] / (st_ms[2] * 1e-3) / 1e12
-            roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": achieved / peaks["bf16_tflops"]}
-        else:
-            achieved = alg["attend"] / (st_ms[2] * 1e-3) / 1e9
-            roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm_gbs"]}
-        roof.update({"traffic": profiled_traffic(kname, sh.name), "kernel": kname,
-                     "peak_source": peak_src + " (burst)"})
-    desc_gbs = alg["descend"] / (st_ms[0] * 1e-3) / 1e9 if st_ms[0] > 0 else None
-    roof["descent"] = {"ms": round(st_ms[0], 4), "algorithmic_bytes": alg["descend"], "achieved": desc_gbs,
-                       "unit": "GB/s", "frac_of_hbm": desc_gbs / peaks["hbm_gbs"] if desc_gbs else None,
-                       "kernels": "root_kernel, score_kernel x2, select_kernel x3, exact_kernel x3"}
-    roof["stage_ms"] = {n: round(v, 4) for n, v in zip(names, st_ms)}
-    roof["algorithmic_bytes"] = {k: alg[k] for k in ("descend", "attend", "staging")}
-    roof["attend_flops"] = alg["attend_flops"]
-    roof["attend_tflops"] = alg["attend_flops"] / (st_ms[2] * 1e-3) / 1e12 if st_ms[2] > 0 else None
-    # the attention's tensor-pipe share: achieved dense bf16 rate / measured burst peak
-    roof["attend_tensor_frac"] = (roof["attend_tflops"] / peaks["bf16_tflops"]
-                                  if roof["attend_tflops"] and sh.dtype == torch.bfloat16 else None)
-    roof["exact_refinement_last_step"] = refine
-
-    clocks = clk.summary()
-    line = {
-        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32" if sh.dtype == torch.float32 else "bf16",
-        "data": "synthetic (seeded hierarchical-Gaussian tree and queries)",
-        "config": config_of(sh, world),
-        "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches,
-        "roofline": roof,
-        "clocks": clocks,
-    }
+    link = pinned_h2d_gbs(torch) if sh.leaf_on_host else None
+    roof = roofline_of(sh, alg, st, ms_per_step, peaks, peak_src, link)
+    roof["exact_refinement"] = refine
+    entry = {"value": value, "unit": "queries/s", "ms_per_step": ms_per_step,
+             "us_per_query": 1e3 * ms_per_step / sh.batch,
+             "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+             "gpu_launches": kernels_per_step(sh) * args.steps, "roofline": roof, "clocks": clk.summary(),
+             "config": config_of(sh, world), "cuda_graph": use_graph,
+             "dtype": "f32" if sh.dtype == torch.float32 else "bf16"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_cpu_baseline(w, sh, args.cpu_seconds)
+        entry["cpu_baseline"] = oracle_cpu_baseline(w, sh, cpu_seconds)
+    if graph is not None:
+        del graph
     tree.close()
+    del w, out, lse, kept, ws, flush, host, dbuf, out_host, lse_host
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return entry
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from hierarchical_kv_pruning_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    sh = workload_shape(args)
+    head = measure(sh, 1000 + args.config + 100 * rank, args, world, rank, local, args.cpu_seconds,
+                   use_graph=(args.config == 0))
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": head["dtype"],
+        "data": "synthetic (seeded hierarchical-Gaussian tree and queries)",
+        "config": head["config"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+        "roofline": head["roofline"], "clocks": head["clocks"],
+    }
+    if "cpu_baseline" in head:
+        line["cpu_baseline"] = head["cpu_baseline"]
+    # every other benchmark shape, one GPU only (the host-leaf shape needs
+    # about 130 GB of pinned host memory per process)
+    if world == 1 and not args.only and not (args.fanout or args.batch):
+        per = {}
+        for c in (0, 1, 2, 3, 4):
+            if c == args.config:
+                continue
+            csh = synth.shape(c)
+            if not host_memory_ok(csh):
+                per[csh.name] = {"skipped": "not enough free host memory to pin the leaves"}
+                continue
+            per[csh.name] = measure(csh, 1000 + c, args, 1, rank, local, args.cpu_seconds / 2, use_graph=(c == 0))
+        line["per_config"] = per
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -460,7 +571,7 @@ def run_reference(args):
     value = statistics.mean(vals)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": 1e3 * sh.batch / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded hierarchical-Gaussian tree and queries)",
         "config": config_of(sh, 1),
         "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -26,7 +26,18 @@ struct AttnParams {
     int B, N, H, H_kv, G, T, K_L;
     float scale_log2;                // scale * log2(e)
     int *status;                     // sticky device status word (bounded waits report here)
+    // tensor-core kernel only: which key sets one launch covers (kAttn*), and
+    // the sequence part's results handed from the sequence launch to the leaf
+    // launch, per (query, KV head) group and group row r = g N + n
+    int mode;
+    float *oseq;                     // [B H_kv][G N][D] normalised sequence-part output
+    float *lse_seq;                  // [B H_kv][G N] its log-sum-exp (natural log)
 };
+
+// attend_tc_kernel modes: both key sets in one online softmax; the causal
+// sequence alone (writes oseq / lse_seq); the kept leaves alone, merged with
+// oseq / lse_seq by the lambda weights in the epilogue.
+enum : int { kAttnFused = 0, kAttnSeq = 1, kAttnLeaf = 2 };
 
 // ---------------------------------------------------------------------------
 // fp32 path: one warp per (b, n, h) output row, CUDA-core FMA, expf.

@@ -75,7 +75,8 @@ constexpr int kBarSFull = kBarEmptyV + kVStages;    // [kWG][2] S in TMEM buffer
 constexpr int kBarPReady = kBarSFull + 2 * kWG;     // [kWG][2] P(w, t) written over it, O_w rescaled (4 warps)
 constexpr int kBarODone = kBarPReady + 2 * kWG;     // [kWG][2] O_w += P V from that buffer done
 constexpr int kBarQReady = kBarODone + 2 * kWG;     // [kWG] Q_w loaded (4 warps)
-constexpr int kNumBars = kBarQReady + kWG;
+constexpr int kBarDrain = kBarQReady + kWG;         // every MMA the issuing thread committed has completed
+constexpr int kNumBars = kBarDrain + 1;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024;   // + slack to align the base to 1024
 constexpr int kTmemCols = 256 * kWG;           // warpgroup w: S / P buffers [256 w, 256 w + 128), O [256 w + 128, 256 w + 256)
@@ -257,12 +258,11 @@ __global__ void wait_timeout_probe_kernel(int *status)
     if (threadIdx.x == 0 && !tc::mbar_wait(b, 0)) set_status(status, kDevTimeout);
 }
 
-// One CTA per (query b, KV head, kWG x 128-row block of the group's G N rows).
-// tm_k / tm_v: the sequence keys / values [B][T][H_kv][D] as 4-D tensor maps
-// (D, H_kv, T, B) with a (64, 1, 64, 1) box and 128-byte swizzle.
-__global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
-    attend_tc_kernel(const AttnParams p, int ctas_per_group, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v)
+// The work of CTA `bid` of a launch: (query b, KV head, kWG x 128-row block
+// of the group's G N rows), keys and values of the sequence by TMA through
+// the tensor maps tm_k / tm_v.
+__device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigned bid, int ctas_per_group,
+                                              const CUtensorMap *tm_k, const CUtensorMap *tm_v)
 {
     using namespace tc;
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
@@ -272,19 +272,19 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffTmemSlot);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int grp_id = blockIdx.x / ctas_per_group;
-    const int cta = blockIdx.x - grp_id * ctas_per_group;
+    const int grp_id = bid / ctas_per_group;
+    const int cta = bid - grp_id * ctas_per_group;
     const int b = grp_id / p.H_kv, hkv = grp_id - b * p.H_kv;
     const int GN = p.G * p.N;
     const int r0 = cta * kCtaRows;                       // first group row of the CTA
     const int r_end = min(GN, r0 + kCtaRows) - 1;        // last valid one
     const int g_first = r0 / p.N, g_last = r_end / p.N;  // heads g_first..g_last own the rows
     const int n_leaf = (g_last - g_first + 1) * p.K_L;   // their kept leaves, head by head
-    const int n_leaf_tiles = (n_leaf + kKeys - 1) / kKeys;
+    const int n_leaf_tiles = p.mode == kAttnSeq ? 0 : (n_leaf + kKeys - 1) / kKeys;
     // causal extent: the largest token index of the CTA is N - 1 when its rows
     // span two heads, else that of its last row
     const int cta_last = p.T - p.N + (r_end / p.N != r0 / p.N ? p.N - 1 : r_end % p.N);
-    const int n_seq_tiles = (cta_last + kKeys) / kKeys;
+    const int n_seq_tiles = p.mode == kAttnLeaf ? 0 : (cta_last + kKeys) / kKeys;
     const int n_tiles = n_leaf_tiles + n_seq_tiles;
     // Warpgroup w takes every sequence tile (if it has rows at all) and the
     // leaf tiles holding its heads' leaves: its heads are contiguous and the
@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) {
-            const bool per_warp = (i >= kBarPReady && i < kBarPReady + 2 * kWG) || (i >= kBarQReady);
+            const bool per_warp = (i >= kBarPReady && i < kBarPReady + 2 * kWG) || (i >= kBarQReady && i < kBarQReady + kWG);
             mbar_init(bar(i), per_warp ? 4 : 1);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kBarQReady + w));
         };
-        load_q(p.q_seq);
+        load_q(p.mode == kAttnLeaf ? p.q_kg : p.q_seq);
         const bool any_leaf = wvalid[w] && wlo[w] <= whi[w];
 
         const float sl2 = p.scale_log2;
@@ -468,26 +468,66 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
         }
         if (!failed && c_w > 0) {
             const float inv = 1.f / l;
+            const size_t grow = (size_t)grp_id * GN + (row_ok ? row : 0);   // row of the group-row layout
+            // lambda merge of the two blocks ("Quick read / How it works" merge
+            // equation): lam_kg = e^{LSE_kg} / (e^{LSE_kg} + e^{LSE_seq}), in log2 units
+            float lam_kg = 1.f, lam_seq = 0.f, lse2 = m_used + log2f(l);
+            const float *os = nullptr;
+            if (p.mode == kAttnLeaf && row_ok) {
+                const float lse_kg2 = lse2;
+                const float lse_seq2 = p.lse_seq[grow] * 1.44269504088896340736f;
+                const float M = fmaxf(lse_kg2, lse_seq2);
+                const float wk = exp2f(lse_kg2 - M), wq = exp2f(lse_seq2 - M);
+                lam_kg = wk / (wk + wq);
+                lam_seq = wq / (wk + wq);
+                lse2 = M + log2f(wk + wq);
+                os = p.oseq + grow * kD;
+            }
             __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.out) + (((size_t)b * p.N + n) * p.H + h) * kD;
+            float *odst = p.mode == kAttnSeq ? p.oseq + grow * kD : nullptr;
+            const float a = inv * lam_kg;
 #pragma unroll
             for (int c = 0; c < kD; c += 32) {
                 float ov[32];
                 tmem_ld32(tO + lane_off + c, ov);
                 tmem_wait_ld();
-                if (row_ok) {
+                if (!row_ok) continue;
+                if (odst) {
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        __nv_bfloat162 a0 = __floats2bfloat162_rn(ov[i] * inv, ov[i + 1] * inv);
-                        __nv_bfloat162 a1 = __floats2bfloat162_rn(ov[i + 2] * inv, ov[i + 3] * inv);
-                        __nv_bfloat162 a2 = __floats2bfloat162_rn(ov[i + 4] * inv, ov[i + 5] * inv);
-                        __nv_bfloat162 a3 = __floats2bfloat162_rn(ov[i + 6] * inv, ov[i + 7] * inv);
-                        *reinterpret_cast<uint4 *>(dst + c + i) =
-                            make_uint4(*reinterpret_cast<uint32_t *>(&a0), *reinterpret_cast<uint32_t *>(&a1),
-                                       *reinterpret_cast<uint32_t *>(&a2), *reinterpret_cast<uint32_t *>(&a3));
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4 *>(odst + c + i) =
+                            make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
+                    continue;
+                }
+                if (os) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 q4 = *reinterpret_cast<const float4 *>(os + c + i);
+                        ov[i] = fmaf(ov[i], a, lam_seq * q4.x);
+                        ov[i + 1] = fmaf(ov[i + 1], a, lam_seq * q4.y);
+                        ov[i + 2] = fmaf(ov[i + 2], a, lam_seq * q4.z);
+                        ov[i + 3] = fmaf(ov[i + 3], a, lam_seq * q4.w);
                     }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ov[i] *= inv;
+                }
+#pragma unroll
+                for (int i = 0; i < 32; i += 8) {
+                    __nv_bfloat162 a0 = __floats2bfloat162_rn(ov[i], ov[i + 1]);
+                    __nv_bfloat162 a1 = __floats2bfloat162_rn(ov[i + 2], ov[i + 3]);
+                    __nv_bfloat162 a2 = __floats2bfloat162_rn(ov[i + 4], ov[i + 5]);
+                    __nv_bfloat162 a3 = __floats2bfloat162_rn(ov[i + 6], ov[i + 7]);
+                    *reinterpret_cast<uint4 *>(dst + c + i) =
+                        make_uint4(*reinterpret_cast<uint32_t *>(&a0), *reinterpret_cast<uint32_t *>(&a1),
+                                   *reinterpret_cast<uint32_t *>(&a2), *reinterpret_cast<uint32_t *>(&a3));
                 }
             }
-            if (row_ok && p.lse) p.lse[((size_t)b * p.N + n) * p.H + h] = (m_used + log2f(l)) * 0.69314718055994530942f;
+            if (row_ok) {
+                const float lse_nat = lse2 * 0.69314718055994530942f;
+                if (p.mode == kAttnSeq) p.lse_seq[grow] = lse_nat;
+                else if (p.lse) p.lse[((size_t)b * p.N + n) * p.H + h] = lse_nat;
+            }
         }
         if (failed && lane == 0) set_status(p.status, kDevTimeout);
     } else if (warp == kProducerWarp) {
@@ -535,6 +575,7 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
             pending = -1;
         };
         int nk[2] = {-1, -1}, nv[2] = {-1, -1};
+        int k_issued = 0, v_issued = 0;   // tiles whose K / V copies have been issued
         if (n_leaf_tiles > 0) fetch_rows(0, nk, nv);
         for (int t = 0; t < n_tiles; ++t) {
             const int sk = t % kKStages, sv = t % kVStages;
@@ -553,14 +594,16 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
                 const int lt = t - n_seq_tiles;
                 if (lt + 1 < n_leaf_tiles) fetch_rows(lt + 1, nk, nv);
                 gather(kd, lkb, rk);
+                k_issued = t + 1;
             } else {
                 if (lane == 0) {
                     mbar_arrive_expect_tx(bar(kBarFullK + sk), kKVBytes);
 #pragma unroll
                     for (int half = 0; half < 2; ++half)
-                        tma_load_4d(kd + half * (kKeys * 128), &tm_k, half * 64, hkv, t * kKeys, b, bar(kBarFullK + sk));
+                        tma_load_4d(kd + half * (kKeys * 128), tm_k, half * 64, hkv, t * kKeys, b, bar(kBarFullK + sk));
                 }
                 __syncwarp();
+                k_issued = t + 1;
             }
             // the previous leaf tile goes out before any wait on a V stage
             if (pending >= 0) announce(leaf ? 1 : 0);
@@ -576,21 +619,25 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
                     mbar_arrive_expect_tx(bar(kBarFullV + sv), kKVBytes);
 #pragma unroll
                     for (int half = 0; half < 2; ++half)
-                        tma_load_4d(vd + half * (kKeys * 128), &tm_v, half * 64, hkv, t * kKeys, b, bar(kBarFullV + sv));
+                        tma_load_4d(vd + half * (kKeys * 128), tm_v, half * 64, hkv, t * kKeys, b, bar(kBarFullV + sv));
                 }
                 __syncwarp();
             }
+            v_issued = t + 1;
         }
         if (!failed && pending >= 0) announce(0);
-        // the CTA must not exit with copies in flight: wait until the last tile of each stage has landed
-        if (!failed) {
-            for (int t = max(0, n_tiles - kKStages); t < n_tiles; ++t)
-                failed |= !mbar_wait(bar(kBarFullK + t % kKStages), (t / kKStages) & 1);
-            for (int t = max(0, n_tiles - kVStages); t < n_tiles; ++t)
-                failed |= !mbar_wait(bar(kBarFullV + t % kVStages), (t / kVStages) & 1);
-        }
+        // The CTA must not exit with copies in flight, on the failure path too:
+        // wait (bounded) until the last issued tile of each stage has landed.
+        // Gathered tiles are drained by cp.async.wait_group; their full barrier
+        // is only announced by this warp, so after a failure only the TMA
+        // (sequence) tiles are waited for.
+        bool drained = true;
+        for (int t = max(0, k_issued - kKStages); t < k_issued; ++t)
+            if (!failed || t < n_seq_tiles) drained &= mbar_wait(bar(kBarFullK + t % kKStages), (t / kKStages) & 1);
+        for (int t = max(0, v_issued - kVStages); t < v_issued; ++t)
+            if (!failed || t < n_seq_tiles) drained &= mbar_wait(bar(kBarFullV + t % kVStages), (t / kVStages) & 1);
         cp_wait_all();
-        if (failed && lane == 0) set_status(p.status, kDevTimeout);
+        if ((failed || !drained) && lane == 0) set_status(p.status, kDevTimeout);
     } else {
         // ================= MMA issue: one thread =================
         if (lane == 0) {
@@ -611,7 +658,8 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
                     const int cs = wg_count(w, t), bs = cs & 1;
                     if (cs == 0 && !mbar_wait(bar(kBarQReady + w), 0)) return false;
                     // the warpgroup's first leaf tile: Q_w has been replaced by q_kg
-                    if (t >= n_seq_tiles && t - n_seq_tiles == wlo[w] && !mbar_wait(bar(kBarQReady + w), 1))
+                    if (n_seq_tiles > 0 && t >= n_seq_tiles && t - n_seq_tiles == wlo[w] &&
+                        !mbar_wait(bar(kBarQReady + w), 1))
                         return false;
                     // buffer bs still holds the P of this warpgroup's tile two back until its P V has completed
                     if (cs >= 2 && !mbar_wait(bar(kBarODone + 2 * w + bs), ((cs - 2) >> 1) & 1)) return false;
@@ -656,7 +704,11 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
                 if (ok && t > 0) ok = issue_pv(t - 1);
             }
             if (ok) ok = issue_pv(n_tiles - 1);
-            if (!ok) set_status(p.status, kDevTimeout);
+            // before TMEM is released, every MMA this thread committed must have
+            // completed, on the failure path too: one more commit tracks them all
+            mma_commit(bar(kBarDrain));
+            const bool drained = mbar_wait(bar(kBarDrain), 0);
+            if (!ok || !drained) set_status(p.status, kDevTimeout);
         }
         __syncwarp();
     }
@@ -665,6 +717,34 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
     __syncthreads();
     fence_after_sync();
     if (warp == kMmaWarp) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+}
+
+// One call: one CTA per (query b, KV head, kWG x 128-row block of the group's
+// G N rows).  tm_k / tm_v: the sequence keys / values [B][T][H_kv][D] as 4-D
+// tensor maps (D, H_kv, T, B) with a (64, 1, 64, 1) box and 128-byte swizzle.
+__global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
+    attend_tc_kernel(const __grid_constant__ AttnParams p, int ctas_per_group, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v)
+{
+    attend_tc_cta(p, blockIdx.x, ctas_per_group, &tm_k, &tm_v);
+}
+
+// Several layers' calls in one launch (same shapes, each layer its own
+// inputs and kept leaves): layer l owns the CTAs [offs[l], offs[l + 1]).
+constexpr int kMaxAttnLayers = 32;
+struct AttnBatch {
+    CUtensorMap mk[kMaxAttnLayers], mv[kMaxAttnLayers];
+    AttnParams p[kMaxAttnLayers];
+    unsigned offs[kMaxAttnLayers + 1];
+    int n, ctas_per_group;
+};
+
+__global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
+    attend_tc_layers_kernel(const __grid_constant__ AttnBatch b)
+{
+    int l = 0;
+    while (l + 1 < b.n && blockIdx.x >= b.offs[l + 1]) ++l;
+    attend_tc_cta(b.p[l], blockIdx.x - b.offs[l], b.ctas_per_group, &b.mk[l], &b.mv[l]);
 }
 
 }  // namespace akv

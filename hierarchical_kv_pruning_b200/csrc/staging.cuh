@@ -1,5 +1,7 @@
-// Host-leaf staging: bring the leaf-key blocks of the kept mids, and later the
-// kept leaves' value rows, from pinned host memory into HBM.
+// Host staging: bring the key blocks of the kept parents (the mid blocks of the
+// kept roots when the mid level lives in host memory, the leaf blocks of the
+// kept mids), and later the kept leaves' value rows, from pinned host memory
+// into HBM.
 //
 // "AtlasKV: Augmenting LLMs with Billion-Scale Knowledge Graphs in 20GB VRAM",
 // section "Quick read / How it works": only the root keys need to stay on the
@@ -92,20 +94,21 @@ __global__ void __launch_bounds__(kDedupeThreads) dedupe_kernel(const int32_t *_
 constexpr int kStageUnroll = 4;
 constexpr int kStageCtasPerSm = 2;
 
-// Copy the b_L leaf-key rows of every unique kept mid of every group into the
-// key pool: pool row (q*n + u) * b_L + j <- host leaf row child(mid, j) of KV
-// head q % H_kv.
+// Copy the b_c child-key rows of every unique kept parent of every group into
+// the key pool: pool row (q*n + u) * b_c + j <- host child row child(parent, j)
+// of KV head q % H_kv, with child() the level's table (or parent * b_c + j).
+// Used for the leaf blocks of kept mids and the mid blocks of kept roots.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) stage_leaf_blocks_kernel(
-    const T *__restrict__ host_leaf_keys, const int32_t *__restrict__ mid_child, long long n_mid, long long n_leaf,
-    int b_leaf, int H_kv, const int32_t *__restrict__ uniq, const int32_t *__restrict__ count, int n, int n_groups,
-    T *pool, int *status)
+__global__ void __launch_bounds__(256) stage_blocks_kernel(
+    const T *__restrict__ host_child_keys, const int32_t *__restrict__ child_tab, long long n_parent,
+    long long n_child, int b_child, int H_kv, const int32_t *__restrict__ uniq, const int32_t *__restrict__ count,
+    int n, int n_groups, T *pool, int *status)
 {
     constexpr int VPR = D * (int)sizeof(T) / 16;   // 16-byte vectors per row = lanes per row
     constexpr int RPI = 32 / VPR;                  // rows per warp instruction
     const int lane = threadIdx.x & 31, sub = lane % VPR, rsel = lane / VPR;
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-    const long long total = (long long)n_groups * n * b_leaf;
+    const long long total = (long long)n_groups * n * b_child;
     for (long long r0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * (RPI * kStageUnroll);
          r0 < total; r0 += warps * RPI * kStageUnroll) {
         uint4 buf[kStageUnroll];
@@ -115,20 +118,20 @@ __global__ void __launch_bounds__(256) stage_leaf_blocks_kernel(
             const long long w = r0 + (long long)k * RPI + rsel;
             dst[k] = nullptr;
             if (w < total) {
-                const long long blk = w / b_leaf;
-                const int j = (int)(w - blk * b_leaf);
+                const long long blk = w / b_child;
+                const int j = (int)(w - blk * b_child);
                 const int b = (int)(blk / n);
                 const int u = (int)(blk - (long long)b * n);
                 if (u < count[b]) {
                     const int hkv = b % H_kv;   // group b = query * H_kv + hkv
-                    const long long mid = uniq[blk];
-                    const long long leaf = mid_child ? (long long)mid_child[((size_t)hkv * n_mid + mid) * b_leaf + j]
-                                                     : mid * b_leaf + j;
-                    if (leaf < 0 || leaf >= n_leaf) {
+                    const long long par = uniq[blk];
+                    const long long ch = child_tab ? (long long)child_tab[((size_t)hkv * n_parent + par) * b_child + j]
+                                                   : par * b_child + j;
+                    if (ch < 0 || ch >= n_child) {
                         set_status(status, kDevBadChild);
                     } else {
-                        buf[k] = reinterpret_cast<const uint4 *>(host_leaf_keys + ((size_t)hkv * n_leaf + leaf) * D)[sub];
-                        dst[k] = reinterpret_cast<uint4 *>(pool + ((size_t)blk * b_leaf + j) * D) + sub;
+                        buf[k] = reinterpret_cast<const uint4 *>(host_child_keys + ((size_t)hkv * n_child + ch) * D)[sub];
+                        dst[k] = reinterpret_cast<uint4 *>(pool + ((size_t)blk * b_child + j) * D) + sub;
                     }
                 }
             }

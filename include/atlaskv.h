@@ -31,7 +31,7 @@
  *
  * Layouts (all row-major, D contiguous, every base pointer 16-byte aligned):
  *   root_keys   [H_kv][b_R][D]            device
- *   mid_keys    [H_kv][b_R*b_I][D]        device
+ *   mid_keys    [H_kv][b_R*b_I][D]        device, or pinned host memory (then the leaves too)
  *   leaf_keys   [H_kv][b_R*b_I*b_L][D]    device, or pinned host memory
  *   leaf_values [H_kv][b_R*b_I*b_L][D]    same location as leaf_keys
  *   root_child  [H_kv][b_R][b_I]    int32 mid row ids, or NULL: child(r,j) = r*b_I + j
@@ -83,7 +83,12 @@ typedef enum {
 } atlaskv_leaf_location;
 
 /* Tree description ("Method details / Hierarchical clustering of KGKVs": three
- * levels, root / intermediate / leaf; only leaves carry values). */
+ * levels, root / intermediate / leaf; only leaves carry values).  Levels below
+ * the roots may live in pinned host memory ("Quick read / How it works": only
+ * the root keys stay in GPU memory, each next level is loaded from CPU memory
+ * after the level above is pruned): the leaves (leaf_location), or the mids
+ * and the leaves (mid_location as well).  Their blocks of children are then
+ * staged into HBM pools in the workspace, per call, for the kept parents only. */
 typedef struct {
     int32_t dtype;             /* atlaskv_dtype of every key/value/query buffer */
     int32_t n_kv_heads;        /* H_kv >= 1: one tree per KV head */
@@ -96,6 +101,7 @@ typedef struct {
     int32_t leaf_location;     /* atlaskv_leaf_location */
     const int32_t *root_child; /* device, optional */
     const int32_t *mid_child;  /* device, optional */
+    int32_t mid_location;      /* atlaskv_leaf_location of mid_keys; HOST_PINNED needs host-pinned leaves too */
 } atlaskv_tree_desc;
 
 typedef struct {
@@ -132,6 +138,57 @@ typedef struct atlaskv_tree atlaskv_tree;
  * {64, 128}, ECUDA if a CUDA call fails.  *out is set only on OK. */
 atlaskv_status atlaskv_create_tree(const atlaskv_tree_desc *desc, void *stream, atlaskv_tree **out);
 
+/* ---- Trees of any depth with a variable number of children per node -------
+ * "Method details / Hierarchical clustering of KGKVs": a clustering gives
+ * clusters of unequal size, and the depth can be set larger than three.  Level
+ * 0 holds the roots, level n_levels - 1 the leaves (the only level with
+ * values).  The children of node p of level l are listed, per KV head, at
+ * positions child_off[l][hkv][p] .. child_off[l][hkv][p + 1] - 1 of level l's
+ * child list; child_id[l][hkv][e] is the row (of level l + 1) at position e,
+ * or, with child_id[l] NULL, the position e is the row itself (children
+ * stored contiguously).  Every row of level l + 1 must be listed exactly once.
+ * The descent is the same: candidates of a level are the children of the
+ * kept nodes above, K[l] are kept per level, ranked exactly, ties to the lower
+ * row id.  All buffers on the device (no host-resident levels).  Calls:
+ * atlaskv_create_tree_csr, atlaskv_workspace_size_csr, atlaskv_attend_csr;
+ * sync_status, profiling and destroy are shared with the uniform trees. */
+#define ATLASKV_MAX_LEVELS 4
+
+typedef struct {
+    int32_t dtype;                                 /* atlaskv_dtype */
+    int32_t n_kv_heads;                            /* H_kv >= 1 */
+    int32_t head_dim;                              /* D: 64 or 128 */
+    int32_t n_levels;                              /* 2 .. ATLASKV_MAX_LEVELS */
+    int64_t rows[ATLASKV_MAX_LEVELS];              /* nodes per KV head at each level, >= 1 */
+    const void *keys[ATLASKV_MAX_LEVELS];          /* [H_kv][rows[l]][D] */
+    const int32_t *child_off[ATLASKV_MAX_LEVELS - 1];   /* [H_kv][rows[l] + 1]: 0, non-decreasing, rows[l + 1] */
+    const int32_t *child_id[ATLASKV_MAX_LEVELS - 1];    /* [H_kv][rows[l + 1]] rows, or NULL (positions are rows) */
+    const void *leaf_values;                       /* [H_kv][rows[n_levels - 1]][D] */
+} atlaskv_csr_tree_desc;
+
+typedef struct {
+    int32_t K[ATLASKV_MAX_LEVELS];   /* kept per level: 1 <= K[0] <= rows[0]; 1 <= K[l] <= K[l-1] * (fewest
+                                        children of a node of level l-1), so every traversal has K[l] candidates */
+    float scale;                     /* logit scale; 0 means 1/sqrt(D) */
+} atlaskv_level_params;
+
+/* Validate and build a CSR tree.  Reads the offsets to the host once (and
+ * synchronises `stream`), checks the child lists on the device, computes the
+ * key-norm bounds of every level.  EINVAL for a bad description or child
+ * list, EUNSUPPORTED for D not in {64, 128}, ECUDA if a CUDA call fails. */
+atlaskv_status atlaskv_create_tree_csr(const atlaskv_csr_tree_desc *desc, void *stream, atlaskv_tree **out);
+
+/* Workspace bytes of atlaskv_attend_csr for these sizes. */
+atlaskv_status atlaskv_workspace_size_csr(const atlaskv_tree *tree, const atlaskv_level_params *params,
+                                          int32_t B, int32_t N, int32_t H, int32_t T, size_t *bytes);
+
+/* atlaskv_attend for a CSR tree.  io is as for atlaskv_attend except that its
+ * kept_root / kept_mid / kept_leaf are ignored: kept, when not NULL, holds
+ * n_levels optional outputs, kept[l] [B][H][K[l]] int32 ascending row ids of
+ * level l.  The attention uses the leaves kept at the last level. */
+atlaskv_status atlaskv_attend_csr(atlaskv_tree *tree, const atlaskv_level_params *params, const atlaskv_io *io,
+                                  int32_t *const *kept, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Bytes of workspace atlaskv_attend needs for these sizes (EINVAL on bad sizes). */
 atlaskv_status atlaskv_workspace_size(const atlaskv_tree *tree, const atlaskv_params *params,
                                       int32_t B, int32_t N, int32_t H, int32_t T, size_t *bytes);
@@ -140,32 +197,92 @@ atlaskv_status atlaskv_workspace_size(const atlaskv_tree *tree, const atlaskv_pa
  * leaves when the tree's leaves are in host memory), knowledge + sequence
  * attention and merge.  `workspace` is device memory of at least
  * atlaskv_workspace_size() bytes, 256-byte aligned, not shared with a
- * concurrent call.  With host-resident leaves the batch is processed in query
- * chunks (four when B >= 8, else one; each chunk launches every kernel of the
- * path) and the leaf blocks are staged on a second stream owned by the tree
- * (joined back into `stream` before the call's last kernel), so the host link
- * works while other chunks compute; calls on one such tree must therefore not
- * overlap.  Returns EINVAL / ENOMEM (workspace too small) / EUNSUPPORTED
- * without enqueuing anything. */
+ * concurrent call.
+ * - bf16, D = 128: the sequence part depends only on the call's inputs, so it
+ *   runs as its own launch on a low-priority stream owned by the tree, beside
+ *   the descent (which runs on a high-priority stream owned by the tree); the
+ *   knowledge part then merges with it by the lambda weights.
+ * - Host-resident leaves: the batch is processed in query chunks (four when
+ *   B >= 8, else one; each chunk launches the descent, the staging and the
+ *   knowledge part) and the leaf blocks are staged on a third stream owned by
+ *   the tree, so the host link works while other chunks compute.
+ * Every stream the tree owns joins `stream` again before the call's last
+ * kernel, so work enqueued on `stream` afterwards sees the complete results.
+ * Because the tree's streams and events are shared by its calls, calls on one
+ * tree must not overlap: serialise them, or create one tree per concurrent
+ * caller (trees only borrow the key buffers).  The tree's streams and events
+ * are created by atlaskv_create_tree; attend creates and allocates nothing.
+ * Returns EINVAL / ENOMEM (workspace too small) / EUNSUPPORTED without
+ * enqueuing anything. */
 atlaskv_status atlaskv_attend(atlaskv_tree *tree, const atlaskv_params *params, const atlaskv_io *io,
                               void *workspace, size_t workspace_bytes, void *stream);
+
+/* Several layers at once (multi-layer batching; per-layer knowledge keys as in
+ * "Background / Rectangular attention in KBLaM", where every layer has its own
+ * knowledge-key projections): layer l runs the whole path of atlaskv_attend on
+ * trees[l] with ios[l], all with the same params.  The layers share one launch
+ * per kernel (descent, sequence part, knowledge part), which is what makes a
+ * decode step (N = 1, tiny per-layer work) cheap to launch.  Requirements:
+ * 1 <= n_layers <= 32; every tree in HBM (no host-resident level), with the
+ * same dtype, head_dim and n_kv_heads; every io with the same B, N, H and T;
+ * fan-outs may differ as long as the descent's plan is the same (EINVAL
+ * otherwise).  The workspace is atlaskv_workspace_size_layers() bytes,
+ * 256-byte aligned.  Layer 0's tree lends its streams and events (and its
+ * stage times, when its profiling is on): no call on trees[0] may overlap this
+ * one.  Device errors of layer l are reported by trees[l]'s sync status. */
+atlaskv_status atlaskv_workspace_size_layers(int32_t n_layers, atlaskv_tree *const *trees,
+                                             const atlaskv_params *params, const atlaskv_io *ios, size_t *bytes);
+atlaskv_status atlaskv_attend_layers(int32_t n_layers, atlaskv_tree *const *trees, const atlaskv_params *params,
+                                     const atlaskv_io *ios, void *workspace, size_t workspace_bytes, void *stream);
 
 /* Synchronise `stream` and return the tree's sticky device status (OK,
  * EDEVICE or ETIMEOUT), or ECUDA if the stream reports a CUDA error. */
 atlaskv_status atlaskv_sync_status(atlaskv_tree *tree, void *stream);
 
-/* Per-stage device times (ms) of the most recent attend call made while
- * profiling was on: [0] descent levels, [1] host-leaf staging (0 when leaves
- * are in HBM), [2] attention + merge.  Synchronises the stream of that call.
- * n is the capacity of ms; returns EINVAL if profiling was never enabled. */
+/* Diagnostics; the paper has no counterpart.  atlaskv_set_profiling takes a
+ * bit mask: ATLASKV_PROFILE_TIMES records CUDA events around each stage of
+ * later attend calls (cheap, no extra device work); ATLASKV_PROFILE_COUNTERS
+ * keeps the descent counters read by atlaskv_refine_stats (a memset and a few
+ * atomics per call); 0 turns both off. */
+#define ATLASKV_PROFILE_TIMES 1
+#define ATLASKV_PROFILE_COUNTERS 2
 atlaskv_status atlaskv_set_profiling(atlaskv_tree *tree, int32_t enable);
+
+/* How the descent is run; the results are the same either way.
+ * ATLASKV_DESCENT_FUSED: one kernel per call, one CTA per (query, KV head,
+ *   chunk of heads), running every level; it reads the child rows of the
+ *   union of its heads' kept parents (few launches: the choice for small
+ *   calls).
+ * ATLASKV_DESCENT_PARENT_MAJOR: a few kernels per level; the kept parents of
+ *   the whole batch are grouped by (KV head, parent) and each parent's child
+ *   rows are read once per group of up to 32 traversals that kept it, so the
+ *   bytes read approach the unique rows a level needs (the choice for large
+ *   batches).
+ * ATLASKV_DESCENT_AUTO (the default): parent-major when B * H >= 512, else
+ *   fused (each where the other's plan does not fit).
+ * The mode changes the workspace size: set it before atlaskv_workspace_size.
+ * atlaskv_attend_layers always runs the fused kernel. */
+#define ATLASKV_DESCENT_AUTO 0
+#define ATLASKV_DESCENT_FUSED 1
+#define ATLASKV_DESCENT_PARENT_MAJOR 2
+atlaskv_status atlaskv_set_descent(atlaskv_tree *tree, int32_t mode);
+
+/* Per-stage device times (ms) of the most recent attend call made with
+ * ATLASKV_PROFILE_TIMES: [0] descent levels, [1] host-leaf staging (0 when
+ * leaves are in HBM), [2] attention + merge ([3] + [4]), [3] the sequence
+ * part when it runs as its own launch (bf16, D = 128; else 0), [4] the leaf
+ * part (or the whole attention when it is one launch).  With host leaves
+ * [0], [1] and [4] are busy times summed over the query chunks.  Synchronises
+ * the stream of that call.  n is the capacity of ms (at most 5 written);
+ * returns EINVAL if that call recorded no times. */
 atlaskv_status atlaskv_stage_times(atlaskv_tree *tree, float *ms, int32_t n);
 
-/* Descent counters of the most recent attend call made while profiling was
- * on, per level l = 0 (roots), 1 (mids), 2 (leaves): counts[4 l + 0] traversals
- * selected, [4 l + 1] selections the fp32 bound could not settle alone,
- * [4 l + 2] ambiguous candidates in those, [4 l + 3] exact scores computed.
- * Synchronises the device; n is the capacity of counts (at most 12 written). */
+/* Descent counters of the most recent attend call made with
+ * ATLASKV_PROFILE_COUNTERS, per level l = 0 (roots), 1 (mids), 2 (leaves) and,
+ * for deeper CSR trees, 3: counts[4 l + 0] traversals selected, [4 l + 1]
+ * selections the fp32 bound could not settle alone, [4 l + 2] ambiguous
+ * candidates in those, [4 l + 3] exact scores computed.  Synchronises the
+ * device; n is the capacity of counts (at most 16 written). */
 atlaskv_status atlaskv_refine_stats(atlaskv_tree *tree, uint64_t *counts, int32_t n);
 
 /* Size in bytes of the static device scratch used by atlaskv_attend_static. */

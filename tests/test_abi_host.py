@@ -46,6 +46,7 @@ def _desc(**kw):
     for f in ("root_keys", "mid_keys", "leaf_keys", "leaf_values"):
         setattr(d, f, kw.get(f, 4096))
     d.leaf_location = kw.get("leaf_location", binding.ATLASKV_LEAVES_DEVICE)
+    d.mid_location = kw.get("mid_location", binding.ATLASKV_LEAVES_DEVICE)
     return d
 
 
@@ -57,6 +58,8 @@ def _desc(**kw):
     (dict(root_keys=None), binding.ATLASKV_EINVAL),
     (dict(mid_keys=4100), binding.ATLASKV_EINVAL),            # not 16-byte aligned
     (dict(leaf_location=5), binding.ATLASKV_EINVAL),
+    (dict(mid_location=5), binding.ATLASKV_EINVAL),
+    (dict(mid_location=binding.ATLASKV_LEAVES_HOST_PINNED), binding.ATLASKV_EINVAL),   # mids on host, leaves not
     (dict(fanout=(2000, 2000, 2000)), binding.ATLASKV_EUNSUPPORTED),
 ])
 def test_create_tree_rejects_bad_descriptions(lib, kw, status):
@@ -78,9 +81,19 @@ def test_null_arguments(lib):
     assert lib.atlaskv_attend(None, ctypes.byref(p), None, None, 0, None) == binding.ATLASKV_EINVAL
     assert lib.atlaskv_sync_status(None, None) == binding.ATLASKV_EINVAL
     assert lib.atlaskv_set_profiling(None, 1) == binding.ATLASKV_EINVAL
+    assert lib.atlaskv_set_descent(None, binding.ATLASKV_DESCENT_FUSED) == binding.ATLASKV_EINVAL
     buf = (ctypes.c_float * 3)()
     assert lib.atlaskv_stage_times(None, buf, 3) == binding.ATLASKV_EINVAL
     assert lib.atlaskv_destroy(None) == binding.ATLASKV_OK
+    trees = (ctypes.c_void_p * 2)(None, None)
+    ios = (binding.atlaskv_io * 2)()
+    assert lib.atlaskv_workspace_size_layers(2, trees, ctypes.byref(p), ios, ctypes.byref(sz)) == \
+        binding.ATLASKV_EINVAL                                         # null trees
+    assert lib.atlaskv_workspace_size_layers(0, trees, ctypes.byref(p), ios, ctypes.byref(sz)) == \
+        binding.ATLASKV_EINVAL                                         # no layers
+    assert lib.atlaskv_workspace_size_layers(binding.MAX_LAYERS + 1, trees, ctypes.byref(p), ios,
+                                             ctypes.byref(sz)) == binding.ATLASKV_EINVAL
+    assert lib.atlaskv_attend_layers(2, trees, ctypes.byref(p), ios, None, 0, None) == binding.ATLASKV_EINVAL
 
 
 def test_error_wrapper_raises(lib):

@@ -67,10 +67,14 @@ def test_kernels_per_step_and_config():
     from hierarchical_kv_pruning_b200 import synth
     dev = synth.shape(2)
     host = synth.shape(4)
-    assert bench.kernels_per_step(dev) == 10
-    assert host.batch >= 8 and bench.kernels_per_step(host) == 4 * 14   # four query chunks
+    # leaves in HBM, bf16 D = 128: the descent, the sequence part, the knowledge part
+    assert bench.kernels_per_step(dev) == 3
+    # host leaves: 7 launches per query chunk (four chunks) plus one sequence part
+    assert host.batch >= 8 and bench.kernels_per_step(host) == 4 * 7 + 1
     import dataclasses
-    assert bench.kernels_per_step(dataclasses.replace(host, batch=7)) == 14
+    assert bench.kernels_per_step(dataclasses.replace(host, batch=7)) == 7 + 1
+    # fp32: the descent and one fused attention launch
+    assert bench.kernels_per_step(synth.shape(0)) == 2
     c = bench.config_of(dev, 4)
     assert c["workload"] == dev.name and c["parallelism"] == "replicas x4"
     assert c["B"] == dev.batch and c["K"] == list(dev.keep)

@@ -3,9 +3,10 @@
 Kept node and leaf sets must be bit-exact.  Outputs: float32 within
 1e-5 * max|y_ref| (max-abs), bfloat16 within 2e-2 max-abs on unit-scale
 outputs; LSE within 1e-4 (float32) / 2e-3 (bfloat16, logits from bfloat16
-inputs accumulated in fp32).  Full-size shapes are checked on sampled
-traversals against the oracle and on every traversal by properties that hold
-at any size (ascending, distinct, in range, nested).
+inputs accumulated in fp32).  At the benchmark shapes the kept sets of every
+traversal are compared with the oracle's descent, the outputs on 256 sampled
+traversals, and every traversal is also checked by properties that hold at any
+size (ascending, distinct, in range, nested).
 """
 import math
 import os
@@ -240,6 +241,106 @@ def test_leaves_in_pinned_host_memory_chunked():
     compare(w, sh.keep, g_host)
 
 
+def _host_levels(w, mids=True):
+    """The same workload with the leaf keys and values (and the mid keys) in
+    pinned host memory: only the root keys stay on the device."""
+    return synth.Workload(w.shape, w.root_keys, w.mid_keys.cpu().pin_memory() if mids else w.mid_keys,
+                          w.leaf_keys.cpu().pin_memory(), w.leaf_values.cpu().pin_memory(), w.root_child,
+                          w.mid_child, w.q_kg, w.q_seq, w.k_seq, w.v_seq, w.targets)
+
+
+@pytest.mark.parametrize("batch", [3, 9])   # one query chunk; four chunks (2, 2, 2, 3)
+def test_mids_and_leaves_in_pinned_host_memory(batch):
+    # Only the roots resident: the kept roots' mid blocks are staged before
+    # level 1, the kept mids' leaf blocks before level 2; results equal the
+    # HBM-resident path bit for bit and match the oracle.
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(12, 10, 9),
+                      keep=(3, 4, 16), batch=batch, n_tokens=16, seq_len=48, permuted=True)
+    w = synth.make_workload(sh, "cuda", 18 + batch)
+    g_dev = gpu_run(w, sh.keep)
+    g_host = gpu_run(_host_levels(w), sh.keep)
+    for k in ("kept_root", "kept_mid", "kept_leaf", "out", "lse"):
+        assert torch.equal(g_dev[k], g_host[k]), k
+    compare(w, sh.keep, g_host)
+
+
+def test_host_mids_fp32_d64():
+    sh = synth.custom(dtype=torch.float32, n_heads=2, n_kv_heads=1, head_dim=64, fanout=(9, 7, 5),
+                      keep=(3, 5, 9), batch=2, n_tokens=5, seq_len=9)
+    w = synth.make_workload(sh, "cuda", 21)
+    g_host = gpu_run(_host_levels(w), sh.keep)
+    compare(w, sh.keep, g_host)
+
+
+def test_mids_on_host_need_leaves_on_host():
+    from hierarchical_kv_pruning_b200.binding import ATLASKV_EINVAL
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=2, n_kv_heads=1, head_dim=128, fanout=(4, 4, 4),
+                      keep=(2, 2, 2), batch=1, n_tokens=2, seq_len=2)
+    w = synth.make_workload(sh, "cuda", 22)
+    with pytest.raises(AtlaskvError) as ei:
+        HikvpTree(w.root_keys, w.mid_keys.cpu().pin_memory(), w.leaf_keys, w.leaf_values, sh.fanout)
+    assert ei.value.status == ATLASKV_EINVAL
+
+
+@pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.bfloat16, 64), (torch.float32, 128)])
+def test_decode_step_single_token(dtype, D):
+    # A decode step: one query token (N = 1) attends to the T - 1 tokens
+    # before it and to itself, and to its kept leaves.
+    sh = synth.custom(dtype=dtype, n_heads=8, n_kv_heads=2, head_dim=D, fanout=(16, 12, 10),
+                      keep=(4, 6, 24), batch=5, n_tokens=1, seq_len=77, permuted=True)
+    w = synth.make_workload(sh, "cuda", 23)
+    g = gpu_run(w, sh.keep)
+    check_structure(w, sh.keep, g)
+    compare(w, sh.keep, g)
+
+
+@pytest.mark.parametrize("n_tokens", [1, 24])
+def test_layers_in_one_call_match_single_calls(n_tokens):
+    # Several layers, each with its own tree and inputs, in one batched call:
+    # every layer's results equal its own single call bit for bit and match
+    # the oracle.
+    from hierarchical_kv_pruning_b200.binding import attend_layers
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(10, 9, 8),
+                      keep=(3, 5, 16), batch=6, n_tokens=n_tokens, seq_len=40)
+    layers = [synth.make_workload(sh, "cuda", 30 + l) for l in range(4)]
+    trees = [HikvpTree.from_workload(w) for w in layers]
+    try:
+        got = attend_layers(trees, [(w.q_kg, w.q_seq, w.k_seq, w.v_seq) for w in layers], sh.keep)
+        for t in trees:
+            t.sync_status()
+        for l, (w, t) in enumerate(zip(layers, trees)):
+            one = gpu_run(w, sh.keep, tree=t)
+            for k in ("kept_root", "kept_mid", "kept_leaf", "out", "lse"):
+                assert torch.equal(got[l][k].cpu(), one[k]), (l, k)
+        compare(layers[1], sh.keep, {k: v.cpu() for k, v in got[1].items() if k != "workspace"})
+    finally:
+        for t in trees:
+            t.close()
+
+
+def test_layers_fp32_and_mismatch_rejected():
+    from hierarchical_kv_pruning_b200.binding import ATLASKV_EINVAL, attend_layers
+    sh = synth.custom(dtype=torch.float32, n_heads=2, n_kv_heads=1, head_dim=64, fanout=(6, 5, 4),
+                      keep=(2, 3, 6), batch=2, n_tokens=3, seq_len=7)
+    layers = [synth.make_workload(sh, "cuda", 40 + l) for l in range(2)]
+    trees = [HikvpTree.from_workload(w) for w in layers]
+    try:
+        got = attend_layers(trees, [(w.q_kg, w.q_seq, w.k_seq, w.v_seq) for w in layers], sh.keep)
+        for t in trees:
+            t.sync_status()
+        for l, w in enumerate(layers):
+            compare(w, sh.keep, {k: v.cpu() for k, v in got[l].items() if k != "workspace"})
+        w0, w1 = layers
+        with pytest.raises(AtlaskvError) as ei:     # T differs between the layers
+            attend_layers(trees, [(w0.q_kg, w0.q_seq, w0.k_seq, w0.v_seq),
+                                  (w1.q_kg, w1.q_seq, w1.k_seq[:, :5].contiguous(), w1.v_seq[:, :5].contiguous())],
+                          sh.keep)
+        assert ei.value.status == ATLASKV_EINVAL
+    finally:
+        for t in trees:
+            t.close()
+
+
 def test_deterministic_and_b0():
     sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(10, 10, 10),
                       keep=(3, 4, 16), batch=4, n_tokens=32, seq_len=64)
@@ -327,13 +428,40 @@ def full_cache():
     return {}
 
 
+def compare_all_indices(w, K, g):
+    """Kept root, mid and leaf sets of EVERY traversal against the oracle's
+    descent (bit-exact)."""
+    sh = w.shape
+    t = oracle_tree(w)
+    q = storage(w.q_kg)
+    kr, km, kl = oracle.descend(t, q, K)
+    for name, ref in (("kept_root", kr), ("kept_mid", km), ("kept_leaf", kl)):
+        got = g[name].reshape(sh.batch * sh.n_heads, -1).numpy()
+        bad = np.nonzero((got != ref).any(axis=1))[0]
+        assert bad.size == 0, (name, "traversals differ", [(int(i) // sh.n_heads, int(i) % sh.n_heads)
+                                                          for i in bad[:8]], bad.size)
+
+
+def gpu_run_profiled(w, K):
+    """gpu_run with the library's descent counters on: returns the outputs and
+    per level the number of selections the fp32 band left open."""
+    with HikvpTree.from_workload(w) as tree:
+        tree.set_profiling(True)
+        g = gpu_run(w, K, tree=tree)
+        stats = tree.refine_stats()
+    return g, stats
+
+
 @pytest.mark.parametrize("i", [1, 2, 3])
 def test_full_size_shapes(i, full_cache):
     sh = synth.shape(i)
     w = synth.make_workload(sh, "cuda", 1000 + i)
-    g = gpu_run(w, sh.keep)
+    g, stats = gpu_run_profiled(w, sh.keep)
+    print("refined selections per level (%s):" % sh.name,
+          {lvl: (v["refined"], v["exact_scores"]) for lvl, v in stats.items()})
     check_structure(w, sh.keep, g)
-    trav = sample_traversals(sh.batch, sh.n_heads, 10, seed=i)
+    compare_all_indices(w, sh.keep, g)
+    trav = sample_traversals(sh.batch, sh.n_heads, 256, seed=i)
     compare(w, sh.keep, g, trav)
     del w
     torch.cuda.empty_cache()
@@ -346,10 +474,35 @@ def test_full_size_host_leaves():
     if free_host < need:
         pytest.skip("host memory %.0f GB below the %.0f GB the host-leaf shape needs" % (free_host / 1e9, need / 1e9))
     w = synth.make_workload(sh, "cuda", 1004)
-    g = gpu_run(w, sh.keep)
+    g, stats = gpu_run_profiled(w, sh.keep)
+    print("refined selections per level (%s):" % sh.name,
+          {lvl: (v["refined"], v["exact_scores"]) for lvl, v in stats.items()})
     check_structure(w, sh.keep, g)
-    trav = sample_traversals(sh.batch, sh.n_heads, 6, seed=4)
+    compare_all_indices(w, sh.keep, g)
+    trav = sample_traversals(sh.batch, sh.n_heads, 256, seed=4)
     compare(w, sh.keep, g, trav)
+
+
+def test_full_size_host_mids():
+    # The host-leaf benchmark shape with the mid level in host memory too:
+    # every output equals the host-leaf path's on the same buffers, and the
+    # kept sets of a sample match the oracle.
+    sh = synth.shape("host_mids")
+    free_host = os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_AVPHYS_PAGES")
+    need = 2 * sh.n_leaves * sh.head_dim * 2 + (8 << 30)
+    if free_host < need:
+        pytest.skip("host memory %.0f GB below the %.0f GB the host-leaf shape needs" % (free_host / 1e9, need / 1e9))
+    w = synth.make_workload(sh, "cuda", 1004)
+    assert not w.mid_keys.is_cuda and w.mid_keys.is_pinned()
+    g_mids = gpu_run(w, sh.keep)
+    w_dev_mids = synth.Workload(sh, w.root_keys, w.mid_keys.cuda(), w.leaf_keys, w.leaf_values, None, None,
+                                w.q_kg, w.q_seq, w.k_seq, w.v_seq, w.targets)
+    g_leaves = gpu_run(w_dev_mids, sh.keep)
+    for k in ("kept_root", "kept_mid", "kept_leaf", "out", "lse"):
+        assert torch.equal(g_mids[k], g_leaves[k]), k
+    check_structure(w, sh.keep, g_mids)
+    trav = sample_traversals(sh.batch, sh.n_heads, 256, seed=5)
+    compare(w, sh.keep, g_mids, trav)
 
 
 def test_bounded_device_wait_reports_timeout():
@@ -369,3 +522,90 @@ def test_bounded_device_wait_reports_timeout():
         assert time.time() - t0 < 60
     g = gpu_run(w, sh.keep)
     compare(w, sh.keep, g)
+
+
+# ---- trees of any depth with variable numbers of children (CSR) ------------
+
+def _csr_oracle(w):
+    return oracle.CsrTree([storage(k) for k in w.keys], storage(w.leaf_values),
+                          [o.cpu().numpy() for o in w.child_off],
+                          [None if c is None else c.cpu().numpy() for c in w.child_id])
+
+
+def _compare_csr(w, K, g, traversals=None):
+    from hierarchical_kv_pruning_b200.binding import CsrHikvpTree  # noqa: F401
+    sh = w.shape
+    inp = dict(q_kg=storage(w.q_kg), q_seq=storage(w.q_seq), k_seq=storage(w.k_seq), v_seq=storage(w.v_seq))
+    r = oracle.hikvp_csr(_csr_oracle(w), inp["q_kg"], inp["q_seq"], inp["k_seq"], inp["v_seq"], K, traversals)
+    for i, (b, h) in enumerate(r["traversals"]):
+        for l in range(len(K)):
+            assert g["kept"][l][b, h].tolist() == r["kept"][l][i].tolist(), ("level", l, b, h)
+        y = g["out"][b, :, h, :].double().numpy()
+        err = np.max(np.abs(y - r["y"][i]))
+        if sh.dtype == torch.float32:
+            assert err <= 1e-5 * np.max(np.abs(r["y"][i])), (b, h, err)
+        else:
+            assert err <= BF16_TOL, (b, h, err)
+        assert np.max(np.abs(g["lse"][b, :, h].double().numpy() - r["lse"][i])) <= LSE_TOL[sh.dtype]
+
+
+CSR_CASES = [
+    # (dtype, H, H_kv, D, n_roots, fan-out ranges, K per level, B, N, T, permuted)
+    (torch.bfloat16, 8, 2, 128, 12, ((3, 9),), (4, 12), 3, 16, 40, False),                  # depth 2
+    (torch.bfloat16, 8, 2, 128, 20, ((2, 12), (3, 15)), (6, 10, 24), 3, 24, 50, True),      # depth 3, permuted
+    (torch.bfloat16, 32, 1, 128, 16, ((4, 9), (2, 7), (3, 6)), (5, 9, 12, 30), 2, 8, 20, True),   # depth 4, G = 32
+    (torch.float32, 4, 2, 64, 10, ((1, 6), (2, 5)), (3, 3, 6), 2, 5, 9, False),             # fp32, single children
+]
+
+
+@pytest.mark.parametrize("case", CSR_CASES, ids=[str(i) for i in range(len(CSR_CASES))])
+def test_csr_trees(case):
+    from hierarchical_kv_pruning_b200.binding import CsrHikvpTree
+    dtype, H, H_kv, D, n_roots, ranges, K, B, N, T, perm = case
+    sh = synth.CsrShape("csr", dtype, H, H_kv, D, n_roots, ranges, K, B, N, T, permuted=perm)
+    w = synth.make_csr_workload(sh, "cuda", 91)
+    with CsrHikvpTree.from_workload(w) as tree:
+        tree.set_profiling(times=False, counters=True)
+        g = tree.attend(w.q_kg, w.q_seq, w.k_seq, w.v_seq, K)
+        tree.sync_status()
+        assert tree.refine_stats()["root"]["selections"] == B * H
+    g = {"out": g["out"].cpu(), "lse": g["lse"].cpu(), "kept": [k.cpu() for k in g["kept"]]}
+    _compare_csr(w, K, g)
+
+
+def test_uniform_tree_as_csr_matches_the_uniform_path():
+    from hierarchical_kv_pruning_b200.binding import CsrHikvpTree
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(12, 10, 9),
+                      keep=(3, 5, 16), batch=3, n_tokens=16, seq_len=48, permuted=True)
+    w = synth.make_workload(sh, "cuda", 92)
+    g_u = gpu_run(w, sh.keep)
+    bR, bI, bL = sh.fanout
+    off0 = (torch.arange(bR + 1, dtype=torch.int32, device="cuda") * bI).expand(2, -1).contiguous()
+    off1 = (torch.arange(bR * bI + 1, dtype=torch.int32, device="cuda") * bL).expand(2, -1).contiguous()
+    ids0 = w.root_child.reshape(2, -1).contiguous()
+    ids1 = w.mid_child.reshape(2, -1).contiguous()
+    with CsrHikvpTree([w.root_keys, w.mid_keys, w.leaf_keys], w.leaf_values, [off0, off1], [ids0, ids1]) as t:
+        g_c = t.attend(w.q_kg, w.q_seq, w.k_seq, w.v_seq, sh.keep)
+        t.sync_status()
+    for l, name in enumerate(("kept_root", "kept_mid", "kept_leaf")):
+        assert torch.equal(g_c["kept"][l].cpu(), g_u[name]), name
+    assert torch.equal(g_c["out"].cpu(), g_u["out"]) and torch.equal(g_c["lse"].cpu(), g_u["lse"])
+
+
+def test_csr_rejects_bad_offsets_and_too_large_K():
+    from hierarchical_kv_pruning_b200.binding import ATLASKV_EINVAL, CsrHikvpTree
+    sh = synth.CsrShape("bad", torch.bfloat16, 2, 1, 128, 6, ((2, 4), (1, 3)), (2, 2, 2), 1, 2, 3)
+    w = synth.make_csr_workload(sh, "cuda", 93)
+    bad = w.child_off[0].clone()
+    bad[0, 2] = bad[0, 3] + 1                    # decreasing offsets
+    with pytest.raises(AtlaskvError) as ei:
+        CsrHikvpTree(w.keys, w.leaf_values, [bad, w.child_off[1]])
+    assert ei.value.status == ATLASKV_EINVAL
+    fewest = int((w.child_off[1][:, 1:] - w.child_off[1][:, :-1]).min())
+    with CsrHikvpTree.from_workload(w) as t:
+        # level 2 asks for more leaves than 2 kept mids with the fewest children have
+        with pytest.raises(AtlaskvError) as ei:
+            t.attend(w.q_kg, w.q_seq, w.k_seq, w.v_seq, (2, 2, 2 * fewest + 1))
+        assert ei.value.status == ATLASKV_EINVAL
+        g = t.attend(w.q_kg, w.q_seq, w.k_seq, w.v_seq, (2, 2, 2 * fewest))
+        t.sync_status()

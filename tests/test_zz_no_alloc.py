@@ -53,6 +53,32 @@ def test_static_scratch_matches_workspace_path(dtype):
             assert (lse - ref["lse"]).abs().max().item() <= 1e-4
 
 
+def test_static_scratch_allocates_nothing():
+    # After one warm call (the first call on a device looks up the static
+    # array's address, and the runtime may load the library's device code
+    # then), further calls change neither the device's free memory nor torch's
+    # allocation count.
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(12, 10, 9),
+                      keep=(3, 5, 16), batch=4, n_tokens=24, seq_len=70, permuted=True)
+    w = synth.make_workload(sh, "cuda", 33)
+    with binding.HikvpTree.from_workload(w) as tree:
+        out, lse, kept = _outputs(w)
+        io = _io(w, out, lse, kept)
+        params = tree.params(sh.keep)
+        stream = torch.cuda.current_stream().cuda_stream
+        binding.atlaskv_attend_static(tree.handle, params, io, stream)
+        tree.sync_status()
+        torch.cuda.synchronize()
+        free0 = torch.cuda.mem_get_info()[0]
+        allocs0 = torch.cuda.memory_stats().get("allocation.all.allocated", 0)
+        for _ in range(3):
+            binding.atlaskv_attend_static(tree.handle, params, io, stream)
+        tree.sync_status()
+        torch.cuda.synchronize()
+        assert torch.cuda.mem_get_info()[0] == free0
+        assert torch.cuda.memory_stats().get("allocation.all.allocated", 0) == allocs0
+
+
 def test_static_scratch_rejects_sizes_above_its_maximum():
     # B * H * D * 4 bytes of token sums alone exceed the 16 MiB maximum.
     sh = synth.custom(dtype=torch.bfloat16, n_heads=32, n_kv_heads=8, head_dim=128, fanout=(4, 4, 4),
