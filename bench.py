@@ -74,25 +74,50 @@ def config_of(sh, world):
 
 
 def splits_attention(sh):
-    """bf16, D = 128: the sequence part is its own launch beside the descent
-    and the knowledge part merges with it (tensor-core attention)."""
+    """bf16, D = 128 with host-resident leaves: the sequence part is its own
+    launch beside the descent and the staging, and the knowledge part merges
+    with it (tensor-core attention)."""
     import torch
-    return sh.dtype == torch.bfloat16 and sh.head_dim == 128
+    return sh.dtype == torch.bfloat16 and sh.head_dim == 128 and sh.leaf_on_host
 
 
-def kernels_per_step(sh):
-    """Kernels one atlaskv_attend call launches.  Leaves in HBM: the fused
-    descent, then the attention as one launch, or as two (sequence part,
-    knowledge part) when it is split.  Host-resident leaves: per query chunk
-    (four chunks when B >= 8, else one) the descent of levels 0-1, a
-    de-duplication and a staging copy of the leaf-key blocks, the descent of
-    level 2, a de-duplication and a staging copy of the value rows, and the
-    knowledge part; plus one sequence-part launch for the whole batch."""
-    split = splits_attention(sh)
+def uses_parent_major(sh, descent="auto"):
+    """The descent the library runs (ATLASKV_DESCENT_AUTO: parent-major from
+    B * H >= 512 traversals)."""
+    if descent != "auto":
+        return descent == "parent_major"
+    return sh.batch * sh.n_heads >= 512
+
+
+def kernels_per_step(sh, descent="auto"):
+    """Kernels one atlaskv_attend call launches.  The fused descent is one
+    launch; the parent-major one is the token sums, then per level a scoring,
+    a selection and a refinement launch, and per level below the roots a scan
+    and a fill.  Leaves in HBM: the descent, then the attention (one launch).
+    Host-resident leaves: per query chunk (four chunks when B >= 8, else one)
+    the descent up to the level above the leaves, a de-duplication and a
+    staging copy of the leaf-key blocks (and, with the mids on the host, of the
+    mid blocks before level 1), the leaf level, a de-duplication and a staging
+    copy of the value rows, and the knowledge part; plus one sequence-part
+    launch for the whole batch (bf16, D = 128)."""
+    pm = uses_parent_major(sh, descent)
+
+    def levels(first, last):
+        if not pm:
+            return 1
+        n = 0
+        for lvl in range(first, last + 1):
+            n += 3 + (1 if lvl == 0 else 2)
+        return n
+
     if not sh.leaf_on_host:
-        return 3 if split else 2
+        return levels(0, 2) + 1
     chunks = 4 if sh.batch >= 8 else 1
-    return 7 * chunks + (1 if split else 0)
+    if sh.mid_on_host:
+        per = levels(0, 0) + 2 + levels(1, 1) + 2 + levels(2, 2) + 2 + 1
+    else:
+        per = levels(0, 1) + 2 + levels(2, 2) + 2 + 1
+    return chunks * per + (1 if splits_attention(sh) else 0)
 
 
 def max_over_ranks(x, world, device):
@@ -487,7 +512,7 @@ def measure(sh, seed, args, world, rank, local, cpu_seconds, use_graph=False):
     entry = {"value": value, "unit": "queries/s", "ms_per_step": ms_per_step,
              "us_per_query": 1e3 * ms_per_step / sh.batch,
              "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-             "gpu_launches": kernels_per_step(sh) * args.steps, "roofline": roof, "clocks": clk.summary(),
+             "gpu_launches": kernels_per_step(sh, args.descent) * args.steps, "roofline": roof, "clocks": clk.summary(),
              "config": config_of(sh, world), "cuda_graph": use_graph,
              "dtype": "f32" if sh.dtype == torch.float32 else "bf16"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

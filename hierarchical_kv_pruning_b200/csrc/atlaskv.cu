@@ -50,10 +50,12 @@ bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 // Raise a kernel's dynamic shared-memory limit to `bytes` once per (kernel,
 // device): later calls configure nothing, so an attend call can be captured
-// into a CUDA graph after a first, uncaptured one.
+// into a CUDA graph after a first, uncaptured one.  (The default limit leaves
+// 48 KB for static and dynamic shared memory together, so any dynamic size is
+// set explicitly.)
 atlaskv_status ensure_smem(const void *kernel, size_t bytes)
 {
-    if (bytes <= 48 * 1024) return ATLASKV_OK;
+    if (bytes == 0) return ATLASKV_OK;
     int dev = 0;
     AKV_CUDA(cudaGetDevice(&dev));
     static std::mutex m;
@@ -234,10 +236,9 @@ PmPlan plan_pm(const atlaskv_tree *t, const Ks &ks, long long Bc, int H, int kca
     PmPlan pp;
     const int D = t->d.head_dim;
     const int esz = (int)(t->d.dtype == ATLASKV_F32 ? 4 : 2);
-    const int lpg = D * esz / 16;
     const int G = H / t->d.n_kv_heads;
-    pp.HT = std::max(4, lpg / 4);
-    pp.EC = akv::kPmWarps * pp.HT;
+    pp.HT = akv::kPmEC;
+    pp.EC = akv::kPmEC;
     const size_t pw = akv::pm_select_warp_bytes(kcap, cap, kp_max(ks));
     if (pw > 200 * 1024) return pp;
     pp.pw = (int)pw;
@@ -251,6 +252,9 @@ PmPlan plan_pm(const atlaskv_tree *t, const Ks &ks, long long Bc, int H, int kca
     pp.ts_smem = akv::token_sums_smem(pp.ts_GC, D, esz);
     pp.BHc = Bc * H;
     pp.cpre = t->csr;
+    // refinement queues: a length per level, one queue of BH entries reused by the levels
+    pp.zero_bytes = 16 * akv::kMaxLevels;
+    pp.data_bytes = r16((size_t)pp.BHc * 16);
     for (int l = 0; l < ks.n; ++l)   // key rows of a level are addressed with 32-bit row numbers
         if ((long long)t->d.n_kv_heads * t->rows[l] > (1LL << 31) - 1) return pp;
     for (int l = 1; l < ks.n; ++l) {
@@ -272,6 +276,12 @@ PmPlan plan_pm(const atlaskv_tree *t, const Ks &ks, long long Bc, int H, int kca
 void pm_bind(const PmPlan &pp, int n_levels, long long BH, uint8_t *zero, uint8_t *data, akv::PmLevel *lv)
 {
     for (int l = 0; l < akv::kMaxLevels; ++l) lv[l] = akv::PmLevel{};
+    for (int l = 0; l < n_levels; ++l) {
+        lv[l].qcount = reinterpret_cast<int32_t *>(zero + 16 * l);
+        lv[l].queue = reinterpret_cast<int4 *>(data);
+    }
+    zero += 16 * akv::kMaxLevels;
+    data += r16((size_t)pp.BHc * 16);
     for (int l = 1; l < n_levels; ++l) {
         akv::PmLevel &v = lv[l];
         const long long Kp = pp.E[l] / pp.BHc;
@@ -523,76 +533,107 @@ atlaskv_status dispatch_descend(int dtype, int D, const akv::DescendParams &dp, 
                    : launch_descend<__nv_bfloat16, 128>(dp, HT, smem, first, last, s);
 }
 
+// Launch with programmatic stream serialization: the kernel may begin while
+// the previous kernel on the stream drains; it waits (griddep_wait) before it
+// reads anything that kernel wrote.
+template <typename... KArgs, typename... Args>
+atlaskv_status launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+                          Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    AKV_CUDA(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
+    return ATLASKV_OK;
+}
+
 // ---- parent-major descent launches -------------------------------------------
 // Levels first..last of one query chunk: token sums, root scores and root
 // selection when first = 0; then per level the inversion of the kept parents
 // (scan, fill), the scores by parent and the selection.  Each selection but
 // the last level's counts its kept entries for the next level's inversion.
-template <typename T, int D, int HT>
-atlaskv_status run_pm_ht(const atlaskv_tree *t, const PmPlan &pp, const akv::DescendParams &dp, const akv::PmLevel *lv,
-                         int first, int last, cudaStream_t s)
+#define AKV_TRY(x)                                 \
+    do {                                           \
+        const atlaskv_status st_ = (x);            \
+        if (st_ != ATLASKV_OK) return st_;         \
+    } while (0)
+
+// zero / zero_bytes: the chunk's zero-initialised inversion region, cleared
+// by the token-sum kernel (first = 0).
+template <typename T, int D>
+atlaskv_status run_pm(const atlaskv_tree *t, const PmPlan &pp, const akv::DescendParams &dp, const akv::PmLevel *lv,
+                      uint8_t *zero, size_t zero_bytes, int first, int last, cudaStream_t s)
 {
     const int nl = dp.n_levels;
     const long long BH = (long long)dp.B * dp.H;
     if (BH == 0) return ATLASKV_OK;
-    const long long score_cap = (long long)t->num_sms * 4;
     const akv::PmLevel none{};
     const size_t sel_smem = (size_t)pp.nsel * pp.pw;
     AKV_SMEM((akv::pm_select_kernel<T, D>), sel_smem);
     const unsigned sel_grid = (unsigned)((BH + pp.nsel - 1) / pp.nsel);
+    const size_t score_smem = akv::pm_score_smem(D, (int)sizeof(T));
+    AKV_SMEM((akv::pm_score_kernel<T, D>), score_smem);
+    // the scoring grid: as many CTAs as fit on the device at once (the warps loop over the items)
+    static thread_local std::map<std::pair<const void *, int>, int> fit;
+    int &per_sm = fit[{reinterpret_cast<const void *>(akv::pm_score_kernel<T, D>), t->num_sms}];
+    if (per_sm == 0) {
+        AKV_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, akv::pm_score_kernel<T, D>, akv::kPmThreads,
+                                                               score_smem));
+        per_sm = std::max(per_sm, 1);
+    }
+    const long long score_cap = (long long)t->num_sms * per_sm;
+    const size_t ref_smem = (size_t)(akv::kSelThreads / 32) * (dp.Kpmax + 1) * 4;
+    AKV_SMEM((akv::pm_refine_kernel<T, D>), ref_smem);
+    const unsigned ref_grid = (unsigned)std::min<long long>((BH + 7) / 8, (long long)t->num_sms * 2);
     auto select = [&](int L) -> atlaskv_status {
-        akv::pm_select_kernel<T, D><<<sel_grid, akv::kSelThreads, sel_smem, s>>>(dp, L + 1 < nl ? lv[L + 1] : none, L,
-                                                                               pp.nsel, pp.pw);
-        AKV_CUDA(cudaGetLastError());
+        const akv::PmLevel &nx = L + 1 < nl ? lv[L + 1] : none;
+        AKV_TRY(launch_pdl(akv::pm_select_kernel<T, D>, sel_grid, akv::kSelThreads, sel_smem, s, dp, lv[L], nx, L,
+                           pp.nsel, pp.pw));
+        AKV_TRY(launch_pdl(akv::pm_refine_kernel<T, D>, ref_grid, akv::kSelThreads, ref_smem, s, dp, lv[L], nx, L));
         return ATLASKV_OK;
     };
     if (first == 0) {
         const long long tsg = (long long)dp.B * dp.H_kv * (dp.G / pp.ts_GC);
-        akv::token_sums_kernel<T, D><<<(unsigned)tsg, akv::kDescThreads, pp.ts_smem, s>>>(dp, pp.ts_GC);
-        AKV_CUDA(cudaGetLastError());
+        AKV_TRY(launch_pdl(akv::token_sums_kernel<T, D>, (unsigned)tsg, akv::kDescThreads, pp.ts_smem, s, dp, pp.ts_GC,
+                           reinterpret_cast<uint4 *>(zero), (long long)(zero_bytes / 16)));
         const long long items = (long long)dp.H_kv * ((dp.B * dp.G + pp.EC - 1) / pp.EC);
-        akv::pm_score_kernel<T, D, HT>
-            <<<(unsigned)std::min(items, score_cap), akv::kPmThreads, 0, s>>>(dp, none, 0, pp.EC);
-        AKV_CUDA(cudaGetLastError());
-        atlaskv_status st = select(0);
-        if (st != ATLASKV_OK) return st;
+        AKV_TRY(launch_pdl(akv::pm_score_kernel<T, D>,
+                           (unsigned)std::min((items + akv::kPmWarps - 1) / akv::kPmWarps, score_cap), akv::kPmThreads,
+                           score_smem, s, dp, none, 0));
+        AKV_TRY(select(0));
     }
     for (int L = std::max(first, 1); L <= last; ++L) {
         const akv::PmLevel &v = lv[L];
-        akv::pm_scan_kernel<<<(unsigned)v.n_tiles, akv::kScanThreads, 0, s>>>(v, pp.EC, dp.status);
-        AKV_CUDA(cudaGetLastError());
+        AKV_TRY(launch_pdl(akv::pm_scan_kernel, (unsigned)v.n_tiles, akv::kScanThreads, 0, s, v, pp.EC, dp.status));
         const unsigned fg = (unsigned)std::min<long long>((v.E + 255) / 256, (long long)t->num_sms * 8);
-        akv::pm_fill_kernel<<<std::max(1u, fg), 256, 0, s>>>(dp.kept[L - 1], dp.K[L - 1], dp.H, dp.G, dp.rows[L - 1], v,
-                                                             dp.status);
-        AKV_CUDA(cudaGetLastError());
-        akv::pm_score_kernel<T, D, HT>
-            <<<(unsigned)std::min<long long>(v.max_items, score_cap), akv::kPmThreads, 0, s>>>(dp, v, L, pp.EC);
-        AKV_CUDA(cudaGetLastError());
-        atlaskv_status st = select(L);
-        if (st != ATLASKV_OK) return st;
+        AKV_TRY(launch_pdl(akv::pm_fill_kernel, std::max(1u, fg), 256, 0, s, (const int32_t *)dp.kept[L - 1],
+                           dp.K[L - 1], dp.H, dp.G, (long long)dp.rows[L - 1], v, dp.status));
+        AKV_TRY(launch_pdl(akv::pm_score_kernel<T, D>,
+                           (unsigned)std::min<long long>((v.max_items + akv::kPmWarps - 1) / akv::kPmWarps, score_cap),
+                           akv::kPmThreads, score_smem, s, dp, v, L));
+        AKV_TRY(select(L));
     }
     return ATLASKV_OK;
 }
 
-template <typename T, int D>
-atlaskv_status run_pm(const atlaskv_tree *t, const PmPlan &pp, const akv::DescendParams &dp, const akv::PmLevel *lv,
-                      int first, int last, cudaStream_t s)
-{
-    // heads per warp: a quarter of a key row's lanes, at least 4 (plan_pm)
-    constexpr int lpg = D * (int)sizeof(T) / 16;
-    if constexpr (lpg == 32) return run_pm_ht<T, D, 8>(t, pp, dp, lv, first, last, s);
-    else return run_pm_ht<T, D, 4>(t, pp, dp, lv, first, last, s);
-}
 
 atlaskv_status dispatch_pm(const atlaskv_tree *t, const PmPlan &pp, const akv::DescendParams &dp,
-                           const akv::PmLevel *lv, int first, int last, cudaStream_t s)
+                           const akv::PmLevel *lv, uint8_t *zero, size_t zero_bytes, int first, int last,
+                           cudaStream_t s)
 {
     const int D = t->d.head_dim;
     if (t->d.dtype == ATLASKV_F32)
-        return D == 64 ? run_pm<float, 64>(t, pp, dp, lv, first, last, s)
-                       : run_pm<float, 128>(t, pp, dp, lv, first, last, s);
-    return D == 64 ? run_pm<__nv_bfloat16, 64>(t, pp, dp, lv, first, last, s)
-                   : run_pm<__nv_bfloat16, 128>(t, pp, dp, lv, first, last, s);
+        return D == 64 ? run_pm<float, 64>(t, pp, dp, lv, zero, zero_bytes, first, last, s)
+                       : run_pm<float, 128>(t, pp, dp, lv, zero, zero_bytes, first, last, s);
+    return D == 64 ? run_pm<__nv_bfloat16, 64>(t, pp, dp, lv, zero, zero_bytes, first, last, s)
+                   : run_pm<__nv_bfloat16, 128>(t, pp, dp, lv, zero, zero_bytes, first, last, s);
 }
 
 // ---- attention launch -----------------------------------------------------
@@ -666,9 +707,7 @@ atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
     st = encode_seq_map(&mv, ap.v_seq, ap.B, ap.T, ap.H_kv);
     if (st != ATLASKV_OK) return st;
     AKV_SMEM(akv::attend_tc_kernel, akv::tc::kSmemBytes);
-    akv::attend_tc_kernel<<<(unsigned)grid, akv::tc::kThreads, akv::tc::kSmemBytes, s>>>(ap, cpg, mk, mv);
-    AKV_CUDA(cudaGetLastError());
-    return ATLASKV_OK;
+    return launch_pdl(akv::attend_tc_kernel, (unsigned)grid, akv::tc::kThreads, akv::tc::kSmemBytes, s, ap, cpg, mk, mv);
 }
 
 atlaskv_status dispatch_attend(int dtype, int D, const akv::AttnParams &ap, cudaStream_t s)
@@ -928,11 +967,14 @@ atlaskv_status inflate_norms(atlaskv_tree *t)
     return ATLASKV_OK;
 }
 
-// The tree's small device words and, for bf16 D = 128, its two streams and
-// events (shared by both create functions).
+// The tree's small device words and, for bf16 D = 128 with host-resident
+// leaves, its two streams and events (shared by both create functions).  The
+// sequence part runs as its own launch only there, where it overlaps the host
+// link; with the leaves in HBM the descent keeps every SM busy and the
+// attention is one launch after it.
 atlaskv_status init_tree_device(atlaskv_tree *t)
 {
-    t->split = t->d.dtype == ATLASKV_BF16 && t->d.head_dim == akv::tc::kD;
+    t->split = t->d.dtype == ATLASKV_BF16 && t->d.head_dim == akv::tc::kD && t->host_leaves;
     if (t->split) {
         // the sequence part runs beside the descent: lowest priority for it,
         // highest for the descent (the critical path); created once here so
@@ -1295,10 +1337,9 @@ atlaskv_status attend_impl(atlaskv_tree *t, const Ks &ks, const atlaskv_io *io, 
     // the whole descent of an HBM call on stream `st`
     auto descend_all = [&](cudaStream_t st) -> atlaskv_status {
         if (!L.pm) return dispatch_descend(t->d.dtype, D, dp, L.desc.HT, L.desc.smem, 0, t->n_levels - 1, st);
-        AKV_CUDA(cudaMemsetAsync(ws + L.pm_zero, 0, L.pmp.zero_bytes, st));
         akv::PmLevel lv[akv::kMaxLevels];
         pm_bind(L.pmp, t->n_levels, (long long)dp.B * dp.H, ws + L.pm_zero, ws + L.pm_data, lv);
-        return dispatch_pm(t, L.pmp, dp, lv, 0, t->n_levels - 1, st);
+        return dispatch_pm(t, L.pmp, dp, lv, ws + L.pm_zero, L.pmp.zero_bytes, 0, t->n_levels - 1, st);
     };
     t->pm_last = L.pm;
     if (!host) {
@@ -1432,7 +1473,6 @@ atlaskv_status attend_impl(atlaskv_tree *t, const Ks &ks, const atlaskv_io *io, 
         add(kPhaseStageValues, 0, 0);
         add(kPhaseAttend, 0, 0);
         t->nphases_last = np;
-        if (L.pm) AKV_CUDA(cudaMemsetAsync(ws + L.pm_zero, 0, nc * L.pmp.zero_bytes, s));
         // the staging stream starts after everything already queued on the caller's stream
         AKV_CUDA(cudaEventRecord(t->cev[kMaxChunks * kChunkEvents], s));
         AKV_CUDA(cudaStreamWaitEvent(s1, t->cev[kMaxChunks * kChunkEvents], 0));
@@ -1451,7 +1491,9 @@ atlaskv_status attend_impl(atlaskv_tree *t, const Ks &ks, const atlaskv_io *io, 
                 AKV_STEP(tmark(c, 2 * k, st));
                 switch (ph.kind) {
                 case kPhaseDescend:
-                    if (L.pm) AKV_STEP(dispatch_pm(t, L.pmp, q.d, q.lv, ph.first, ph.last, s));
+                    if (L.pm)
+                        AKV_STEP(dispatch_pm(t, L.pmp, q.d, q.lv, ws + L.pm_zero + c * L.pmp.zero_bytes,
+                                             L.pmp.zero_bytes, ph.first, ph.last, s));
                     else AKV_STEP(dispatch_descend(t->d.dtype, D, q.d, L.desc.HT, L.desc.smem, ph.first, ph.last, s));
                     break;
                 case kPhaseStageKeys:
@@ -1627,7 +1669,10 @@ atlaskv_status atlaskv_attend_layers(int32_t n_layers, atlaskv_tree *const *tree
         AKV_STEP(dispatch_descend_layers(t0->d.dtype, D, db, pl.HT, pl.smem, dgrid, s));
         AKV_STEP(tm(1, s));
         AKV_STEP(tm(4, s));
-        for (int l = 0; l < n_layers; ++l) AKV_STEP(dispatch_attend(t0->d.dtype, D, calls[l].ap, s));
+        if (t0->d.dtype == ATLASKV_BF16 && D == akv::tc::kD)   // every layer's attention in one launch
+            AKV_STEP(launch_attend_tc_layers(calls, n_layers, akv::kAttnFused, s));
+        else
+            for (int l = 0; l < n_layers; ++l) AKV_STEP(dispatch_attend(t0->d.dtype, D, calls[l].ap, s));
         AKV_STEP(tm(5, s));
     }
 #undef AKV_STEP

@@ -726,6 +726,8 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
     attend_tc_kernel(const __grid_constant__ AttnParams p, int ctas_per_group, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v)
 {
+    griddep_launch();
+    griddep_wait();   // the kept lists (and everything else) of the previous grid are visible
     attend_tc_cta(p, blockIdx.x, ctas_per_group, &tm_k, &tm_v);
 }
 

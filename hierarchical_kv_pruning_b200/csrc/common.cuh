@@ -10,6 +10,14 @@ namespace akv {
 // Device status word values (sticky; first error wins).
 enum : int { kDevOk = 0, kDevBadChild = 1, kDevTimeout = 2 };
 
+// Programmatic dependent launch.  griddep_wait: wait until the grid this one
+// depends on (the previous kernel on the stream, when this one was launched
+// with programmatic stream serialization) has completed and its writes are
+// visible; a no-op otherwise.  griddep_launch: allow the next grid on the
+// stream to start launching (its CTAs then wait in griddep_wait).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void set_status(int *status, int code)
 {
     atomicCAS(status, kDevOk, code);

@@ -34,6 +34,8 @@
 
 #include <float.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "exact.cuh"
 
@@ -325,36 +327,49 @@ __device__ __noinline__ void token_sums(const DescendParams &p, const T *qb, lon
 // ==========================================================================
 
 // Ascending bitonic sort of the warp's 32 E values held in registers, lane l
-// holding elements l E .. l E + E - 1 (E a power of two): partners within a
-// lane are compared in place, the others exchanged by shuffles.
+// holding elements l E .. l E + E - 1 (E = 1, 2 or 4): partners within a lane
+// are compared in place, the others exchanged by shuffles.  The stage loops
+// stay rolled (small code: the selection runs beside many other warps).
+__device__ __forceinline__ void cmp_swap(uint64_t &a, uint64_t &b, bool asc)
+{
+    const uint64_t lo = a < b ? a : b, hi = a < b ? b : a;
+    a = asc ? lo : hi;
+    b = asc ? hi : lo;
+}
+
+template <int S, int E>
+__device__ __forceinline__ void lane_stage(uint64_t (&v)[E], int i0, int size)
+{
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if ((e & S) == 0) cmp_swap(v[e], v[e + S], ((i0 + e) & size) == 0);
+}
+
 template <int E>
 __device__ __forceinline__ void reg_bitonic(uint64_t (&v)[E])
 {
+    static_assert(E == 1 || E == 2 || E == 4 || E == 8, "E");
     const int lane = threadIdx.x & 31;
     constexpr int n = 32 * E;
-#pragma unroll
+#pragma unroll 1
     for (int size = 2; size <= n; size <<= 1) {
-#pragma unroll
+#pragma unroll 1
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            if (stride < E) {
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    if (e & stride) continue;   // e is the lower of the pair (e, e + stride)
-                    const int i = lane * E + e;
-                    const bool asc = (i & size) == 0;
-                    const uint64_t a = v[e], b = v[e + stride];
-                    if ((a > b) == asc) {
-                        v[e] = b;
-                        v[e + stride] = a;
-                    }
-                }
-            } else {
+            if (stride >= E) {
 #pragma unroll
                 for (int e = 0; e < E; ++e) {
                     const int i = lane * E + e;
                     const uint64_t o = __shfl_xor_sync(0xffffffffu, v[e], stride / E);
                     const bool lower = (i & stride) == 0, asc = (i & size) == 0;
                     v[e] = (lower == asc) ? (v[e] < o ? v[e] : o) : (v[e] > o ? v[e] : o);
+                }
+            } else if constexpr (E >= 2) {
+                const int i0 = lane * E;
+                if (stride == 1) {
+                    lane_stage<1, E>(v, i0, size);
+                } else if constexpr (E >= 4) {
+                    if (stride == 2) lane_stage<2, E>(v, i0, size);
+                    else if constexpr (E >= 8) lane_stage<4, E>(v, i0, size);
                 }
             }
         }
@@ -501,7 +516,8 @@ __device__ __forceinline__ void write_kept_reg(const DescendParams &p, const Lev
     __syncwarp();
 }
 
-__device__ void write_kept(const DescendParams &p, const LevelView &lv, int L, long long bh, uint64_t *kbuf, int K)
+__device__ __forceinline__ void write_kept(const DescendParams &p, const LevelView &lv, int L, long long bh,
+                                           uint64_t *kbuf, int K)
 {
     const int lane = threadIdx.x & 31;
     __syncwarp();
@@ -563,7 +579,8 @@ __device__ __forceinline__ void warp_pick_bin(const uint32_t *hist, int kk, int 
 // map); the bucket holding the k-th largest is then searched exactly: sorted
 // when it holds at most 64, else narrowed by MSB-first radix passes over the
 // order-preserving bit image.  hist: 256 bins; tmp: 64 uint64.
-__device__ float warp_kth_largest(const float *f, int n, int k, float mn, float mx, uint32_t *hist, uint64_t *tmp)
+__device__ __forceinline__ float warp_kth_largest(const float *f, int n, int k, float mn, float mx, uint32_t *hist,
+                                                  uint64_t *tmp)
 {
     const int lane = threadIdx.x & 31;
     if (mx == mn) return mx;   // all equal
@@ -718,6 +735,95 @@ struct ExactScratch {
     }
 };
 
+// Tier 2 of the refinement (see warp_refine): the listed candidates (at most
+// 32, all scores finite) in float64 with their own bounds.  Returns true when
+// that settles the selection (kbuf then holds K entries); otherwise the
+// candidates kept for sure are appended (nsel, r updated) and list / nlist
+// name the still-ambiguous ones (in sc.list2).
+template <typename T, int D>
+__device__ __forceinline__ bool refine_tier2(const DescendParams &p, const LevelView &lv, long long bh,
+                                             uint64_t *kbuf, int &nsel, int &r, const int *&list, int &nlist,
+                                             ExactScratch &sc)
+{
+    const int lane = threadIdx.x & 31;
+    const T *kbase = reinterpret_cast<const T *>(p.keys[lv.L]);
+    // lane d holds elements d, d + 32, ... of s64 and a64; every listed
+    // candidate's fp64 dot product is split over the lanes and summed by
+    // shuffles (binary64 in any order: the g64_D bound below holds), four
+    // candidates' rows in flight at a time; lane j keeps candidate j's.
+    constexpr int DL = D / 32;
+    const double *s64 = p.s64_ws + (size_t)bh * D;
+    const double *a64 = p.a64_ws + (size_t)bh * D;
+    double sv[DL], av[DL];
+#pragma unroll
+    for (int j = 0; j < DL; ++j) {
+        sv[j] = s64[lane + 32 * j];
+        av[j] = a64[lane + 32 * j];
+    }
+    const int my_pos = lane < nlist ? list[lane] : -1;
+    const long long my_row = my_pos >= 0 ? lv.row(my_pos) : 0;
+    double y = -INFINITY, e2 = 0.0;
+    const double g64d = (double)D * 0x1p-53 / (1.0 - (double)D * 0x1p-53);
+    const double g64n = (double)p.N * 0x1p-53 / (1.0 - (double)p.N * 0x1p-53);
+    for (int c0 = 0; c0 < nlist; c0 += 4) {
+        float x[4][DL];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const long long rr = __shfl_sync(0xffffffffu, my_row, min(c0 + u, nlist - 1));
+            const T *krow = kbase + (size_t)rr * D;
+#pragma unroll
+            for (int j = 0; j < DL; ++j) x[u][j] = elem_f32(krow[lane + 32 * j]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            double acc = 0.0, mag = 0.0;
+#pragma unroll
+            for (int j = 0; j < DL; ++j) {
+                acc = fma(sv[j], (double)x[u][j], acc);
+                mag = fma(av[j], fabs((double)x[u][j]), mag);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                mag += __shfl_xor_sync(0xffffffffu, mag, o);
+            }
+            if (lane == c0 + u && lane < nlist) {
+                y = acc;
+                e2 = (g64d * (1.0 + g64n) + g64n) * mag * (1.0 + 1e-6) + 0x1p-1000;
+            }
+        }
+    }
+    double E2 = e2;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) E2 = fmax(E2, __shfl_xor_sync(0xffffffffu, E2, o));
+    int rank = 0;
+    for (int j = 0; j < nlist; ++j) {
+        const double yj = __shfl_sync(0xffffffffu, y, j);
+        rank += (yj > y) || (yj == y && j < lane);
+    }
+    const int tl = __ffs(__ballot_sync(0xffffffffu, my_pos >= 0 && rank == r - 1)) - 1;
+    const double t2 = __shfl_sync(0xffffffffu, y, tl);
+    const double hi2 = __dadd_ru(t2, 2.0 * E2), lo2 = __dsub_rd(t2, 2.0 * E2);
+    const bool in2 = my_pos >= 0 && y > hi2;
+    const bool amb2 = my_pos >= 0 && !in2 && y >= lo2;
+    const unsigned min2 = __ballot_sync(0xffffffffu, in2);
+    const unsigned ma2 = __ballot_sync(0xffffffffu, amb2);
+    const int n_in2 = __popc(min2), nA2 = __popc(ma2);
+    const bool settle = nA2 == r - n_in2;
+    if (in2 || (settle && amb2)) {
+        const unsigned m = settle ? (min2 | ma2) : min2;
+        kbuf[nsel + __popc(m & lanemask_lt())] = ((uint64_t)(uint32_t)lv.id(my_pos) << 32) | (uint32_t)my_pos;
+    }
+    if (!settle && amb2) sc.list2[__popc(ma2 & lanemask_lt())] = my_pos;
+    __syncwarp();
+    if (settle) return true;
+    nsel += n_in2;
+    r -= n_in2;
+    nlist = nA2;
+    list = sc.list2;
+    return false;
+}
+
 // A selection tier 1 left open: nsel entries are kept in kbuf already and
 // r = K - nsel places remain among the nlist band candidates `list`.
 //   tier 2: when at most 32 are listed (and all scores were finite), each lane
@@ -747,62 +853,7 @@ __device__ __noinline__ void warp_refine(const DescendParams &p, const LevelView
     int32_t *best_id = sc.ids, *ch_id = sc.ids + RC, *tmp_id = sc.ids + 2 * RC;
     int32_t *best_pos = sc.poss, *ch_pos = sc.poss + RC, *tmp_pos = sc.poss + 2 * RC;
 
-    if (!bad && nlist <= 32) {
-        // ---- tier 2 ----
-        const double *s64 = p.s64_ws + (size_t)bh * D;
-        const double *a64 = p.a64_ws + (size_t)bh * D;
-        const int my_pos = lane < nlist ? list[lane] : -1;
-        double y = -INFINITY, e2 = 0.0;
-        if (my_pos >= 0) {
-            const T *krow = kbase + (size_t)lv.row(my_pos) * D;
-            uint4 w[D / EV];
-#pragma unroll
-            for (int v = 0; v < D / EV; ++v) w[v] = ldg16(krow + v * EV);
-            double acc = 0.0, mag = 0.0;
-#pragma unroll
-            for (int v = 0; v < D / EV; ++v) {
-                float x[EV];
-                Vec16<T>::unpack(w[v], x);
-#pragma unroll
-                for (int q = 0; q < EV; ++q) {
-                    acc = fma(s64[v * EV + q], (double)x[q], acc);
-                    mag = fma(a64[v * EV + q], fabs((double)x[q]), mag);
-                }
-            }
-            const double g64d = (double)D * 0x1p-53 / (1.0 - (double)D * 0x1p-53);
-            const double g64n = (double)p.N * 0x1p-53 / (1.0 - (double)p.N * 0x1p-53);
-            y = acc;
-            e2 = (g64d * (1.0 + g64n) + g64n) * mag * (1.0 + 1e-6) + 0x1p-1000;
-        }
-        double E2 = e2;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) E2 = fmax(E2, __shfl_xor_sync(0xffffffffu, E2, o));
-        int rank = 0;
-        for (int j = 0; j < nlist; ++j) {
-            const double yj = __shfl_sync(0xffffffffu, y, j);
-            rank += (yj > y) || (yj == y && j < lane);
-        }
-        const int tl = __ffs(__ballot_sync(0xffffffffu, my_pos >= 0 && rank == r - 1)) - 1;
-        const double t2 = __shfl_sync(0xffffffffu, y, tl);
-        const double hi2 = __dadd_ru(t2, 2.0 * E2), lo2 = __dsub_rd(t2, 2.0 * E2);
-        const bool in2 = my_pos >= 0 && y > hi2;
-        const bool amb2 = my_pos >= 0 && !in2 && y >= lo2;
-        const unsigned min2 = __ballot_sync(0xffffffffu, in2);
-        const unsigned ma2 = __ballot_sync(0xffffffffu, amb2);
-        const int n_in2 = __popc(min2), nA2 = __popc(ma2);
-        const bool settle = nA2 == r - n_in2;
-        if (in2 || (settle && amb2)) {
-            const unsigned m = settle ? (min2 | ma2) : min2;
-            kbuf[nsel + __popc(m & lanemask_lt())] = ((uint64_t)(uint32_t)lv.id(my_pos) << 32) | (uint32_t)my_pos;
-        }
-        if (!settle && amb2) sc.list2[__popc(ma2 & lanemask_lt())] = my_pos;
-        __syncwarp();
-        if (settle) return;
-        nsel += n_in2;
-        r -= n_in2;
-        nlist = nA2;
-        list = sc.list2;
-    }
+    if (!bad && nlist <= 32 && refine_tier2<T, D>(p, lv, bh, kbuf, nsel, r, list, nlist, sc)) return;
     // ---- tier 3 ----
     int chosen = 0;
     bool have_pivot = false;
@@ -872,11 +923,15 @@ __device__ __noinline__ void warp_refine(const DescendParams &p, const LevelView
 // Top-K of traversal bh at level L by one warp, from its fp32 scores f[0..C)
 // (tier 1): the scores and their rigorous bound E settle every candidate
 // outside the band [t - 2E, t + 2E] around the K-th largest score t; when the
-// band holds more candidates than places left, warp_refine decides them.
-template <typename T, int D>
-__device__ __noinline__ void warp_select(const DescendParams &p, int L, long long bh, const int32_t *cpre,
-                                         const int32_t *prev_sh, uint32_t *hist, uint64_t *tmp, uint64_t *kbuf,
-                                         float *f, ExactScratch &xs)
+// band holds more candidates than places left, warp_refine decides them --
+// here, or (kDefer) in a later kernel: the band list goes to the traversal's
+// score row, the entries kept so far to its kept-entry area behind the scores,
+// and (bh, kept so far, listed, bad) to the queue; then it returns false.
+template <typename T, int D, bool kDefer = false>
+__device__ __forceinline__ bool warp_select(const DescendParams &p, int L, long long bh, const int32_t *cpre,
+                                            const int32_t *prev_sh, uint32_t *hist, uint64_t *tmp, uint64_t *kbuf,
+                                            float *f, ExactScratch &xs, int4 *queue = nullptr,
+                                            int *qcount = nullptr)
 {
     const int lane = threadIdx.x & 31;
     const LevelView lv = level_view(p, L, bh, cpre, prev_sh);
@@ -913,6 +968,13 @@ __device__ __noinline__ void warp_select(const DescendParams &p, int L, long lon
                 }
         };
         int v = lane;
+        for (; v + 224 < nv; v += 256) {
+            float4 t[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) t[u] = __ldcg(src + v + 32 * u);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) take(t[u], v + 32 * u);
+        }
         for (; v + 96 < nv; v += 128) {
             float4 t[4];
 #pragma unroll
@@ -930,7 +992,7 @@ __device__ __noinline__ void warp_select(const DescendParams &p, int L, long lon
         resolve_ids(C);
         __syncwarp();
         write_kept(p, lv, L, bh, kbuf, K);
-        return;
+        return true;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -948,21 +1010,43 @@ __device__ __noinline__ void warp_select(const DescendParams &p, int L, long lon
     // class of a candidate: 1 kept for sure, 2 ambiguous, 0 dropped.  The band
     // list is compacted in place over the scores: a list entry is stored at an
     // index below every score not yet read.
+    // Four scores per lane per step; the step's reads all precede its writes
+    // (the counts pass through the warp scan), and a step writes list entries
+    // only below 4 (step + 1) 32.
     int *list = reinterpret_cast<int *>(f);
     int n_in = 0, nA = 0;
-    for (int c0 = 0; c0 < C; c0 += 32) {
-        const int c = c0 + lane;
-        int k = 0;
-        if (c < C) {
-            const float fv = f[c];
-            k = bad2 ? 2 : (fv > hi32 ? 1 : (fv >= lo32 ? 2 : 0));
+    {
+        const float4 *f4 = reinterpret_cast<const float4 *>(f);
+        const int nv = (C + 3) >> 2;
+        for (int b4 = 0; b4 < nv; b4 += 32) {
+            const int v4 = b4 + lane;
+            float e[4] = {0.f, 0.f, 0.f, 0.f};
+            if (v4 < nv) {
+                const float4 x = f4[v4];
+                e[0] = x.x;
+                e[1] = x.y;
+                e[2] = x.z;
+                e[3] = x.w;
+            }
+            int k[4], c1 = 0, c2 = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const bool in = v4 < nv && 4 * v4 + q < C;
+                k[q] = !in ? 0 : bad2 ? 2 : (e[q] > hi32 ? 1 : (e[q] >= lo32 ? 2 : 0));
+                c1 += k[q] == 1;
+                c2 += k[q] == 2;
+            }
+            int tot;
+            const int pre = warp_excl_scan(c1 | (c2 << 16), tot);
+            int o1 = n_in + (pre & 0xffff), o2 = nA + (pre >> 16);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (k[q] == 1) kbuf[o1++] = (uint32_t)(4 * v4 + q);
+                if (k[q] == 2) list[o2++] = 4 * v4 + q;
+            }
+            n_in += tot & 0xffff;
+            nA += tot >> 16;
         }
-        const unsigned mi = __ballot_sync(0xffffffffu, k == 1);
-        const unsigned ma = __ballot_sync(0xffffffffu, k == 2);
-        if (k == 1) kbuf[n_in + __popc(mi & lanemask_lt())] = (uint32_t)c;
-        if (k == 2) list[nA + __popc(ma & lanemask_lt())] = c;
-        n_in += __popc(mi);
-        nA += __popc(ma);
     }
     __syncwarp();
     const int r = K - n_in;
@@ -974,16 +1058,243 @@ __device__ __noinline__ void warp_select(const DescendParams &p, int L, long lon
         __syncwarp();
         resolve_ids(K);
         write_kept(p, lv, L, bh, kbuf, K);
-        return;
+        return true;
     }
     if (p.stats && lane == 0) {
         atomicAdd(p.stats + L * 4 + 1, 1ull);
         atomicAdd(p.stats + L * 4 + 2, (unsigned long long)nA);
     }
     resolve_ids(n_in);
-    warp_refine<T, D>(p, lv, L, bh, kbuf, n_in, list, nA, bad2, xs);
+    if constexpr (kDefer) {
+        int *glist = reinterpret_cast<int *>(p.f_ws + (size_t)bh * p.fstride);
+        uint64_t *gk = reinterpret_cast<uint64_t *>(p.f_ws + (size_t)bh * p.fstride + p.cap);
+        for (int i = lane; i < nA; i += 32) glist[i] = list[i];
+        if (gk != kbuf)
+            for (int i = lane; i < n_in; i += 32) gk[i] = kbuf[i];
+        __syncwarp();
+        if (lane == 0) queue[atomicAdd(qcount, 1)] = make_int4((int)bh, n_in, nA, bad2 ? 1 : 0);
+        (void)xs;
+        return false;
+    } else {
+        warp_refine<T, D>(p, lv, L, bh, kbuf, n_in, list, nA, bad2, xs);
+        __syncwarp();
+        write_kept(p, lv, L, bh, kbuf, K);
+        return true;
+    }
+}
+
+// The same as a call: the fused kernel keeps the selection out of line (its
+// registers go to the scoring loop).
+template <typename T, int D>
+__device__ __noinline__ void warp_select_call(const DescendParams &p, int L, long long bh, const int32_t *cpre,
+                                              const int32_t *prev_sh, uint32_t *hist, uint64_t *tmp, uint64_t *kbuf,
+                                              float *f, ExactScratch &xs)
+{
+    warp_select<T, D>(p, L, bh, cpre, prev_sh, hist, tmp, kbuf, f, xs);
+}
+
+// The same with the selection kept out of line and deferred refinement: the
+// parent-major path's rare fallback.
+template <typename T, int D>
+__device__ __noinline__ bool warp_select_defer_call(const DescendParams &p, int L, long long bh, const int32_t *cpre,
+                                                    const int32_t *prev_sh, uint32_t *hist, uint64_t *tmp,
+                                                    uint64_t *kbuf, float *f, ExactScratch &xs, int4 *queue,
+                                                    int *qcount)
+{
+    return warp_select<T, D, true>(p, L, bh, cpre, prev_sh, hist, tmp, kbuf, f, xs, queue, qcount);
+}
+
+// Tier 1 in one pass over the scores (read from the traversal's workspace
+// row), for the parent-major path:
+//   1. a sample of 128 scores (all of them when C <= 128), sorted, gives t0,
+//      the j-th largest sample value with j chosen so that about 1.5 K + 3
+//      sample-strides of scores lie above it: t0 <= t (the K-th largest score)
+//      unless fewer than K scores are >= t0, which the pass counts;
+//   2. the pass collects every candidate with f >= fl_down(t0 - 2E) and counts
+//      those >= t0;
+//   3. with at least K counted (so t >= t0), every candidate of the band
+//      [t - 2E, t + 2E] and above was collected: t is the K-th largest of the
+//      collected, which are sorted; the sorted prefix above t + 2E is kept for
+//      sure, the next ones down to t - 2E are the band.
+// Non-finite scores, too many collected (more than kCollectCap) or too few
+// counted fall back to warp_select on the same row.  The certified band and
+// the refinement are those of warp_select, so the kept sets are the same.
+constexpr int kCollectCap = 512;
+
+template <typename T, int D>
+__device__ __forceinline__ bool warp_select_pm(const DescendParams &p, int L, long long bh, const int32_t *cpre,
+                                               const int32_t *prev_sh, uint32_t *hist, uint64_t *tmp, uint64_t *kbuf,
+                                               uint64_t *col, ExactScratch &xs, int4 *queue, int *qcount)
+{
+    const int lane = threadIdx.x & 31;
+    const LevelView lv = level_view(p, L, bh, cpre, prev_sh);
+    const int C = lv.C, K = p.K[L];
+    float *f = p.f_ws + (size_t)bh * p.fstride;
+    auto fallback = [&]() {
+        return warp_select_defer_call<T, D>(p, L, bh, cpre, prev_sh, hist, tmp, kbuf, f, xs, queue, qcount);
+    };
+    auto resolve_ids = [&](int n) {
+        for (int i = lane; i < n; i += 32) {
+            const int c = (int)(uint32_t)kbuf[i];
+            kbuf[i] = ((uint64_t)(uint32_t)lv.id(c) << 32) | (uint32_t)c;
+        }
+        __syncwarp();
+    };
+    if (K >= C) return fallback();
+    const float anorm = p.anorm_ws[bh], knorm = p.norm_bound[L * p.H_kv + lv.hkv];
+    const double E = p.cprime * (double)anorm * (double)knorm * (1.0 + 1e-6) + D * 0x1p-148;
+    if (!isfinite(E)) return fallback();
+
+    // ---- 1. the sample threshold (all scores when C <= 128) ----
+    const bool all = C <= 128;
+    uint64_t sv[4];
+    int bad = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int i = lane * 4 + e;
+        const int idx = all ? i : (int)(((long long)i * C) >> 7);
+        const float v = (!all || i < C) ? __ldcg(f + idx) : -INFINITY;
+        bad |= (!all || i < C) && !isfinite(v);
+        sv[e] = ((uint64_t)(~float_key(v)) << 32) | (uint32_t)idx;   // ascending keys: descending values
+    }
+    if (__any_sync(0xffffffffu, bad)) return fallback();
+    reg_bitonic<4>(sv);
+    int ncol;
+    if (all) {   // every score is in the sorted sample: it is the collected set
+#pragma unroll
+        for (int e = 0; e < 4; ++e) col[lane * 4 + e] = sv[e];
+        ncol = C;
+    } else {
+        const int j = (3 * K * 128 + 2 * C - 1) / (2 * C) + 3;
+        if (j > 127) return fallback();
+        const uint64_t kj0 = __shfl_sync(0xffffffffu, sv[0], j >> 2), kj1 = __shfl_sync(0xffffffffu, sv[1], j >> 2);
+        const uint64_t kj2 = __shfl_sync(0xffffffffu, sv[2], j >> 2), kj3 = __shfl_sync(0xffffffffu, sv[3], j >> 2);
+        const uint64_t kj = (j & 3) == 0 ? kj0 : (j & 3) == 1 ? kj1 : (j & 3) == 2 ? kj2 : kj3;
+        const float t0 = key_float(~(uint32_t)(kj >> 32));
+        const float c_lo = __double2float_rd(__dsub_rd((double)t0, 2.0 * E));
+
+        // ---- 2. one pass: collect, count, check (four 16-byte loads in flight per lane) ----
+        int cnt = 0;
+        ncol = 0;
+        const float4 *f4 = reinterpret_cast<const float4 *>(f);
+        const int nv = (C + 3) >> 2;
+        for (int b4 = 0; b4 < nv; b4 += 128) {
+            float4 x[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int v4 = b4 + 32 * u + lane;
+                x[u] = v4 < nv ? __ldcg(f4 + v4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int v4 = b4 + 32 * u + lane;
+                const float e[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+                bool take[4];
+                int c1 = 0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const bool in = v4 < nv && 4 * v4 + q < C;
+                    bad |= in && !isfinite(e[q]);
+                    take[q] = in && e[q] >= c_lo;
+                    cnt += in && e[q] >= t0;
+                    c1 += take[q];
+                }
+                int tot;
+                int off = ncol + warp_excl_scan(c1, tot);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (take[q]) {
+                        if (off < kCollectCap)
+                            col[off] = ((uint64_t)(~float_key(e[q])) << 32) | (uint32_t)(4 * v4 + q);
+                        ++off;
+                    }
+                ncol += tot;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        bad = __any_sync(0xffffffffu, bad);
+        if (bad || !isfinite(t0) || cnt < K || ncol > kCollectCap) return fallback();
+        __syncwarp();
+
+        // ---- 3. the collected, sorted ----
+        auto sort_reg = [&](auto tag) {
+            constexpr int EE = decltype(tag)::value;
+            uint64_t v[EE];
+#pragma unroll
+            for (int e = 0; e < EE; ++e) v[e] = lane * EE + e < ncol ? col[lane * EE + e] : ~0ull;
+            reg_bitonic<EE>(v);
+            __syncwarp();
+#pragma unroll
+            for (int e = 0; e < EE; ++e) col[lane * EE + e] = v[e];
+        };
+        if (ncol <= 64) {
+            sort_reg(std::integral_constant<int, 2>());
+        } else if (ncol <= 128) {
+            sort_reg(std::integral_constant<int, 4>());
+        } else if (ncol <= 256) {
+            sort_reg(std::integral_constant<int, 8>());
+        } else {
+            int n2 = 512;
+            for (int i = ncol + lane; i < n2; i += 32) col[i] = ~0ull;
+            __syncwarp();
+            warp_sort_u64(col, n2);
+        }
+    }
     __syncwarp();
-    write_kept(p, lv, L, bh, kbuf, K);
+    // the K-th largest; the sure prefix above t + 2E and the band down to t - 2E
+    const float t = key_float(~(uint32_t)(col[K - 1] >> 32));
+    const float hi32 = __double2float_ru(__dadd_ru((double)t, 2.0 * E));
+    const float lo32 = __double2float_rd(__dsub_rd((double)t, 2.0 * E));
+    int n_in = 0, nA = 0;
+    for (int i0 = 0; i0 < ncol; i0 += 32) {
+        const int i = i0 + lane;
+        const float v = i < ncol ? key_float(~(uint32_t)(col[i] >> 32)) : -INFINITY;
+        n_in += __popc(__ballot_sync(0xffffffffu, i < ncol && v > hi32));
+        nA += __popc(__ballot_sync(0xffffffffu, i < ncol && v <= hi32 && v >= lo32));
+    }
+    if (p.stats && lane == 0) atomicAdd(p.stats + L * 4, 1ull);
+    const int r = K - n_in;
+    for (int i = lane; i < n_in; i += 32) kbuf[i] = (uint32_t)col[i];
+    if (nA == r) {   // every band candidate is kept
+        for (int i = lane; i < nA; i += 32) kbuf[n_in + i] = (uint32_t)col[n_in + i];
+        __syncwarp();
+        resolve_ids(K);
+        write_kept(p, lv, L, bh, kbuf, K);
+        return true;
+    }
+    if (p.stats && lane == 0) {
+        atomicAdd(p.stats + L * 4 + 1, 1ull);
+        atomicAdd(p.stats + L * 4 + 2, (unsigned long long)nA);
+    }
+    resolve_ids(n_in);
+    // tier 2 here when the band is short (the band's positions in hist)
+    int nsel = n_in, rr = r, nl = nA;
+    const int *lst = reinterpret_cast<const int *>(hist);
+    if (nA <= 32) {
+        if (lane < nA) hist[lane] = (uint32_t)col[n_in + lane];
+        __syncwarp();
+        if (refine_tier2<T, D>(p, lv, bh, kbuf, nsel, rr, lst, nl, xs)) {
+            write_kept(p, lv, L, bh, kbuf, K);
+            return true;
+        }
+    }
+    // hand over to the refinement kernel: the open candidates' positions over
+    // the scores (consumed), the entries kept so far behind them, a queue entry
+    int *glist = reinterpret_cast<int *>(f);
+    uint64_t *gk = reinterpret_cast<uint64_t *>(f + p.cap);
+    __syncwarp();
+    if (nA <= 32) {
+        for (int i = lane; i < nl; i += 32) glist[i] = lst[i];
+    } else {
+        for (int i = lane; i < nA; i += 32) glist[i] = (int)(uint32_t)col[n_in + i];
+    }
+    if (gk != kbuf)
+        for (int i = lane; i < nsel; i += 32) gk[i] = kbuf[i];
+    __syncwarp();
+    if (lane == 0) queue[atomicAdd(qcount, 1)] = make_int4((int)bh, nsel, nl, 0);
+    (void)rr;
+    return false;
 }
 
 // ==========================================================================
@@ -1317,7 +1628,7 @@ __device__ __forceinline__ void descend_cta(const DescendParams &p, const unsign
                                                  : reinterpret_cast<uint64_t *>(p.f_ws + (size_t)(bh0 + g) * fstride +
                                                                                 p.cap);
             float *fs = reinterpret_cast<float *>(ws + warp_sel_bytes(p.kcap, 0));
-            warp_select<T, D>(p, L, bh0 + g, csr ? cpre + g * (Kp + 1) : nullptr, L == 0 ? nullptr : lists + g * Kp,
+            warp_select_call<T, D>(p, L, bh0 + g, csr ? cpre + g * (Kp + 1) : nullptr, L == 0 ? nullptr : lists + g * Kp,
                               hist, tmp, kbuf, fs, xs);
         }
     }

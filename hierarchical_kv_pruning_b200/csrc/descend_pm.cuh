@@ -54,6 +54,8 @@ struct PmLevel {
     int32_t *tflag;               // [n_tiles] 0, 1 aggregate ready, 2 prefix ready (zero at the start)
     int32_t *ctr;                 // [4] tile ticket, number of work items (zero at the start)
     int32_t *cpre;                // CSR level: [BH][Kp + 1] first candidate of each kept parent, else null
+    int4 *queue;                  // [BH] traversals of level L whose selection waits for refinement
+    int32_t *qcount;              // queue length (zero at the start)
     long long NK;
     int E, max_items, n_tiles;
 };
@@ -79,11 +81,18 @@ __device__ __forceinline__ void st_release(int32_t *p, int v)
 }
 
 // ---------------------------------------------------------------------------
-// Token sums: one CTA per (query, KV head, chunk of GC heads).
+// Token sums: one CTA per (query, KV head, chunk of GC heads).  The grid also
+// clears the call's zero-initialised inversion region (zero, zwords 16-byte
+// words) once the previous grid on the stream is done.
 template <typename T, int D>
-__global__ void __launch_bounds__(kDescThreads) token_sums_kernel(const __grid_constant__ DescendParams p, int GC)
+__global__ void __launch_bounds__(kDescThreads)
+    token_sums_kernel(const __grid_constant__ DescendParams p, int GC, uint4 *zero, long long zwords)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
+    griddep_launch();
+    griddep_wait();
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < zwords; i += (long long)gridDim.x * blockDim.x)
+        zero[i] = make_uint4(0u, 0u, 0u, 0u);
     const int hchunks = p.G / GC;
     const int hc = (int)(blockIdx.x % hchunks);
     const int grp = (int)(blockIdx.x / hchunks);
@@ -103,212 +112,272 @@ __host__ __device__ constexpr size_t token_sums_smem(int GC, int D, int esz)
 }
 
 // ---------------------------------------------------------------------------
-// Scoring: work items in turn (blockIdx.x, + gridDim.x, ...).  A warp serves
-// HT traversals of the item and holds their token-sum slices in registers; a
-// key row spans LPG lanes (one 16-byte vector each) and a lane group takes R
-// = LPG / HT rows at a time, reducing its R x HT partial dot products by
-// recursive halving (as in the fused kernel).  The hgn = ceil(ne / HT) head
-// groups of an item share the row stream; 4 / hgn streams split the rows.
-template <typename T, int D, int HT>
-__global__ void __launch_bounds__(kPmThreads, 4)
-    pm_score_kernel(const __grid_constant__ DescendParams p0, const __grid_constant__ PmLevel pl, int L, int EC)
-{
-    constexpr int EV = Vec16<T>::E;
-    constexpr int LPG = D / EV;
-    constexpr int GPW = 32 / LPG;
-    constexpr int R = LPG / HT;
-    static_assert(LPG >= 8 && LPG <= 32 && R >= 1 && R * HT == LPG, "one score per lane");
-    constexpr int RCH = GPW * R;
-    constexpr int ROWB = D * (int)sizeof(T);
-    static_assert(R <= 4 && RCH * ROWB <= kChunkBytes, "a chunk fits its ring stage");
-    static_assert(kPmWarps * HT <= kPmMaxEC, "entries per item");
+// Scoring: a small GEMM per work item.  Each warp takes items on its own
+// (global warp gw: items gw, gw + all warps, ...; no CTA barrier), so an SM
+// keeps many items in flight.  An item's child rows are taken kPmRP = 128 at
+// a time (a pass); lane l owns rows l, l + 32, l + 64, l + 96 of the pass and
+// holds a 4 x kPmEC register tile of partial scores (rows x traversals).  The
+// contraction over D streams through two shared-memory stages of the warp:
+// per stage a 64-byte slice of every row of the pass (cp.async, 16-byte
+// pieces; piece c of row r at c ^ ((r >> 1) & 3), so a quarter-warp's eight
+// rows sit in distinct banks) and the same slice of the item's token sums
+// (read as broadcasts).  The next stage loads while this one is multiplied;
+// the next item's table entry and traversals are loaded one item ahead.
+// Scores go to the traversals' candidate slots, consecutive lanes to
+// consecutive slots.  Products in fp32 pairs; the fp32 sum of D products, in
+// whatever order, stays within the g_D bound of the filter.
+constexpr int kPmEC = 8;        // traversals per work item
+constexpr int kPmRP = 128;      // rows per pass (4 per lane)
+constexpr int kPmSlice = 64;    // bytes of a row per stage
 
+__host__ __device__ constexpr size_t pm_stage_bytes(int esz)
+{
+    return (size_t)kPmRP * kPmSlice + (size_t)kPmEC * (kPmSlice / esz) * 4;
+}
+__host__ __device__ constexpr size_t pm_score_smem(int D, int esz)
+{
+    return (size_t)kPmWarps * 2 * pm_stage_bytes(esz) + 0 * D;
+}
+
+// One item as a warp sees it: every lane holds the item's fields and, lane
+// j < ne, traversal j's row index and first candidate slot.
+struct PmItem {
+    int hkv, par, ne, n_c;
+    long long base;   // CSR: the first child entry; slot: the pool row of child 0
+    long long bh;     // this lane's traversal
+    int c0;           // its first candidate slot
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kPmThreads, 3)
+    pm_score_kernel(const __grid_constant__ DescendParams p0, const __grid_constant__ PmLevel pl, int L)
+{
+    constexpr int ESZ = (int)sizeof(T);
+    constexpr int EV = Vec16<T>::E;             // elements per 16-byte piece
+    constexpr int KE = kPmSlice / ESZ;          // elements of a row per stage
+    constexpr int NKC = D / KE;                 // stages per pass
+    constexpr int PPR = kPmSlice / 16;          // pieces per row slice (4)
+    constexpr int EC = kPmEC, R = kPmRP / 32;
+    constexpr int SB = (int)pm_stage_bytes(ESZ);
+    static_assert(NKC >= 2 && PPR == 4 && R == 4, "layout");
+
+    extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ DescendParams p;
-    __shared__ __align__(16) uint8_t ring_all[kPmWarps * kRingStages * kChunkBytes];
-    __shared__ int32_t trow[kPmPassRows];
-    __shared__ long long ent_bh[kPmMaxEC];
-    __shared__ int ent_c0[kPmMaxEC];
-    __shared__ long long item_base;
-    __shared__ int item_i[5];
+    griddep_launch();
     copy_params(p, p0);
-    __syncthreads();
+    griddep_wait();
+    __syncthreads();   // the only CTA barrier: the warps are independent from here on
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int lg = lane / LPG, sub = lane % LPG;
-    const int k_mine = sub / HT, h_mine = sub - (sub / HT) * HT;
+    uint8_t *wsm = smem_raw + (size_t)warp * 2 * SB;
+    const uint32_t wsm_s = (uint32_t)__cvta_generic_to_shared(wsm);
+
     const int BG = p.B * p.G;
     const int Kp = L == 0 ? 1 : p.K[L - 1];
     const int fo = p.fanout[L];
     const long long prow = L == 0 ? 1 : p.rows[L - 1], rows = p.rows[L];
     const T *kbase = reinterpret_cast<const T *>(p.keys[L]);
+    const float *s_ws = p.s_ws;
+    float *f_ws = p.f_ws;
+    const int fstride = p.fstride;
     const int32_t *coff = L >= 1 ? p.coff[L - 1] : nullptr;
     const int32_t *cid = L >= 1 ? p.cid[L - 1] : nullptr;
     const int32_t *tab = L >= 1 ? p.child[L - 1] : nullptr;
     const int32_t *slot = L >= 1 ? p.slot[L] : nullptr;
     const int per_hkv = (BG + EC - 1) / EC;
     const int n_items = L == 0 ? p.H_kv * per_hkv : min(pl.ctr[1], pl.max_items);
+    const int gw = blockIdx.x * kPmWarps + warp, nw = gridDim.x * kPmWarps;
+    if (gw >= n_items) return;
 
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        __syncthreads();   // the previous item's entries, row table and rings are free
-        if (threadIdx.x == 0) {
-            int hkv, par = 0, e0, ne, n_c;
-            long long base = 0;   // CSR: the first child entry; slot: the pool row of child 0
-            if (L == 0) {
-                hkv = item / per_hkv;
-                e0 = (item - hkv * per_hkv) * EC;
-                ne = min(EC, BG - e0);
-                n_c = (int)rows;
-            } else {
-                const int4 it = pl.ctab[item];
-                hkv = (int)(it.x / prow);
-                par = (int)(it.x - (long long)hkv * prow);
-                e0 = it.y;
-                ne = min(it.z, EC);
-                if (coff) {
-                    const int32_t *off_h = coff + (size_t)hkv * (prow + 1);
-                    base = off_h[par];
-                    n_c = off_h[par + 1] - (int)base;
-                } else {
-                    n_c = fo;
-                    if (slot) base = (long long)slot[pl.list[e0]] * fo;   // any copy of the block will do
-                }
-            }
-            item_i[0] = hkv;
-            item_i[1] = par;
-            item_i[2] = e0;
-            item_i[3] = ne;
-            item_i[4] = n_c;
-            item_base = base;
-        }
-        __syncthreads();
-        const int hkv = item_i[0], par = item_i[1], e0 = item_i[2], ne = item_i[3], n_c = item_i[4];
-        const long long base = item_base;
-        if ((int)threadIdx.x < ne) {
-            long long bh;
-            int c0;
-            if (L == 0) {
-                const int i = e0 + threadIdx.x;
-                const int b = i / p.G;
-                bh = (long long)b * p.H + (long long)hkv * p.G + (i - b * p.G);
-                c0 = 0;
-            } else {
-                const int e = pl.list[e0 + threadIdx.x];
-                bh = e / Kp;
-                const int k = e - (int)bh * Kp;
-                c0 = pl.cpre ? pl.cpre[bh * (Kp + 1) + k] : k * fo;
-            }
-            ent_bh[threadIdx.x] = bh;
-            ent_c0[threadIdx.x] = c0;
-        }
-        __syncthreads();
-
-        const int hgn = (ne + HT - 1) / HT;
-        const int streams = kPmWarps / hgn;
-        const bool computes = warp < streams * hgn;
-        const int hg = warp % hgn, rs = warp / hgn;
-        const int g_mine = hg * HT + h_mine;
-        const bool stores = computes && g_mine < ne;
-
-        // this lane's slice of the head group's token sums, as packed pairs
-        uint64_t sreg[HT][EV / 2];
-#pragma unroll
-        for (int h = 0; h < HT; ++h) {
-            const int g = hg * HT + h;
-            const bool ok = computes && g < ne;
-            const float *sp = p.s_ws + (size_t)(ok ? ent_bh[g] : 0) * D + sub * EV;
-#pragma unroll
-            for (int e = 0; e < EV; e += 4) {
-                float4 t4 = *reinterpret_cast<const float4 *>(sp + e);
-                if (!ok) t4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                sreg[h][e / 2] = pack2(t4.x, t4.y);
-                sreg[h][e / 2 + 1] = pack2(t4.z, t4.w);
-            }
-        }
-        float *f_mine = p.f_ws + (size_t)(stores ? ent_bh[g_mine] : 0) * p.fstride + (stores ? ent_c0[g_mine] : 0);
-        uint8_t *ring = ring_all + (size_t)(rs < kPmWarps ? rs : 0) * kRingStages * kChunkBytes;
-        const int tg = (int)threadIdx.x - rs * hgn * 32;
-        auto stream_sync = [&]() {
-            if (hgn == 1) __syncwarp();
-            else asm volatile("bar.sync %0, %1;" ::"r"(1 + rs), "r"(hgn * 32) : "memory");
-        };
-        // key row of child j of the item's parent
-        auto row_of = [&](int j) -> long long {
-            if (L == 0) return (long long)hkv * rows + j;
-            if (slot) return base + j;
-            long long id;
+    auto load_item = [&](int item) {
+        PmItem m;
+        if (L == 0) {
+            m.hkv = item / per_hkv;
+            const int e0 = (item - m.hkv * per_hkv) * EC;
+            m.par = 0;
+            m.ne = min(EC, BG - e0);
+            m.n_c = (int)rows;
+            m.base = 0;
+            const int i = e0 + (lane < m.ne ? lane : 0);
+            const int b = i / p.G;
+            m.bh = (long long)b * p.H + (long long)m.hkv * p.G + (i - b * p.G);
+            m.c0 = 0;
+        } else {
+            const int4 it = pl.ctab[item];
+            m.hkv = (int)(it.x / prow);
+            m.par = (int)(it.x - (long long)m.hkv * prow);
+            m.ne = min(it.z, EC);
+            const int e = pl.list[it.y + (lane < m.ne ? lane : 0)];
+            m.bh = e / Kp;
+            const int k = e - (int)m.bh * Kp;
+            m.c0 = pl.cpre ? pl.cpre[m.bh * (Kp + 1) + k] : k * fo;
             if (coff) {
-                const long long e = base + j;
-                id = cid ? (long long)cid[(size_t)hkv * rows + e] : e;
+                const int32_t *off_h = coff + (size_t)m.hkv * (prow + 1);
+                m.base = off_h[m.par];
+                m.n_c = off_h[m.par + 1] - (int)m.base;
             } else {
-                id = tab ? (long long)tab[((size_t)hkv * prow + par) * fo + j] : (long long)par * fo + j;
+                m.n_c = fo;
+                // any staged copy of the block will do: the first traversal's
+                m.base = slot ? (long long)__shfl_sync(0xffffffffu, slot[e], 0) * fo : 0;
             }
-            if (id < 0 || id >= rows) {
-                set_status(p.status, kDevBadChild);
-                id = 0;
-            }
-            return (long long)hkv * rows + id;
-        };
+        }
+        return m;
+    };
+    // key row of child j of item m
+    auto row_of = [&](const PmItem &m, int j) -> int {
+        if (L == 0) return (int)((long long)m.hkv * rows + j);
+        if (slot) return (int)(m.base + j);
+        long long id;
+        if (coff) {
+            const long long e = m.base + j;
+            id = cid ? (long long)cid[(size_t)m.hkv * rows + e] : e;
+        } else {
+            id = tab ? (long long)tab[((size_t)m.hkv * prow + m.par) * fo + j] : (long long)m.par * fo + j;
+        }
+        if (id < 0 || id >= rows) {
+            set_status(p.status, kDevBadChild);
+            id = 0;
+        }
+        return (int)((long long)m.hkv * rows + id);
+    };
+    // stage: slice kc of rows [q0, q0 + 128) of item m (row ids rid[j] of
+    // rows q0 + lane + 32 j) and of its token sums, into buffer b
+    auto issue = [&](const PmItem &m, int q0, int kc, const int (&rid)[R], int b) {
+        const uint32_t dst = wsm_s + (uint32_t)(b * SB);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {   // 512 pieces: row (lane >> 2) + 8 i, piece lane & 3
+            const int row = (lane >> 2) + 8 * i, pc = lane & 3;
+            const int rr = __shfl_sync(0xffffffffu, rid[i >> 2], row & 31);
+            const bool ok = q0 + row < m.n_c;
+            const T *src = kbase + (size_t)(ok ? rr : 0) * D + kc * KE + pc * EV;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(
+                             dst + (uint32_t)(row * kPmSlice + ((pc ^ ((row >> 1) & 3)) << 4))),
+                         "l"(src), "r"(ok ? 16 : 0));
+        }
+        constexpr int SP = KE / 4;   // 16-byte pieces of a traversal's slice
+        const uint32_t sdst = dst + kPmRP * kPmSlice;
+#pragma unroll
+        for (int i = 0; i < (EC * SP + 31) / 32; ++i) {
+            const int q = lane + 32 * i;
+            const int e = min(q / SP, m.ne - 1), v = q - (q / SP) * SP;
+            const long long bhe = __shfl_sync(0xffffffffu, m.bh, e);
+            if (q < m.ne * SP)
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sdst + (uint32_t)(e * KE + v * 4) * 4),
+                             "l"(s_ws + (size_t)bhe * D + kc * KE + v * 4));
+        }
+    };
+    auto row_ids = [&](const PmItem &m, int q0, int (&rid)[R]) {
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+            const int row = q0 + lane + 32 * j;
+            rid[j] = row < m.n_c ? row_of(m, row) : 0;
+        }
+    };
 
-        for (int q0 = 0; q0 < n_c; q0 += kPmPassRows) {
-            const int pr = min(kPmPassRows, n_c - q0);
-            for (int r = threadIdx.x; r < pr; r += kPmThreads) trow[r] = (int32_t)row_of(q0 + r);
-            __syncthreads();   // the pass's row table is complete
-            if (computes) {
-                const int nck = (pr + RCH - 1) / RCH;
-                auto issue = [&](int t) {
-                    const int c = rs + t * streams;
-                    if (c < nck) {
-                        const uint32_t dst0 = (uint32_t)__cvta_generic_to_shared(ring + (t % kRingStages) * kChunkBytes);
-                        for (int q = tg; q < RCH * LPG; q += hgn * 32) {
-                            const int r = q / LPG, v = q - (q / LPG) * LPG;
-                            const int rr = c * RCH + r;
-                            const bool ok = rr < pr;
-                            const T *src = kbase + (size_t)(ok ? trow[rr] : 0) * D + v * EV;
-                            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst0 + r * ROWB + v * 16),
-                                         "l"(src), "r"(ok ? 16 : 0));
-                        }
+    // issue side (one stage ahead) and compute side
+    int i_item = gw, i_q0 = 0, i_kc = 0;
+    PmItem ii = load_item(gw);
+    int pf_item = gw + nw;
+    PmItem pf = ii;
+    if (pf_item < n_items) pf = load_item(pf_item);
+    int rid[R];
+    row_ids(ii, 0, rid);
+    issue(ii, 0, 0, rid, 0);
+    asm volatile("cp.async.commit_group;\n" ::);
+    bool i_done = false;
+    PmItem ci = ii;
+    int c_item = gw, c_q0 = 0, c_kc = 0;
+    uint64_t acc[R][EC];
+    for (int t = 0;; ++t) {
+        // the issue side moves one stage on and loads it
+        if (!i_done) {
+            if (++i_kc == NKC) {
+                i_kc = 0;
+                i_q0 += kPmRP;
+                if (i_q0 >= ii.n_c) {
+                    i_q0 = 0;
+                    i_item = pf_item;
+                    if (i_item < n_items) {
+                        ii = pf;
+                        pf_item += nw;
+                        if (pf_item < n_items) pf = load_item(pf_item);
+                    } else {
+                        i_done = true;
                     }
-                    asm volatile("cp.async.commit_group;\n" ::);
-                };
-#pragma unroll
-                for (int t = 0; t < kRingStages - 1; ++t) issue(t);
-                for (int t = 0; rs + t * streams < nck; ++t) {   // the same bound for the whole stream
-                    asm volatile("cp.async.wait_group %0;\n" ::"n"(kRingStages - 2));
-                    stream_sync();   // chunk t landed for the stream; the stage of chunk t - 1 is free
-                    issue(t + kRingStages - 1);
-                    const int c = rs + t * streams;
-                    const uint8_t *tb = ring + (t % kRingStages) * kChunkBytes;
-                    float v[LPG];
-#pragma unroll
-                    for (int k = 0; k < R; ++k) {
-                        uint64_t xp[EV / 2];
-                        Pairs16<T>::get(*reinterpret_cast<const uint4 *>(tb + (lg * R + k) * ROWB + sub * 16), xp);
-#pragma unroll
-                        for (int h = 0; h < HT; ++h) {
-                            uint64_t acc = 0;
-#pragma unroll
-                            for (int e = 0; e < EV / 2; ++e) acc = ffma2(sreg[h][e], xp[e], acc);
-                            v[k * HT + h] = sum2(acc);
-                        }
-                    }
-#pragma unroll
-                    for (int m = LPG / 2; m >= 1; m >>= 1) {
-                        const bool upper = (sub & m) != 0;
-#pragma unroll
-                        for (int q = 0; q < m; ++q) {
-                            const float send = upper ? v[q] : v[q + m];
-                            const float keep = upper ? v[q + m] : v[q];
-                            v[q] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-                        }
-                    }
-                    const int rr = c * RCH + lg * R + k_mine;
-                    if (stores && rr < pr) f_mine[q0 + rr] = v[0];
                 }
-                asm volatile("cp.async.wait_group 0;\n" ::);
+                if (!i_done) row_ids(ii, i_q0, rid);
             }
-            __syncthreads();   // the rings and the table are free for the next pass
+            if (!i_done) issue(ii, i_q0, i_kc, rid, (t + 1) & 1);
+        }
+        asm volatile("cp.async.commit_group;\n" ::);
+        asm volatile("cp.async.wait_group 1;\n" ::);
+        __syncwarp();   // stage t landed for every lane
+        if (c_kc == 0) {
+#pragma unroll
+            for (int j = 0; j < R; ++j)
+#pragma unroll
+                for (int h = 0; h < EC; ++h) acc[j][h] = 0;
+        }
+        {
+            const uint8_t *st = wsm + (size_t)(t & 1) * SB;
+            const float *ss = reinterpret_cast<const float *>(st + kPmRP * kPmSlice);
+#pragma unroll
+            for (int pc = 0; pc < PPR; ++pc) {
+                uint64_t xp[R][EV / 2];
+#pragma unroll
+                for (int j = 0; j < R; ++j) {
+                    const int row = lane + 32 * j;
+                    Pairs16<T>::get(*reinterpret_cast<const uint4 *>(st + row * kPmSlice + ((pc ^ ((row >> 1) & 3)) << 4)),
+                                    xp[j]);
+                }
+#pragma unroll
+                for (int h = 0; h < EC; ++h) {
+                    if (h < ci.ne) {
+                        const uint64_t *sp = reinterpret_cast<const uint64_t *>(ss + h * KE + pc * EV);
+                        uint64_t sv[EV / 2];
+#pragma unroll
+                        for (int e = 0; e < EV / 2; e += 2) {
+                            const ulonglong2 w = *reinterpret_cast<const ulonglong2 *>(sp + e);
+                            sv[e] = w.x;
+                            sv[e + 1] = w.y;
+                        }
+#pragma unroll
+                        for (int j = 0; j < R; ++j)
+#pragma unroll
+                            for (int e = 0; e < EV / 2; ++e) acc[j][h] = ffma2(sv[e], xp[j][e], acc[j][h]);
+                    }
+                }
+            }
+        }
+        if (c_kc == NKC - 1) {
+#pragma unroll
+            for (int h = 0; h < EC; ++h) {
+                const long long bhh = __shfl_sync(0xffffffffu, ci.bh, h);
+                const int c0h = __shfl_sync(0xffffffffu, ci.c0, h);
+                if (h < ci.ne) {
+                    float *dst = f_ws + (size_t)bhh * fstride + c0h + c_q0;
+#pragma unroll
+                    for (int j = 0; j < R; ++j) {
+                        const int row = lane + 32 * j;
+                        if (c_q0 + row < ci.n_c) dst[row] = sum2(acc[j][h]);
+                    }
+                }
+            }
+        }
+        __syncwarp();   // buffer t & 1 is free for stage t + 2
+        // the compute side moves one stage on
+        if (++c_kc == NKC) {
+            c_kc = 0;
+            c_q0 += kPmRP;
+            if (c_q0 >= ci.n_c) {
+                c_q0 = 0;
+                c_item += nw;
+                if (c_item >= n_items) break;
+                ci = ii;   // the issue side is on this item's second stage (NKC >= 2)
+            }
         }
     }
+    asm volatile("cp.async.wait_group 0;\n" ::);
 }
 
 // ---------------------------------------------------------------------------
@@ -319,16 +388,94 @@ __global__ void __launch_bounds__(kPmThreads, 4)
 // writes their candidate prefix.
 __host__ __device__ constexpr size_t pm_select_warp_bytes(int kcap, int cap, int Kpmax)
 {
-    return (warp_sel_bytes(kcap, cap) + (size_t)(2 * Kpmax + 2) * 4 + 15) & ~size_t(15);
+    return (warp_sel_bytes(kcap, 0) + (size_t)kCollectCap * 8 + (size_t)(2 * Kpmax + 2) * 4 + 15 + 0 * cap) &
+           ~size_t(15);
+}
+
+// Counts traversal bh's kept entries of level L per key of the next level's
+// inversion nx (and, on a CSR next level, their candidate prefix).  One warp.
+__device__ __forceinline__ void pm_count_next(const DescendParams &p, const PmLevel &nx, int L, long long bh)
+{
+    const int lane = threadIdx.x & 31;
+    const int hkv = (int)(bh % p.H) / p.G;
+    const int K = p.K[L];
+    const long long rws = p.rows[L];
+    const int32_t *kl = p.kept[L] + bh * K;
+    for (int k = lane; k < K; k += 32) {
+        const int id = kl[k];
+        if (id < 0 || id >= rws) {
+            set_status(p.status, kDevBadChild);
+            nx.rank[bh * K + k] = -1;
+            continue;
+        }
+        nx.rank[bh * K + k] = atomicAdd(nx.cnt + (size_t)hkv * rws + id, 1);
+    }
+    if (nx.cpre) {
+        const int32_t *off_h = p.coff[L] + (size_t)hkv * (rws + 1);
+        warp_prefix_counts(
+            K,
+            [&](int k) {
+                const int id = kl[k];
+                return (id < 0 || id >= rws) ? 0 : off_h[id + 1] - off_h[id];
+            },
+            nx.cpre + bh * (K + 1));
+    }
+}
+
+// Selections the fp32 band left open (queued by pm_select_kernel): one warp
+// per queued traversal runs the refinement, writes the kept list and counts
+// it for the next level.  Rare, and register-hungry (exact arithmetic), so it
+// is kept out of the selection kernel.  Shared memory: per warp the kept
+// parents' candidate prefix (CSR), Kpmax + 1 ints.
+template <typename T, int D>
+__global__ void __launch_bounds__(kSelThreads, 1)
+    pm_refine_kernel(const __grid_constant__ DescendParams p0, const __grid_constant__ PmLevel self,
+                     const __grid_constant__ PmLevel nx, int L)
+{
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    __shared__ DescendParams p;
+    griddep_launch();
+    copy_params(p, p0);
+    griddep_wait();
+    __syncthreads();
+    const int warp = threadIdx.x >> 5;
+    constexpr int NW = kSelThreads / 32;
+    int32_t *cpre = reinterpret_cast<int32_t *>(smem_raw) + warp * (p.Kpmax + 1);
+    const int nq = *self.qcount;
+    const int K = p.K[L];
+    const int Kp = L == 0 ? 0 : p.K[L - 1];
+    const bool csr = L >= 1 && p.coff[L - 1] != nullptr;
+    for (int i = blockIdx.x * NW + warp; i < nq; i += gridDim.x * NW) {
+        const int4 q = self.queue[i];
+        const long long bh = q.x;
+        if (csr) {
+            const int hkv = (int)(bh % p.H) / p.G;
+            const int32_t *off_h = p.coff[L - 1] + (size_t)hkv * (p.rows[L - 1] + 1);
+            const int32_t *prev = p.kept[L - 1] + bh * Kp;
+            warp_prefix_counts(Kp, [&](int k) { return off_h[prev[k] + 1] - off_h[prev[k]]; }, cpre);
+        }
+        const LevelView lv = level_view(p, L, bh, csr ? cpre : nullptr);
+        uint64_t *kbuf = reinterpret_cast<uint64_t *>(p.f_ws + (size_t)bh * p.fstride + p.cap);
+        const int *list = reinterpret_cast<const int *>(p.f_ws + (size_t)bh * p.fstride);
+        ExactScratch xs(p.xs_ws + (size_t)bh * ExactScratch::bytes());
+        warp_refine<T, D>(p, lv, L, bh, kbuf, q.y, list, q.z, q.w != 0, xs);
+        __syncwarp();
+        write_kept(p, lv, L, bh, kbuf, K);
+        if (nx.cnt) pm_count_next(p, nx, L, bh);
+        __syncwarp();
+    }
 }
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kSelThreads, 2)
-    pm_select_kernel(const __grid_constant__ DescendParams p0, const __grid_constant__ PmLevel nx, int L, int nsel, int pw)
+    pm_select_kernel(const __grid_constant__ DescendParams p0, const __grid_constant__ PmLevel self,
+                     const __grid_constant__ PmLevel nx, int L, int nsel, int pw)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ DescendParams p;
+    griddep_launch();
     copy_params(p, p0);
+    griddep_wait();
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long BH = (long long)p.B * p.H;
@@ -339,8 +486,8 @@ __global__ void __launch_bounds__(kSelThreads, 2)
     uint64_t *tmp = reinterpret_cast<uint64_t *>(ws + 1024);
     uint64_t *kbuf = p.kcap <= kKbufSmem ? reinterpret_cast<uint64_t *>(ws + 1536)
                                          : reinterpret_cast<uint64_t *>(p.f_ws + (size_t)bh * p.fstride + p.cap);
-    float *fs = reinterpret_cast<float *>(ws + warp_sel_bytes(p.kcap, 0));
-    int32_t *prev = reinterpret_cast<int32_t *>(ws + warp_sel_bytes(p.kcap, p.cap));
+    uint64_t *col = reinterpret_cast<uint64_t *>(ws + warp_sel_bytes(p.kcap, 0));
+    int32_t *prev = reinterpret_cast<int32_t *>(ws + warp_sel_bytes(p.kcap, 0) + (size_t)kCollectCap * 8);
     int32_t *cpre = prev + p.Kpmax;
     const int hkv = (int)(bh % p.H) / p.G;
     const int Kp = L == 0 ? 0 : p.K[L - 1];
@@ -354,32 +501,11 @@ __global__ void __launch_bounds__(kSelThreads, 2)
         }
     }
     ExactScratch xs(p.xs_ws + (size_t)bh * ExactScratch::bytes());
-    warp_select<T, D>(p, L, bh, csr ? cpre : nullptr, L == 0 ? nullptr : prev, hist, tmp, kbuf, fs, xs);
+    const bool done = warp_select_pm<T, D>(p, L, bh, csr ? cpre : nullptr, L == 0 ? nullptr : prev, hist, tmp, kbuf,
+                                           col, xs, self.queue, self.qcount);
     __syncwarp();
-    if (nx.cnt) {
-        const int K = p.K[L];
-        const long long rws = p.rows[L];
-        const int32_t *kl = p.kept[L] + bh * K;
-        for (int k = lane; k < K; k += 32) {
-            const int id = kl[k];
-            if (id < 0 || id >= rws) {
-                set_status(p.status, kDevBadChild);
-                nx.rank[bh * K + k] = -1;
-                continue;
-            }
-            nx.rank[bh * K + k] = atomicAdd(nx.cnt + (size_t)hkv * rws + id, 1);
-        }
-        if (nx.cpre) {
-            const int32_t *off_h = p.coff[L] + (size_t)hkv * (rws + 1);
-            warp_prefix_counts(
-                K,
-                [&](int k) {
-                    const int id = kl[k];
-                    return (id < 0 || id >= rws) ? 0 : off_h[id + 1] - off_h[id];
-                },
-                nx.cpre + bh * (K + 1));
-        }
-    }
+    if (done && nx.cnt) pm_count_next(p, nx, L, bh);
+    (void)lane;
 }
 
 // ---------------------------------------------------------------------------
@@ -393,6 +519,8 @@ __global__ void __launch_bounds__(kScanThreads) pm_scan_kernel(const __grid_cons
     __shared__ int tile_sh;
     __shared__ unsigned long long wsum[kScanThreads / 32];
     __shared__ unsigned long long pre_sh;
+    griddep_launch();
+    griddep_wait();
     if (threadIdx.x == 0) tile_sh = atomicAdd(pl.ctr, 1);
     __syncthreads();
     const int tile = tile_sh;
@@ -419,36 +547,51 @@ __global__ void __launch_bounds__(kScanThreads) pm_scan_kernel(const __grid_cons
         if (w < warp) wpre += wsum[w];
         agg += wsum[w];
     }
-    if (threadIdx.x == 0) {
+    if (warp == 0) {
+        // publish this tile's aggregate, then look back over the predecessors
+        // 32 at a time: sum aggregates down to the nearest published prefix
         unsigned long long pre = 0;
         if (tile == 0) {
-            pl.tval[1] = agg;
-            st_release(pl.tflag, 2);
+            if (lane == 0) {
+                pl.tval[1] = agg;
+                st_release(pl.tflag, 2);
+            }
         } else {
-            pl.tval[2 * tile] = agg;
-            st_release(pl.tflag + tile, 1);
+            if (lane == 0) {
+                pl.tval[2 * tile] = agg;
+                st_release(pl.tflag + tile, 1);
+            }
             int j = tile - 1, spins = 0;
             while (j >= 0) {
-                const int f = ld_acquire(pl.tflag + j);
-                if (f == 2) {
-                    pre += pl.tval[2 * j + 1];
-                    break;
-                }
-                if (f == 1) {
-                    pre += pl.tval[2 * j];
-                    --j;
+                const int idx = j - lane;
+                const int f = idx >= 0 ? ld_acquire(pl.tflag + idx) : 2;
+                if (__any_sync(0xffffffffu, f == 0)) {
+                    if (++spins > kScanSpinLimit) {
+                        if (lane == 0) set_status(status, kDevTimeout);
+                        break;
+                    }
                     continue;
                 }
-                if (++spins > kScanSpinLimit) {
-                    set_status(status, kDevTimeout);
-                    break;
-                }
+                const unsigned inc = __ballot_sync(0xffffffffu, f == 2);
+                const int first = inc ? __ffs(inc) - 1 : 32;   // the nearest published prefix
+                unsigned long long v = 0;
+                if (idx >= 0 && lane < first) v = pl.tval[2 * idx];
+                if (idx >= 0 && lane == first) v = pl.tval[2 * idx + 1];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                pre += v;
+                if (inc) break;
+                j -= 32;
             }
-            pl.tval[2 * tile + 1] = pre + agg;
-            st_release(pl.tflag + tile, 2);
+            if (lane == 0) {
+                pl.tval[2 * tile + 1] = pre + agg;
+                st_release(pl.tflag + tile, 2);
+            }
         }
-        pre_sh = pre;
-        if (tile == pl.n_tiles - 1) pl.ctr[1] = (int)((pre + agg) >> 32);
+        if (lane == 0) {
+            pre_sh = pre;
+            if (tile == pl.n_tiles - 1) pl.ctr[1] = (int)((pre + agg) >> 32);
+        }
     }
     __syncthreads();
     unsigned long long run = pre_sh + wpre + incl - loc;
@@ -470,6 +613,8 @@ __global__ void __launch_bounds__(kScanThreads) pm_scan_kernel(const __grid_cons
 __global__ void pm_fill_kernel(const int32_t *__restrict__ kept_prev, int Kp, int H, int G, long long prow,
                                const __grid_constant__ PmLevel pl, int *status)
 {
+    griddep_launch();
+    griddep_wait();
     for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < pl.E;
          e += (long long)gridDim.x * blockDim.x) {
         const long long bh = e / Kp;

@@ -64,17 +64,24 @@ def test_single_rank_helpers():
 
 
 def test_kernels_per_step_and_config():
+    import dataclasses
+
     from hierarchical_kv_pruning_b200 import synth
     dev = synth.shape(2)
     host = synth.shape(4)
-    # leaves in HBM, bf16 D = 128: the descent, the sequence part, the knowledge part
-    assert bench.kernels_per_step(dev) == 3
-    # host leaves: 7 launches per query chunk (four chunks) plus one sequence part
-    assert host.batch >= 8 and bench.kernels_per_step(host) == 4 * 7 + 1
-    import dataclasses
-    assert bench.kernels_per_step(dataclasses.replace(host, batch=7)) == 7 + 1
-    # fp32: the descent and one fused attention launch
-    assert bench.kernels_per_step(synth.shape(0)) == 2
+    # leaves in HBM, B H >= 512: parent-major descent (token sums; 3 levels of
+    # score, select, refine; scan and fill below the roots) and one attention
+    assert bench.uses_parent_major(dev) and bench.kernels_per_step(dev) == 1 + 3 * 3 + 2 * 2 + 1
+    assert bench.kernels_per_step(dev, "fused") == 2
+    # host leaves: per query chunk (four) levels 0-1, leaf-block staging (2),
+    # level 2, value staging (2), knowledge part; plus one sequence part
+    per = (1 + 3 + 3 + 2) + 2 + (3 + 2) + 2 + 1
+    assert host.batch >= 8 and bench.kernels_per_step(host) == 4 * per + 1
+    assert bench.kernels_per_step(dataclasses.replace(host, batch=7), "fused") == 7 + 1
+    mids = dataclasses.replace(host, mid_on_host=True)
+    assert bench.kernels_per_step(mids, "fused") == 4 * 10 + 1
+    # fp32, one query: the fused descent and one attention launch
+    assert not bench.uses_parent_major(synth.shape(0)) and bench.kernels_per_step(synth.shape(0)) == 2
     c = bench.config_of(dev, 4)
     assert c["workload"] == dev.name and c["parallelism"] == "replicas x4"
     assert c["B"] == dev.batch and c["K"] == list(dev.keep)

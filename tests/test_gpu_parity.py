@@ -220,14 +220,14 @@ def test_leaves_in_pinned_host_memory_small():
                         w.leaf_values.cpu().pin_memory(), w.root_child, w.mid_child, w.q_kg, w.q_seq, w.k_seq,
                         w.v_seq, w.targets)
     g_host = gpu_run(hw, sh.keep)
-    for k in ("kept_root", "kept_mid", "kept_leaf", "out", "lse"):
-        assert torch.equal(g_dev[k], g_host[k]), k
+    same_as_hbm_path(g_dev, g_host)
     compare(w, sh.keep, g_host)
 
 
 def test_leaves_in_pinned_host_memory_chunked():
     # B = 9 splits into four query chunks (2, 2, 2, 3) staged on a second stream
-    # while the other chunks compute; results equal the HBM-resident path.
+    # while the other chunks compute; kept sets equal the HBM-resident path's,
+    # outputs to rounding.
     sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(12, 10, 9),
                       keep=(3, 4, 16), batch=9, n_tokens=16, seq_len=48, permuted=True)
     w = synth.make_workload(sh, "cuda", 15)
@@ -236,9 +236,19 @@ def test_leaves_in_pinned_host_memory_chunked():
                         w.leaf_values.cpu().pin_memory(), w.root_child, w.mid_child, w.q_kg, w.q_seq, w.k_seq,
                         w.v_seq, w.targets)
     g_host = gpu_run(hw, sh.keep)
-    for k in ("kept_root", "kept_mid", "kept_leaf", "out", "lse"):
-        assert torch.equal(g_dev[k], g_host[k]), k
+    same_as_hbm_path(g_dev, g_host)
     compare(w, sh.keep, g_host)
+
+
+def same_as_hbm_path(g_dev, g_host):
+    """Host-resident leaves against the same workload in HBM: identical kept
+    sets; the attention is the same softmax but runs as a sequence part merged
+    with the knowledge part (host leaves) against one launch (HBM), so the
+    outputs agree to rounding: within one bfloat16 ulp at unit scale."""
+    for k in ("kept_root", "kept_mid", "kept_leaf"):
+        assert torch.equal(g_dev[k], g_host[k]), k
+    assert float((g_dev["out"].float() - g_host["out"].float()).abs().max()) <= 2 ** -7
+    assert float((g_dev["lse"] - g_host["lse"]).abs().max()) <= 1e-4
 
 
 def _host_levels(w, mids=True):
@@ -252,15 +262,15 @@ def _host_levels(w, mids=True):
 @pytest.mark.parametrize("batch", [3, 9])   # one query chunk; four chunks (2, 2, 2, 3)
 def test_mids_and_leaves_in_pinned_host_memory(batch):
     # Only the roots resident: the kept roots' mid blocks are staged before
-    # level 1, the kept mids' leaf blocks before level 2; results equal the
-    # HBM-resident path bit for bit and match the oracle.
+    # level 1, the kept mids' leaf blocks before level 2; the kept sets equal
+    # the HBM-resident path's, the outputs agree to rounding, and both match
+    # the oracle.
     sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(12, 10, 9),
                       keep=(3, 4, 16), batch=batch, n_tokens=16, seq_len=48, permuted=True)
     w = synth.make_workload(sh, "cuda", 18 + batch)
     g_dev = gpu_run(w, sh.keep)
     g_host = gpu_run(_host_levels(w), sh.keep)
-    for k in ("kept_root", "kept_mid", "kept_leaf", "out", "lse"):
-        assert torch.equal(g_dev[k], g_host[k]), k
+    same_as_hbm_path(g_dev, g_host)
     compare(w, sh.keep, g_host)
 
 
