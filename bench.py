@@ -83,10 +83,10 @@ def splits_attention(sh):
 
 def uses_parent_major(sh, descent="auto"):
     """The descent the library runs (ATLASKV_DESCENT_AUTO: parent-major from
-    B * H >= 512 traversals)."""
+    B * H >= 1024 traversals)."""
     if descent != "auto":
         return descent == "parent_major"
-    return sh.batch * sh.n_heads >= 512
+    return sh.batch * sh.n_heads >= 1024
 
 
 def kernels_per_step(sh, descent="auto"):
@@ -144,19 +144,28 @@ def attend_kernel_name(sh):
     return "attend_tc_kernel" if sh.head_dim == 128 else "attend_bf16_kernel"
 
 
-KERNEL_SOURCES = {"attend_tc_kernel": "attend_tc.cuh", "attend_bf16_kernel": "attend.cuh",
-                  "attend_f32_kernel": "attend.cuh", "descend_kernel": "descend.cuh",
-                  "stage_leaf_blocks_kernel": "staging.cuh"}
+# Source files of each profiled stage (the descent is a chain of kernels).
+KERNEL_SOURCES = {"attend_tc_kernel": ["attend_tc.cuh"], "attend_bf16_kernel": ["attend.cuh"],
+                  "attend_f32_kernel": ["attend.cuh"], "descent": ["descend.cuh", "descend_pm.cuh"],
+                  "stage_blocks_kernel": ["staging.cuh"]}
+
+
+def sources_digest(kernel):
+    """sha256 over the stage's source files, concatenated in order."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES.get(kernel, []):
+        with open(os.path.join(ROOT, "hierarchical_kv_pruning_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def profiled_traffic(kernel, workload):
-    """DRAM bytes per launch (read + write) from the committed ncu summary of
-    this kernel on this workload, if the kernel source still hashes to the one
-    profiled; otherwise None."""
-    import hashlib
+    """DRAM bytes per launch (read + write; for the descent, per call: the sum
+    over its kernels) from the committed ncu summary of this stage on this
+    workload, if its sources still hash to the ones profiled; otherwise None."""
     summ = os.path.join(ROOT, "profiles", "%s__%s.md" % (kernel, workload))
-    src = os.path.join(ROOT, "hierarchical_kv_pruning_b200", "csrc", KERNEL_SOURCES.get(kernel, ""))
-    if not (os.path.exists(summ) and os.path.isfile(src)):
+    if not (os.path.exists(summ) and kernel in KERNEL_SOURCES):
         return None
     fields = {}
     with open(summ) as f:
@@ -164,9 +173,7 @@ def profiled_traffic(kernel, workload):
             if line.startswith("- ") and ": " in line:
                 k, v = line[2:].split(": ", 1)
                 fields[k.strip()] = v.strip().strip("`")
-    with open(src, "rb") as f:
-        digest = hashlib.sha256(f.read()).hexdigest()
-    if fields.get("source_sha256") != digest or "dram_bytes_per_launch" not in fields:
+    if fields.get("source_sha256") != sources_digest(kernel) or "dram_bytes_per_launch" not in fields:
         return None
     return int(fields["dram_bytes_per_launch"])
 
@@ -335,7 +342,7 @@ def host_memory_ok(sh):
     return free_host >= 2 * sh.n_leaves * sh.n_kv_heads * sh.head_dim * 2 + (8 << 30)
 
 
-def roofline_of(sh, alg, st, ms_per_step, peaks, peak_src, link_gbs):
+def roofline_of(sh, alg, st, ms_per_step, peaks, peak_src, link_gbs, descent="auto"):
     """Rooflines from the algorithmic bytes and the per-launch stage times
     (CUDA events on each kernel's own stream, averaged over the stage pass).
     The headline is the kernel with the largest time; `kernels` lists each
@@ -352,7 +359,9 @@ def roofline_of(sh, alg, st, ms_per_step, peaks, peak_src, link_gbs):
         kernels[name] = {"kernel": kernel, "ms": round(ms, 5), "algorithmic_bytes": nbytes, "achieved": ach,
                          "unit": "GB/s", "frac": ach / hbm, "bound": "hbm"}
 
-    entry("descend", alg["descend"], st["descend"], "descend_kernel")
+    entry("descend", alg["descend"], st["descend"],
+          "descent (parent-major chain: token sums; per level score, select, refine; scan and fill)"
+          if uses_parent_major(sh, descent) else "descent (descend_kernel)")
     if splits_attention(sh):
         entry("attend_seq", alg["attend_seq"], st["attend_seq"], "attend_tc_kernel (sequence part)")
         entry("attend_leaf", alg["attend_leaf"], st["attend_leaf"], "attend_tc_kernel (knowledge part + merge)")
@@ -360,7 +369,7 @@ def roofline_of(sh, alg, st, ms_per_step, peaks, peak_src, link_gbs):
         entry("attend", alg["attend"], st["attend"], attend_kernel_name(sh))
     if sh.leaf_on_host:
         ach = alg["staging"] / (st["staging"] * 1e-3) / 1e9 if st["staging"] > 0 else 0.0
-        kernels["staging"] = {"kernel": "stage_leaf_blocks_kernel + stage_value_rows_kernel",
+        kernels["staging"] = {"kernel": "stage_blocks_kernel + stage_value_rows_kernel",
                               "ms": round(st["staging"], 5), "algorithmic_bytes": alg["staging"], "achieved": ach,
                               "unit": "GB/s", "frac": ach / link_gbs, "bound": "host_link",
                               "peak": link_gbs, "peak_source": "pinned cudaMemcpyAsync H2D measured in this run"}
@@ -507,7 +516,7 @@ def measure(sh, seed, args, world, rank, local, cpu_seconds, use_graph=False):
     alg = algorithmic_bytes(sh, res, w)
     peaks, peak_src = measured_peaks()
     link = pinned_h2d_gbs(torch) if sh.leaf_on_host else None
-    roof = roofline_of(sh, alg, st, ms_per_step, peaks, peak_src, link)
+    roof = roofline_of(sh, alg, st, ms_per_step, peaks, peak_src, link, args.descent)
     roof["exact_refinement"] = refine
     entry = {"value": value, "unit": "queries/s", "ms_per_step": ms_per_step,
              "us_per_query": 1e3 * ms_per_step / sh.batch,

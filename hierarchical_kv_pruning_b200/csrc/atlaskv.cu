@@ -212,8 +212,10 @@ DescPlan plan_descent(int G, const Ks &ks, int kcap, int cap, int D, int esz, lo
 
 // ---- parent-major descent plan ---------------------------------------------
 // Traversals with at least this many (B H) take the parent-major descent in
-// ATLASKV_DESCENT_AUTO; fewer run the fused kernel (one launch).
-constexpr long long kPmAutoMinTraversals = 512;
+// ATLASKV_DESCENT_AUTO; fewer run the fused kernel (one launch).  Measured on
+// B200: 512 traversals (47x47x47, B 16) run faster fused, 2048 (100x100x100,
+// B 64) faster parent-major.
+constexpr long long kPmAutoMinTraversals = 1024;
 constexpr size_t kPmSelBudget = 56 * 1024;   // selection CTA's shared memory (several CTAs per SM)
 
 struct PmPlan {

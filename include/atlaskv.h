@@ -258,7 +258,7 @@ atlaskv_status atlaskv_set_profiling(atlaskv_tree *tree, int32_t enable);
  *   rows are read once per group of up to 32 traversals that kept it, so the
  *   bytes read approach the unique rows a level needs (the choice for large
  *   batches).
- * ATLASKV_DESCENT_AUTO (the default): parent-major when B * H >= 512, else
+ * ATLASKV_DESCENT_AUTO (the default): parent-major when B * H >= 1024, else
  *   fused (each where the other's plan does not fit).
  * The mode changes the workspace size: set it before atlaskv_workspace_size.
  * atlaskv_attend_layers always runs the fused kernel. */

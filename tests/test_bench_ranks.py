@@ -80,8 +80,9 @@ def test_kernels_per_step_and_config():
     assert bench.kernels_per_step(dataclasses.replace(host, batch=7), "fused") == 7 + 1
     mids = dataclasses.replace(host, mid_on_host=True)
     assert bench.kernels_per_step(mids, "fused") == 4 * 10 + 1
-    # fp32, one query: the fused descent and one attention launch
+    # fp32, one query, and 16 queries of 32 heads: the fused descent and one attention launch
     assert not bench.uses_parent_major(synth.shape(0)) and bench.kernels_per_step(synth.shape(0)) == 2
+    assert not bench.uses_parent_major(synth.shape(1)) and bench.kernels_per_step(synth.shape(1)) == 2
     c = bench.config_of(dev, 4)
     assert c["workload"] == dev.name and c["parallelism"] == "replicas x4"
     assert c["B"] == dev.batch and c["K"] == list(dev.keep)
@@ -141,6 +142,14 @@ def test_profiled_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic("attend_tc_kernel", "other") is None     # no summary for that workload
     src.write_bytes(b"// kernel v2\n")
     assert bench.profiled_traffic("attend_tc_kernel", "w") is None         # source changed since the capture
+    # the descent is a chain of kernels from two files: the digest covers both, in order
+    (csrc / "descend.cuh").write_bytes(b"a")
+    (csrc / "descend_pm.cuh").write_bytes(b"b")
+    (tmp_path / "profiles" / "descent__w.md").write_text(
+        "- source_sha256: `%s`\n- dram_bytes_per_launch: 7\n" % hashlib.sha256(b"ab").hexdigest())
+    assert bench.profiled_traffic("descent", "w") == 7
+    (csrc / "descend_pm.cuh").write_bytes(b"c")
+    assert bench.profiled_traffic("descent", "w") is None
 
 
 def test_peaks_fall_back_when_unmeasured(tmp_path, monkeypatch):

@@ -438,13 +438,19 @@ def full_cache():
     return {}
 
 
-def compare_all_indices(w, K, g):
+def compare_all_indices(w, K, g, cache=None):
     """Kept root, mid and leaf sets of EVERY traversal against the oracle's
-    descent (bit-exact)."""
+    descent (bit-exact).  cache: a dict keeping the oracle's kept sets per
+    workload name across calls."""
     sh = w.shape
-    t = oracle_tree(w)
-    q = storage(w.q_kg)
-    kr, km, kl = oracle.descend(t, q, K)
+    if cache is not None and sh.name in cache:
+        kr, km, kl = cache[sh.name]
+    else:
+        t = oracle_tree(w)
+        q = storage(w.q_kg)
+        kr, km, kl = oracle.descend(t, q, K)
+        if cache is not None:
+            cache[sh.name] = (kr, km, kl)
     for name, ref in (("kept_root", kr), ("kept_mid", km), ("kept_leaf", kl)):
         got = g[name].reshape(sh.batch * sh.n_heads, -1).numpy()
         bad = np.nonzero((got != ref).any(axis=1))[0]
@@ -452,25 +458,28 @@ def compare_all_indices(w, K, g):
                                                           for i in bad[:8]], bad.size)
 
 
-def gpu_run_profiled(w, K):
+def gpu_run_profiled(w, K, descent=0):
     """gpu_run with the library's descent counters on: returns the outputs and
     per level the number of selections the fp32 band left open."""
     with HikvpTree.from_workload(w) as tree:
+        tree.set_descent(descent)
         tree.set_profiling(True)
         g = gpu_run(w, K, tree=tree)
         stats = tree.refine_stats()
     return g, stats
 
 
+@pytest.mark.parametrize("descent", ["fused", "parent_major"])
 @pytest.mark.parametrize("i", [1, 2, 3])
-def test_full_size_shapes(i, full_cache):
+def test_full_size_shapes(i, descent, full_cache):
+    # both descents at the benchmark sizes: every traversal's kept sets
     sh = synth.shape(i)
     w = synth.make_workload(sh, "cuda", 1000 + i)
-    g, stats = gpu_run_profiled(w, sh.keep)
-    print("refined selections per level (%s):" % sh.name,
+    g, stats = gpu_run_profiled(w, sh.keep, {"fused": 1, "parent_major": 2}[descent])
+    print("refined selections per level (%s, %s):" % (sh.name, descent),
           {lvl: (v["refined"], v["exact_scores"]) for lvl, v in stats.items()})
     check_structure(w, sh.keep, g)
-    compare_all_indices(w, sh.keep, g)
+    compare_all_indices(w, sh.keep, g, full_cache)
     trav = sample_traversals(sh.batch, sh.n_heads, 256, seed=i)
     compare(w, sh.keep, g, trav)
     del w
