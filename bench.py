@@ -49,6 +49,9 @@ def parse():
     ap.add_argument("--only", action="store_true", help="time the --config workload only (no per_config block)")
     ap.add_argument("--descent", default="auto", choices=["auto", "fused", "parent_major"],
                     help="how the descent runs (the results are the same)")
+    ap.add_argument("--leaf-cache", type=int, default=0,
+                    help="host-resident leaves: an HBM cache of this many staged leaf blocks across steps "
+                         "(every step repeats the same batch, so this measures the all-hit case)")
     return ap.parse_args()
 
 
@@ -89,7 +92,7 @@ def uses_parent_major(sh, descent="auto"):
     return sh.batch * sh.n_heads >= 1024
 
 
-def kernels_per_step(sh, descent="auto"):
+def kernels_per_step(sh, descent="auto", leaf_cache=False):
     """Kernels one atlaskv_attend call launches.  The fused descent is one
     launch; the parent-major one is the token sums, then per level a scoring,
     a selection and a refinement launch, and per level below the roots a scan
@@ -99,7 +102,8 @@ def kernels_per_step(sh, descent="auto"):
     staging copy of the leaf-key blocks (and, with the mids on the host, of the
     mid blocks before level 1), the leaf level, a de-duplication and a staging
     copy of the value rows, and the knowledge part; plus one sequence-part
-    launch for the whole batch (bf16, D = 128)."""
+    launch for the whole batch (bf16, D = 128).  A leaf-block cache adds its
+    map and commit launches per chunk."""
     pm = uses_parent_major(sh, descent)
 
     def levels(first, last):
@@ -117,6 +121,8 @@ def kernels_per_step(sh, descent="auto"):
         per = levels(0, 0) + 2 + levels(1, 1) + 2 + levels(2, 2) + 2 + 1
     else:
         per = levels(0, 1) + 2 + levels(2, 2) + 2 + 1
+    if leaf_cache:
+        per += 2
     return chunks * per + (1 if splits_attention(sh) else 0)
 
 
@@ -412,6 +418,8 @@ def measure(sh, seed, args, world, rank, local, cpu_seconds, use_graph=False):
     stream = torch.cuda.current_stream()
     tree = HikvpTree.from_workload(w)
     tree.set_descent({"auto": 0, "fused": 1, "parent_major": 2}[args.descent])
+    if args.leaf_cache and sh.leaf_on_host:
+        tree.set_leaf_cache(args.leaf_cache)
     K = sh.keep
     out = torch.empty_like(w.q_kg)
     lse = torch.empty((sh.batch, sh.n_tokens, sh.n_heads), dtype=torch.float32, device=dev)
@@ -521,9 +529,14 @@ def measure(sh, seed, args, world, rank, local, cpu_seconds, use_graph=False):
     entry = {"value": value, "unit": "queries/s", "ms_per_step": ms_per_step,
              "us_per_query": 1e3 * ms_per_step / sh.batch,
              "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-             "gpu_launches": kernels_per_step(sh, args.descent) * args.steps, "roofline": roof, "clocks": clk.summary(),
+             "gpu_launches": kernels_per_step(sh, args.descent, bool(args.leaf_cache) and sh.leaf_on_host) * args.steps, "roofline": roof, "clocks": clk.summary(),
              "config": config_of(sh, world), "cuda_graph": use_graph,
              "dtype": "f32" if sh.dtype == torch.float32 else "bf16"}
+    if args.leaf_cache and sh.leaf_on_host:
+        entry["leaf_cache"] = dict(tree.leaf_cache_stats(), blocks=args.leaf_cache,
+                                   note="cumulative over warm-up, timed and profiling steps; every step "
+                                        "repeats the same batch, so blocks hit after the first; the staging "
+                                        "roofline still counts every staged block as host-link bytes")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         entry["cpu_baseline"] = oracle_cpu_baseline(w, sh, cpu_seconds)
     if graph is not None:
@@ -561,6 +574,8 @@ def run_ours(args):
     }
     if "cpu_baseline" in head:
         line["cpu_baseline"] = head["cpu_baseline"]
+    if "leaf_cache" in head:
+        line["leaf_cache"] = head["leaf_cache"]
     # every other benchmark shape, one GPU only (the host-leaf shape needs
     # about 130 GB of pinned host memory per process)
     if world == 1 and not args.only and not (args.fanout or args.batch):

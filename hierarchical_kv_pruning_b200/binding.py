@@ -32,7 +32,7 @@ EXPORTED = ("atlaskv_create_tree", "atlaskv_workspace_size", "atlaskv_attend", "
             "atlaskv_set_profiling", "atlaskv_stage_times", "atlaskv_refine_stats", "atlaskv_attend_static",
             "atlaskv_probe_wait_timeout", "atlaskv_destroy", "atlaskv_last_error", "atlaskv_workspace_size_layers",
             "atlaskv_attend_layers", "atlaskv_create_tree_csr", "atlaskv_workspace_size_csr", "atlaskv_attend_csr",
-            "atlaskv_set_descent")
+            "atlaskv_set_descent", "atlaskv_set_leaf_cache", "atlaskv_leaf_cache_stats")
 MAX_LAYERS = 32
 MAX_LEVELS = 4
 # Size of the library's static device scratch (ATLASKV_STATIC_SCRATCH_BYTES).
@@ -125,6 +125,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
             lib.atlaskv_sync_status.argtypes = [V, V]
             lib.atlaskv_set_profiling.argtypes = [V, I32]
             lib.atlaskv_set_descent.argtypes = [V, I32]
+            lib.atlaskv_set_leaf_cache.argtypes = [V, ctypes.c_int64, V]
+            lib.atlaskv_leaf_cache_stats.argtypes = [V, ctypes.POINTER(ctypes.c_uint64), I32]
             lib.atlaskv_stage_times.argtypes = [V, ctypes.POINTER(ctypes.c_float), I32]
             lib.atlaskv_refine_stats.argtypes = [V, ctypes.POINTER(ctypes.c_uint64), I32]
             lib.atlaskv_probe_wait_timeout.argtypes = [V, V]
@@ -227,6 +229,18 @@ def atlaskv_set_profiling(tree: int, enable: int) -> None:
 def atlaskv_set_descent(tree: int, mode: int) -> None:
     """mode: ATLASKV_DESCENT_AUTO, ATLASKV_DESCENT_FUSED or ATLASKV_DESCENT_PARENT_MAJOR."""
     _check(load_library().atlaskv_set_descent(ctypes.c_void_p(tree), int(mode)))
+
+
+def atlaskv_set_leaf_cache(tree: int, blocks: int, stream: int = 0) -> None:
+    """HBM cache of `blocks` staged leaf-key blocks across calls (0: none)."""
+    _check(load_library().atlaskv_set_leaf_cache(ctypes.c_void_p(tree), int(blocks), ctypes.c_void_p(stream)))
+
+
+def atlaskv_leaf_cache_stats(tree: int):
+    """Cumulative cache counters: dict(hits, fills, bypasses)."""
+    out = (ctypes.c_uint64 * 3)()
+    _check(load_library().atlaskv_leaf_cache_stats(ctypes.c_void_p(tree), out, 3))
+    return {"hits": int(out[0]), "fills": int(out[1]), "bypasses": int(out[2])}
 
 
 def atlaskv_stage_times(tree: int):
@@ -376,6 +390,13 @@ class HikvpTree:
     def set_descent(self, mode: int):
         """ATLASKV_DESCENT_AUTO, ATLASKV_DESCENT_FUSED or ATLASKV_DESCENT_PARENT_MAJOR (same results)."""
         atlaskv_set_descent(self.handle, mode)
+
+    def set_leaf_cache(self, blocks: int, stream=None):
+        """HBM cache of staged leaf blocks across calls (host-resident leaves; 0 removes it)."""
+        atlaskv_set_leaf_cache(self.handle, blocks, _stream(stream))
+
+    def leaf_cache_stats(self):
+        return atlaskv_leaf_cache_stats(self.handle)
 
     def stage_times(self):
         return atlaskv_stage_times(self.handle)

@@ -157,6 +157,12 @@ struct atlaskv_tree {
     int nphases_last;
     int descent_mode;                                 // ATLASKV_DESCENT_*
     bool pm_last;                                     // the last attend ran the parent-major descent
+    // HBM cache of staged leaf blocks (host leaves; atlaskv_set_leaf_cache)
+    unsigned long long *cache_tag;                    // [sets * kCacheWays] way words
+    void *cache_pool;                                 // [sets * kCacheWays][b_L][D]
+    long long cache_sets;
+    uint32_t cache_epoch;                             // calls that used the cache
+    unsigned long long *cache_stats;                  // [3] hits, fills, bypasses (cumulative)
 };
 
 namespace {
@@ -317,6 +323,7 @@ void pm_bind(const PmPlan &pp, int n_levels, long long BH, uint8_t *zero, uint8_
 
 struct Layout {
     size_t s_ws, s64_ws, a64_ws, anorm_ws, f_ws, xs, kept[akv::kMaxLevels], leaf_slot, kept_leaf_row, vslot, umid, ucount_mid,
+        csrc, cfill,
         uleaf, ucount_leaf, key_pool, val_pool, oseq, lse_seq, mid_slot, uroot, ucount_root, mid_pool, total;
     int cap, kcap, fstride;
     DescPlan desc;
@@ -393,6 +400,8 @@ Layout plan(const atlaskv_tree *t, const Ks &ks, int B, int N, int H, int T, boo
         L.vslot = take(BH * ks.K[2] * 4);
         L.umid = take(groups * n_mid * 4);
         L.ucount_mid = take(groups * 4);
+        L.csrc = take(groups * n_mid * 4);    // leaf-block cache map (used when the tree has a cache)
+        L.cfill = take(groups * n_mid * 4);
         L.uleaf = take(groups * n_leaf * 4);
         L.ucount_leaf = take(groups * 4);
         L.key_pool = take(groups * n_mid * (size_t)t->d.fanout[2] * D * esize(t->d.dtype));
@@ -744,13 +753,14 @@ atlaskv_status launch_dedupe(const int32_t *ids, int n, int groups, int32_t *uni
 // roots, 2: leaves of kept mids) from host memory into the pool.
 template <typename T, int D>
 atlaskv_status stage_keys(const atlaskv_tree *t, int L, const int32_t *uniq, const int32_t *cnt, int n, int groups,
-                          void *pool, cudaStream_t s)
+                          void *pool, const int32_t *csrc, const int32_t *cfill, cudaStream_t s)
 {
     const void *src = L == 1 ? t->mid_keys_dev : t->leaf_keys_dev;
     const int32_t *tab = L == 1 ? t->d.root_child : t->d.mid_child;
+    T *cache = csrc ? reinterpret_cast<T *>(t->cache_pool) : nullptr;
     akv::stage_blocks_kernel<T, D><<<akv::kStageCtasPerSm * t->num_sms, 256, 0, s>>>(
         reinterpret_cast<const T *>(src), tab, t->rows[L - 1], t->rows[L], t->d.fanout[L], t->d.n_kv_heads, uniq, cnt,
-        n, groups, reinterpret_cast<T *>(pool), t->status);
+        n, groups, reinterpret_cast<T *>(pool), t->status, cache, csrc, cfill);
     AKV_CUDA(cudaGetLastError());
     return ATLASKV_OK;
 }
@@ -766,15 +776,39 @@ atlaskv_status stage_values(const atlaskv_tree *t, const int32_t *uleaf, const i
     return ATLASKV_OK;
 }
 
+// csrc / cfill: the chunk's cache map (null without the leaf-block cache)
 atlaskv_status dispatch_stage_keys(const atlaskv_tree *t, int L, const int32_t *uniq, const int32_t *cnt, int n,
-                                   int groups, void *pool, cudaStream_t s)
+                                   int groups, void *pool, cudaStream_t s, const int32_t *csrc = nullptr,
+                                   const int32_t *cfill = nullptr)
 {
     const int D = t->d.head_dim;
     if (t->d.dtype == ATLASKV_F32)
-        return D == 64 ? stage_keys<float, 64>(t, L, uniq, cnt, n, groups, pool, s)
-                       : stage_keys<float, 128>(t, L, uniq, cnt, n, groups, pool, s);
-    return D == 64 ? stage_keys<__nv_bfloat16, 64>(t, L, uniq, cnt, n, groups, pool, s)
-                   : stage_keys<__nv_bfloat16, 128>(t, L, uniq, cnt, n, groups, pool, s);
+        return D == 64 ? stage_keys<float, 64>(t, L, uniq, cnt, n, groups, pool, csrc, cfill, s)
+                       : stage_keys<float, 128>(t, L, uniq, cnt, n, groups, pool, csrc, cfill, s);
+    return D == 64 ? stage_keys<__nv_bfloat16, 64>(t, L, uniq, cnt, n, groups, pool, csrc, cfill, s)
+                   : stage_keys<__nv_bfloat16, 128>(t, L, uniq, cnt, n, groups, pool, csrc, cfill, s);
+}
+
+// The leaf-block cache's map and commit for one chunk's unique kept mids.
+atlaskv_status cache_map(const atlaskv_tree *t, const int32_t *umid, const int32_t *cnt, int n, int groups,
+                         int32_t *csrc, int32_t *cfill, cudaStream_t s)
+{
+    const unsigned g = (unsigned)std::max<long long>(1, std::min<long long>(((long long)groups * n + 255) / 256,
+                                                                            (long long)t->num_sms * 4));
+    akv::cache_map_kernel<<<g, 256, 0, s>>>(umid, cnt, n, groups, t->d.n_kv_heads, t->rows[1], t->cache_tag,
+                                            t->cache_sets, t->cache_epoch, csrc, cfill, t->cache_stats);
+    AKV_CUDA(cudaGetLastError());
+    return ATLASKV_OK;
+}
+
+atlaskv_status cache_commit(const atlaskv_tree *t, const int32_t *cnt, int n, int groups, const int32_t *cfill,
+                            cudaStream_t s)
+{
+    const unsigned g = (unsigned)std::max<long long>(1, std::min<long long>(((long long)groups * n + 255) / 256,
+                                                                            (long long)t->num_sms * 4));
+    akv::cache_commit_kernel<<<g, 256, 0, s>>>(cnt, n, groups, cfill, t->cache_tag);
+    AKV_CUDA(cudaGetLastError());
+    return ATLASKV_OK;
 }
 
 atlaskv_status dispatch_stage_values(const atlaskv_tree *t, const int32_t *uleaf, const int32_t *cnt, int n,
@@ -1390,7 +1424,7 @@ atlaskv_status attend_impl(atlaskv_tree *t, const Ks &ks, const atlaskv_io *io, 
             akv::AttnParams a;
             akv::PmLevel lv[akv::kMaxLevels];
             int groups;
-            int32_t *uroot, *croot, *mid_slot, *umid, *cmid, *leaf_slot, *uleaf, *cleaf, *vslot;
+            int32_t *uroot, *croot, *mid_slot, *umid, *cmid, *leaf_slot, *uleaf, *cleaf, *vslot, *csrc, *cfill;
         };
         Chunk ch[kMaxChunks];
         for (int c = 0; c < nc; ++c) {
@@ -1417,6 +1451,8 @@ atlaskv_status attend_impl(atlaskv_tree *t, const Ks &ks, const atlaskv_io *io, 
             k.vslot = reinterpret_cast<int32_t *>(ws + L.vslot) + bh0 * p->K_leaf;
             k.umid = reinterpret_cast<int32_t *>(ws + L.umid) + g0 * n_mid;
             k.cmid = reinterpret_cast<int32_t *>(ws + L.ucount_mid) + g0;
+            k.csrc = reinterpret_cast<int32_t *>(ws + L.csrc) + g0 * n_mid;
+            k.cfill = reinterpret_cast<int32_t *>(ws + L.cfill) + g0 * n_mid;
             k.uleaf = reinterpret_cast<int32_t *>(ws + L.uleaf) + g0 * n_leaf;
             k.cleaf = reinterpret_cast<int32_t *>(ws + L.ucount_leaf) + g0;
             uint8_t *pool = ws + L.key_pool + g0 * n_mid * (size_t)t->d.fanout[2] * D * esz;
@@ -1482,6 +1518,7 @@ atlaskv_status attend_impl(atlaskv_tree *t, const Ks &ks, const atlaskv_io *io, 
             AKV_CUDA(cudaEventRecord(t->fev[0], s));
             AKV_STEP(fork_sequence_part());
         }
+        if (t->cache_pool) ++t->cache_epoch;   // this call's stamp (epoch 0 marks empty ways)
         for (int k = 0; k < np; ++k) {
             const Phase ph = t->phase[k];
             const bool on_stage = ph.kind == kPhaseStageKeys || ph.kind == kPhaseStageValues;
@@ -1505,8 +1542,15 @@ atlaskv_status attend_impl(atlaskv_tree *t, const Ks &ks, const atlaskv_io *io, 
                                                      const_cast<void *>(q.d.keys[1]), s1));
                     } else {
                         AKV_STEP(launch_dedupe(q.d.kept[1], n_mid, q.groups, q.umid, q.leaf_slot, q.cmid, s1));
-                        AKV_STEP(dispatch_stage_keys(t, 2, q.umid, q.cmid, n_mid, q.groups,
-                                                     const_cast<void *>(q.d.keys[2]), s1));
+                        if (t->cache_pool) {
+                            AKV_STEP(cache_map(t, q.umid, q.cmid, n_mid, q.groups, q.csrc, q.cfill, s1));
+                            AKV_STEP(dispatch_stage_keys(t, 2, q.umid, q.cmid, n_mid, q.groups,
+                                                         const_cast<void *>(q.d.keys[2]), s1, q.csrc, q.cfill));
+                            AKV_STEP(cache_commit(t, q.cmid, n_mid, q.groups, q.cfill, s1));
+                        } else {
+                            AKV_STEP(dispatch_stage_keys(t, 2, q.umid, q.cmid, n_mid, q.groups,
+                                                         const_cast<void *>(q.d.keys[2]), s1));
+                        }
                     }
                     break;
                 case kPhaseStageValues:
@@ -1711,6 +1755,61 @@ atlaskv_status atlaskv_set_profiling(atlaskv_tree *t, int32_t enable)
     return ATLASKV_OK;
 }
 
+atlaskv_status atlaskv_set_leaf_cache(atlaskv_tree *t, int64_t blocks, void *stream)
+{
+    if (!t) return fail(ATLASKV_EINVAL, "null tree");
+    if (blocks < 0) return fail(ATLASKV_EINVAL, "blocks = %lld < 0", (long long)blocks);
+    if (blocks > 0 && (!t->host_leaves || t->csr))
+        return fail(ATLASKV_EUNSUPPORTED, "the leaf-block cache is for three-level trees with host-resident leaves");
+    if (blocks > 0 && (long long)t->d.n_kv_heads * t->rows[1] >= (1LL << 31) - 1)
+        return fail(ATLASKV_EUNSUPPORTED, "too many mids for the cache's keys");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    AKV_CUDA(cudaStreamSynchronize(s));
+    if (t->stage_stream) AKV_CUDA(cudaStreamSynchronize(t->stage_stream));
+    if (t->cache_tag) AKV_CUDA(cudaFree(t->cache_tag));
+    if (t->cache_pool) AKV_CUDA(cudaFree(t->cache_pool));
+    if (t->cache_stats) AKV_CUDA(cudaFree(t->cache_stats));
+    t->cache_tag = nullptr;
+    t->cache_pool = nullptr;
+    t->cache_stats = nullptr;
+    t->cache_sets = 0;
+    t->cache_epoch = 0;
+    if (blocks == 0) return ATLASKV_OK;
+    long long sets = 1;
+    while (sets * akv::kCacheWays < blocks) sets <<= 1;
+    const size_t slots = (size_t)sets * akv::kCacheWays;
+    const size_t block_bytes = (size_t)t->d.fanout[2] * t->d.head_dim * esize(t->d.dtype);
+    cudaError_t e = cudaMalloc(&t->cache_pool, slots * block_bytes);
+    if (e == cudaSuccess) e = cudaMalloc(&t->cache_tag, slots * 8);
+    if (e == cudaSuccess) e = cudaMalloc(&t->cache_stats, 3 * sizeof(unsigned long long));
+    if (e == cudaSuccess) e = cudaMemsetAsync(t->cache_tag, 0, slots * 8, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(t->cache_stats, 0, 3 * sizeof(unsigned long long), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        if (t->cache_pool) cudaFree(t->cache_pool);
+        if (t->cache_tag) cudaFree(t->cache_tag);
+        if (t->cache_stats) cudaFree(t->cache_stats);
+        t->cache_pool = nullptr;
+        t->cache_tag = nullptr;
+        t->cache_stats = nullptr;
+        return fail(ATLASKV_ENOMEM, "leaf-block cache of %zu blocks: %s", slots, cudaGetErrorString(e));
+    }
+    t->cache_sets = sets;
+    return ATLASKV_OK;
+}
+
+atlaskv_status atlaskv_leaf_cache_stats(atlaskv_tree *t, uint64_t *counts, int32_t n)
+{
+    if (!t || !counts || n < 0) return fail(ATLASKV_EINVAL, "null tree or counts");
+    if (!t->cache_stats) return fail(ATLASKV_EINVAL, "the tree has no leaf-block cache");
+    unsigned long long v[3];
+    AKV_CUDA(cudaDeviceSynchronize());
+    AKV_CUDA(cudaMemcpy(v, t->cache_stats, sizeof(v), cudaMemcpyDeviceToHost));
+    for (int i = 0; i < n && i < 3; ++i) counts[i] = v[i];
+    return ATLASKV_OK;
+}
+
 atlaskv_status atlaskv_set_descent(atlaskv_tree *t, int32_t mode)
 {
     if (!t) return fail(ATLASKV_EINVAL, "null tree");
@@ -1773,6 +1872,9 @@ atlaskv_status atlaskv_destroy(atlaskv_tree *t)
     if (t->norm_bound) cudaFree(t->norm_bound);
     if (t->status) cudaFree(t->status);
     if (t->stats) cudaFree(t->stats);
+    if (t->cache_tag) cudaFree(t->cache_tag);
+    if (t->cache_pool) cudaFree(t->cache_pool);
+    if (t->cache_stats) cudaFree(t->cache_stats);
     for (int i = 0; i < kNumEvents; ++i)
         if (t->ev[i]) cudaEventDestroy(t->ev[i]);
     for (cudaEvent_t e : t->cev)

@@ -98,11 +98,15 @@ constexpr int kStageCtasPerSm = 2;
 // the key pool: pool row (q*n + u) * b_c + j <- host child row child(parent, j)
 // of KV head q % H_kv, with child() the level's table (or parent * b_c + j).
 // Used for the leaf blocks of kept mids and the mid blocks of kept roots.
+// With a leaf-block cache (cache non-null): block blk is read from cache slot
+// csrc[blk] when that is >= 0 (HBM) instead of host memory, and also written
+// to cache slot cfill[blk] when that is >= 0.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) stage_blocks_kernel(
     const T *__restrict__ host_child_keys, const int32_t *__restrict__ child_tab, long long n_parent,
     long long n_child, int b_child, int H_kv, const int32_t *__restrict__ uniq, const int32_t *__restrict__ count,
-    int n, int n_groups, T *pool, int *status)
+    int n, int n_groups, T *pool, int *status, T *cache, const int32_t *__restrict__ csrc,
+    const int32_t *__restrict__ cfill)
 {
     constexpr int VPR = D * (int)sizeof(T) / 16;   // 16-byte vectors per row = lanes per row
     constexpr int RPI = 32 / VPR;                  // rows per warp instruction
@@ -112,11 +116,11 @@ __global__ void __launch_bounds__(256) stage_blocks_kernel(
     for (long long r0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * (RPI * kStageUnroll);
          r0 < total; r0 += warps * RPI * kStageUnroll) {
         uint4 buf[kStageUnroll];
-        uint4 *dst[kStageUnroll];
+        uint4 *dst[kStageUnroll], *dst2[kStageUnroll];
 #pragma unroll
         for (int k = 0; k < kStageUnroll; ++k) {
             const long long w = r0 + (long long)k * RPI + rsel;
-            dst[k] = nullptr;
+            dst[k] = dst2[k] = nullptr;
             if (w < total) {
                 const long long blk = w / b_child;
                 const int j = (int)(w - blk * b_child);
@@ -124,21 +128,131 @@ __global__ void __launch_bounds__(256) stage_blocks_kernel(
                 const int u = (int)(blk - (long long)b * n);
                 if (u < count[b]) {
                     const int hkv = b % H_kv;   // group b = query * H_kv + hkv
-                    const long long par = uniq[blk];
-                    const long long ch = child_tab ? (long long)child_tab[((size_t)hkv * n_parent + par) * b_child + j]
-                                                   : par * b_child + j;
-                    if (ch < 0 || ch >= n_child) {
-                        set_status(status, kDevBadChild);
-                    } else {
-                        buf[k] = reinterpret_cast<const uint4 *>(host_child_keys + ((size_t)hkv * n_child + ch) * D)[sub];
+                    const int from = cache ? csrc[blk] : -1;
+                    if (from >= 0) {   // a cached block: copied within HBM
+                        buf[k] = reinterpret_cast<const uint4 *>(cache + ((size_t)from * b_child + j) * D)[sub];
                         dst[k] = reinterpret_cast<uint4 *>(pool + ((size_t)blk * b_child + j) * D) + sub;
+                    } else {
+                        const long long par = uniq[blk];
+                        const long long ch = child_tab
+                                                 ? (long long)child_tab[((size_t)hkv * n_parent + par) * b_child + j]
+                                                 : par * b_child + j;
+                        if (ch < 0 || ch >= n_child) {
+                            set_status(status, kDevBadChild);
+                        } else {
+                            buf[k] =
+                                reinterpret_cast<const uint4 *>(host_child_keys + ((size_t)hkv * n_child + ch) * D)[sub];
+                            dst[k] = reinterpret_cast<uint4 *>(pool + ((size_t)blk * b_child + j) * D) + sub;
+                            const int to = cache ? cfill[blk] : -1;
+                            if (to >= 0) dst2[k] = reinterpret_cast<uint4 *>(cache + ((size_t)to * b_child + j) * D) + sub;
+                        }
                     }
                 }
             }
         }
 #pragma unroll
-        for (int k = 0; k < kStageUnroll; ++k)
+        for (int k = 0; k < kStageUnroll; ++k) {
             if (dst[k]) *dst[k] = buf[k];
+            if (dst2[k]) *dst2[k] = buf[k];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// HBM cache of staged leaf blocks across calls, keyed by the kept mid
+// ("Quick read / Results": the CPU-GPU movement between levels is the I/O
+// cost; blocks of branches that recur need not cross the host link again).
+// Set-associative: kCacheWays ways per set, least recently used way evicted.
+// A way is one 64-bit word: call epoch (high 32 bits) | pending (bit 31) |
+// key + 1 (bits 0..30, key = hkv rows_mid + mid; 0 = empty).  Claiming a
+// victim and pinning a hit are single compare-and-swaps on that word, so a
+// way cannot change owner between the check and the use.  A way claimed in
+// this call stays pending until its block has been staged (cache_commit):
+// other groups wanting the same block meanwhile read it from host memory.
+// Ways stamped with the current epoch are never evicted in this call.
+constexpr int kCacheWays = 8;
+constexpr uint32_t kCachePending = 0x80000000u;
+constexpr int kCacheAttempts = 16;
+
+__device__ __forceinline__ uint32_t cache_hash(uint32_t key)
+{
+    uint32_t h = key * 0x9E3779B1u;
+    return h ^ (h >> 15);
+}
+
+// One thread per unique block of the chunk: csrc[blk] = cache slot holding it
+// (a hit), or -1; cfill[blk] = cache slot to fill while staging it (a miss
+// that claimed a way), or -1.  stats: hits, fills, bypasses.
+__global__ void cache_map_kernel(const int32_t *__restrict__ uniq, const int32_t *__restrict__ count, int n,
+                                 int n_groups, int H_kv, long long rows_mid, unsigned long long *tag, long long n_sets,
+                                 uint32_t epoch, int32_t *csrc, int32_t *cfill, unsigned long long *stats)
+{
+    const long long total = (long long)n_groups * n;
+    for (long long blk = (long long)blockIdx.x * blockDim.x + threadIdx.x; blk < total;
+         blk += (long long)gridDim.x * blockDim.x) {
+        const int b = (int)(blk / n);
+        const int u = (int)(blk - (long long)b * n);
+        if (u >= count[b]) continue;
+        const uint32_t key = (uint32_t)((long long)(b % H_kv) * rows_mid + uniq[blk]);
+        const uint32_t kw = key + 1u;
+        const long long set = (long long)(cache_hash(key) & (uint32_t)(n_sets - 1));
+        unsigned long long *ways = tag + set * kCacheWays;
+        int src = -1, fill = -1, kind = 2;   // 0 hit, 1 fill, 2 bypass
+        for (int attempt = 0; attempt < kCacheAttempts; ++attempt) {
+            unsigned long long w[kCacheWays];
+#pragma unroll
+            for (int i = 0; i < kCacheWays; ++i) w[i] = atomicAdd(ways + i, 0ull);
+            int hit = -1, victim = -1;
+            uint32_t oldest = 0xffffffffu;
+#pragma unroll
+            for (int i = 0; i < kCacheWays; ++i) {
+                const uint32_t lo = (uint32_t)w[i], stamp = (uint32_t)(w[i] >> 32);
+                if ((lo & ~kCachePending) == kw && hit < 0) hit = i;
+                if (stamp != epoch && stamp < oldest) {
+                    oldest = stamp;
+                    victim = i;
+                }
+            }
+            if (hit >= 0) {
+                const uint32_t lo = (uint32_t)w[hit], stamp = (uint32_t)(w[hit] >> 32);
+                if (lo & kCachePending) break;   // being filled in this call: bypass
+                if (stamp == epoch) {            // pinned already
+                    src = (int)(set * kCacheWays + hit);
+                    kind = 0;
+                    break;
+                }
+                const unsigned long long want = ((unsigned long long)epoch << 32) | kw;
+                if (atomicCAS(ways + hit, w[hit], want) == w[hit]) {
+                    src = (int)(set * kCacheWays + hit);
+                    kind = 0;
+                    break;
+                }
+                continue;   // the way changed: look again
+            }
+            if (victim < 0) break;   // every way holds a block of this call: bypass
+            const unsigned long long want = ((unsigned long long)epoch << 32) | kCachePending | kw;
+            if (atomicCAS(ways + victim, w[victim], want) == w[victim]) {
+                fill = (int)(set * kCacheWays + victim);
+                kind = 1;
+                break;
+            }
+        }
+        csrc[blk] = src;
+        cfill[blk] = fill;
+        if (stats) atomicAdd(stats + kind, 1ull);
+    }
+}
+
+// After the chunk's staging: the ways it filled are no longer pending.
+__global__ void cache_commit_kernel(const int32_t *__restrict__ count, int n, int n_groups,
+                                    const int32_t *__restrict__ cfill, unsigned long long *tag)
+{
+    const long long total = (long long)n_groups * n;
+    for (long long blk = (long long)blockIdx.x * blockDim.x + threadIdx.x; blk < total;
+         blk += (long long)gridDim.x * blockDim.x) {
+        const int b = (int)(blk / n);
+        const int u = (int)(blk - (long long)b * n);
+        if (u < count[b] && cfill[blk] >= 0) atomicAnd(tag + cfill[blk], ~(unsigned long long)kCachePending);
     }
 }
 

@@ -248,6 +248,30 @@ atlaskv_status atlaskv_sync_status(atlaskv_tree *tree, void *stream);
 #define ATLASKV_PROFILE_COUNTERS 2
 atlaskv_status atlaskv_set_profiling(atlaskv_tree *tree, int32_t enable);
 
+/* HBM cache of staged leaf blocks across calls (host-resident leaves of a
+ * three-level tree).  "Quick read / Results" names the CPU-GPU movement
+ * between levels as HiKVP's I/O cost; a branch that recurs over calls need
+ * not cross the host link again.  The cache holds `blocks` leaf-key blocks
+ * (rounded up to a power of two of 8-way sets; each block is the b_L child
+ * key rows of one mid, b_L * head_dim elements) in device memory that the
+ * tree allocates here and frees on destroy or on a later call with
+ * blocks = 0.  Keyed by (KV head, mid row); least recently used way of a set
+ * evicted; blocks of the current call are never evicted by it.  On a hit the
+ * block is copied within HBM instead of over the host link; results are
+ * identical with and without the cache.  Synchronises `stream` and the
+ * tree's staging stream first.  EUNSUPPORTED for HBM-resident or CSR trees,
+ * ENOMEM if the allocation fails (the tree then has no cache).  Not during a
+ * stream capture. */
+atlaskv_status atlaskv_set_leaf_cache(atlaskv_tree *tree, int64_t blocks, void *stream);
+
+/* Cumulative leaf-block cache counters since atlaskv_set_leaf_cache:
+ * counts[0] hits (block copied from the cache), [1] fills (read from host
+ * memory and kept), [2] bypasses (read from host memory, not kept: its set
+ * was full of this call's blocks, or another group of the call was filling
+ * it).  Synchronises the device; n is the capacity of counts (at most 3
+ * written).  EINVAL without a cache. */
+atlaskv_status atlaskv_leaf_cache_stats(atlaskv_tree *tree, uint64_t *counts, int32_t n);
+
 /* How the descent is run; the results are the same either way.
  * ATLASKV_DESCENT_FUSED: one kernel per call, one CTA per (query, KV head,
  *   chunk of heads), running every level; it reads the child rows of the

@@ -82,6 +82,9 @@ def test_null_arguments(lib):
     assert lib.atlaskv_sync_status(None, None) == binding.ATLASKV_EINVAL
     assert lib.atlaskv_set_profiling(None, 1) == binding.ATLASKV_EINVAL
     assert lib.atlaskv_set_descent(None, binding.ATLASKV_DESCENT_FUSED) == binding.ATLASKV_EINVAL
+    assert lib.atlaskv_set_leaf_cache(None, 8, None) == binding.ATLASKV_EINVAL
+    cnt = (ctypes.c_uint64 * 3)()
+    assert lib.atlaskv_leaf_cache_stats(None, cnt, 3) == binding.ATLASKV_EINVAL
     buf = (ctypes.c_float * 3)()
     assert lib.atlaskv_stage_times(None, buf, 3) == binding.ATLASKV_EINVAL
     assert lib.atlaskv_destroy(None) == binding.ATLASKV_OK

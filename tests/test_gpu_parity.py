@@ -274,6 +274,56 @@ def test_mids_and_leaves_in_pinned_host_memory(batch):
     compare(w, sh.keep, g_host)
 
 
+def _cached_runs(w_host, batches, blocks):
+    """Run the batches in turn on one host-leaf tree with a leaf-block cache of
+    `blocks` blocks (0: none); return the outputs and the cache counters."""
+    outs = []
+    with HikvpTree.from_workload(w_host) as tree:
+        if blocks:
+            tree.set_leaf_cache(blocks)
+        for q in batches:
+            r = tree.attend(q[0], q[1], q[2], q[3], w_host.shape.keep)
+            tree.sync_status()
+            outs.append({k: (v.cpu() if torch.is_tensor(v) and k != "workspace" else v) for k, v in r.items()})
+        stats = tree.leaf_cache_stats() if blocks else None
+    return outs, stats
+
+
+@pytest.mark.parametrize("blocks", [4096, 8])   # room for every block; one set of 8 ways (evictions, bypasses)
+def test_leaf_block_cache_gives_the_same_results(blocks):
+    # Batches A, A, B, A on one tree: with the cache every output equals the
+    # uncached path's, and the repeated batch finds its blocks in the cache.
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(12, 10, 9),
+                      keep=(3, 4, 16), batch=9, n_tokens=16, seq_len=48, permuted=True)
+    wa = synth.make_workload(sh, "cuda", 31)
+    wb = synth.make_workload(sh, "cuda", 32)
+    hw = _host_levels(wa, mids=False)
+    qa = (wa.q_kg, wa.q_seq, wa.k_seq, wa.v_seq)
+    qb = (wb.q_kg, wb.q_seq, wb.k_seq, wb.v_seq)
+    plain, _ = _cached_runs(hw, [qa, qb], 0)
+    got, stats = _cached_runs(hw, [qa, qa, qb, qa], blocks)
+    for g, ref in zip(got, [plain[0], plain[0], plain[1], plain[0]]):
+        for k in ("kept_root", "kept_mid", "kept_leaf", "out", "lse"):
+            assert torch.equal(g[k], ref[k]), k
+    compare(wa, sh.keep, got[1])
+    assert stats["hits"] + stats["fills"] + stats["bypasses"] > 0
+    if blocks == 4096:
+        assert stats["hits"] > 0 and stats["hits"] >= stats["fills"]
+    else:
+        assert stats["bypasses"] > 0
+
+
+def test_leaf_block_cache_needs_host_leaves():
+    from hierarchical_kv_pruning_b200.binding import ATLASKV_EUNSUPPORTED
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=2, n_kv_heads=1, head_dim=128, fanout=(4, 4, 4),
+                      keep=(2, 2, 2), batch=1, n_tokens=2, seq_len=2)
+    w = synth.make_workload(sh, "cuda", 33)
+    with HikvpTree.from_workload(w) as tree:
+        with pytest.raises(AtlaskvError) as ei:
+            tree.set_leaf_cache(64)
+        assert ei.value.status == ATLASKV_EUNSUPPORTED
+
+
 def test_host_mids_fp32_d64():
     sh = synth.custom(dtype=torch.float32, n_heads=2, n_kv_heads=1, head_dim=64, fanout=(9, 7, 5),
                       keep=(3, 5, 9), batch=2, n_tokens=5, seq_len=9)
