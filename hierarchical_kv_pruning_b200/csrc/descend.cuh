@@ -1107,9 +1107,10 @@ __device__ __noinline__ bool warp_select_defer_call(const DescendParams &p, int 
 // Tier 1 in one pass over the scores (read from the traversal's workspace
 // row), for the parent-major path:
 //   1. a sample of 128 scores (all of them when C <= 128), sorted, gives t0,
-//      the j-th largest sample value with j chosen so that about 1.5 K + 3
-//      sample-strides of scores lie above it: t0 <= t (the K-th largest score)
-//      unless fewer than K scores are >= t0, which the pass counts;
+//      the j-th largest sample value with j = ceil(1.25 K 128 / C) + 2, so
+//      that about 1.25 K scores are expected above it: t0 <= t (the K-th
+//      largest score) unless fewer than K scores are >= t0, which the pass
+//      counts;
 //   2. the pass collects every candidate with f >= fl_down(t0 - 2E) and counts
 //      those >= t0;
 //   3. with at least K counted (so t >= t0), every candidate of the band
@@ -1165,7 +1166,7 @@ __device__ __forceinline__ bool warp_select_pm(const DescendParams &p, int L, lo
         for (int e = 0; e < 4; ++e) col[lane * 4 + e] = sv[e];
         ncol = C;
     } else {
-        const int j = (3 * K * 128 + 2 * C - 1) / (2 * C) + 3;
+        const int j = (5 * K * 128 + 4 * C - 1) / (4 * C) + 2;
         if (j > 127) return fallback();
         const uint64_t kj0 = __shfl_sync(0xffffffffu, sv[0], j >> 2), kj1 = __shfl_sync(0xffffffffu, sv[1], j >> 2);
         const uint64_t kj2 = __shfl_sync(0xffffffffu, sv[2], j >> 2), kj3 = __shfl_sync(0xffffffffu, sv[3], j >> 2);
