@@ -1104,10 +1104,28 @@ __device__ __noinline__ bool warp_select_defer_call(const DescendParams &p, int 
     return warp_select<T, D, true>(p, L, bh, cpre, prev_sh, hist, tmp, kbuf, f, xs, queue, qcount);
 }
 
+// The k-th largest (1-based) of the warp's 32 E order-preserving float keys,
+// k at most the number of real keys (padding keys are 0, below every real
+// one): MSB-first, keep each bit while at least k keys are >= the prefix.
+template <int E>
+__device__ __forceinline__ uint32_t warp_kth_key(const uint32_t (&key)[E], int k)
+{
+    uint32_t t = 0;
+#pragma unroll 1
+    for (int b = 31; b >= 0; --b) {
+        const uint32_t c = t | (1u << b);
+        unsigned cnt = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) cnt += key[e] >= c;
+        if (__reduce_add_sync(0xffffffffu, cnt) >= (unsigned)k) t = c;
+    }
+    return t;
+}
+
 // Tier 1 in one pass over the scores (read from the traversal's workspace
 // row), for the parent-major path:
-//   1. a sample of 128 scores (all of them when C <= 128), sorted, gives t0,
-//      the j-th largest sample value with j = ceil(1.25 K 128 / C) + 2, so
+//   1. a sample of 128 scores (all of them when C <= 128) gives t0, the j-th
+//      largest sample value (a radix select) with j = ceil(1.25 K 128 / C) + 2, so
 //      that about 1.25 K scores are expected above it: t0 <= t (the K-th
 //      largest score) unless fewer than K scores are >= t0, which the pass
 //      counts;
@@ -1115,8 +1133,9 @@ __device__ __noinline__ bool warp_select_defer_call(const DescendParams &p, int 
 //      those >= t0;
 //   3. with at least K counted (so t >= t0), every candidate of the band
 //      [t - 2E, t + 2E] and above was collected: t is the K-th largest of the
-//      collected, which are sorted; the sorted prefix above t + 2E is kept for
-//      sure, the next ones down to t - 2E are the band.
+//      collected (a radix select over their order-preserving keys); those
+//      above t + 2E are kept for sure, those down to t - 2E are the band.
+//      (With C <= 128 the sample is every score: t comes from it directly.)
 // Non-finite scores, too many collected (more than kCollectCap) or too few
 // counted fall back to warp_select on the same row.  The certified band and
 // the refinement are those of warp_select, so the kept sets are the same.
@@ -1148,35 +1167,30 @@ __device__ __forceinline__ bool warp_select_pm(const DescendParams &p, int L, lo
 
     // ---- 1. the sample threshold (all scores when C <= 128) ----
     const bool all = C <= 128;
-    uint64_t sv[4];
+    uint32_t skey[4];
+    float sval[4];
     int bad = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         const int i = lane * 4 + e;
         const int idx = all ? i : (int)(((long long)i * C) >> 7);
-        const float v = (!all || i < C) ? __ldcg(f + idx) : -INFINITY;
-        bad |= (!all || i < C) && !isfinite(v);
-        sv[e] = ((uint64_t)(~float_key(v)) << 32) | (uint32_t)idx;   // ascending keys: descending values
+        sval[e] = (!all || i < C) ? __ldcg(f + idx) : -INFINITY;
+        bad |= (!all || i < C) && !isfinite(sval[e]);
+        skey[e] = float_key(sval[e]);
     }
     if (__any_sync(0xffffffffu, bad)) return fallback();
-    reg_bitonic<4>(sv);
-    int ncol;
-    if (all) {   // every score is in the sorted sample: it is the collected set
-#pragma unroll
-        for (int e = 0; e < 4; ++e) col[lane * 4 + e] = sv[e];
-        ncol = C;
+    float t;
+    int ncol = 0;
+    if (all) {   // every score is in the sample: t is exact
+        t = key_float(warp_kth_key<4>(skey, K));
     } else {
         const int j = (5 * K * 128 + 4 * C - 1) / (4 * C) + 2;
         if (j > 127) return fallback();
-        const uint64_t kj0 = __shfl_sync(0xffffffffu, sv[0], j >> 2), kj1 = __shfl_sync(0xffffffffu, sv[1], j >> 2);
-        const uint64_t kj2 = __shfl_sync(0xffffffffu, sv[2], j >> 2), kj3 = __shfl_sync(0xffffffffu, sv[3], j >> 2);
-        const uint64_t kj = (j & 3) == 0 ? kj0 : (j & 3) == 1 ? kj1 : (j & 3) == 2 ? kj2 : kj3;
-        const float t0 = key_float(~(uint32_t)(kj >> 32));
+        const float t0 = key_float(warp_kth_key<4>(skey, j + 1));
         const float c_lo = __double2float_rd(__dsub_rd((double)t0, 2.0 * E));
 
         // ---- 2. one pass: collect, count, check (four 16-byte loads in flight per lane) ----
         int cnt = 0;
-        ncol = 0;
         const float4 *f4 = reinterpret_cast<const float4 *>(f);
         const int nv = (C + 3) >> 2;
         for (int b4 = 0; b4 < nv; b4 += 128) {
@@ -1205,60 +1219,75 @@ __device__ __forceinline__ bool warp_select_pm(const DescendParams &p, int L, lo
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                     if (take[q]) {
-                        if (off < kCollectCap)
-                            col[off] = ((uint64_t)(~float_key(e[q])) << 32) | (uint32_t)(4 * v4 + q);
+                        if (off < kCollectCap) col[off] = ((uint64_t)float_key(e[q]) << 32) | (uint32_t)(4 * v4 + q);
                         ++off;
                     }
                 ncol += tot;
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        cnt = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt);
         bad = __any_sync(0xffffffffu, bad);
         if (bad || !isfinite(t0) || cnt < K || ncol > kCollectCap) return fallback();
         __syncwarp();
 
-        // ---- 3. the collected, sorted ----
-        auto sort_reg = [&](auto tag) {
-            constexpr int EE = decltype(tag)::value;
-            uint64_t v[EE];
+        // ---- 3. t: the K-th largest of the collected ----
+        if (ncol <= 256) {
+            uint32_t key[8];
 #pragma unroll
-            for (int e = 0; e < EE; ++e) v[e] = lane * EE + e < ncol ? col[lane * EE + e] : ~0ull;
-            reg_bitonic<EE>(v);
-            __syncwarp();
-#pragma unroll
-            for (int e = 0; e < EE; ++e) col[lane * EE + e] = v[e];
-        };
-        if (ncol <= 64) {
-            sort_reg(std::integral_constant<int, 2>());
-        } else if (ncol <= 128) {
-            sort_reg(std::integral_constant<int, 4>());
-        } else if (ncol <= 256) {
-            sort_reg(std::integral_constant<int, 8>());
+            for (int e = 0; e < 8; ++e) key[e] = lane * 8 + e < ncol ? (uint32_t)(col[lane * 8 + e] >> 32) : 0u;
+            t = key_float(warp_kth_key<8>(key, K));
         } else {
-            int n2 = 512;
-            for (int i = ncol + lane; i < n2; i += 32) col[i] = ~0ull;
-            __syncwarp();
-            warp_sort_u64(col, n2);
+            uint32_t key[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) key[e] = lane * 16 + e < ncol ? (uint32_t)(col[lane * 16 + e] >> 32) : 0u;
+            t = key_float(warp_kth_key<16>(key, K));
         }
     }
-    __syncwarp();
-    // the K-th largest; the sure prefix above t + 2E and the band down to t - 2E
-    const float t = key_float(~(uint32_t)(col[K - 1] >> 32));
+    // the sure set above t + 2E (positions into kbuf) and the band down to
+    // t - 2E (positions compacted to the front of col)
     const float hi32 = __double2float_ru(__dadd_ru((double)t, 2.0 * E));
     const float lo32 = __double2float_rd(__dsub_rd((double)t, 2.0 * E));
     int n_in = 0, nA = 0;
-    for (int i0 = 0; i0 < ncol; i0 += 32) {
-        const int i = i0 + lane;
-        const float v = i < ncol ? key_float(~(uint32_t)(col[i] >> 32)) : -INFINITY;
-        n_in += __popc(__ballot_sync(0xffffffffu, i < ncol && v > hi32));
-        nA += __popc(__ballot_sync(0xffffffffu, i < ncol && v <= hi32 && v >= lo32));
+    if (all) {
+        int c_in = 0, c_b = 0;
+        bool sin[4], sb[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const bool valid = lane * 4 + e < C;
+            sin[e] = valid && sval[e] > hi32;
+            sb[e] = valid && !sin[e] && sval[e] >= lo32;
+            c_in += sin[e];
+            c_b += sb[e];
+        }
+        int tot;
+        const int pre = warp_excl_scan(c_in | (c_b << 16), tot);
+        int o1 = pre & 0xffff, o2 = pre >> 16;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (sin[e]) kbuf[o1++] = (uint32_t)(lane * 4 + e);
+            if (sb[e]) col[o2++] = (uint32_t)(lane * 4 + e);
+        }
+        n_in = tot & 0xffff;
+        nA = tot >> 16;
+    } else {
+        for (int i0 = 0; i0 < ncol; i0 += 32) {
+            const int i = i0 + lane;
+            const uint64_t ent = i < ncol ? col[i] : 0ull;
+            const float v = key_float((uint32_t)(ent >> 32));
+            const bool sin = i < ncol && v > hi32;
+            const bool sb = i < ncol && !sin && v >= lo32;
+            const unsigned mi = __ballot_sync(0xffffffffu, sin), mb = __ballot_sync(0xffffffffu, sb);
+            if (sin) kbuf[n_in + __popc(mi & lanemask_lt())] = (uint32_t)ent;
+            if (sb) col[nA + __popc(mb & lanemask_lt())] = (uint32_t)ent;   // at or below i: already read
+            n_in += __popc(mi);
+            nA += __popc(mb);
+        }
     }
+    __syncwarp();
     if (p.stats && lane == 0) atomicAdd(p.stats + L * 4, 1ull);
     const int r = K - n_in;
-    for (int i = lane; i < n_in; i += 32) kbuf[i] = (uint32_t)col[i];
     if (nA == r) {   // every band candidate is kept
-        for (int i = lane; i < nA; i += 32) kbuf[n_in + i] = (uint32_t)col[n_in + i];
+        for (int i = lane; i < nA; i += 32) kbuf[n_in + i] = (uint32_t)col[i];
         __syncwarp();
         resolve_ids(K);
         write_kept(p, lv, L, bh, kbuf, K);
@@ -1273,7 +1302,7 @@ __device__ __forceinline__ bool warp_select_pm(const DescendParams &p, int L, lo
     int nsel = n_in, rr = r, nl = nA;
     const int *lst = reinterpret_cast<const int *>(hist);
     if (nA <= 32) {
-        if (lane < nA) hist[lane] = (uint32_t)col[n_in + lane];
+        if (lane < nA) hist[lane] = (uint32_t)col[lane];
         __syncwarp();
         if (refine_tier2<T, D>(p, lv, bh, kbuf, nsel, rr, lst, nl, xs)) {
             write_kept(p, lv, L, bh, kbuf, K);
@@ -1288,7 +1317,7 @@ __device__ __forceinline__ bool warp_select_pm(const DescendParams &p, int L, lo
     if (nA <= 32) {
         for (int i = lane; i < nl; i += 32) glist[i] = lst[i];
     } else {
-        for (int i = lane; i < nA; i += 32) glist[i] = (int)(uint32_t)col[n_in + i];
+        for (int i = lane; i < nA; i += 32) glist[i] = (int)(uint32_t)col[i];
     }
     if (gk != kbuf)
         for (int i = lane; i < nsel; i += 32) gk[i] = kbuf[i];
