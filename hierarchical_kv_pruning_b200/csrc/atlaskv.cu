@@ -587,8 +587,11 @@ atlaskv_status run_pm(const atlaskv_tree *t, const PmPlan &pp, const akv::Descen
     if (BH == 0) return ATLASKV_OK;
     const akv::PmLevel none{};
     const size_t sel_smem = (size_t)pp.nsel * pp.pw;
-    AKV_SMEM((akv::pm_select_kernel<T, D>), sel_smem);
+    AKV_SMEM((akv::pm_select_kernel<T, D, 2>), sel_smem);
+    AKV_SMEM((akv::pm_select_kernel<T, D, 3>), sel_smem);
     const unsigned sel_grid = (unsigned)((BH + pp.nsel - 1) / pp.nsel);
+    // more traversals than one wave of 2 CTAs per SM: the 3-CTA register budget
+    const bool sel3 = (long long)sel_grid > 2LL * t->num_sms;
     const size_t score_smem = akv::pm_score_smem(D, (int)sizeof(T));
     AKV_SMEM((akv::pm_score_kernel<T, D>), score_smem);
     // the scoring grid: as many CTAs as fit on the device at once (the warps loop over the items)
@@ -605,8 +608,12 @@ atlaskv_status run_pm(const atlaskv_tree *t, const PmPlan &pp, const akv::Descen
     const unsigned ref_grid = (unsigned)std::min<long long>((BH + 7) / 8, (long long)t->num_sms * 2);
     auto select = [&](int L) -> atlaskv_status {
         const akv::PmLevel &nx = L + 1 < nl ? lv[L + 1] : none;
-        AKV_TRY(launch_pdl(akv::pm_select_kernel<T, D>, sel_grid, akv::kSelThreads, sel_smem, s, dp, lv[L], nx, L,
-                           pp.nsel, pp.pw));
+        if (sel3)
+            AKV_TRY(launch_pdl(akv::pm_select_kernel<T, D, 3>, sel_grid, akv::kSelThreads, sel_smem, s, dp, lv[L], nx,
+                               L, pp.nsel, pp.pw));
+        else
+            AKV_TRY(launch_pdl(akv::pm_select_kernel<T, D, 2>, sel_grid, akv::kSelThreads, sel_smem, s, dp, lv[L], nx,
+                               L, pp.nsel, pp.pw));
         AKV_TRY(launch_pdl(akv::pm_refine_kernel<T, D>, ref_grid, akv::kSelThreads, ref_smem, s, dp, lv[L], nx, L));
         return ATLASKV_OK;
     };

@@ -466,8 +466,11 @@ __global__ void __launch_bounds__(kSelThreads, 1)
     }
 }
 
-template <typename T, int D>
-__global__ void __launch_bounds__(kSelThreads, 2)
+// MINB: CTAs per SM the registers are budgeted for (2: 128 registers, the
+// fastest per warp; 3: 80, more warps resident when the traversals exceed one
+// wave).
+template <typename T, int D, int MINB>
+__global__ void __launch_bounds__(kSelThreads, MINB)
     pm_select_kernel(const __grid_constant__ DescendParams p0, const __grid_constant__ PmLevel self,
                      const __grid_constant__ PmLevel nx, int L, int nsel, int pw)
 {
