@@ -27,10 +27,11 @@ BF16_TOL = 2e-2
 LSE_TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-3}
 
 
-def gpu_run(w, K, scale=0.0, tree=None):
+def gpu_run(w, K, scale=0.0, tree=None, descent=0):
     own = tree is None
     if own:
         tree = HikvpTree.from_workload(w)
+        tree.set_descent(descent)
     r = tree.attend(w.q_kg, w.q_seq, w.k_seq, w.v_seq, K, scale=scale)
     tree.sync_status()
     out = {k: (v.cpu() if torch.is_tensor(v) and k != "workspace" else v) for k, v in r.items()}
@@ -168,30 +169,37 @@ def test_scale_argument():
     compare(w, sh.keep, g, scale=0.05)
 
 
-def test_all_keys_identical_mass_ties():
+DESCENTS = pytest.mark.parametrize("descent", [1, 2], ids=["fused", "parent_major"])
+
+
+@DESCENTS
+def test_all_keys_identical_mass_ties(descent):
     # Every score ties exactly; more ambiguous candidates than one refinement
-    # chunk: the lowest row ids must win at every level.
+    # chunk: the lowest row ids must win at every level (parent-major: the
+    # selection's fallback and the queued exact tier).
     sh = synth.custom(dtype=torch.bfloat16, n_heads=2, n_kv_heads=1, head_dim=128, fanout=(40, 30, 20),
                       keep=(5, 70, 150), batch=2, n_tokens=4, seq_len=8, permuted=True)
     w = synth.make_workload(sh, "cuda", 9)
     for t in (w.root_keys, w.mid_keys, w.leaf_keys):
         t.copy_(w.leaf_keys[0, 0].expand_as(t))
-    g = gpu_run(w, sh.keep)
+    g = gpu_run(w, sh.keep, descent=descent)
     compare(w, sh.keep, g)
     assert g["kept_root"][0, 0].tolist() == list(range(5))
 
 
-def test_zero_queries():
+@DESCENTS
+def test_zero_queries(descent):
     sh = synth.custom(dtype=torch.bfloat16, n_heads=2, n_kv_heads=1, head_dim=128, fanout=(8, 8, 8),
                       keep=(3, 5, 7), batch=2, n_tokens=4, seq_len=8)
     w = synth.make_workload(sh, "cuda", 10)
     w.q_kg.zero_()
-    g = gpu_run(w, sh.keep)
+    g = gpu_run(w, sh.keep, descent=descent)
     compare(w, sh.keep, g)
     assert g["kept_leaf"][0, 0].tolist() == list(range(7))
 
 
-def test_near_ties_need_exact_arithmetic():
+@DESCENTS
+def test_near_ties_need_exact_arithmetic(descent):
     # Pairs of float32 keys that differ in one component by one unit in the
     # last place, and duplicated keys: the fp32 filter cannot order them,
     # exact arithmetic must.
@@ -207,7 +215,7 @@ def test_near_ties_need_exact_arithmetic():
             k[i, j] = torch.nextafter(k[i - 1, j], torch.tensor(float("inf"), device=k.device))
         for i in range(3, n, 7):
             k[i] = k[i - 3]
-    g = gpu_run(w, sh.keep)
+    g = gpu_run(w, sh.keep, descent=descent)
     compare(w, sh.keep, g)
 
 
@@ -401,11 +409,15 @@ def test_layers_fp32_and_mismatch_rejected():
             t.close()
 
 
-def test_deterministic_and_b0():
+@DESCENTS
+def test_deterministic_and_b0(descent):
+    # the parent-major path groups traversals with atomics: its results must
+    # not depend on the order they land in
     sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(10, 10, 10),
                       keep=(3, 4, 16), batch=4, n_tokens=32, seq_len=64)
     w = synth.make_workload(sh, "cuda", 13)
     with HikvpTree.from_workload(w) as tree:
+        tree.set_descent(descent)
         a = gpu_run(w, sh.keep, tree=tree)
         b = gpu_run(w, sh.keep, tree=tree)
         for k in ("kept_root", "kept_mid", "kept_leaf", "out", "lse"):
