@@ -226,7 +226,7 @@ constexpr size_t kPmSelBudget = 56 * 1024;   // selection CTA's shared memory (s
 
 struct PmPlan {
     bool ok = false;               // supported for this call
-    int HT = 0, EC = 0;            // traversals per warp / per work item
+    int EC = 0;                    // traversals per scoring work item
     int nsel = 0, pw = 0;          // selection: warps per CTA, shared bytes per warp
     int ts_GC = 0;                 // token sums: heads per CTA
     size_t ts_smem = 0;
@@ -239,15 +239,14 @@ struct PmPlan {
 
 size_t r16(size_t b) { return (b + 15) & ~size_t(15); }
 
-PmPlan plan_pm(const atlaskv_tree *t, const Ks &ks, long long Bc, int H, int kcap, int cap)
+PmPlan plan_pm(const atlaskv_tree *t, const Ks &ks, long long Bc, int H, int kcap)
 {
     PmPlan pp;
     const int D = t->d.head_dim;
     const int esz = (int)(t->d.dtype == ATLASKV_F32 ? 4 : 2);
     const int G = H / t->d.n_kv_heads;
-    pp.HT = akv::kPmEC;
     pp.EC = akv::kPmEC;
-    const size_t pw = akv::pm_select_warp_bytes(kcap, cap, kp_max(ks));
+    const size_t pw = akv::pm_select_warp_bytes(kcap, kp_max(ks));
     if (pw > 200 * 1024) return pp;
     pp.pw = (int)pw;
     pp.nsel = (int)std::max<size_t>(1, std::min<size_t>(8, kPmSelBudget / pw));
@@ -381,7 +380,7 @@ Layout plan(const atlaskv_tree *t, const Ks &ks, int B, int N, int H, int T, boo
     L.desc = plan_descent(G, ks, L.kcap, L.cap, D, (int)esize(t->d.dtype), (long long)chunk_b * t->d.n_kv_heads,
                           t->num_sms);
     const int gc = L.desc.GC > 0 ? L.desc.GC : 1;
-    L.pmp = plan_pm(t, ks, chunk_b, H, L.kcap, L.cap);
+    L.pmp = plan_pm(t, ks, chunk_b, H, L.kcap);
     L.pm = allow_pm && use_pm(t, L.pmp.ok, L.desc.GC > 0, (long long)B * H);
     // refinement scratch: one slot per selecting warp of every descent CTA
     // (parent-major: one per traversal)
@@ -453,7 +452,7 @@ atlaskv_status check_params(const atlaskv_tree *t, const Ks &ks, int B, int N, i
                                        (int)esize(t->d.dtype), (long long)B * t->d.n_kv_heads, t->num_sms)
                               .GC > 0;
     const int nc = t->host_leaves ? query_chunks(B) : 1;
-    const bool pm_ok = plan_pm(t, ks, (B + nc - 1) / nc, H, kcap, score_cap(t, ks)).ok;
+    const bool pm_ok = plan_pm(t, ks, (B + nc - 1) / nc, H, kcap).ok;
     if (t->descent_mode == ATLASKV_DESCENT_FUSED && !fused_ok)
         return fail(ATLASKV_EUNSUPPORTED, "the fused descent's shared-memory plan does not fit for these K");
     if (t->descent_mode == ATLASKV_DESCENT_PARENT_MAJOR && !pm_ok)
@@ -570,7 +569,7 @@ atlaskv_status launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned bloc
 // selection when first = 0; then per level the inversion of the kept parents
 // (scan, fill), the scores by parent and the selection.  Each selection but
 // the last level's counts its kept entries for the next level's inversion.
-#define AKV_TRY(x)                                 \
+#define AKV_RET(x)                                 \
     do {                                           \
         const atlaskv_status st_ = (x);            \
         if (st_ != ATLASKV_OK) return st_;         \
@@ -592,7 +591,7 @@ atlaskv_status run_pm(const atlaskv_tree *t, const PmPlan &pp, const akv::Descen
     const unsigned sel_grid = (unsigned)((BH + pp.nsel - 1) / pp.nsel);
     // more traversals than one wave of 2 CTAs per SM: the 3-CTA register budget
     const bool sel3 = (long long)sel_grid > 2LL * t->num_sms;
-    const size_t score_smem = akv::pm_score_smem(D, (int)sizeof(T));
+    const size_t score_smem = akv::pm_score_smem((int)sizeof(T));
     AKV_SMEM((akv::pm_score_kernel<T, D>), score_smem);
     // the scoring grid: as many CTAs as fit on the device at once (the warps loop over the items)
     static thread_local std::map<std::pair<const void *, int>, int> fit;
@@ -609,34 +608,34 @@ atlaskv_status run_pm(const atlaskv_tree *t, const PmPlan &pp, const akv::Descen
     auto select = [&](int L) -> atlaskv_status {
         const akv::PmLevel &nx = L + 1 < nl ? lv[L + 1] : none;
         if (sel3)
-            AKV_TRY(launch_pdl(akv::pm_select_kernel<T, D, 3>, sel_grid, akv::kSelThreads, sel_smem, s, dp, lv[L], nx,
+            AKV_RET(launch_pdl(akv::pm_select_kernel<T, D, 3>, sel_grid, akv::kSelThreads, sel_smem, s, dp, lv[L], nx,
                                L, pp.nsel, pp.pw));
         else
-            AKV_TRY(launch_pdl(akv::pm_select_kernel<T, D, 2>, sel_grid, akv::kSelThreads, sel_smem, s, dp, lv[L], nx,
+            AKV_RET(launch_pdl(akv::pm_select_kernel<T, D, 2>, sel_grid, akv::kSelThreads, sel_smem, s, dp, lv[L], nx,
                                L, pp.nsel, pp.pw));
-        AKV_TRY(launch_pdl(akv::pm_refine_kernel<T, D>, ref_grid, akv::kSelThreads, ref_smem, s, dp, lv[L], nx, L));
+        AKV_RET(launch_pdl(akv::pm_refine_kernel<T, D>, ref_grid, akv::kSelThreads, ref_smem, s, dp, lv[L], nx, L));
         return ATLASKV_OK;
     };
     if (first == 0) {
         const long long tsg = (long long)dp.B * dp.H_kv * (dp.G / pp.ts_GC);
-        AKV_TRY(launch_pdl(akv::token_sums_kernel<T, D>, (unsigned)tsg, akv::kDescThreads, pp.ts_smem, s, dp, pp.ts_GC,
+        AKV_RET(launch_pdl(akv::token_sums_kernel<T, D>, (unsigned)tsg, akv::kDescThreads, pp.ts_smem, s, dp, pp.ts_GC,
                            reinterpret_cast<uint4 *>(zero), (long long)(zero_bytes / 16)));
         const long long items = (long long)dp.H_kv * ((dp.B * dp.G + pp.EC - 1) / pp.EC);
-        AKV_TRY(launch_pdl(akv::pm_score_kernel<T, D>,
+        AKV_RET(launch_pdl(akv::pm_score_kernel<T, D>,
                            (unsigned)std::min((items + akv::kPmWarps - 1) / akv::kPmWarps, score_cap), akv::kPmThreads,
                            score_smem, s, dp, none, 0));
-        AKV_TRY(select(0));
+        AKV_RET(select(0));
     }
     for (int L = std::max(first, 1); L <= last; ++L) {
         const akv::PmLevel &v = lv[L];
-        AKV_TRY(launch_pdl(akv::pm_scan_kernel, (unsigned)v.n_tiles, akv::kScanThreads, 0, s, v, pp.EC, dp.status));
+        AKV_RET(launch_pdl(akv::pm_scan_kernel, (unsigned)v.n_tiles, akv::kScanThreads, 0, s, v, pp.EC, dp.status));
         const unsigned fg = (unsigned)std::min<long long>((v.E + 255) / 256, (long long)t->num_sms * 8);
-        AKV_TRY(launch_pdl(akv::pm_fill_kernel, std::max(1u, fg), 256, 0, s, (const int32_t *)dp.kept[L - 1],
+        AKV_RET(launch_pdl(akv::pm_fill_kernel, std::max(1u, fg), 256, 0, s, (const int32_t *)dp.kept[L - 1],
                            dp.K[L - 1], dp.H, dp.G, (long long)dp.rows[L - 1], v, dp.status));
-        AKV_TRY(launch_pdl(akv::pm_score_kernel<T, D>,
+        AKV_RET(launch_pdl(akv::pm_score_kernel<T, D>,
                            (unsigned)std::min<long long>((v.max_items + akv::kPmWarps - 1) / akv::kPmWarps, score_cap),
                            akv::kPmThreads, score_smem, s, dp, v, L));
-        AKV_TRY(select(L));
+        AKV_RET(select(L));
     }
     return ATLASKV_OK;
 }

@@ -841,7 +841,6 @@ __device__ __noinline__ void warp_refine(const DescendParams &p, const LevelView
                                          ExactScratch &sc)
 {
     constexpr int RC = kRefineChunk;
-    constexpr int EV = Vec16<T>::E;
     const int lane = threadIdx.x & 31;
     const int K = p.K[L];
     int r = K - nsel;

@@ -33,8 +33,6 @@ namespace akv {
 
 constexpr int kPmThreads = 128;                 // scoring CTA: 4 warps, one ring each
 constexpr int kPmWarps = kPmThreads / 32;
-constexpr int kPmPassRows = 1024;               // child rows whose table is built at a time
-constexpr int kPmMaxEC = 32;                    // traversals per work item, at most
 constexpr int kScanThreads = 256;
 constexpr int kScanPerThread = 8;
 constexpr int kScanTile = kScanThreads * kScanPerThread;
@@ -134,9 +132,9 @@ __host__ __device__ constexpr size_t pm_stage_bytes(int esz)
 {
     return (size_t)kPmRP * kPmSlice + (size_t)kPmEC * (kPmSlice / esz) * 4;
 }
-__host__ __device__ constexpr size_t pm_score_smem(int D, int esz)
+__host__ __device__ constexpr size_t pm_score_smem(int esz)
 {
-    return (size_t)kPmWarps * 2 * pm_stage_bytes(esz) + 0 * D;
+    return (size_t)kPmWarps * 2 * pm_stage_bytes(esz);
 }
 
 // One item as a warp sees it: every lane holds the item's fields and, lane
@@ -386,10 +384,9 @@ __global__ void __launch_bounds__(kPmThreads, 3)
 // (CSR) their candidate prefix.  With nx.cnt set, the warp then counts its
 // kept entries per key for the next level (nx) and, on a CSR next level,
 // writes their candidate prefix.
-__host__ __device__ constexpr size_t pm_select_warp_bytes(int kcap, int cap, int Kpmax)
+__host__ __device__ constexpr size_t pm_select_warp_bytes(int kcap, int Kpmax)
 {
-    return (warp_sel_bytes(kcap, 0) + (size_t)kCollectCap * 8 + (size_t)(2 * Kpmax + 2) * 4 + 15 + 0 * cap) &
-           ~size_t(15);
+    return (warp_sel_bytes(kcap, 0) + (size_t)kCollectCap * 8 + (size_t)(2 * Kpmax + 2) * 4 + 15) & ~size_t(15);
 }
 
 // Counts traversal bh's kept entries of level L per key of the next level's
