@@ -351,9 +351,12 @@ def host_memory_ok(sh):
 def roofline_of(sh, alg, st, ms_per_step, peaks, peak_src, link_gbs, descent="auto"):
     """Rooflines from the algorithmic bytes and the per-launch stage times
     (CUDA events on each kernel's own stream, averaged over the stage pass).
-    The headline is the kernel with the largest time; `kernels` lists each
-    launch kind; `step` is the whole step against HBM (and, with host leaves,
-    the staged bytes against the host link)."""
+    Leaves in HBM: the headline is the whole step against HBM (descent and
+    attention bytes over the step time), `dominant` the stage with the largest
+    time.  Host-resident leaves: the headline is the staging against the host
+    link (the streams overlap).  `kernels` lists each stage; `step` is the
+    whole step against HBM (and, with host leaves, the staged bytes against
+    the host link)."""
     import torch
     hbm = peaks["hbm_gbs"]
     kernels = {}
@@ -390,13 +393,20 @@ def roofline_of(sh, alg, st, ms_per_step, peaks, peak_src, link_gbs, descent="au
                              "frac": link_ach / link_gbs}
         top = dict(kernels["staging"])
         top["bound"] = "host_link"
+        top["traffic"] = None   # host-link bytes are not DRAM counters
     else:
+        # the headline is the whole step against HBM (its stages run one after
+        # the other); the stage with the largest time is kept as `dominant`
         name = max(kernels, key=lambda k: kernels[k]["ms"])
-        top = dict(kernels[name])
-        top["peak"] = hbm
+        dom = dict(kernels[name])
+        dom["peak"] = hbm
+        dom["traffic"] = profiled_traffic(dom["kernel"].split(" ")[0], sh.name)
+        parts = [profiled_traffic(kernels[k]["kernel"].split(" ")[0], sh.name) for k in kernels]
+        top = {"kernel": "whole step (descent + attention)", "bound": "hbm", "achieved": step["achieved"],
+               "peak": hbm, "unit": "GB/s", "frac": step["frac"], "algorithmic_bytes": step_bytes,
+               "ms": ms_per_step, "traffic": sum(parts) if parts and None not in parts else None,
+               "dominant": dom}
         top["peak_source"] = peak_src + " (burst)"
-    kname = top["kernel"].split(" ")[0]
-    top["traffic"] = profiled_traffic(kname, sh.name)
     attend_ms = st["attend"]
     tflops = alg["attend_flops"] / (attend_ms * 1e-3) / 1e12 if attend_ms > 0 else None
     top.update({"kernels": kernels, "step": step, "stage_ms": {k: round(v, 5) for k, v in st.items()},

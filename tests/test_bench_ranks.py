@@ -196,3 +196,20 @@ def test_reference_arm_contract():
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["config"]["workload"] == "tiny_fp32_10x10x10"
     r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, env=dict(env, RANK="1"), cwd=ROOT)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_headline_roofline_is_the_whole_step():
+    # leaves in HBM: frac = (descent + attention bytes) / step time / peak;
+    # the slowest stage is reported beside it, not instead of it
+    from hierarchical_kv_pruning_b200 import synth
+    sh = synth.shape(2)
+    alg = {"descend": 200e6, "attend": 400e6, "attend_seq": 300e6, "attend_leaf": 100e6, "attend_flops": 7e10,
+           "staging": 0}
+    st = {"descend": 0.25, "staging": 0.0, "attend": 0.15, "attend_seq": 0.0, "attend_leaf": 0.15}
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0}
+    top = bench.roofline_of(sh, alg, st, 0.4, peaks, "measured", 50.0)
+    assert top["frac"] == pytest.approx(600e6 / 0.4e-3 / 1e9 / 6000.0)
+    assert top["kernel"].startswith("whole step") and top["bound"] == "hbm"
+    assert top["dominant"]["kernel"].startswith("descent")
+    assert top["dominant"]["frac"] == pytest.approx(200e6 / 0.25e-3 / 1e9 / 6000.0)
+    assert set(top["kernels"]) == {"descend", "attend"}
