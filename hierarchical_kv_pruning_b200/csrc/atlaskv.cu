@@ -679,11 +679,11 @@ atlaskv_status launch_attend_f32(const akv::AttnParams &ap, cudaStream_t s)
     return ATLASKV_OK;
 }
 
-// Tensor map of a sequence K or V tensor [B][T][H_kv][D] (bf16, D = 128) for
-// the attention kernel: dims (D, H_kv, T, B), box (64, 1, 64, 1), 128-byte
-// swizzle, zero fill outside.  cuTensorMapEncodeTiled is a host-only call,
-// reached through the runtime's driver entry point.
-atlaskv_status encode_seq_map(CUtensorMap *map, const void *base, int B, int T, int H_kv)
+// 4-D tensor map (bf16, 128-byte swizzle, zero fill outside) over a tensor
+// [d3][d2][d1][D] (D = 128 innermost) with a (64, 1, rows, 1) box, for the
+// attention kernel.  cuTensorMapEncodeTiled is a host-only call, reached
+// through the runtime's driver entry point.
+atlaskv_status encode_tc_map(CUtensorMap *map, const void *base, long long d1, long long d2, long long d3, int rows)
 {
     // looked up once per process (thread-safe static initialisation)
     static const PFN_cuTensorMapEncodeTiled_v12000 encode = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
@@ -695,11 +695,11 @@ atlaskv_status encode_seq_map(CUtensorMap *map, const void *base, int B, int T, 
         return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }();
     if (!encode) return fail(ATLASKV_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
-    if (reinterpret_cast<uintptr_t>(base) & 15u) return fail(ATLASKV_EINVAL, "sequence K/V must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(base) & 15u) return fail(ATLASKV_EINVAL, "attention inputs must be 16-byte aligned");
     const int D = akv::tc::kD;
-    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H_kv, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H_kv * D * 2, (cuuint64_t)T * H_kv * D * 2};
-    const cuuint32_t box[4] = {64, 1, (cuuint32_t)akv::tc::kKeys, 1};
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)d1, (cuuint64_t)d2, (cuuint64_t)d3};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)(d1 * D * 2), (cuuint64_t)(d2 * d1 * D * 2)};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -709,7 +709,10 @@ atlaskv_status encode_seq_map(CUtensorMap *map, const void *base, int B, int T, 
 }
 
 // bf16, D = 128: tcgen05 tensor cores, one CTA per kWG x 128 query rows of a
-// (query, KV head) group, sequence tiles by TMA.
+// (query, KV head) group.  Sequence K / V [B][T][H_kv][D] by TMA (box of 64
+// keys); Q [B][N][H][D] by TMA too (box of min(N, 128) tokens of one head)
+// when every head's rows start on a swizzle atom of the Q tile, i.e. N is a
+// multiple of 8 that divides 128 or is divisible by it, else by cp.async.
 atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
 {
     const int rows = ap.G * ap.N;
@@ -718,13 +721,28 @@ atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
     if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "attention grid too large");
     if (ap.lk_rows >= (1LL << 31) || ap.lv_rows >= (1LL << 31))
         return fail(ATLASKV_EUNSUPPORTED, "more than 2^31 leaf rows");
-    CUtensorMap mk, mv;
-    atlaskv_status st = encode_seq_map(&mk, ap.k_seq, ap.B, ap.T, ap.H_kv);
+    CUtensorMap mk, mv, mqs, mqk;
+    atlaskv_status st = encode_tc_map(&mk, ap.k_seq, ap.H_kv, ap.T, ap.B, akv::tc::kKeys);
     if (st != ATLASKV_OK) return st;
-    st = encode_seq_map(&mv, ap.v_seq, ap.B, ap.T, ap.H_kv);
+    st = encode_tc_map(&mv, ap.v_seq, ap.H_kv, ap.T, ap.B, akv::tc::kKeys);
     if (st != ATLASKV_OK) return st;
+    // a mode that reads only one of the two query tensors uses it for both maps
+    const void *qs = ap.q_seq ? ap.q_seq : ap.q_kg, *qk = ap.q_kg ? ap.q_kg : ap.q_seq;
+    const auto aligned = [](const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    int q_maps = ap.N % 8 == 0 && (128 % ap.N == 0 || ap.N % 128 == 0) && aligned(qs) && aligned(qk);
+    if (q_maps) {
+        const int bn = ap.N < akv::tc::kRows ? ap.N : akv::tc::kRows;
+        st = encode_tc_map(&mqs, qs, ap.H, ap.N, ap.B, bn);
+        if (st != ATLASKV_OK) return st;
+        st = encode_tc_map(&mqk, qk, ap.H, ap.N, ap.B, bn);
+        if (st != ATLASKV_OK) return st;
+    } else {
+        mqs = mk;   // unused
+        mqk = mk;
+    }
     AKV_SMEM(akv::attend_tc_kernel, akv::tc::kSmemBytes);
-    return launch_pdl(akv::attend_tc_kernel, (unsigned)grid, akv::tc::kThreads, akv::tc::kSmemBytes, s, ap, cpg, mk, mv);
+    return launch_pdl(akv::attend_tc_kernel, (unsigned)grid, akv::tc::kThreads, akv::tc::kSmemBytes, s, ap, cpg, mk, mv,
+                      mqs, mqk, q_maps);
 }
 
 atlaskv_status dispatch_attend(int dtype, int D, const akv::AttnParams &ap, cudaStream_t s)
@@ -981,9 +999,9 @@ atlaskv_status launch_attend_tc_layers(const Call *calls, int n, int mode, cudaS
         b.p[l].mode = mode;
         b.offs[l] = (unsigned)(per * l);
         if (b.p[l].lk_rows >= (1LL << 31)) return fail(ATLASKV_EUNSUPPORTED, "more than 2^31 leaf rows");
-        atlaskv_status st = encode_seq_map(&b.mk[l], b.p[l].k_seq, a0.B, a0.T, a0.H_kv);
+        atlaskv_status st = encode_tc_map(&b.mk[l], b.p[l].k_seq, a0.H_kv, a0.T, a0.B, akv::tc::kKeys);
         if (st != ATLASKV_OK) return st;
-        st = encode_seq_map(&b.mv[l], b.p[l].v_seq, a0.B, a0.T, a0.H_kv);
+        st = encode_tc_map(&b.mv[l], b.p[l].v_seq, a0.H_kv, a0.T, a0.B, akv::tc::kKeys);
         if (st != ATLASKV_OK) return st;
     }
     b.offs[n] = (unsigned)(per * n);
@@ -1745,6 +1763,7 @@ atlaskv_status atlaskv_sync_status(atlaskv_tree *t, void *stream)
     AKV_CUDA(cudaStreamSynchronize(s));
     if (v == akv::kDevBadChild) return fail(ATLASKV_EDEVICE, "a child id was out of range on the device");
     if (v == akv::kDevTimeout) return fail(ATLASKV_ETIMEOUT, "a bounded device wait gave up");
+    if (v == akv::kDevBadSmem) return fail(ATLASKV_EDEVICE, "the attention kernel's shared memory base was not 1024-byte aligned");
     if (v != akv::kDevOk) return fail(ATLASKV_EDEVICE, "device status %d", v);
     return ATLASKV_OK;
 }

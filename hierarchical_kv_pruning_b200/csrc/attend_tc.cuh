@@ -6,17 +6,20 @@
 // sequence softmaxes equals one softmax over both key sets), organised for
 // sm_100a as a warp-specialised pipeline.  A CTA owns kWG 128-row tiles of
 // one (query b, KV head) group (row r = g N + n is token n of head g), one per
-// softmax warpgroup, and streams 64-key tiles shared by them: first the causal
-// sequence, then the kept leaves of the CTA's heads (each visible only to its
-// own head's rows); the online softmax is order-free.  kWG = 1 (TMEM 256
-// columns, 96 KB of shared memory) runs two CTAs per SM, so one CTA's MMA,
+// softmax warpgroup, and streams 64-key tiles shared by them: first the kept
+// leaves of the CTA's heads (each visible only to its own head's rows), then
+// the causal sequence; the online softmax is order-free.  Leaves first: their
+// gathers are the slowest copies of the CTA and start while the rings are
+// empty, and the switch from q_kg to q_seq is then a TMA load that runs under
+// the softmax of the last leaf tile.  kWG = 1 (TMEM 256
+// columns, 112 KB of shared memory) runs two CTAs per SM, so one CTA's MMA,
 // copy and softmax bubbles overlap the other's work; this measured faster than
 // two warpgroups sharing the key tiles in one CTA per SM.
 //
 //   producer warp   sequence K/V tiles by TMA (4-D tensor maps, 128-byte
 //                   swizzle) and gathered leaf rows by cp.async, into a K ring
-//                   (a stage is released as soon as S has read it) and a V
-//                   ring, each guarded by full / empty mbarriers;
+//                   (a stage is released as soon as S has read it) and a
+//                   three-stage V ring, each guarded by full / empty mbarriers;
 //   MMA warp        one thread issues S(w, t) = Q_w K_t^T (M 128, N 64,
 //                   K 128, both operands in shared memory) into a double-
 //                   buffered S in TMEM for each warpgroup, then
@@ -49,7 +52,7 @@ constexpr int kKeys = 64;                  // keys per tile
 constexpr int kD = 128;                    // head dim
 constexpr int kWG = 1;                     // softmax warpgroups per CTA (1: two CTAs per SM)
 constexpr int kKStages = kWG == 2 ? 4 : 2; // K ring depth (a stage is freed when S = Q K^T completes)
-constexpr int kVStages = kWG == 2 ? 3 : 2; // V ring depth (freed when P V completes)
+constexpr int kVStages = 3;                // V ring depth (freed when P V completes; its wait bounds the K issue too)
 constexpr int kMinCtasPerSm = kWG == 2 ? 1 : 2;
 constexpr int kProducerWarp = 4 * kWG;
 constexpr int kMmaWarp = 4 * kWG + 1;
@@ -78,7 +81,10 @@ constexpr int kBarQReady = kBarODone + 2 * kWG;     // [kWG] Q_w loaded (4 warps
 constexpr int kBarDrain = kBarQReady + kWG;         // every MMA the issuing thread committed has completed
 constexpr int kNumBars = kBarDrain + 1;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024;   // + slack to align the base to 1024
+// No alignment slack: with no static shared memory the dynamic base is 1024-byte
+// aligned (the kernel checks it and reports EDEVICE otherwise), and 112 KB
+// keeps two CTAs per SM.
+constexpr int kSmemBytes = kOffTmemSlot + 16;
 constexpr int kTmemCols = 256 * kWG;           // warpgroup w: S / P buffers [256 w, 256 w + 128), O [256 w + 128, 256 w + 256)
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -262,12 +268,17 @@ __global__ void wait_timeout_probe_kernel(int *status)
 // of the group's G N rows), keys and values of the sequence by TMA through
 // the tensor maps tm_k / tm_v.
 __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigned bid, int ctas_per_group,
-                                              const CUtensorMap *tm_k, const CUtensorMap *tm_v)
+                                              const CUtensorMap *tm_k, const CUtensorMap *tm_v,
+                                              const CUtensorMap *tm_qs, const CUtensorMap *tm_qk)
 {
     using namespace tc;
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem = tc_smem_raw;
     const uint32_t sb = smem_addr(smem);
+    if (sb & 1023u) {   // the 128-byte swizzle atoms need a 1024-byte aligned base (CTA-uniform exit)
+        if (threadIdx.x == 0) set_status(p.status, kDevBadSmem);
+        return;
+    }
     auto bar = [&](int i) -> uint32_t { return sb + kOffBar + 8 * i; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffTmemSlot);
 
@@ -286,11 +297,16 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
     const int cta_last = p.T - p.N + (r_end / p.N != r0 / p.N ? p.N - 1 : r_end % p.N);
     const int n_seq_tiles = p.mode == kAttnLeaf ? 0 : (cta_last + kKeys) / kKeys;
     const int n_tiles = n_leaf_tiles + n_seq_tiles;
+    // Tiles 0 .. n_leaf_tiles - 1 are leaf tiles, the rest sequence tiles.
     // Warpgroup w takes every sequence tile (if it has rows at all) and the
     // leaf tiles holding its heads' leaves: its heads are contiguous and the
     // leaves are stored head by head, so those are the leaf tiles
     // [wlo[w], whi[w]] (empty when wlo > whi).  It skips the others, and so do
     // its MMAs; its count of taken tiles drives its S / P buffers and phases.
+    // Q by TMA (tm_qs / tm_qk non-null) needs whole heads of N rows, N a
+    // multiple of 8 dividing 128 (or 128 dividing N): every head then starts
+    // on a swizzle atom of the Q tile.
+    const bool q_tma = tm_qs != nullptr && p.N % 8 == 0 && (128 % p.N == 0 || p.N % 128 == 0);
     int wlo[kWG], whi[kWG];
     bool wvalid[kWG];
 #pragma unroll
@@ -306,14 +322,16 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
         }
     }
     auto wg_takes = [&](int w, int t) -> bool {
-        return wvalid[w] && (t < n_seq_tiles || (t - n_seq_tiles >= wlo[w] && t - n_seq_tiles <= whi[w]));
+        return wvalid[w] && (t >= n_leaf_tiles || (t >= wlo[w] && t <= whi[w]));
     };
-    // position of a taken tile t among warpgroup w's tiles
-    auto wg_count = [&](int w, int t) -> int { return t < n_seq_tiles ? t : n_seq_tiles + (t - n_seq_tiles - wlo[w]); };
+    // leaf tiles of warpgroup w, and the position of a taken tile t among its tiles
+    auto wg_leaves = [&](int w) -> int { return wlo[w] <= whi[w] ? whi[w] - wlo[w] + 1 : 0; };
+    auto wg_count = [&](int w, int t) -> int { return t < n_leaf_tiles ? t - wlo[w] : wg_leaves(w) + (t - n_leaf_tiles); };
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) {
-            const bool per_warp = (i >= kBarPReady && i < kBarPReady + 2 * kWG) || (i >= kBarQReady && i < kBarQReady + kWG);
+            const bool per_warp = (i >= kBarPReady && i < kBarPReady + 2 * kWG) ||
+                                  (!q_tma && i >= kBarQReady && i < kBarQReady + kWG);
             mbar_init(bar(i), per_warp ? 4 : 1);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -343,7 +361,27 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
         const uint32_t qa = sb + kOffQ + w * kQBytes;
         bool failed = false;
 
-        // Q_w rows into the swizzled A tile: 16 consecutive threads per 256-byte row
+        // Q_w rows into the swizzled A tile.  By TMA: one thread, one box of the
+        // head's N rows per 64-column half, completion counted in bytes on
+        // QReady; it returns at once.  Else cp.async, 16 consecutive threads per
+        // 256-byte row; it returns once the rows have landed.
+        auto load_q_tma = [&](const CUtensorMap *m) {
+            if (lrow != 0) return;
+            const int wr0 = r0 + w * kRows, wr1 = min(GN, wr0 + kRows);
+            const int bn = min(p.N, kRows);
+            if (wr1 <= wr0) {   // a warpgroup without rows: nothing to load (and no MMA waits for it)
+                mbar_arrive(bar(kBarQReady + w));
+                return;
+            }
+            mbar_arrive_expect_tx(bar(kBarQReady + w), (uint32_t)(wr1 - wr0) * kD * 2);
+            for (int rr = wr0; rr < wr1; rr += bn) {
+                const int gg = rr / p.N, tok = rr - gg * p.N;
+#pragma unroll
+                for (int half = 0; half < 2; ++half)
+                    tma_load_4d(qa + half * (kRows * 128) + (rr - wr0) * 128, m, half * 64, hkv * p.G + gg, tok, b,
+                                bar(kBarQReady + w));
+            }
+        };
         auto load_q = [&](const void *qptr) {
             const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(qptr);
             const int lc = lrow & 15, lr = lrow >> 4;
@@ -362,8 +400,10 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kBarQReady + w));
         };
-        load_q(p.mode == kAttnLeaf ? p.q_kg : p.q_seq);
-        const bool any_leaf = wvalid[w] && wlo[w] <= whi[w];
+        const int n_lw = wvalid[w] ? wg_leaves(w) : 0;   // this warpgroup's leaf tiles come first
+        const bool swap_q = n_lw > 0 && n_seq_tiles > 0;
+        if (q_tma) load_q_tma(n_lw > 0 ? tm_qk : tm_qs);
+        else load_q(n_lw > 0 ? p.q_kg : p.q_seq);
 
         const float sl2 = p.scale_log2;
         float m_used = -INFINITY, l = 0.f;
@@ -378,19 +418,22 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
             tmem_ld32(tS + 64 * bs + lane_off, sc);
             tmem_ld32(tS + 64 * bs + 32 + lane_off, sc + 32);
             tmem_wait_ld();
-            // S(w, last sequence tile) has completed: Q_w may now be replaced by q_kg
-            if (t == n_seq_tiles - 1 && any_leaf) load_q(p.q_kg);
+            // S(w, its last leaf tile) has completed: Q_w may now be replaced by q_seq
+            if (swap_q && c_w == n_lw - 1) {
+                if (q_tma) load_q_tma(tm_qs);
+                else load_q(p.q_seq);
+            }
 
             // visible keys of this tile, [lo, hi) in tile-local index: the leaves
             // are stored head by head, K_L per head; a sequence tile is cut by
             // the causal limit
             int lo, hi;
-            if (t >= n_seq_tiles) {
-                lo = (g - g_first) * p.K_L - (t - n_seq_tiles) * kKeys;
+            if (t < n_leaf_tiles) {
+                lo = (g - g_first) * p.K_L - t * kKeys;
                 hi = lo + p.K_L;
             } else {
                 lo = 0;
-                hi = last_key + 1 - t * kKeys;
+                hi = last_key + 1 - (t - n_leaf_tiles) * kKeys;
             }
             if (!row_ok) hi = lo;
             if (!(lo <= 0 && hi >= kKeys)) {
@@ -579,7 +622,8 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
         if (n_leaf_tiles > 0) fetch_rows(0, nk, nv);
         for (int t = 0; t < n_tiles; ++t) {
             const int sk = t % kKStages, sv = t % kVStages;
-            const bool leaf = t >= n_seq_tiles;
+            const bool leaf = t < n_leaf_tiles;
+            const int st = t - n_leaf_tiles;   // sequence tile index
             const uint32_t kd = sb + kOffK + sk * kKVBytes, vd = sb + kOffV + sv * kKVBytes;
             if (t >= kKStages) {
                 failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarEmptyK + sk), ((t / kKStages) + 1) & 1));
@@ -591,8 +635,7 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
                 rk[1] = nk[1];
                 rv[0] = nv[0];
                 rv[1] = nv[1];
-                const int lt = t - n_seq_tiles;
-                if (lt + 1 < n_leaf_tiles) fetch_rows(lt + 1, nk, nv);
+                if (t + 1 < n_leaf_tiles) fetch_rows(t + 1, nk, nv);
                 gather(kd, lkb, rk);
                 k_issued = t + 1;
             } else {
@@ -600,7 +643,7 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
                     mbar_arrive_expect_tx(bar(kBarFullK + sk), kKVBytes);
 #pragma unroll
                     for (int half = 0; half < 2; ++half)
-                        tma_load_4d(kd + half * (kKeys * 128), tm_k, half * 64, hkv, t * kKeys, b, bar(kBarFullK + sk));
+                        tma_load_4d(kd + half * (kKeys * 128), tm_k, half * 64, hkv, st * kKeys, b, bar(kBarFullK + sk));
                 }
                 __syncwarp();
                 k_issued = t + 1;
@@ -619,7 +662,7 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
                     mbar_arrive_expect_tx(bar(kBarFullV + sv), kKVBytes);
 #pragma unroll
                     for (int half = 0; half < 2; ++half)
-                        tma_load_4d(vd + half * (kKeys * 128), tm_v, half * 64, hkv, t * kKeys, b, bar(kBarFullV + sv));
+                        tma_load_4d(vd + half * (kKeys * 128), tm_v, half * 64, hkv, st * kKeys, b, bar(kBarFullV + sv));
                 }
                 __syncwarp();
             }
@@ -633,9 +676,9 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
         // (sequence) tiles are waited for.
         bool drained = true;
         for (int t = max(0, k_issued - kKStages); t < k_issued; ++t)
-            if (!failed || t < n_seq_tiles) drained &= mbar_wait(bar(kBarFullK + t % kKStages), (t / kKStages) & 1);
+            if (!failed || t >= n_leaf_tiles) drained &= mbar_wait(bar(kBarFullK + t % kKStages), (t / kKStages) & 1);
         for (int t = max(0, v_issued - kVStages); t < v_issued; ++t)
-            if (!failed || t < n_seq_tiles) drained &= mbar_wait(bar(kBarFullV + t % kVStages), (t / kVStages) & 1);
+            if (!failed || t >= n_leaf_tiles) drained &= mbar_wait(bar(kBarFullV + t % kVStages), (t / kVStages) & 1);
         cp_wait_all();
         if ((failed || !drained) && lane == 0) set_status(p.status, kDevTimeout);
     } else {
@@ -657,10 +700,8 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
                     if (!wg_takes(w, t)) continue;
                     const int cs = wg_count(w, t), bs = cs & 1;
                     if (cs == 0 && !mbar_wait(bar(kBarQReady + w), 0)) return false;
-                    // the warpgroup's first leaf tile: Q_w has been replaced by q_kg
-                    if (n_seq_tiles > 0 && t >= n_seq_tiles && t - n_seq_tiles == wlo[w] &&
-                        !mbar_wait(bar(kBarQReady + w), 1))
-                        return false;
+                    // the warpgroup's first sequence tile after its leaves: Q_w has been replaced by q_seq
+                    if (t == n_leaf_tiles && cs > 0 && !mbar_wait(bar(kBarQReady + w), 1)) return false;
                     // buffer bs still holds the P of this warpgroup's tile two back until its P V has completed
                     if (cs >= 2 && !mbar_wait(bar(kBarODone + 2 * w + bs), ((cs - 2) >> 1) & 1)) return false;
                     fence_after_sync();
@@ -721,14 +762,17 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
 
 // One call: one CTA per (query b, KV head, kWG x 128-row block of the group's
 // G N rows).  tm_k / tm_v: the sequence keys / values [B][T][H_kv][D] as 4-D
-// tensor maps (D, H_kv, T, B) with a (64, 1, 64, 1) box and 128-byte swizzle.
+// tensor maps (D, H_kv, T, B) with a (64, 1, 64, 1) box and 128-byte swizzle;
+// with q_maps, tm_qs / tm_qk: q_seq / q_kg [B][N][H][D] as (D, H, N, B) with a
+// (64, 1, min(N, 128), 1) box (else Q is loaded by cp.async).
 __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
     attend_tc_kernel(const __grid_constant__ AttnParams p, int ctas_per_group, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v)
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
+                     const __grid_constant__ CUtensorMap tm_qk, int q_maps)
 {
     griddep_launch();
     griddep_wait();   // the kept lists (and everything else) of the previous grid are visible
-    attend_tc_cta(p, blockIdx.x, ctas_per_group, &tm_k, &tm_v);
+    attend_tc_cta(p, blockIdx.x, ctas_per_group, &tm_k, &tm_v, q_maps ? &tm_qs : nullptr, q_maps ? &tm_qk : nullptr);
 }
 
 // Several layers' calls in one launch (same shapes, each layer its own
@@ -746,7 +790,7 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
 {
     int l = 0;
     while (l + 1 < b.n && blockIdx.x >= b.offs[l + 1]) ++l;
-    attend_tc_cta(b.p[l], blockIdx.x - b.offs[l], b.ctas_per_group, &b.mk[l], &b.mv[l]);
+    attend_tc_cta(b.p[l], blockIdx.x - b.offs[l], b.ctas_per_group, &b.mk[l], &b.mv[l], nullptr, nullptr);
 }
 
 }  // namespace akv

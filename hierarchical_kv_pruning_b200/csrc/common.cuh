@@ -8,7 +8,7 @@
 namespace akv {
 
 // Device status word values (sticky; first error wins).
-enum : int { kDevOk = 0, kDevBadChild = 1, kDevTimeout = 2 };
+enum : int { kDevOk = 0, kDevBadChild = 1, kDevTimeout = 2, kDevBadSmem = 3 };
 
 // Programmatic dependent launch.  griddep_wait: wait until the grid this one
 // depends on (the previous kernel on the stream, when this one was launched
