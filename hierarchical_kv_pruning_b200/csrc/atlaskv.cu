@@ -708,17 +708,21 @@ atlaskv_status encode_tc_map(CUtensorMap *map, const void *base, long long d1, l
     return ATLASKV_OK;
 }
 
-// bf16, D = 128: tcgen05 tensor cores, one CTA per kWG x 128 query rows of a
-// (query, KV head) group.  Sequence K / V [B][T][H_kv][D] by TMA (box of 64
-// keys); Q [B][N][H][D] by TMA too (box of min(N, 128) tokens of one head)
-// when every head's rows start on a swizzle atom of the Q tile, i.e. N is a
-// multiple of 8 that divides 128 or is divisible by it, else by cp.async.
+int num_sms();
+
+// bf16, D = 128: tcgen05 tensor cores, units of 128 query rows of a (query,
+// KV head) group on a persistent grid.  Sequence K / V [B][T][H_kv][D] by TMA
+// (box of 64 keys); Q [B][N][H][D] by TMA too (box of min(N, 128) tokens of
+// one head) when every head's rows start on a swizzle atom of the Q tile, i.e.
+// N is a multiple of 8 that divides 128 or is divisible by it, else by
+// cp.async.
 atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
 {
     const int rows = ap.G * ap.N;
     const int cpg = (rows + akv::tc::kCtaRows - 1) / akv::tc::kCtaRows;
-    const long long grid = (long long)ap.B * ap.H_kv * cpg;
-    if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "attention grid too large");
+    const long long units = (long long)ap.B * ap.H_kv * cpg;
+    if (units > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "attention grid too large");
+    if (units == 0) return ATLASKV_OK;
     if (ap.lk_rows >= (1LL << 31) || ap.lv_rows >= (1LL << 31))
         return fail(ATLASKV_EUNSUPPORTED, "more than 2^31 leaf rows");
     CUtensorMap mk, mv, mqs, mqk;
@@ -729,7 +733,7 @@ atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
     // a mode that reads only one of the two query tensors uses it for both maps
     const void *qs = ap.q_seq ? ap.q_seq : ap.q_kg, *qk = ap.q_kg ? ap.q_kg : ap.q_seq;
     const auto aligned = [](const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-    int q_maps = ap.N % 8 == 0 && (128 % ap.N == 0 || ap.N % 128 == 0) && aligned(qs) && aligned(qk);
+    const int q_maps = ap.N % 8 == 0 && (128 % ap.N == 0 || ap.N % 128 == 0) && aligned(qs) && aligned(qk);
     if (q_maps) {
         const int bn = ap.N < akv::tc::kRows ? ap.N : akv::tc::kRows;
         st = encode_tc_map(&mqs, qs, ap.H, ap.N, ap.B, bn);
@@ -737,12 +741,18 @@ atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
         st = encode_tc_map(&mqk, qk, ap.H, ap.N, ap.B, bn);
         if (st != ATLASKV_OK) return st;
     } else {
-        mqs = mk;   // unused
-        mqk = mk;
+        mqs = mqk = mk;   // unused
     }
     AKV_SMEM(akv::attend_tc_kernel, akv::tc::kSmemBytes);
-    return launch_pdl(akv::attend_tc_kernel, (unsigned)grid, akv::tc::kThreads, akv::tc::kSmemBytes, s, ap, cpg, mk, mv,
-                      mqs, mqk, q_maps);
+    // persistent grid: as many CTAs as are resident at once, each taking units
+    // round-robin.  Two per SM by construction (112 KB of shared memory, 256
+    // TMEM columns, the launch bounds); the occupancy query reports one here
+    // (it assumes the default shared-memory carve-out), and a grid of one per SM
+    // measured 1.4x slower.
+    const long long resident = (long long)akv::tc::kMinCtasPerSm * num_sms();
+    const unsigned grid = (unsigned)(units < resident ? units : resident);
+    return launch_pdl(akv::attend_tc_kernel, grid, akv::tc::kThreads, akv::tc::kSmemBytes, s, ap, cpg,
+                      (unsigned)units, mk, mv, mqs, mqk, q_maps);
 }
 
 atlaskv_status dispatch_attend(int dtype, int D, const akv::AttnParams &ap, cudaStream_t s)

@@ -4,34 +4,35 @@
 // Same computation as attend.cuh ("AtlasKV: Augmenting LLMs with Billion-Scale
 // Knowledge Graphs in 20GB VRAM": the lambda-weighted merge of the knowledge and
 // sequence softmaxes equals one softmax over both key sets), organised for
-// sm_100a as a warp-specialised pipeline.  A CTA owns kWG 128-row tiles of
-// one (query b, KV head) group (row r = g N + n is token n of head g), one per
-// softmax warpgroup, and streams 64-key tiles shared by them: first the kept
-// leaves of the CTA's heads (each visible only to its own head's rows), then
-// the causal sequence; the online softmax is order-free.  Leaves first: their
-// gathers are the slowest copies of the CTA and start while the rings are
-// empty, and the switch from q_kg to q_seq is then a TMA load that runs under
-// the softmax of the last leaf tile.  kWG = 1 (TMEM 256
-// columns, 112 KB of shared memory) runs two CTAs per SM, so one CTA's MMA,
-// copy and softmax bubbles overlap the other's work; this measured faster than
-// two warpgroups sharing the key tiles in one CTA per SM.
+// sm_100a as a warp-specialised, persistent pipeline.  A unit of work is a
+// 128-row block of one (query b, KV head) group (row r = g N + n is token n of
+// head g) and its 64-key tiles: first the kept leaves of the block's heads
+// (each visible only to its own head's rows), then the causal sequence; the
+// online softmax is order-free.  A CTA (TMEM 256 columns, 112 KB of shared
+// memory, two per SM, so one CTA's MMA, copy and softmax bubbles overlap the
+// other's work) runs its units back to back through one pipeline, so a unit's
+// start (leaf gathers, the Q load, the first S) overlaps the previous unit's
+// last tiles and epilogue.
 //
 //   producer warp   sequence K/V tiles by TMA (4-D tensor maps, 128-byte
 //                   swizzle) and gathered leaf rows by cp.async, into a K ring
 //                   (a stage is released as soon as S has read it) and a
 //                   three-stage V ring, each guarded by full / empty mbarriers;
-//   MMA warp        one thread issues S(w, t) = Q_w K_t^T (M 128, N 64,
-//                   K 128, both operands in shared memory) into a double-
-//                   buffered S in TMEM for each warpgroup, then
-//                   O_w += P_w V_{t-1} (M 128, N 128, K 64) with P_w read from
-//                   TMEM, so S(t) runs under softmax(t - 1); tcgen05.commit
-//                   arrives on the mbarriers;
-//   kWG warpgroups  one thread per query row: read its S row (tcgen05.ld),
+//   MMA warp        one thread issues S(t) = Q K_t^T (M 128, N 64, K 128, both
+//                   operands in shared memory) into a double-buffered S in
+//                   TMEM, then O += P V_{t-1} (M 128, N 128, K 64) with P read
+//                   from TMEM, so S(t) runs under softmax(t - 1); a unit's
+//                   first P V starts O afresh once the previous unit's O has
+//                   been read out; tcgen05.commit arrives on the mbarriers;
+//   4 softmax warps one thread per query row: read its S row (tcgen05.ld),
 //                   mask, online softmax with a lazily rescaled running max
 //                   (O in TMEM is rescaled only when the row max grows by more
 //                   than 2^8), P (bf16 pairs) written back over the first half
 //                   of the same S buffer (tcgen05.st), so P never touches
-//                   shared memory; finally O / l and the log-sum-exp.
+//                   shared memory; the Q loads (q_kg, then q_seq, then the
+//                   next unit's), each started as soon as the last S that
+//                   reads the old Q has completed; finally O / l and the
+//                   log-sum-exp.
 // Shared-memory bandwidth is what the tensor core waits on here (the MMA
 // operands plus the K/V copies); P in TMEM removes its store and its reread.
 //
@@ -50,14 +51,13 @@ namespace tc {
 constexpr int kRows = 128;                 // query rows per warpgroup (UMMA M)
 constexpr int kKeys = 64;                  // keys per tile
 constexpr int kD = 128;                    // head dim
-constexpr int kWG = 1;                     // softmax warpgroups per CTA (1: two CTAs per SM)
-constexpr int kKStages = kWG == 2 ? 4 : 2; // K ring depth (a stage is freed when S = Q K^T completes)
+constexpr int kKStages = 2;                // K ring depth (a stage is freed when S = Q K^T completes)
 constexpr int kVStages = 3;                // V ring depth (freed when P V completes; its wait bounds the K issue too)
-constexpr int kMinCtasPerSm = kWG == 2 ? 1 : 2;
-constexpr int kProducerWarp = 4 * kWG;
-constexpr int kMmaWarp = 4 * kWG + 1;
-constexpr int kThreads = 32 * (4 * kWG + 2);
-constexpr int kCtaRows = kWG * kRows;
+constexpr int kMinCtasPerSm = 2;           // one softmax warpgroup per CTA, two CTAs per SM
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kThreads = 32 * 6;
+constexpr int kCtaRows = kRows;
 constexpr long long kSpinLimit = 1ll << 18;   // bounded mbarrier waits: try_wait iterations, not a fixed time
 constexpr float kRescaleLog2 = 8.f;            // rescale O only when the row max grows by more than this
 
@@ -65,27 +65,29 @@ constexpr float kRescaleLog2 = 8.f;            // rescale O only when the row ma
 // canonical 128-byte-swizzled UMMA layouts)
 constexpr int kQBytes = kRows * kD * 2;       // 32 KB: 2 K-blocks of [128 rows][64]
 constexpr int kKVBytes = kKeys * kD * 2;      // 16 KB: 2 blocks of [64 keys][64]
-constexpr int kOffQ = 0;                                  // [kWG]
-constexpr int kOffK = kOffQ + kWG * kQBytes;              // [kKStages]
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kQBytes;                    // [kKStages]
 constexpr int kOffV = kOffK + kKStages * kKVBytes;        // [kVStages]
 constexpr int kOffBar = kOffV + kVStages * kKVBytes;
-// mbarriers (8 bytes each); [kWG][2] arrays are indexed by warpgroup and tile parity
+// mbarriers (8 bytes each); the [2] arrays are indexed by the parity of the
+// CTA's running tile count (tiles of all its units, in order)
 constexpr int kBarFullK = 0;                        // [kKStages] K tile landed
 constexpr int kBarEmptyK = kBarFullK + kKStages;    // [kKStages] S of the tile done
 constexpr int kBarFullV = kBarEmptyK + kKStages;    // [kVStages] V tile landed
 constexpr int kBarEmptyV = kBarFullV + kVStages;    // [kVStages] P V of the tile done
-constexpr int kBarSFull = kBarEmptyV + kVStages;    // [kWG][2] S in TMEM buffer (tiles taken by w so far) & 1
-constexpr int kBarPReady = kBarSFull + 2 * kWG;     // [kWG][2] P(w, t) written over it, O_w rescaled (4 warps)
-constexpr int kBarODone = kBarPReady + 2 * kWG;     // [kWG][2] O_w += P V from that buffer done
-constexpr int kBarQReady = kBarODone + 2 * kWG;     // [kWG] Q_w loaded (4 warps)
-constexpr int kBarDrain = kBarQReady + kWG;         // every MMA the issuing thread committed has completed
+constexpr int kBarSFull = kBarEmptyV + kVStages;    // [2] S in TMEM buffer (tile & 1)
+constexpr int kBarPReady = kBarSFull + 2;           // [2] P written over it, O rescaled (4 warps)
+constexpr int kBarODone = kBarPReady + 2;           // [2] O += P V from that buffer done
+constexpr int kBarQReady = kBarODone + 2;           // Q loaded (one phase per load; 4 warps with cp.async)
+constexpr int kBarODrained = kBarQReady + 1;        // a unit's O read out of TMEM (4 warps)
+constexpr int kBarDrain = kBarODrained + 1;         // every MMA the issuing thread committed has completed
 constexpr int kNumBars = kBarDrain + 1;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 // No alignment slack: with no static shared memory the dynamic base is 1024-byte
 // aligned (the kernel checks it and reports EDEVICE otherwise), and 112 KB
 // keeps two CTAs per SM.
 constexpr int kSmemBytes = kOffTmemSlot + 16;
-constexpr int kTmemCols = 256 * kWG;           // warpgroup w: S / P buffers [256 w, 256 w + 128), O [256 w + 128, 256 w + 256)
+constexpr int kTmemCols = 256;                 // S / P buffers [0, 128), O [128, 256)
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -264,11 +266,49 @@ __global__ void wait_timeout_probe_kernel(int *status)
     if (threadIdx.x == 0 && !tc::mbar_wait(b, 0)) set_status(status, kDevTimeout);
 }
 
-// The work of CTA `bid` of a launch: (query b, KV head, kWG x 128-row block
-// of the group's G N rows), keys and values of the sequence by TMA through
-// the tensor maps tm_k / tm_v.
-__device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigned bid, int ctas_per_group,
-                                              const CUtensorMap *tm_k, const CUtensorMap *tm_v,
+// One unit of attention work: (query b, KV head, 128-row block of the group's
+// G N rows; row r = g N + n is token n of head g).  Its tiles 0 ..
+// n_leaf_tiles - 1 hold the kept leaves of the block's heads (stored head by
+// head, K_L per head), the rest the causal sequence.
+struct TcUnit {
+    int b, hkv, grp, r0, rows, g_first, n_leaf, n_leaf_tiles, n_seq_tiles, n_tiles;
+};
+
+__device__ __forceinline__ TcUnit tc_unit(const AttnParams &p, unsigned u, int ctas_per_group)
+{
+    TcUnit U;
+    U.grp = (int)(u / (unsigned)ctas_per_group);
+    const int blk = (int)u - U.grp * ctas_per_group;
+    U.b = U.grp / p.H_kv;
+    U.hkv = U.grp - U.b * p.H_kv;
+    const int GN = p.G * p.N;
+    U.r0 = blk * tc::kRows;
+    const int r_end = min(GN, U.r0 + tc::kRows) - 1;   // last valid row
+    U.rows = r_end + 1 - U.r0;
+    U.g_first = U.r0 / p.N;
+    const int g_last = r_end / p.N;
+    U.n_leaf = (g_last - U.g_first + 1) * p.K_L;
+    U.n_leaf_tiles = p.mode == kAttnSeq ? 0 : (U.n_leaf + tc::kKeys - 1) / tc::kKeys;
+    // causal extent: the largest token index of the block is N - 1 when its
+    // rows span two heads, else that of its last row
+    const int last = p.T - p.N + (g_last != U.g_first ? p.N - 1 : r_end % p.N);
+    U.n_seq_tiles = p.mode == kAttnLeaf ? 0 : (last + tc::kKeys) / tc::kKeys;
+    U.n_tiles = U.n_leaf_tiles + U.n_seq_tiles;
+    return U;
+}
+
+// A CTA runs the units u0, u0 + ustride, ... below n_units back to back
+// through one pipeline: the rings, the S / P buffers and every barrier phase
+// run on over the units' tiles in order (T counts them), so the next unit's
+// leaf gathers, Q load and first S overlap the last tiles and the epilogue of
+// the current one.  Leaves come first in a unit: their gathers are its
+// slowest copies, and the switch from q_kg to q_seq is then a load that runs
+// under the softmax of the unit's last leaf tile.  Sequence K / V by TMA
+// through tm_k / tm_v; Q by TMA through tm_qs / tm_qk when they are given and
+// every head of a block starts on a swizzle atom of the Q tile (N a multiple
+// of 8 that divides 128 or is divisible by it), else by cp.async.
+__device__ __forceinline__ void attend_tc_run(const AttnParams &p, int ctas_per_group, unsigned u0, unsigned ustride,
+                                              unsigned n_units, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                                               const CUtensorMap *tm_qs, const CUtensorMap *tm_qk)
 {
     using namespace tc;
@@ -279,59 +319,17 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
         if (threadIdx.x == 0) set_status(p.status, kDevBadSmem);
         return;
     }
+    if (u0 >= n_units) return;   // CTA-uniform: no unit, nothing allocated yet
     auto bar = [&](int i) -> uint32_t { return sb + kOffBar + 8 * i; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffTmemSlot);
-
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int grp_id = bid / ctas_per_group;
-    const int cta = bid - grp_id * ctas_per_group;
-    const int b = grp_id / p.H_kv, hkv = grp_id - b * p.H_kv;
     const int GN = p.G * p.N;
-    const int r0 = cta * kCtaRows;                       // first group row of the CTA
-    const int r_end = min(GN, r0 + kCtaRows) - 1;        // last valid one
-    const int g_first = r0 / p.N, g_last = r_end / p.N;  // heads g_first..g_last own the rows
-    const int n_leaf = (g_last - g_first + 1) * p.K_L;   // their kept leaves, head by head
-    const int n_leaf_tiles = p.mode == kAttnSeq ? 0 : (n_leaf + kKeys - 1) / kKeys;
-    // causal extent: the largest token index of the CTA is N - 1 when its rows
-    // span two heads, else that of its last row
-    const int cta_last = p.T - p.N + (r_end / p.N != r0 / p.N ? p.N - 1 : r_end % p.N);
-    const int n_seq_tiles = p.mode == kAttnLeaf ? 0 : (cta_last + kKeys) / kKeys;
-    const int n_tiles = n_leaf_tiles + n_seq_tiles;
-    // Tiles 0 .. n_leaf_tiles - 1 are leaf tiles, the rest sequence tiles.
-    // Warpgroup w takes every sequence tile (if it has rows at all) and the
-    // leaf tiles holding its heads' leaves: its heads are contiguous and the
-    // leaves are stored head by head, so those are the leaf tiles
-    // [wlo[w], whi[w]] (empty when wlo > whi).  It skips the others, and so do
-    // its MMAs; its count of taken tiles drives its S / P buffers and phases.
-    // Q by TMA (tm_qs / tm_qk non-null) needs whole heads of N rows, N a
-    // multiple of 8 dividing 128 (or 128 dividing N): every head then starts
-    // on a swizzle atom of the Q tile.
     const bool q_tma = tm_qs != nullptr && p.N % 8 == 0 && (128 % p.N == 0 || p.N % 128 == 0);
-    int wlo[kWG], whi[kWG];
-    bool wvalid[kWG];
-#pragma unroll
-    for (int w = 0; w < kWG; ++w) {
-        const int wr0 = r0 + w * kRows;
-        wvalid[w] = wr0 < GN;
-        wlo[w] = 1;
-        whi[w] = 0;
-        if (wvalid[w] && n_leaf_tiles > 0) {
-            const int wr1 = min(GN, wr0 + kRows) - 1;
-            wlo[w] = ((wr0 / p.N - g_first) * p.K_L) / kKeys;
-            whi[w] = min(n_leaf_tiles - 1, ((wr1 / p.N - g_first + 1) * p.K_L - 1) / kKeys);
-        }
-    }
-    auto wg_takes = [&](int w, int t) -> bool {
-        return wvalid[w] && (t >= n_leaf_tiles || (t >= wlo[w] && t <= whi[w]));
-    };
-    // leaf tiles of warpgroup w, and the position of a taken tile t among its tiles
-    auto wg_leaves = [&](int w) -> int { return wlo[w] <= whi[w] ? whi[w] - wlo[w] + 1 : 0; };
-    auto wg_count = [&](int w, int t) -> int { return t < n_leaf_tiles ? t - wlo[w] : wg_leaves(w) + (t - n_leaf_tiles); };
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) {
-            const bool per_warp = (i >= kBarPReady && i < kBarPReady + 2 * kWG) ||
-                                  (!q_tma && i >= kBarQReady && i < kBarQReady + kWG);
+            const bool per_warp = i == kBarPReady || i == kBarPReady + 1 || i == kBarODrained ||
+                                  (!q_tma && i == kBarQReady);
             mbar_init(bar(i), per_warp ? 4 : 1);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -346,172 +344,169 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp < 4 * kWG) {
-        // ================= softmax warpgroup w: one thread per query row =================
-        const int w = warp >> 2;
-        const int lrow = tid & (kRows - 1);                    // row of the Q tile = TMEM lane
-        const int row = r0 + w * kRows + lrow;
-        const bool row_ok = row < GN;
-        const int g = row_ok ? row / p.N : g_first;
-        const int n = row_ok ? row - g * p.N : 0;
-        const int h = hkv * p.G + g;
-        const int last_key = p.T - p.N + n;
-        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + 256 * w, tO = tmem + 256 * w + 128;
-        const uint32_t qa = sb + kOffQ + w * kQBytes;
+    if (warp < 4) {
+        // ================= softmax warpgroup: one thread per query row =================
+        const int lrow = tid;                                   // row of the Q tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t tS = tmem, tO = tmem + 128;
+        const uint32_t qa = sb + kOffQ;
+        const float sl2 = p.scale_log2;
         bool failed = false;
 
-        // Q_w rows into the swizzled A tile.  By TMA: one thread, one box of the
-        // head's N rows per 64-column half, completion counted in bytes on
-        // QReady; it returns at once.  Else cp.async, 16 consecutive threads per
-        // 256-byte row; it returns once the rows have landed.
-        auto load_q_tma = [&](const CUtensorMap *m) {
-            if (lrow != 0) return;
-            const int wr0 = r0 + w * kRows, wr1 = min(GN, wr0 + kRows);
-            const int bn = min(p.N, kRows);
-            if (wr1 <= wr0) {   // a warpgroup without rows: nothing to load (and no MMA waits for it)
-                mbar_arrive(bar(kBarQReady + w));
+        // Q rows of unit U into the swizzled A tile.  By TMA: one thread, one box
+        // of min(N, 128) rows of one head per 64-column half, completion counted
+        // in bytes on QReady; it returns at once.  Else cp.async, 16 consecutive
+        // threads per 256-byte row; it returns once the rows have landed.
+        auto load_q = [&](const TcUnit &U, bool seq) {
+            if (q_tma) {
+                if (tid != 0) return;
+                const CUtensorMap *m = seq ? tm_qs : tm_qk;
+                const int bn = min(p.N, kRows);
+                mbar_arrive_expect_tx(bar(kBarQReady), (uint32_t)U.rows * kD * 2);
+                for (int rr = U.r0; rr < U.r0 + U.rows; rr += bn) {
+                    const int gg = rr / p.N, tok = rr - gg * p.N;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half)
+                        tma_load_4d(qa + half * (kRows * 128) + (rr - U.r0) * 128, m, half * 64, U.hkv * p.G + gg, tok,
+                                    U.b, bar(kBarQReady));
+                }
                 return;
             }
-            mbar_arrive_expect_tx(bar(kBarQReady + w), (uint32_t)(wr1 - wr0) * kD * 2);
-            for (int rr = wr0; rr < wr1; rr += bn) {
-                const int gg = rr / p.N, tok = rr - gg * p.N;
-#pragma unroll
-                for (int half = 0; half < 2; ++half)
-                    tma_load_4d(qa + half * (kRows * 128) + (rr - wr0) * 128, m, half * 64, hkv * p.G + gg, tok, b,
-                                bar(kBarQReady + w));
-            }
-        };
-        auto load_q = [&](const void *qptr) {
-            const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(qptr);
+            const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(seq ? p.q_seq : p.q_kg);
             const int lc = lrow & 15, lr = lrow >> 4;
             const uint32_t dst0 = qa + (lc >> 3) * (kRows * 128);
 #pragma unroll 4
             for (int i = 0; i < kRows / 8; ++i) {
-                const int rl = lr + 8 * i, rr = r0 + w * kRows + rl;
-                const bool ok = rr < GN;
-                const int gg = ok ? rr / p.N : 0, nn = ok ? rr - gg * p.N : 0;
-                const __nv_bfloat16 *src = q + (((size_t)b * p.N + nn) * p.H + hkv * p.G + gg) * kD + lc * 8;
+                const int rl = lr + 8 * i;
+                const bool ok = rl < U.rows;
+                const int rr = U.r0 + (ok ? rl : 0);
+                const int gg = rr / p.N, nn = rr - gg * p.N;
+                const __nv_bfloat16 *src = q + (((size_t)U.b * p.N + nn) * p.H + U.hkv * p.G + gg) * kD + lc * 8;
                 cp16(dst0 + sw128(rl, lc & 7), src, ok);
             }
             cp_commit();
             cp_wait_all();
             fence_async_smem();   // visible to the tensor cores once the barrier is passed
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kBarQReady + w));
+            if (lane == 0) mbar_arrive(bar(kBarQReady));
         };
-        const int n_lw = wvalid[w] ? wg_leaves(w) : 0;   // this warpgroup's leaf tiles come first
-        const bool swap_q = n_lw > 0 && n_seq_tiles > 0;
-        if (q_tma) load_q_tma(n_lw > 0 ? tm_qk : tm_qs);
-        else load_q(n_lw > 0 ? p.q_kg : p.q_seq);
 
-        const float sl2 = p.scale_log2;
-        float m_used = -INFINITY, l = 0.f;
-        int c_w = 0;   // tiles this warpgroup has taken so far
-        for (int t = 0; t < n_tiles; ++t) {
-            if (!wg_takes(w, t)) continue;
-            const int bs = c_w & 1;
-            failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarSFull + 2 * w + bs), (c_w >> 1) & 1));
+        int T = 0;   // tiles of this CTA so far
+        unsigned u = u0;
+        TcUnit U = tc_unit(p, u, ctas_per_group);
+        load_q(U, U.n_leaf_tiles == 0);
+        for (int ui = 0; !failed; ++ui) {
+            const unsigned un = u + ustride;
+            const bool has_next = un < n_units;
+            const int row = U.r0 + lrow;
+            const bool row_ok = lrow < U.rows;
+            const int g = row_ok ? row / p.N : U.g_first;
+            const int n = row_ok ? row - g * p.N : 0;
+            const int h = U.hkv * p.G + g;
+            const int last_key = p.T - p.N + n;
+            float m_used = -INFINITY, l = 0.f;
+            for (int t = 0; t < U.n_tiles; ++t, ++T) {
+                const int bs = T & 1;
+                failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarSFull + bs), (T >> 1) & 1));
+                if (failed) break;
+                fence_after_sync();
+                float sc[kKeys];
+                tmem_ld32(tS + 64 * bs + lane_off, sc);
+                tmem_ld32(tS + 64 * bs + 32 + lane_off, sc + 32);
+                tmem_wait_ld();
+                // the last S that reads this Q has completed: start the next Q
+                if (t == U.n_leaf_tiles - 1 && U.n_seq_tiles > 0) load_q(U, true);
+                else if (t == U.n_tiles - 1 && has_next) {
+                    const TcUnit Un = tc_unit(p, un, ctas_per_group);
+                    load_q(Un, Un.n_leaf_tiles == 0);
+                }
+
+                // visible keys of this tile, [lo, hi) in tile-local index: the
+                // leaves are stored head by head, K_L per head; a sequence tile is
+                // cut by the causal limit
+                int lo, hi;
+                if (t < U.n_leaf_tiles) {
+                    lo = (g - U.g_first) * p.K_L - t * kKeys;
+                    hi = lo + p.K_L;
+                } else {
+                    lo = 0;
+                    hi = last_key + 1 - (t - U.n_leaf_tiles) * kKeys;
+                }
+                if (!row_ok) hi = lo;
+                if (!(lo <= 0 && hi >= kKeys)) {
+#pragma unroll
+                    for (int j = 0; j < kKeys; ++j) sc[j] = (j >= lo && j < hi) ? sc[j] : -INFINITY;
+                }
+                // row max with 8 independent chains
+                float mx8[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mx8[k] = sc[k];
+#pragma unroll
+                for (int j = 8; j < kKeys; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], sc[j]);
+                const float tmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                const float m_new = fmaxf(m_used, tmax * sl2);   // scores in log2 units (sl2 > 0)
+                if (t == 0) {
+                    m_used = m_new;   // O is initialised by the unit's first P V
+                } else {
+                    const bool need = m_new > m_used + kRescaleLog2;   // also when m_used is still -inf
+                    if (__any_sync(0xffffffffu, need)) {
+                        // O may be rescaled only once the previous P V has landed in it
+                        failed = __any_sync(0xffffffffu,
+                                            !mbar_wait(bar(kBarODone + ((T - 1) & 1)), ((T - 1) >> 1) & 1));
+                        if (failed) break;
+                        fence_after_sync();
+                        const float f = need ? fast_exp2(m_used - m_new) : 1.f;
+#pragma unroll
+                        for (int c = 0; c < kD; c += 32) {
+                            float ov[32];
+                            tmem_ld32(tO + lane_off + c, ov);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) ov[i] *= f;
+                            tmem_st32(tO + lane_off + c, ov);
+                        }
+                        tmem_wait_st();
+                        if (need) {
+                            l *= f;
+                            m_used = m_new;
+                        }
+                    }
+                }
+                float psum = 0.f;
+                uint32_t pk[kKeys / 2];
+                if (m_used != -INFINITY) {
+                    const float neg = -m_used;
+                    float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int j = 0; j < kKeys; j += 2) {
+                        const float e0 = fast_exp2(fmaf(sc[j], sl2, neg));
+                        const float e1 = fast_exp2(fmaf(sc[j + 1], sl2, neg));
+                        ps8[(j >> 1) & 7] += e0 + e1;
+                        __nv_bfloat162 v2 = __floats2bfloat162_rn(e0, e1);
+                        pk[j / 2] = *reinterpret_cast<uint32_t *>(&v2);
+                    }
+                    psum = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < kKeys / 2; ++j) pk[j] = 0u;
+                }
+                l += psum;
+                // P over the first 32 columns of S buffer bs (bf16 pairs: key 2c in
+                // the low half of column c), the A operand of P V
+                tmem_st32(tS + 64 * bs + lane_off, reinterpret_cast<const float *>(pk));
+                tmem_wait_st();
+                fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarPReady + bs));
+            }
+            if (failed) break;
+            // the unit's last P V has landed in O
+            failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarODone + ((T - 1) & 1)), ((T - 1) >> 1) & 1));
             if (failed) break;
             fence_after_sync();
-            float sc[kKeys];
-            tmem_ld32(tS + 64 * bs + lane_off, sc);
-            tmem_ld32(tS + 64 * bs + 32 + lane_off, sc + 32);
-            tmem_wait_ld();
-            // S(w, its last leaf tile) has completed: Q_w may now be replaced by q_seq
-            if (swap_q && c_w == n_lw - 1) {
-                if (q_tma) load_q_tma(tm_qs);
-                else load_q(p.q_seq);
-            }
-
-            // visible keys of this tile, [lo, hi) in tile-local index: the leaves
-            // are stored head by head, K_L per head; a sequence tile is cut by
-            // the causal limit
-            int lo, hi;
-            if (t < n_leaf_tiles) {
-                lo = (g - g_first) * p.K_L - t * kKeys;
-                hi = lo + p.K_L;
-            } else {
-                lo = 0;
-                hi = last_key + 1 - (t - n_leaf_tiles) * kKeys;
-            }
-            if (!row_ok) hi = lo;
-            if (!(lo <= 0 && hi >= kKeys)) {
-#pragma unroll
-                for (int j = 0; j < kKeys; ++j) sc[j] = (j >= lo && j < hi) ? sc[j] : -INFINITY;
-            }
-            // row max with 8 independent chains
-            float mx8[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mx8[k] = sc[k];
-#pragma unroll
-            for (int j = 8; j < kKeys; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], sc[j]);
-            const float tmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-            const float m_new = fmaxf(m_used, tmax * sl2);   // scores in log2 units (sl2 > 0)
-            if (c_w == 0) {
-                m_used = m_new;   // O_w is initialised by the first P V
-            } else {
-                const bool need = m_new > m_used + kRescaleLog2;   // also when m_used is still -inf
-                if (__any_sync(0xffffffffu, need)) {
-                    // O_w may be rescaled only once the previous P V has landed in it
-                    failed = __any_sync(0xffffffffu,
-                                        !mbar_wait(bar(kBarODone + 2 * w + ((c_w - 1) & 1)), ((c_w - 1) >> 1) & 1));
-                    if (failed) break;
-                    fence_after_sync();
-                    const float f = need ? fast_exp2(m_used - m_new) : 1.f;
-#pragma unroll
-                    for (int c = 0; c < kD; c += 32) {
-                        float ov[32];
-                        tmem_ld32(tO + lane_off + c, ov);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) ov[i] *= f;
-                        tmem_st32(tO + lane_off + c, ov);
-                    }
-                    tmem_wait_st();
-                    if (need) {
-                        l *= f;
-                        m_used = m_new;
-                    }
-                }
-            }
-            float psum = 0.f;
-            uint32_t pk[kKeys / 2];
-            if (m_used != -INFINITY) {
-                const float neg = -m_used;
-                float ps8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int j = 0; j < kKeys; j += 2) {
-                    const float e0 = fast_exp2(fmaf(sc[j], sl2, neg));
-                    const float e1 = fast_exp2(fmaf(sc[j + 1], sl2, neg));
-                    ps8[(j >> 1) & 7] += e0 + e1;
-                    __nv_bfloat162 v2 = __floats2bfloat162_rn(e0, e1);
-                    pk[j / 2] = *reinterpret_cast<uint32_t *>(&v2);
-                }
-                psum = ((ps8[0] + ps8[1]) + (ps8[2] + ps8[3])) + ((ps8[4] + ps8[5]) + (ps8[6] + ps8[7]));
-            } else {
-#pragma unroll
-                for (int j = 0; j < kKeys / 2; ++j) pk[j] = 0u;
-            }
-            l += psum;
-            // P(t) over the first 32 columns of S buffer bs (bf16 pairs: key 2c in
-            // the low half of column c), the A operand of P V
-            tmem_st32(tS + 64 * bs + lane_off, reinterpret_cast<const float *>(pk));
-            tmem_wait_st();
-            fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kBarPReady + 2 * w + bs));
-            ++c_w;
-        }
-        if (!failed && c_w > 0) {
-            failed = __any_sync(0xffffffffu,
-                                !mbar_wait(bar(kBarODone + 2 * w + ((c_w - 1) & 1)), ((c_w - 1) >> 1) & 1));
-            fence_after_sync();
-        }
-        if (!failed && c_w > 0) {
             const float inv = 1.f / l;
-            const size_t grow = (size_t)grp_id * GN + (row_ok ? row : 0);   // row of the group-row layout
+            const size_t grow = (size_t)U.grp * GN + (row_ok ? row : 0);   // row of the group-row layout
             // lambda merge of the two blocks ("Quick read / How it works" merge
             // equation): lam_kg = e^{LSE_kg} / (e^{LSE_kg} + e^{LSE_seq}), in log2 units
             float lam_kg = 1.f, lam_seq = 0.f, lse2 = m_used + log2f(l);
@@ -526,7 +521,7 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
                 lse2 = M + log2f(wk + wq);
                 os = p.oseq + grow * kD;
             }
-            __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.out) + (((size_t)b * p.N + n) * p.H + h) * kD;
+            __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.out) + (((size_t)U.b * p.N + n) * p.H + h) * kD;
             float *odst = p.mode == kAttnSeq ? p.oseq + grow * kD : nullptr;
             const float a = inv * lam_kg;
 #pragma unroll
@@ -534,6 +529,12 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
                 float ov[32];
                 tmem_ld32(tO + lane_off + c, ov);
                 tmem_wait_ld();
+                if (c == kD - 32) {
+                    // O has been read: the next unit's first P V may overwrite it
+                    fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(kBarODrained));
+                }
                 if (!row_ok) continue;
                 if (odst) {
 #pragma unroll
@@ -569,8 +570,11 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
             if (row_ok) {
                 const float lse_nat = lse2 * 0.69314718055994530942f;
                 if (p.mode == kAttnSeq) p.lse_seq[grow] = lse_nat;
-                else if (p.lse) p.lse[((size_t)b * p.N + n) * p.H + h] = lse_nat;
+                else if (p.lse) p.lse[((size_t)U.b * p.N + n) * p.H + h] = lse_nat;
             }
+            if (!has_next) break;
+            u = un;
+            U = tc_unit(p, u, ctas_per_group);
         }
         if (failed && lane == 0) set_status(p.status, kDevTimeout);
     } else if (warp == kProducerWarp) {
@@ -578,18 +582,19 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
         const __nv_bfloat16 *lkb = reinterpret_cast<const __nv_bfloat16 *>(p.lk_base);
         const __nv_bfloat16 *lvb = reinterpret_cast<const __nv_bfloat16 *>(p.lv_base);
         bool failed = false;
-        int pending = -1;   // leaf tile whose cp.async copies are in flight, not yet announced
-        // leaf rows of keys `lane` and `lane + 32` of leaf tile lt (-1: none), fetched one tile ahead
-        auto fetch_rows = [&](int lt, int *rk, int *rv) {
+        int pending = -1;      // leaf tile (running count) whose cp.async copies are in flight, not yet announced
+        uint32_t leafbits = 0; // bit (T mod 32): tile T was gathered (its full barrier is announced by this warp)
+        // leaf rows of keys `lane` and `lane + 32` of leaf tile lt of unit U (-1: none)
+        auto fetch_rows = [&](const TcUnit &U, int lt, int *rk, int *rv) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int j = lt * kKeys + lane + 32 * u;
-                rk[u] = rv[u] = -1;
-                if (j < n_leaf) {
-                    const int gg = g_first + j / p.K_L, jj = j - (j / p.K_L) * p.K_L;
-                    const long long e = ((long long)b * p.H + hkv * p.G + gg) * p.K_L + jj;
-                    rk[u] = (int)(p.leaf_head_stride * hkv + p.lk_idx[e]);
-                    rv[u] = (int)(p.leaf_head_stride * hkv + p.lv_idx[e]);
+            for (int v = 0; v < 2; ++v) {
+                const int j = lt * kKeys + lane + 32 * v;
+                rk[v] = rv[v] = -1;
+                if (j < U.n_leaf) {
+                    const int gg = U.g_first + j / p.K_L, jj = j - (j / p.K_L) * p.K_L;
+                    const long long e = ((long long)U.b * p.H + U.hkv * p.G + gg) * p.K_L + jj;
+                    rk[v] = (int)(p.leaf_head_stride * U.hkv + p.lk_idx[e]);
+                    rv[v] = (int)(p.leaf_head_stride * U.hkv + p.lv_idx[e]);
                 }
             }
         };
@@ -617,56 +622,62 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
             }
             pending = -1;
         };
-        int nk[2] = {-1, -1}, nv[2] = {-1, -1};
-        int k_issued = 0, v_issued = 0;   // tiles whose K / V copies have been issued
-        if (n_leaf_tiles > 0) fetch_rows(0, nk, nv);
-        for (int t = 0; t < n_tiles; ++t) {
-            const int sk = t % kKStages, sv = t % kVStages;
-            const bool leaf = t < n_leaf_tiles;
-            const int st = t - n_leaf_tiles;   // sequence tile index
-            const uint32_t kd = sb + kOffK + sk * kKVBytes, vd = sb + kOffV + sv * kKVBytes;
-            if (t >= kKStages) {
-                failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarEmptyK + sk), ((t / kKStages) + 1) & 1));
-                if (failed) break;
-            }
-            int rk[2] = {-1, -1}, rv[2] = {-1, -1};
-            if (leaf) {
-                rk[0] = nk[0];
-                rk[1] = nk[1];
-                rv[0] = nv[0];
-                rv[1] = nv[1];
-                if (t + 1 < n_leaf_tiles) fetch_rows(t + 1, nk, nv);
-                gather(kd, lkb, rk);
-                k_issued = t + 1;
-            } else {
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(bar(kBarFullK + sk), kKVBytes);
-#pragma unroll
-                    for (int half = 0; half < 2; ++half)
-                        tma_load_4d(kd + half * (kKeys * 128), tm_k, half * 64, hkv, st * kKeys, b, bar(kBarFullK + sk));
+        int T = 0, k_issued = 0, v_issued = 0;   // tiles so far; tiles whose K / V copies have been issued
+        for (unsigned u = u0; u < n_units && !failed; u += ustride) {
+            const TcUnit U = tc_unit(p, u, ctas_per_group);
+            int nk[2] = {-1, -1}, nv[2] = {-1, -1};
+            if (U.n_leaf_tiles > 0) fetch_rows(U, 0, nk, nv);
+            for (int t = 0; t < U.n_tiles; ++t, ++T) {
+                const int sk = T % kKStages, sv = T % kVStages;
+                const bool leaf = t < U.n_leaf_tiles;
+                const int st = t - U.n_leaf_tiles;   // sequence tile index
+                const uint32_t kd = sb + kOffK + sk * kKVBytes, vd = sb + kOffV + sv * kKVBytes;
+                if (T >= kKStages) {
+                    failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarEmptyK + sk), ((T / kKStages) + 1) & 1));
+                    if (failed) break;
                 }
-                __syncwarp();
-                k_issued = t + 1;
-            }
-            // the previous leaf tile goes out before any wait on a V stage
-            if (pending >= 0) announce(leaf ? 1 : 0);
-            if (t >= kVStages) {
-                failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarEmptyV + sv), ((t / kVStages) + 1) & 1));
-                if (failed) break;
-            }
-            if (leaf) {
-                gather(vd, lvb, rv);
-                pending = t;
-            } else {
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(bar(kBarFullV + sv), kKVBytes);
+                int rk[2] = {-1, -1}, rv[2] = {-1, -1};
+                if (leaf) {
+                    rk[0] = nk[0];
+                    rk[1] = nk[1];
+                    rv[0] = nv[0];
+                    rv[1] = nv[1];
+                    if (t + 1 < U.n_leaf_tiles) fetch_rows(U, t + 1, nk, nv);
+                    gather(kd, lkb, rk);
+                    leafbits |= 1u << (T & 31);
+                } else {
+                    leafbits &= ~(1u << (T & 31));
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar(kBarFullK + sk), kKVBytes);
 #pragma unroll
-                    for (int half = 0; half < 2; ++half)
-                        tma_load_4d(vd + half * (kKeys * 128), tm_v, half * 64, hkv, st * kKeys, b, bar(kBarFullV + sv));
+                        for (int half = 0; half < 2; ++half)
+                            tma_load_4d(kd + half * (kKeys * 128), tm_k, half * 64, U.hkv, st * kKeys, U.b,
+                                        bar(kBarFullK + sk));
+                    }
+                    __syncwarp();
                 }
-                __syncwarp();
+                k_issued = T + 1;
+                // the previous leaf tile goes out before any wait on a V stage
+                if (pending >= 0) announce(leaf ? 1 : 0);
+                if (T >= kVStages) {
+                    failed = __any_sync(0xffffffffu, !mbar_wait(bar(kBarEmptyV + sv), ((T / kVStages) + 1) & 1));
+                    if (failed) break;
+                }
+                if (leaf) {
+                    gather(vd, lvb, rv);
+                    pending = T;
+                } else {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar(kBarFullV + sv), kKVBytes);
+#pragma unroll
+                        for (int half = 0; half < 2; ++half)
+                            tma_load_4d(vd + half * (kKeys * 128), tm_v, half * 64, U.hkv, st * kKeys, U.b,
+                                        bar(kBarFullV + sv));
+                    }
+                    __syncwarp();
+                }
+                v_issued = T + 1;
             }
-            v_issued = t + 1;
         }
         if (!failed && pending >= 0) announce(0);
         // The CTA must not exit with copies in flight, on the failure path too:
@@ -676,9 +687,11 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
         // (sequence) tiles are waited for.
         bool drained = true;
         for (int t = max(0, k_issued - kKStages); t < k_issued; ++t)
-            if (!failed || t >= n_leaf_tiles) drained &= mbar_wait(bar(kBarFullK + t % kKStages), (t / kKStages) & 1);
+            if (!failed || !((leafbits >> (t & 31)) & 1u))
+                drained &= mbar_wait(bar(kBarFullK + t % kKStages), (t / kKStages) & 1);
         for (int t = max(0, v_issued - kVStages); t < v_issued; ++t)
-            if (!failed || t >= n_leaf_tiles) drained &= mbar_wait(bar(kBarFullV + t % kVStages), (t / kVStages) & 1);
+            if (!failed || !((leafbits >> (t & 31)) & 1u))
+                drained &= mbar_wait(bar(kBarFullV + t % kVStages), (t / kVStages) & 1);
         cp_wait_all();
         if ((failed || !drained) && lane == 0) set_status(p.status, kDevTimeout);
     } else {
@@ -692,59 +705,60 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
             const uint64_t dq0 = make_desc(sb + kOffQ, 16, 1024);
             const uint64_t dk0 = make_desc(sb + kOffK, 16, 1024);
             const uint64_t dv0 = make_desc(sb + kOffV, kKeys * 128, 1024);
-            auto issue_s = [&](int t) -> bool {
-                const int sk = t % kKStages;
-                if (!mbar_wait(bar(kBarFullK + sk), (t / kKStages) & 1)) return false;
-#pragma unroll
-                for (int w = 0; w < kWG; ++w) {
-                    if (!wg_takes(w, t)) continue;
-                    const int cs = wg_count(w, t), bs = cs & 1;
-                    if (cs == 0 && !mbar_wait(bar(kBarQReady + w), 0)) return false;
-                    // the warpgroup's first sequence tile after its leaves: Q_w has been replaced by q_seq
-                    if (t == n_leaf_tiles && cs > 0 && !mbar_wait(bar(kBarQReady + w), 1)) return false;
-                    // buffer bs still holds the P of this warpgroup's tile two back until its P V has completed
-                    if (cs >= 2 && !mbar_wait(bar(kBarODone + 2 * w + bs), ((cs - 2) >> 1) & 1)) return false;
-                    fence_after_sync();
-                    const uint64_t qd = dq0 + (uint64_t)((w * kQBytes) >> 4);
-                    const uint64_t kdsc = dk0 + (uint64_t)((sk * kKVBytes) >> 4);
-                    const uint32_t td = tmem + 256 * w + 64 * bs;
-#pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
-                        mma_bf16(td, qd + (uint64_t)(((ks >> 2) * (kRows * 128) + (ks & 3) * 32) >> 4),
-                                 kdsc + (uint64_t)(((ks >> 2) * (kKeys * 128) + (ks & 3) * 32) >> 4), idesc_s,
-                                 ks > 0 ? 1u : 0u);
-                    }
-                    mma_commit(bar(kBarSFull + 2 * w + bs));
+            int q_loads = 0;   // Q loads consumed so far (QReady phase)
+            auto issue_s = [&](int T, bool new_q) -> bool {
+                const int sk = T % kKStages, bs = T & 1;
+                if (!mbar_wait(bar(kBarFullK + sk), (T / kKStages) & 1)) return false;
+                if (new_q) {
+                    if (!mbar_wait(bar(kBarQReady), q_loads & 1)) return false;
+                    ++q_loads;
                 }
+                // buffer bs still holds the P of tile T - 2 until its P V has completed
+                if (T >= 2 && !mbar_wait(bar(kBarODone + bs), ((T - 2) >> 1) & 1)) return false;
+                fence_after_sync();
+                const uint64_t kdsc = dk0 + (uint64_t)((sk * kKVBytes) >> 4);
+                const uint32_t td = tmem + 64 * bs;
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks)
+                    mma_bf16(td, dq0 + (uint64_t)(((ks >> 2) * (kRows * 128) + (ks & 3) * 32) >> 4),
+                             kdsc + (uint64_t)(((ks >> 2) * (kKeys * 128) + (ks & 3) * 32) >> 4), idesc_s,
+                             ks > 0 ? 1u : 0u);
+                mma_commit(bar(kBarSFull + bs));
                 mma_commit(bar(kBarEmptyK + sk));
                 return true;
             };
-            auto issue_pv = [&](int u) -> bool {
-                const int sv = u % kVStages;
-                if (!mbar_wait(bar(kBarFullV + sv), (u / kVStages) & 1)) return false;
+            // P V of tile T; first: the first tile of unit ui (O starts from zero
+            // once the previous unit's O has been read out)
+            auto issue_pv = [&](int T, bool first, int ui) -> bool {
+                const int sv = T % kVStages, bs = T & 1;
+                if (!mbar_wait(bar(kBarFullV + sv), (T / kVStages) & 1)) return false;
+                if (!mbar_wait(bar(kBarPReady + bs), (T >> 1) & 1)) return false;
+                if (first && ui > 0 && !mbar_wait(bar(kBarODrained), (ui - 1) & 1)) return false;
+                fence_after_sync();
+                const uint32_t ta = tmem + 64 * bs, td = tmem + 128;
+                const uint64_t vdsc = dv0 + (uint64_t)((sv * kKVBytes) >> 4);
 #pragma unroll
-                for (int w = 0; w < kWG; ++w) {
-                    if (!wg_takes(w, u)) continue;
-                    const int lc = wg_count(w, u), bs = lc & 1;
-                    if (!mbar_wait(bar(kBarPReady + 2 * w + bs), (lc >> 1) & 1)) return false;
-                    fence_after_sync();
-                    const uint32_t ta = tmem + 256 * w + 64 * bs, td = tmem + 256 * w + 128;
-                    const uint64_t vdsc = dv0 + (uint64_t)((sv * kKVBytes) >> 4);
-#pragma unroll
-                    for (int ks = 0; ks < kKeys / 16; ++ks)
-                        mma_bf16_ts(td, ta + 8 * ks, vdsc + (uint64_t)((ks * 16 * 128) >> 4), idesc_o,
-                                    (lc > 0 || ks > 0) ? 1u : 0u);
-                    mma_commit(bar(kBarODone + 2 * w + bs));
-                }
+                for (int ks = 0; ks < kKeys / 16; ++ks)
+                    mma_bf16_ts(td, ta + 8 * ks, vdsc + (uint64_t)((ks * 16 * 128) >> 4), idesc_o,
+                                (!first || ks > 0) ? 1u : 0u);
+                mma_commit(bar(kBarODone + bs));
                 mma_commit(bar(kBarEmptyV + sv));
                 return true;
             };
             bool ok = true;
-            for (int t = 0; t < n_tiles && ok; ++t) {
-                ok = issue_s(t);
-                if (ok && t > 0) ok = issue_pv(t - 1);
+            int T = 0, ui = 0, prev_ui = 0;
+            bool prev_first = false;
+            for (unsigned u = u0; u < n_units && ok; u += ustride, ++ui) {
+                const TcUnit U = tc_unit(p, u, ctas_per_group);
+                for (int t = 0; t < U.n_tiles && ok; ++t, ++T) {
+                    // a new Q: the unit's first tile, and its first sequence tile after leaves
+                    ok = issue_s(T, t == 0 || (t == U.n_leaf_tiles && t > 0));
+                    if (ok && T > 0) ok = issue_pv(T - 1, prev_first, prev_ui);
+                    prev_first = t == 0;
+                    prev_ui = ui;
+                }
             }
-            if (ok) ok = issue_pv(n_tiles - 1);
+            if (ok && T > 0) ok = issue_pv(T - 1, prev_first, prev_ui);
             // before TMEM is released, every MMA this thread committed must have
             // completed, on the failure path too: one more commit tracks them all
             mma_commit(bar(kBarDrain));
@@ -760,23 +774,26 @@ __device__ __forceinline__ void attend_tc_cta(const AttnParams &p, const unsigne
     if (warp == kMmaWarp) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
-// One call: one CTA per (query b, KV head, kWG x 128-row block of the group's
-// G N rows).  tm_k / tm_v: the sequence keys / values [B][T][H_kv][D] as 4-D
-// tensor maps (D, H_kv, T, B) with a (64, 1, 64, 1) box and 128-byte swizzle;
-// with q_maps, tm_qs / tm_qk: q_seq / q_kg [B][N][H][D] as (D, H, N, B) with a
-// (64, 1, min(N, 128), 1) box (else Q is loaded by cp.async).
+// One call: n_units units of (query b, KV head, 128-row block of the group's
+// G N rows), a persistent grid (at most as many CTAs as fit on the device)
+// taking them round-robin.  tm_k / tm_v: the sequence keys / values
+// [B][T][H_kv][D] as 4-D tensor maps (D, H_kv, T, B) with a (64, 1, 64, 1) box
+// and 128-byte swizzle; with q_maps, tm_qs / tm_qk: q_seq / q_kg [B][N][H][D]
+// as (D, H, N, B) with a (64, 1, min(N, 128), 1) box (else Q by cp.async).
 __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
-    attend_tc_kernel(const __grid_constant__ AttnParams p, int ctas_per_group, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qs,
-                     const __grid_constant__ CUtensorMap tm_qk, int q_maps)
+    attend_tc_kernel(const __grid_constant__ AttnParams p, int ctas_per_group, unsigned n_units,
+                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_qk, int q_maps)
 {
     griddep_launch();
     griddep_wait();   // the kept lists (and everything else) of the previous grid are visible
-    attend_tc_cta(p, blockIdx.x, ctas_per_group, &tm_k, &tm_v, q_maps ? &tm_qs : nullptr, q_maps ? &tm_qk : nullptr);
+    attend_tc_run(p, ctas_per_group, blockIdx.x, gridDim.x, n_units, &tm_k, &tm_v, q_maps ? &tm_qs : nullptr,
+                  q_maps ? &tm_qk : nullptr);
 }
 
 // Several layers' calls in one launch (same shapes, each layer its own
-// inputs and kept leaves): layer l owns the CTAs [offs[l], offs[l + 1]).
+// inputs and kept leaves): layer l owns the CTAs [offs[l], offs[l + 1]), one
+// unit each.
 constexpr int kMaxAttnLayers = 32;
 struct AttnBatch {
     CUtensorMap mk[kMaxAttnLayers], mv[kMaxAttnLayers];
@@ -790,7 +807,8 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
 {
     int l = 0;
     while (l + 1 < b.n && blockIdx.x >= b.offs[l + 1]) ++l;
-    attend_tc_cta(b.p[l], blockIdx.x - b.offs[l], b.ctas_per_group, &b.mk[l], &b.mv[l], nullptr, nullptr);
+    const unsigned u = blockIdx.x - b.offs[l];
+    attend_tc_run(b.p[l], b.ctas_per_group, u, 1u, u + 1, &b.mk[l], &b.mv[l], nullptr, nullptr);
 }
 
 }  // namespace akv
