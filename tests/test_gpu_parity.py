@@ -150,6 +150,35 @@ def test_small_trees(case):
     compare(w, K, g)
 
 
+# The bf16 tensor-core attention runs a persistent grid of two CTAs per SM over
+# units of 128 query rows; these shapes have more units than a B200 has CTA
+# slots (296), a ragged last round, and short units (one leaf tile, one or two
+# sequence tiles), so a CTA crosses many unit boundaries: the Q switch to the
+# next unit, O started afresh once the previous unit's O has been read.
+PERSISTENT = [
+    # (H, H_kv, N, T, B): N = 64 loads Q by TMA, N = 48 by cp.async (heads cut by row blocks)
+    (8, 2, 64, 70, 80),     # 320 units
+    (6, 2, 48, 50, 100),    # 400 units
+]
+
+
+@pytest.mark.parametrize("case", PERSISTENT, ids=["q_tma", "q_cp_async"])
+def test_persistent_attention_many_units(case):
+    H, H_kv, N, T, B = case
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=H, n_kv_heads=H_kv, head_dim=128, fanout=(6, 6, 6),
+                      keep=(3, 3, 9), batch=B, n_tokens=N, seq_len=T, permuted=True)
+    w = synth.make_workload(sh, "cuda", 99)
+    g = gpu_run(w, sh.keep)
+    check_structure(w, sh.keep, g)
+    compare(w, sh.keep, g, traversals=sample_traversals(B, H, 40, seed=3))
+    # the same units through the host-leaf path: sequence part and knowledge
+    # part as separate persistent launches, merged
+    hw = synth.Workload(sh, w.root_keys, w.mid_keys, w.leaf_keys.cpu().pin_memory(),
+                        w.leaf_values.cpu().pin_memory(), w.root_child, w.mid_child, w.q_kg, w.q_seq, w.k_seq,
+                        w.v_seq, w.targets)
+    same_as_hbm_path(g, gpu_run(hw, sh.keep))
+
+
 def test_balanced_lambda_regime():
     # KG queries scaled so the KG and sequence log-sum-exps are comparable and
     # both lambda weights matter.
