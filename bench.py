@@ -147,12 +147,11 @@ def attend_kernel_name(sh):
     import torch
     if sh.dtype == torch.float32:
         return "attend_f32_kernel"
-    return "attend_tc_kernel" if sh.head_dim == 128 else "attend_bf16_kernel"
+    return "attend_tc_kernel"
 
 
 # Source files of each profiled stage (the descent is a chain of kernels).
-KERNEL_SOURCES = {"attend_tc_kernel": ["attend_tc.cuh"], "attend_bf16_kernel": ["attend.cuh"],
-                  "attend_f32_kernel": ["attend.cuh"], "descent": ["descend.cuh", "descend_pm.cuh"],
+KERNEL_SOURCES = {"attend_tc_kernel": ["attend_tc.cuh"], "attend_f32_kernel": ["attend.cuh"], "descent": ["descend.cuh", "descend_pm.cuh"],
                   "stage_blocks_kernel": ["staging.cuh"]}
 
 

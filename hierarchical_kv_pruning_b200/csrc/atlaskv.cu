@@ -655,20 +655,6 @@ atlaskv_status dispatch_pm(const atlaskv_tree *t, const PmPlan &pp, const akv::D
 
 // ---- attention launch -----------------------------------------------------
 template <int D>
-atlaskv_status launch_attend_bf16(const akv::AttnParams &ap, cudaStream_t s)
-{
-    const int nchunks = (ap.N + 15) / 16;
-    const int bpg = (ap.G * nchunks + akv::kAttnWarps - 1) / akv::kAttnWarps;
-    const long long grid = (long long)ap.B * ap.H_kv * bpg;
-    if (grid > 0x7fffffffLL) return fail(ATLASKV_EUNSUPPORTED, "attention grid too large");
-    const int smem = akv::AttnSmem<D>::BYTES;
-    AKV_SMEM(akv::attend_bf16_kernel<D>, smem);
-    akv::attend_bf16_kernel<D><<<(unsigned)grid, akv::kAttnWarps * 32, smem, s>>>(ap, bpg);
-    AKV_CUDA(cudaGetLastError());
-    return ATLASKV_OK;
-}
-
-template <int D>
 atlaskv_status launch_attend_f32(const akv::AttnParams &ap, cudaStream_t s)
 {
     const long long rows = (long long)ap.B * ap.N * ap.H;
@@ -680,10 +666,11 @@ atlaskv_status launch_attend_f32(const akv::AttnParams &ap, cudaStream_t s)
 }
 
 // 4-D tensor map (bf16, 128-byte swizzle, zero fill outside) over a tensor
-// [d3][d2][d1][D] (D = 128 innermost) with a (64, 1, rows, 1) box, for the
-// attention kernel.  cuTensorMapEncodeTiled is a host-only call, reached
+// [d3][d2][d1][D] (D = 64 or 128 innermost) with a (64, 1, rows, 1) box, for
+// the attention kernel.  cuTensorMapEncodeTiled is a host-only call, reached
 // through the runtime's driver entry point.
-atlaskv_status encode_tc_map(CUtensorMap *map, const void *base, long long d1, long long d2, long long d3, int rows)
+atlaskv_status encode_tc_map(CUtensorMap *map, const void *base, int D, long long d1, long long d2, long long d3,
+                             int rows)
 {
     // looked up once per process (thread-safe static initialisation)
     static const PFN_cuTensorMapEncodeTiled_v12000 encode = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
@@ -696,7 +683,6 @@ atlaskv_status encode_tc_map(CUtensorMap *map, const void *base, long long d1, l
     }();
     if (!encode) return fail(ATLASKV_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
     if (reinterpret_cast<uintptr_t>(base) & 15u) return fail(ATLASKV_EINVAL, "attention inputs must be 16-byte aligned");
-    const int D = akv::tc::kD;
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)d1, (cuuint64_t)d2, (cuuint64_t)d3};
     const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)(d1 * D * 2), (cuuint64_t)(d2 * d1 * D * 2)};
     const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
@@ -710,12 +696,13 @@ atlaskv_status encode_tc_map(CUtensorMap *map, const void *base, long long d1, l
 
 int num_sms();
 
-// bf16, D = 128: tcgen05 tensor cores, units of 128 query rows of a (query,
-// KV head) group on a persistent grid.  Sequence K / V [B][T][H_kv][D] by TMA
+// bf16, D = 64 or 128: tcgen05 tensor cores, units of 128 query rows of a
+// (query, KV head) group on a persistent grid.  Sequence K / V [B][T][H_kv][D] by TMA
 // (box of 64 keys); Q [B][N][H][D] by TMA too (box of min(N, 128) tokens of
 // one head) when every head's rows start on a swizzle atom of the Q tile, i.e.
 // N is a multiple of 8 that divides 128 or is divisible by it, else by
 // cp.async.
+template <int D>
 atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
 {
     const int rows = ap.G * ap.N;
@@ -726,9 +713,9 @@ atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
     if (ap.lk_rows >= (1LL << 31) || ap.lv_rows >= (1LL << 31))
         return fail(ATLASKV_EUNSUPPORTED, "more than 2^31 leaf rows");
     CUtensorMap mk, mv, mqs, mqk;
-    atlaskv_status st = encode_tc_map(&mk, ap.k_seq, ap.H_kv, ap.T, ap.B, akv::tc::kKeys);
+    atlaskv_status st = encode_tc_map(&mk, ap.k_seq, D, ap.H_kv, ap.T, ap.B, akv::tc::kKeys);
     if (st != ATLASKV_OK) return st;
-    st = encode_tc_map(&mv, ap.v_seq, ap.H_kv, ap.T, ap.B, akv::tc::kKeys);
+    st = encode_tc_map(&mv, ap.v_seq, D, ap.H_kv, ap.T, ap.B, akv::tc::kKeys);
     if (st != ATLASKV_OK) return st;
     // a mode that reads only one of the two query tensors uses it for both maps
     const void *qs = ap.q_seq ? ap.q_seq : ap.q_kg, *qk = ap.q_kg ? ap.q_kg : ap.q_seq;
@@ -736,14 +723,15 @@ atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
     const int q_maps = ap.N % 8 == 0 && (128 % ap.N == 0 || ap.N % 128 == 0) && aligned(qs) && aligned(qk);
     if (q_maps) {
         const int bn = ap.N < akv::tc::kRows ? ap.N : akv::tc::kRows;
-        st = encode_tc_map(&mqs, qs, ap.H, ap.N, ap.B, bn);
+        st = encode_tc_map(&mqs, qs, D, ap.H, ap.N, ap.B, bn);
         if (st != ATLASKV_OK) return st;
-        st = encode_tc_map(&mqk, qk, ap.H, ap.N, ap.B, bn);
+        st = encode_tc_map(&mqk, qk, D, ap.H, ap.N, ap.B, bn);
         if (st != ATLASKV_OK) return st;
     } else {
         mqs = mqk = mk;   // unused
     }
-    AKV_SMEM(akv::attend_tc_kernel, akv::tc::kSmemBytes);
+    constexpr int smem = akv::tc::TcSmem<D>::kBytes;
+    AKV_SMEM(akv::attend_tc_kernel<D>, smem);
     // persistent grid: as many CTAs as are resident at once, each taking units
     // round-robin.  Two per SM by construction (112 KB of shared memory, 256
     // TMEM columns, the launch bounds); the occupancy query reports one here
@@ -751,14 +739,14 @@ atlaskv_status launch_attend_tc(const akv::AttnParams &ap, cudaStream_t s)
     // measured 1.4x slower.
     const long long resident = (long long)akv::tc::kMinCtasPerSm * num_sms();
     const unsigned grid = (unsigned)(units < resident ? units : resident);
-    return launch_pdl(akv::attend_tc_kernel, grid, akv::tc::kThreads, akv::tc::kSmemBytes, s, ap, cpg,
+    return launch_pdl(akv::attend_tc_kernel<D>, grid, akv::tc::kThreads, smem, s, ap, cpg,
                       (unsigned)units, mk, mv, mqs, mqk, q_maps);
 }
 
 atlaskv_status dispatch_attend(int dtype, int D, const akv::AttnParams &ap, cudaStream_t s)
 {
     if (dtype == ATLASKV_F32) return D == 64 ? launch_attend_f32<64>(ap, s) : launch_attend_f32<128>(ap, s);
-    return D == 64 ? launch_attend_bf16<64>(ap, s) : launch_attend_tc(ap, s);
+    return D == 64 ? launch_attend_tc<64>(ap, s) : launch_attend_tc<128>(ap, s);
 }
 
 // ---- staging launches -----------------------------------------------------
@@ -992,6 +980,7 @@ atlaskv_status dispatch_descend_layers(int dtype, int D, const akv::DescendBatch
 }
 
 // The tensor-core attention of every layer in one launch, in `mode`.
+template <int D>
 atlaskv_status launch_attend_tc_layers(const Call *calls, int n, int mode, cudaStream_t s)
 {
     static akv::AttnBatch b;   // large: not on the stack; guarded below
@@ -1009,14 +998,15 @@ atlaskv_status launch_attend_tc_layers(const Call *calls, int n, int mode, cudaS
         b.p[l].mode = mode;
         b.offs[l] = (unsigned)(per * l);
         if (b.p[l].lk_rows >= (1LL << 31)) return fail(ATLASKV_EUNSUPPORTED, "more than 2^31 leaf rows");
-        atlaskv_status st = encode_tc_map(&b.mk[l], b.p[l].k_seq, a0.H_kv, a0.T, a0.B, akv::tc::kKeys);
+        atlaskv_status st = encode_tc_map(&b.mk[l], b.p[l].k_seq, D, a0.H_kv, a0.T, a0.B, akv::tc::kKeys);
         if (st != ATLASKV_OK) return st;
-        st = encode_tc_map(&b.mv[l], b.p[l].v_seq, a0.H_kv, a0.T, a0.B, akv::tc::kKeys);
+        st = encode_tc_map(&b.mv[l], b.p[l].v_seq, D, a0.H_kv, a0.T, a0.B, akv::tc::kKeys);
         if (st != ATLASKV_OK) return st;
     }
     b.offs[n] = (unsigned)(per * n);
-    AKV_SMEM(akv::attend_tc_layers_kernel, akv::tc::kSmemBytes);
-    akv::attend_tc_layers_kernel<<<(unsigned)(per * n), akv::tc::kThreads, akv::tc::kSmemBytes, s>>>(b);
+    constexpr int smem = akv::tc::TcSmem<D>::kBytes;
+    AKV_SMEM(akv::attend_tc_layers_kernel<D>, smem);
+    akv::attend_tc_layers_kernel<D><<<(unsigned)(per * n), akv::tc::kThreads, smem, s>>>(b);
     AKV_CUDA(cudaGetLastError());
     return ATLASKV_OK;
 }
@@ -1044,7 +1034,7 @@ atlaskv_status inflate_norms(atlaskv_tree *t)
 // attention is one launch after it.
 atlaskv_status init_tree_device(atlaskv_tree *t)
 {
-    t->split = t->d.dtype == ATLASKV_BF16 && t->d.head_dim == akv::tc::kD && t->host_leaves;
+    t->split = t->d.dtype == ATLASKV_BF16 && t->host_leaves;
     if (t->split) {
         // the sequence part runs beside the descent: lowest priority for it,
         // highest for the descent (the critical path); created once here so
@@ -1399,7 +1389,7 @@ atlaskv_status attend_impl(atlaskv_tree *t, const Ks &ks, const atlaskv_io *io, 
         akv::AttnParams a = ap;
         a.mode = akv::kAttnSeq;
         AKV_STEP(tm(2, t->seq_stream));
-        AKV_STEP(launch_attend_tc(a, t->seq_stream));
+        AKV_STEP(D == 64 ? launch_attend_tc<64>(a, t->seq_stream) : launch_attend_tc<128>(a, t->seq_stream));
         AKV_STEP(tm(3, t->seq_stream));
         AKV_CUDA(cudaEventRecord(t->fev[2], t->seq_stream));
         return ATLASKV_OK;
@@ -1736,21 +1726,24 @@ atlaskv_status atlaskv_attend_layers(int32_t n_layers, atlaskv_tree *const *tree
         AKV_STEP(tm(1, t0->desc_stream));
         AKV_CUDA(cudaEventRecord(t0->fev[1], t0->desc_stream));
         AKV_STEP(tm(2, t0->seq_stream));
-        AKV_STEP(launch_attend_tc_layers(calls, n_layers, akv::kAttnSeq, t0->seq_stream));
+        AKV_STEP(D == 64 ? launch_attend_tc_layers<64>(calls, n_layers, akv::kAttnSeq, t0->seq_stream)
+                         : launch_attend_tc_layers<128>(calls, n_layers, akv::kAttnSeq, t0->seq_stream));
         AKV_STEP(tm(3, t0->seq_stream));
         AKV_CUDA(cudaEventRecord(t0->fev[2], t0->seq_stream));
         AKV_CUDA(cudaStreamWaitEvent(s, t0->fev[1], 0));
         AKV_CUDA(cudaStreamWaitEvent(s, t0->fev[2], 0));
         AKV_STEP(tm(4, s));
-        AKV_STEP(launch_attend_tc_layers(calls, n_layers, akv::kAttnLeaf, s));
+        AKV_STEP(D == 64 ? launch_attend_tc_layers<64>(calls, n_layers, akv::kAttnLeaf, s)
+                         : launch_attend_tc_layers<128>(calls, n_layers, akv::kAttnLeaf, s));
         AKV_STEP(tm(5, s));
     } else {
         AKV_STEP(tm(0, s));
         AKV_STEP(dispatch_descend_layers(t0->d.dtype, D, db, pl.HT, pl.smem, dgrid, s));
         AKV_STEP(tm(1, s));
         AKV_STEP(tm(4, s));
-        if (t0->d.dtype == ATLASKV_BF16 && D == akv::tc::kD)   // every layer's attention in one launch
-            AKV_STEP(launch_attend_tc_layers(calls, n_layers, akv::kAttnFused, s));
+        if (t0->d.dtype == ATLASKV_BF16)   // every layer's attention in one launch
+            AKV_STEP(D == 64 ? launch_attend_tc_layers<64>(calls, n_layers, akv::kAttnFused, s)
+                             : launch_attend_tc_layers<128>(calls, n_layers, akv::kAttnFused, s));
         else
             for (int l = 0; l < n_layers; ++l) AKV_STEP(dispatch_attend(t0->d.dtype, D, calls[l].ap, s));
         AKV_STEP(tm(5, s));

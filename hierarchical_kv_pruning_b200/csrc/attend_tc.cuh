@@ -1,5 +1,5 @@
 // Knowledge + causal-sequence attention on the 5th-generation tensor cores
-// (tcgen05.mma, accumulators in Tensor Memory), bf16 inputs, D = 128.
+// (tcgen05.mma, accumulators in Tensor Memory), bf16 inputs, D = 64 or 128.
 //
 // Same computation as attend.cuh ("AtlasKV: Augmenting LLMs with Billion-Scale
 // Knowledge Graphs in 20GB VRAM": the lambda-weighted merge of the knowledge and
@@ -50,7 +50,6 @@ namespace tc {
 
 constexpr int kRows = 128;                 // query rows per warpgroup (UMMA M)
 constexpr int kKeys = 64;                  // keys per tile
-constexpr int kD = 128;                    // head dim
 constexpr int kKStages = 2;                // K ring depth (a stage is freed when S = Q K^T completes)
 constexpr int kVStages = 3;                // V ring depth (freed when P V completes; its wait bounds the K issue too)
 constexpr int kMinCtasPerSm = 2;           // one softmax warpgroup per CTA, two CTAs per SM
@@ -61,14 +60,6 @@ constexpr int kCtaRows = kRows;
 constexpr long long kSpinLimit = 1ll << 18;   // bounded mbarrier waits: try_wait iterations, not a fixed time
 constexpr float kRescaleLog2 = 8.f;            // rescale O only when the row max grows by more than this
 
-// shared memory (byte offsets from a 1024-aligned base; operand tiles in the
-// canonical 128-byte-swizzled UMMA layouts)
-constexpr int kQBytes = kRows * kD * 2;       // 32 KB: 2 K-blocks of [128 rows][64]
-constexpr int kKVBytes = kKeys * kD * 2;      // 16 KB: 2 blocks of [64 keys][64]
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;                    // [kKStages]
-constexpr int kOffV = kOffK + kKStages * kKVBytes;        // [kVStages]
-constexpr int kOffBar = kOffV + kVStages * kKVBytes;
 // mbarriers (8 bytes each); the [2] arrays are indexed by the parity of the
 // CTA's running tile count (tiles of all its units, in order)
 constexpr int kBarFullK = 0;                        // [kKStages] K tile landed
@@ -82,12 +73,27 @@ constexpr int kBarQReady = kBarODone + 2;           // Q loaded (one phase per l
 constexpr int kBarODrained = kBarQReady + 1;        // a unit's O read out of TMEM (4 warps)
 constexpr int kBarDrain = kBarODrained + 1;         // every MMA the issuing thread committed has completed
 constexpr int kNumBars = kBarDrain + 1;
-constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
-// No alignment slack: with no static shared memory the dynamic base is 1024-byte
-// aligned (the kernel checks it and reports EDEVICE otherwise), and 112 KB
+
+// Shared memory for head dim D (64 or 128): byte offsets from a 1024-aligned
+// base; operand tiles in the canonical 128-byte-swizzled UMMA layouts, made of
+// D / 64 blocks of 64 columns (one 128-byte row per block).  No alignment
+// slack: with no static shared memory the dynamic base is 1024-byte aligned
+// (the kernel checks it and reports EDEVICE otherwise); 112 KB at D = 128
 // keeps two CTAs per SM.
-constexpr int kSmemBytes = kOffTmemSlot + 16;
-constexpr int kTmemCols = 256;                 // S / P buffers [0, 128), O [128, 256)
+template <int D>
+struct TcSmem {
+    static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    static constexpr int kBlocks = D / 64;
+    static constexpr int kQBytes = kRows * D * 2;       // 32 / 16 KB
+    static constexpr int kKVBytes = kKeys * D * 2;      // 16 / 8 KB
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQBytes;                    // [kKStages]
+    static constexpr int kOffV = kOffK + kKStages * kKVBytes;        // [kVStages]
+    static constexpr int kOffBar = kOffV + kVStages * kKVBytes;
+    static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+    static constexpr int kBytes = kOffTmemSlot + 16;
+};
+constexpr int kTmemCols = 256;                 // S / P buffers [0, 128), O [128, 128 + D)
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -307,11 +313,15 @@ __device__ __forceinline__ TcUnit tc_unit(const AttnParams &p, unsigned u, int c
 // through tm_k / tm_v; Q by TMA through tm_qs / tm_qk when they are given and
 // every head of a block starts on a swizzle atom of the Q tile (N a multiple
 // of 8 that divides 128 or is divisible by it), else by cp.async.
+template <int D>
 __device__ __forceinline__ void attend_tc_run(const AttnParams &p, int ctas_per_group, unsigned u0, unsigned ustride,
                                               unsigned n_units, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
                                               const CUtensorMap *tm_qs, const CUtensorMap *tm_qk)
 {
     using namespace tc;
+    using SM = TcSmem<D>;
+    constexpr int kKVBytes = SM::kKVBytes, kOffQ = SM::kOffQ, kOffK = SM::kOffK, kOffV = SM::kOffV,
+                  kOffBar = SM::kOffBar, kOffTmemSlot = SM::kOffTmemSlot, kBlocks = SM::kBlocks;
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
     uint8_t *smem = tc_smem_raw;
     const uint32_t sb = smem_addr(smem);
@@ -362,26 +372,27 @@ __device__ __forceinline__ void attend_tc_run(const AttnParams &p, int ctas_per_
                 if (tid != 0) return;
                 const CUtensorMap *m = seq ? tm_qs : tm_qk;
                 const int bn = min(p.N, kRows);
-                mbar_arrive_expect_tx(bar(kBarQReady), (uint32_t)U.rows * kD * 2);
+                mbar_arrive_expect_tx(bar(kBarQReady), (uint32_t)U.rows * D * 2);
                 for (int rr = U.r0; rr < U.r0 + U.rows; rr += bn) {
                     const int gg = rr / p.N, tok = rr - gg * p.N;
 #pragma unroll
-                    for (int half = 0; half < 2; ++half)
+                    for (int half = 0; half < kBlocks; ++half)
                         tma_load_4d(qa + half * (kRows * 128) + (rr - U.r0) * 128, m, half * 64, U.hkv * p.G + gg, tok,
                                     U.b, bar(kBarQReady));
                 }
                 return;
             }
             const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(seq ? p.q_seq : p.q_kg);
-            const int lc = lrow & 15, lr = lrow >> 4;
+            constexpr int TPR = D / 8;   // threads per row: one 16-byte chunk each
+            const int lc = lrow % TPR, lr = lrow / TPR;
             const uint32_t dst0 = qa + (lc >> 3) * (kRows * 128);
 #pragma unroll 4
-            for (int i = 0; i < kRows / 8; ++i) {
-                const int rl = lr + 8 * i;
+            for (int i = 0; i < kRows * TPR / 128; ++i) {
+                const int rl = lr + (128 / TPR) * i;
                 const bool ok = rl < U.rows;
                 const int rr = U.r0 + (ok ? rl : 0);
                 const int gg = rr / p.N, nn = rr - gg * p.N;
-                const __nv_bfloat16 *src = q + (((size_t)U.b * p.N + nn) * p.H + U.hkv * p.G + gg) * kD + lc * 8;
+                const __nv_bfloat16 *src = q + (((size_t)U.b * p.N + nn) * p.H + U.hkv * p.G + gg) * D + lc * 8;
                 cp16(dst0 + sw128(rl, lc & 7), src, ok);
             }
             cp_commit();
@@ -458,7 +469,7 @@ __device__ __forceinline__ void attend_tc_run(const AttnParams &p, int ctas_per_
                         fence_after_sync();
                         const float f = need ? fast_exp2(m_used - m_new) : 1.f;
 #pragma unroll
-                        for (int c = 0; c < kD; c += 32) {
+                        for (int c = 0; c < D; c += 32) {
                             float ov[32];
                             tmem_ld32(tO + lane_off + c, ov);
                             tmem_wait_ld();
@@ -519,17 +530,17 @@ __device__ __forceinline__ void attend_tc_run(const AttnParams &p, int ctas_per_
                 lam_kg = wk / (wk + wq);
                 lam_seq = wq / (wk + wq);
                 lse2 = M + log2f(wk + wq);
-                os = p.oseq + grow * kD;
+                os = p.oseq + grow * D;
             }
-            __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.out) + (((size_t)U.b * p.N + n) * p.H + h) * kD;
-            float *odst = p.mode == kAttnSeq ? p.oseq + grow * kD : nullptr;
+            __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.out) + (((size_t)U.b * p.N + n) * p.H + h) * D;
+            float *odst = p.mode == kAttnSeq ? p.oseq + grow * D : nullptr;
             const float a = inv * lam_kg;
 #pragma unroll
-            for (int c = 0; c < kD; c += 32) {
+            for (int c = 0; c < D; c += 32) {
                 float ov[32];
                 tmem_ld32(tO + lane_off + c, ov);
                 tmem_wait_ld();
-                if (c == kD - 32) {
+                if (c == D - 32) {
                     // O has been read: the next unit's first P V may overwrite it
                     fence_before_sync();
                     __syncwarp();
@@ -598,14 +609,15 @@ __device__ __forceinline__ void attend_tc_run(const AttnParams &p, int ctas_per_
                 }
             }
         };
-        // cp.async of 64 gathered rows (two per warp instruction, 16 lanes per 256-byte row)
+        // cp.async of 64 gathered rows (D / 8 lanes per row, 256 / D rows per warp instruction)
         auto gather = [&](uint32_t dst, const __nv_bfloat16 *base, const int *rows2) {
-            const int c = lane & 15;
+            constexpr int CPR = D / 8, RPI = 32 / CPR;
+            const int c = lane % CPR;
 #pragma unroll 4
-            for (int i = 0; i < kKeys / 2; ++i) {
-                const int r = 2 * i + (lane >> 4);
-                const int x = __shfl_sync(0xffffffffu, i < 16 ? rows2[0] : rows2[1], r & 31);
-                cp16(dst + (c >> 3) * (kKeys * 128) + sw128(r, c & 7), x >= 0 ? base + (size_t)x * kD + c * 8 : base,
+            for (int i = 0; i < kKeys / RPI; ++i) {
+                const int r = RPI * i + lane / CPR;
+                const int x = __shfl_sync(0xffffffffu, RPI * i < 32 ? rows2[0] : rows2[1], r & 31);
+                cp16(dst + (c >> 3) * (kKeys * 128) + sw128(r, c & 7), x >= 0 ? base + (size_t)x * D + c * 8 : base,
                      x >= 0);
             }
             cp_commit();
@@ -650,7 +662,7 @@ __device__ __forceinline__ void attend_tc_run(const AttnParams &p, int ctas_per_
                     if (lane == 0) {
                         mbar_arrive_expect_tx(bar(kBarFullK + sk), kKVBytes);
 #pragma unroll
-                        for (int half = 0; half < 2; ++half)
+                        for (int half = 0; half < kBlocks; ++half)
                             tma_load_4d(kd + half * (kKeys * 128), tm_k, half * 64, U.hkv, st * kKeys, U.b,
                                         bar(kBarFullK + sk));
                     }
@@ -670,7 +682,7 @@ __device__ __forceinline__ void attend_tc_run(const AttnParams &p, int ctas_per_
                     if (lane == 0) {
                         mbar_arrive_expect_tx(bar(kBarFullV + sv), kKVBytes);
 #pragma unroll
-                        for (int half = 0; half < 2; ++half)
+                        for (int half = 0; half < kBlocks; ++half)
                             tma_load_4d(vd + half * (kKeys * 128), tm_v, half * 64, U.hkv, st * kKeys, U.b,
                                         bar(kBarFullV + sv));
                     }
@@ -698,7 +710,7 @@ __device__ __forceinline__ void attend_tc_run(const AttnParams &p, int ctas_per_
         // ================= MMA issue: one thread =================
         if (lane == 0) {
             const uint32_t idesc_s = make_idesc(kRows, kKeys, 0, 0);   // Q (K-major) x K^T (K-major)
-            const uint32_t idesc_o = make_idesc(kRows, kD, 0, 1);      // P (K-major) x V (MN-major)
+            const uint32_t idesc_o = make_idesc(kRows, D, 0, 1);      // P (K-major) x V (MN-major)
             // descriptors of the first tile of each operand region; a tile or
             // K-step offset is added to the start-address field (the low 14 bits,
             // in 16-byte units: shared addresses stay below 256 KB, so no carry)
@@ -719,7 +731,7 @@ __device__ __forceinline__ void attend_tc_run(const AttnParams &p, int ctas_per_
                 const uint64_t kdsc = dk0 + (uint64_t)((sk * kKVBytes) >> 4);
                 const uint32_t td = tmem + 64 * bs;
 #pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks)
+                for (int ks = 0; ks < D / 16; ++ks)
                     mma_bf16(td, dq0 + (uint64_t)(((ks >> 2) * (kRows * 128) + (ks & 3) * 32) >> 4),
                              kdsc + (uint64_t)(((ks >> 2) * (kKeys * 128) + (ks & 3) * 32) >> 4), idesc_s,
                              ks > 0 ? 1u : 0u);
@@ -780,6 +792,7 @@ __device__ __forceinline__ void attend_tc_run(const AttnParams &p, int ctas_per_
 // [B][T][H_kv][D] as 4-D tensor maps (D, H_kv, T, B) with a (64, 1, 64, 1) box
 // and 128-byte swizzle; with q_maps, tm_qs / tm_qk: q_seq / q_kg [B][N][H][D]
 // as (D, H, N, B) with a (64, 1, min(N, 128), 1) box (else Q by cp.async).
+template <int D>
 __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
     attend_tc_kernel(const __grid_constant__ AttnParams p, int ctas_per_group, unsigned n_units,
                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -787,7 +800,7 @@ __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
 {
     griddep_launch();
     griddep_wait();   // the kept lists (and everything else) of the previous grid are visible
-    attend_tc_run(p, ctas_per_group, blockIdx.x, gridDim.x, n_units, &tm_k, &tm_v, q_maps ? &tm_qs : nullptr,
+    attend_tc_run<D>(p, ctas_per_group, blockIdx.x, gridDim.x, n_units, &tm_k, &tm_v, q_maps ? &tm_qs : nullptr,
                   q_maps ? &tm_qk : nullptr);
 }
 
@@ -802,13 +815,14 @@ struct AttnBatch {
     int n, ctas_per_group;
 };
 
+template <int D>
 __global__ void __launch_bounds__(tc::kThreads, tc::kMinCtasPerSm)
     attend_tc_layers_kernel(const __grid_constant__ AttnBatch b)
 {
     int l = 0;
     while (l + 1 < b.n && blockIdx.x >= b.offs[l + 1]) ++l;
     const unsigned u = blockIdx.x - b.offs[l];
-    attend_tc_run(b.p[l], b.ctas_per_group, u, 1u, u + 1, &b.mk[l], &b.mv[l], nullptr, nullptr);
+    attend_tc_run<D>(b.p[l], b.ctas_per_group, u, 1u, u + 1, &b.mk[l], &b.mv[l], nullptr, nullptr);
 }
 
 }  // namespace akv

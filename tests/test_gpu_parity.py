@@ -156,16 +156,18 @@ def test_small_trees(case):
 # sequence tiles), so a CTA crosses many unit boundaries: the Q switch to the
 # next unit, O started afresh once the previous unit's O has been read.
 PERSISTENT = [
-    # (H, H_kv, N, T, B): N = 64 loads Q by TMA, N = 48 by cp.async (heads cut by row blocks)
-    (8, 2, 64, 70, 80),     # 320 units
-    (6, 2, 48, 50, 100),    # 400 units
+    # (H, H_kv, N, T, B, D): N = 64 loads Q by TMA, N = 48 by cp.async (heads cut by row blocks)
+    (8, 2, 64, 70, 80, 128),     # 320 units
+    (6, 2, 48, 50, 100, 128),    # 400 units
+    (8, 2, 64, 70, 80, 64),      # the same at D = 64 (one 64-column block per tile)
+    (6, 2, 48, 50, 100, 64),
 ]
 
 
-@pytest.mark.parametrize("case", PERSISTENT, ids=["q_tma", "q_cp_async"])
+@pytest.mark.parametrize("case", PERSISTENT, ids=["q_tma", "q_cp_async", "q_tma_d64", "q_cp_async_d64"])
 def test_persistent_attention_many_units(case):
-    H, H_kv, N, T, B = case
-    sh = synth.custom(dtype=torch.bfloat16, n_heads=H, n_kv_heads=H_kv, head_dim=128, fanout=(6, 6, 6),
+    H, H_kv, N, T, B, D = case
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=H, n_kv_heads=H_kv, head_dim=D, fanout=(6, 6, 6),
                       keep=(3, 3, 9), batch=B, n_tokens=N, seq_len=T, permuted=True)
     w = synth.make_workload(sh, "cuda", 99)
     g = gpu_run(w, sh.keep)
