@@ -393,13 +393,14 @@ def test_decode_step_single_token(dtype, D):
     compare(w, sh.keep, g)
 
 
+@pytest.mark.parametrize("D", [128, 64])
 @pytest.mark.parametrize("n_tokens", [1, 24])
-def test_layers_in_one_call_match_single_calls(n_tokens):
+def test_layers_in_one_call_match_single_calls(n_tokens, D):
     # Several layers, each with its own tree and inputs, in one batched call:
     # every layer's results equal its own single call bit for bit and match
     # the oracle.
     from hierarchical_kv_pruning_b200.binding import attend_layers
-    sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=128, fanout=(10, 9, 8),
+    sh = synth.custom(dtype=torch.bfloat16, n_heads=8, n_kv_heads=2, head_dim=D, fanout=(10, 9, 8),
                       keep=(3, 5, 16), batch=6, n_tokens=n_tokens, seq_len=40)
     layers = [synth.make_workload(sh, "cuda", 30 + l) for l in range(4)]
     trees = [HikvpTree.from_workload(w) for w in layers]
